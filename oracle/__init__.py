@@ -1,0 +1,193 @@
+"""fp64 CPU oracle for block-hybrid attention -- TEST INFRASTRUCTURE.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg (and its ``--impl reference`` arm) may import this package.  The product
+path (``block_hybrid_linear_b200``) never imports it, and this package never
+imports the product path: the two share no code.
+
+Method (paper "Retrofitting Linear Attention into Diffusion Language
+Models", arXiv 2608.06628; paper-daily summary page, sections "核心公式与算法"
+(core formula) and "具体技术细节示例" (worked example); fugumt abstract page):
+
+    y = softmax(Q_a K_a^T * scale) V_a + phi(Q_a) S_p,
+    S_p = sum over committed tokens of phi(k)^T v,   phi = ReLU.
+
+Readings where the pages are silent or garbled (each listed in the design
+notes): the feature term uses the active block's queries (the worked example
+writes phi(Q_2) S_1); the softmax is scaled by 1/sqrt(d); attention inside
+the block is bidirectional; the linear term is added unnormalised (weight 1)
+unless the shared-denominator option is selected.
+
+Every function takes float arrays (float32 values are widened to float64
+exactly), returns float64, and computes the plain definition in
+``bha_oracle.c``.  "parity unpinned": the shared-denominator variant is not
+on the pages; it is pinned only by its reduction to softmax when S = z = 0
+and by a brute-force restatement over prefix tokens.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        lib = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        lp = ctypes.POINTER(ctypes.c_long)
+        L = ctypes.c_long
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_threads.restype = ctypes.c_int
+        lib.oracle_max_threads.argtypes = []
+        lib.oracle_max_threads.restype = ctypes.c_int
+        lib.oracle_state_prefill.argtypes = [dp, dp, L, L, L, dp, dp]
+        lib.oracle_state_prefill.restype = None
+        lib.oracle_state_commit.argtypes = [dp, dp, dp, dp, L, L, L]
+        lib.oracle_state_commit.restype = None
+        lib.oracle_hybrid_step.argtypes = [dp, dp, dp, dp, dp, dp, L, L, L, L,
+                                           L, ctypes.c_double, ctypes.c_int]
+        lib.oracle_hybrid_step.restype = None
+        lib.oracle_prefix_softmax.argtypes = [dp, dp, dp, L, L, dp, dp, dp, L,
+                                              L, L, L, L, ctypes.c_double]
+        lib.oracle_prefix_softmax.restype = None
+        lib.oracle_block_partition.argtypes = [L, L, lp]
+        lib.oracle_block_partition.restype = L
+        _lib = lib
+    return _lib
+
+
+def _f64(a):
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def set_threads(n: int) -> int:
+    """OpenMP threads used by the oracle (parallel over independent units)."""
+    return _load().oracle_set_threads(int(n))
+
+
+def max_threads() -> int:
+    return _load().oracle_max_threads()
+
+
+def state_prefill(K, V, with_z=True):
+    """S = phi(K)^T V and z = sum_t phi(k_t) over a prompt.
+
+    K, V: [..., T, d] (leading dims are independent units, e.g. [n, hkv]).
+    Returns (S [..., d, d], z [..., d] or None).
+    """
+    K = _f64(K)
+    V = _f64(V)
+    assert K.shape == V.shape and K.ndim >= 2
+    lead, (T, d) = K.shape[:-2], K.shape[-2:]
+    units = int(np.prod(lead)) if lead else 1
+    S = np.zeros(lead + (d, d))
+    z = np.zeros(lead + (d,)) if with_z else None
+    _load().oracle_state_prefill(_ptr(K), _ptr(V), units, T, d, _ptr(S),
+                                 _ptr(z))
+    return S, z
+
+
+def state_commit(S, z, Kb, Vb):
+    """Return (S + phi(Kb)^T Vb, z + sum_t phi(kb_t)); inputs are not modified.
+
+    S [..., d, d], z [..., d] or None, Kb/Vb [..., b, d].
+    """
+    S = _f64(S).copy()
+    z = None if z is None else _f64(z).copy()
+    Kb = _f64(Kb)
+    Vb = _f64(Vb)
+    lead, (b, d) = Kb.shape[:-2], Kb.shape[-2:]
+    assert S.shape == lead + (d, d)
+    units = int(np.prod(lead)) if lead else 1
+    _load().oracle_state_commit(_ptr(S), _ptr(z), _ptr(Kb), _ptr(Vb), units,
+                                b, d)
+    return S, z
+
+
+def hybrid_step(Q, K, V, S, z=None, scale=0.0, shared=False):
+    """Block-hybrid attention output for the active block.
+
+    Q [n, hq, b, d]; K, V [n, hkv, b, d]; S [n, hkv, d, d]; z [n, hkv, d]
+    (required when shared).  scale <= 0 means 1/sqrt(d).
+    Returns Y [n, hq, b, d] in float64.
+    """
+    Q, K, V, S = _f64(Q), _f64(K), _f64(V), _f64(S)
+    n, hq, b, d = Q.shape
+    hkv = K.shape[1]
+    assert K.shape == (n, hkv, b, d) and V.shape == K.shape
+    assert S.shape == (n, hkv, d, d) and hq % hkv == 0
+    if shared:
+        assert z is not None
+    zz = None if z is None else _f64(z)
+    Y = np.zeros((n, hq, b, d))
+    _load().oracle_hybrid_step(_ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(zz),
+                               _ptr(Y), n, hq, hkv, b, d, float(scale),
+                               1 if shared else 0)
+    return Y
+
+
+def prefix_softmax(Q, Kc, Vc, P, K, V, scale=0.0):
+    """Exact softmax attention of the active block over [cache[:P] || block].
+
+    Q [n, hq, b, d]; Kc, Vc [n, hkv, cap, d] (first P tokens valid);
+    K, V [n, hkv, b, d].  Returns Y [n, hq, b, d] in float64.
+    """
+    Q, Kc, Vc, K, V = _f64(Q), _f64(Kc), _f64(Vc), _f64(K), _f64(V)
+    n, hq, b, d = Q.shape
+    hkv, cap = Kc.shape[1], Kc.shape[2]
+    assert 0 <= P <= cap and Kc.shape == (n, hkv, cap, d)
+    Y = np.zeros((n, hq, b, d))
+    _load().oracle_prefix_softmax(_ptr(Q), _ptr(Kc), _ptr(Vc), int(P), cap,
+                                  _ptr(K), _ptr(V), _ptr(Y), n, hq, hkv, b, d,
+                                  float(scale))
+    return Y
+
+
+def block_partition(L: int, B: int):
+    """Block boundaries [0, B, 2B, ..., L] (last block may be short)."""
+    k_max = (L + B - 1) // B if B > 0 else 0
+    out = (ctypes.c_long * (k_max + 2))()
+    k = _load().oracle_block_partition(int(L), int(B), out)
+    if k < 0:
+        raise ValueError("bad block partition arguments")
+    return [int(out[i]) for i in range(k + 1)]
+
+
+def generate(Q_steps, K_steps, V_steps, K_prompt=None, V_prompt=None,
+             scale=0.0, shared=False):
+    """Blockwise decoding loop of the worked example, on given inputs.
+
+    Q_steps[blk][step] etc. hold the active block's tensors at each
+    denoising step ([n, hq, b_blk, d] / [n, hkv, b_blk, d]).  The prompt
+    (optional) is folded into S first; every block's outputs use the state
+    of all earlier blocks, and after its last step the block is committed
+    with the K/V of that step.  Returns outputs[blk][step] and the final S, z.
+    """
+    first_k = K_steps[0][0]
+    n, hkv, _, dd = first_k.shape
+    if K_prompt is not None:
+        S, z = state_prefill(K_prompt, V_prompt)
+    else:
+        S = np.zeros((n, hkv, dd, dd))
+        z = np.zeros((n, hkv, dd))
+    outs = []
+    for blk in range(len(Q_steps)):
+        ob = []
+        for st in range(len(Q_steps[blk])):
+            ob.append(hybrid_step(Q_steps[blk][st], K_steps[blk][st],
+                                  V_steps[blk][st], S, z, scale, shared))
+        outs.append(ob)
+        S, z = state_commit(S, z, K_steps[blk][-1], V_steps[blk][-1])
+    return outs, S, z

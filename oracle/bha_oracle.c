@@ -1,0 +1,279 @@
+/*
+ * Plain fp64 CPU oracle for block-hybrid attention.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  It shares no code,
+ * header, table or helper with the CUDA library and never calls it.
+ *
+ * Source of the method: "Retrofitting Linear Attention into Diffusion
+ * Language Models" (Kim, Roh, Kim; arXiv 2608.06628) as summarised on the
+ * paper-daily page (sections "核心公式与算法" = core formula and
+ * "具体技术细节示例" = worked example) and the fugumt abstract page.
+ *
+ *   y = Softmax(Q_a K_a^T) V_a + phi(Q_a) S_p,   S_p = sum_t phi(k_t)^T v_t
+ *
+ * with phi = ReLU (worked example), the softmax scaled by 1/sqrt(d) and the
+ * query feature term taken on the active block's queries (the worked example
+ * writes phi(Q_2) S_1 for block 2).  Every routine here is written as the
+ * plain definition, one output element at a time, in double precision; no
+ * blocking, fusion or reordering beyond the definition.
+ *
+ * Layouts (all row-major, contiguous):
+ *   Q, Y            [n][hq][b][d]
+ *   K, V (block)    [n][hkv][b][d]
+ *   K, V (prompt)   [units][T][d]           (units = n*hkv)
+ *   K, V (cache)    [n][hkv][cap][d], the first P tokens valid
+ *   S               [units][d][d]   S[r][c] = sum_t phi(k_t)[r] * v_t[c]
+ *   z               [units][d]      z[r]    = sum_t phi(k_t)[r]
+ * GQA: query head h reads KV head h / (hq/hkv) (contiguous grouping).
+ *
+ * parity pins: see tests/test_oracle_pins.py.  The shared-denominator
+ * variant is not on the pages (an engineer-added option); it is pinned only
+ * by its own reduction cases and a brute-force restatement over prefix
+ * tokens, not by any page value.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdlib.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+static double relu(double x) { return x > 0.0 ? x : 0.0; }
+
+static int g_threads = 1;
+
+/* Number of OpenMP threads the routines below use (1 = single-threaded). */
+int oracle_set_threads(int n)
+{
+    if (n < 1) n = 1;
+    g_threads = n;
+    return g_threads;
+}
+
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_num_procs();
+#else
+    return 1;
+#endif
+}
+
+/*
+ * Prefix state of a prompt (the prompt counts as "previous blocks"):
+ *   S[u][r][c] = sum_{t<T} relu(K[u][t][r]) * V[u][t][c]
+ *   z[u][r]    = sum_{t<T} relu(K[u][t][r])
+ * T = 0 gives S = 0, z = 0.  z may be NULL.
+ * Worked example: S_1 = phi(K_1)^T V_1.
+ */
+void oracle_state_prefill(const double *K, const double *V, long units, long T,
+                          long d, double *S, double *z)
+{
+    long u;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (u = 0; u < units; ++u) {
+        const double *Ku = K + u * T * d;
+        const double *Vu = V + u * T * d;
+        double *Su = S + u * d * d;
+        for (long r = 0; r < d; ++r) {
+            for (long c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (long t = 0; t < T; ++t)
+                    acc += relu(Ku[t * d + r]) * Vu[t * d + c];
+                Su[r * d + c] = acc;
+            }
+            if (z) {
+                double zs = 0.0;
+                for (long t = 0; t < T; ++t)
+                    zs += relu(Ku[t * d + r]);
+                z[u * d + r] = zs;
+            }
+        }
+    }
+}
+
+/*
+ * Block commit when a block is finalised:
+ *   S[u] += phi(Kb[u])^T Vb[u],   z[u] += sum_t phi(Kb[u][t])
+ * Worked example: S_{1,2} = phi(K_1)^T V_1 + phi(K_2)^T V_2.
+ * Kb, Vb are [units][b][d].  z may be NULL.
+ */
+void oracle_state_commit(double *S, double *z, const double *Kb,
+                         const double *Vb, long units, long b, long d)
+{
+    long u;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (u = 0; u < units; ++u) {
+        const double *Ku = Kb + u * b * d;
+        const double *Vu = Vb + u * b * d;
+        double *Su = S + u * d * d;
+        for (long r = 0; r < d; ++r) {
+            for (long c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (long t = 0; t < b; ++t)
+                    acc += relu(Ku[t * d + r]) * Vu[t * d + c];
+                Su[r * d + c] += acc;
+            }
+            if (z) {
+                double zs = 0.0;
+                for (long t = 0; t < b; ++t)
+                    zs += relu(Ku[t * d + r]);
+                z[u * d + r] += zs;
+            }
+        }
+    }
+}
+
+/*
+ * One denoising step of block-hybrid attention for every query row of the
+ * active block (core formula; worked example, blocks 2 and 3).
+ *
+ * For request n, query head h (KV head g = h / (hq/hkv)), query row i:
+ *   s_j  = scale * q_i . k_{g,j}            j over the b block tokens, no mask
+ *   m    = max_j s_j,  e_j = exp(s_j - m),  l = sum_j e_j
+ *   lin  = phi(q_i) S_g                     (row vector, length d)
+ *   default:  y_i = sum_j (e_j / l) v_{g,j} + lin
+ *   shared :  y_i = (sum_j e_j v_{g,j} + e^{-m} lin) /
+ *                   (l + e^{-m} phi(q_i) . z_g)
+ * scale <= 0 selects 1/sqrt(d).  z is read only when shared != 0.
+ */
+void oracle_hybrid_step(const double *Q, const double *K, const double *V,
+                        const double *S, const double *z, double *Y, long n,
+                        long hq, long hkv, long b, long d, double scale,
+                        int shared)
+{
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    const long G = hq / hkv;
+    long nh;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (nh = 0; nh < n * hq; ++nh) {
+        const long ni = nh / hq, h = nh % hq, g = h / G;
+        const double *Kg = K + (ni * hkv + g) * b * d;
+        const double *Vg = V + (ni * hkv + g) * b * d;
+        const double *Sg = S + (ni * hkv + g) * d * d;
+        const double *zg = z ? z + (ni * hkv + g) * d : NULL;
+        double *s = (double *)malloc(sizeof(double) * (size_t)b);
+        double *lin = (double *)malloc(sizeof(double) * (size_t)d);
+        for (long i = 0; i < b; ++i) {
+            const double *q = Q + ((ni * hq + h) * b + i) * d;
+            double *y = Y + ((ni * hq + h) * b + i) * d;
+            double m = -INFINITY;
+            for (long j = 0; j < b; ++j) {
+                double dot = 0.0;
+                for (long c = 0; c < d; ++c)
+                    dot += q[c] * Kg[j * d + c];
+                s[j] = scale * dot;
+                if (s[j] > m) m = s[j];
+            }
+            double l = 0.0;
+            for (long j = 0; j < b; ++j) {
+                s[j] = exp(s[j] - m); /* s now holds e_j */
+                l += s[j];
+            }
+            for (long c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (long r = 0; r < d; ++r)
+                    acc += relu(q[r]) * Sg[r * d + c];
+                lin[c] = acc;
+            }
+            if (!shared) {
+                for (long c = 0; c < d; ++c) {
+                    double soft = 0.0;
+                    for (long j = 0; j < b; ++j)
+                        soft += (s[j] / l) * Vg[j * d + c];
+                    y[c] = soft + lin[c];
+                }
+            } else {
+                double qz = 0.0;
+                for (long r = 0; r < d; ++r)
+                    qz += relu(q[r]) * zg[r];
+                const double em = exp(-m);
+                const double den = l + em * qz;
+                for (long c = 0; c < d; ++c) {
+                    double num = 0.0;
+                    for (long j = 0; j < b; ++j)
+                        num += s[j] * Vg[j * d + c];
+                    y[c] = (num + em * lin[c]) / den;
+                }
+            }
+        }
+        free(s);
+        free(lin);
+    }
+}
+
+/*
+ * Exact prefix softmax (the baseline the abstract describes: every denoising
+ * step attends to all previous blocks through the KV cache).  One joint
+ * softmax over the P cached tokens followed by the b active-block tokens,
+ * bidirectional (no mask):
+ *   y_i = sum_j softmax_j(scale * q_i . k_j) v_j,  j in [cache[0:P] || block]
+ * Kc, Vc are [n][hkv][cap][d]; K, V are [n][hkv][b][d].
+ */
+void oracle_prefix_softmax(const double *Q, const double *Kc, const double *Vc,
+                           long P, long cap, const double *K, const double *V,
+                           double *Y, long n, long hq, long hkv, long b, long d,
+                           double scale)
+{
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    const long G = hq / hkv;
+    const long L = P + b;
+    long nh;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (nh = 0; nh < n * hq; ++nh) {
+        const long ni = nh / hq, h = nh % hq, g = h / G;
+        const double *Kcg = Kc + (ni * hkv + g) * cap * d;
+        const double *Vcg = Vc + (ni * hkv + g) * cap * d;
+        const double *Kg = K + (ni * hkv + g) * b * d;
+        const double *Vg = V + (ni * hkv + g) * b * d;
+        double *s = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        for (long i = 0; i < b; ++i) {
+            const double *q = Q + ((ni * hq + h) * b + i) * d;
+            double *y = Y + ((ni * hq + h) * b + i) * d;
+            double m = -INFINITY;
+            for (long j = 0; j < L; ++j) {
+                const double *k = j < P ? Kcg + j * d : Kg + (j - P) * d;
+                double dot = 0.0;
+                for (long c = 0; c < d; ++c)
+                    dot += q[c] * k[c];
+                s[j] = scale * dot;
+                if (s[j] > m) m = s[j];
+            }
+            double l = 0.0;
+            for (long j = 0; j < L; ++j) {
+                s[j] = exp(s[j] - m);
+                l += s[j];
+            }
+            for (long c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (long j = 0; j < L; ++j) {
+                    const double *v = j < P ? Vcg + j * d : Vg + (j - P) * d;
+                    acc += (s[j] / l) * v[c];
+                }
+                y[c] = acc;
+            }
+        }
+        free(s);
+    }
+}
+
+/*
+ * Block partition of a length-L sequence into blocks of B tokens; the last
+ * block may be short (worked example: L=10, B=4 gives tokens 1-4, 5-8, 9-10).
+ * Writes the boundaries 0 = bounds[0] < bounds[1] < ... < bounds[k] = L and
+ * returns k, the number of blocks (0 for L = 0; -1 for bad arguments).
+ * bounds needs room for k + 1 entries.
+ */
+long oracle_block_partition(long L, long B, long *bounds)
+{
+    if (L < 0 || B < 1) return -1;
+    long k = 0;
+    bounds[0] = 0;
+    for (long start = 0; start < L; start += B) {
+        long end = start + B;
+        if (end > L) end = L;
+        bounds[++k] = end;
+    }
+    return k;
+}
