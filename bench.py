@@ -1,0 +1,501 @@
+#!/usr/bin/env python
+"""Benchmark: block-hybrid attention, active-block tokens/s per layer on B200.
+
+Workload (default): the long-prefix regime of a 16B dLLM attention layer --
+batch 64, 16 query / 4 KV heads, head dim 128, active block B = 32, a
+committed prefix of 32768 tokens folded into the fp32 prefix state by the
+GPU prefill.  One timed step is one block of the decoding loop: 8 denoising
+steps (bha_hybrid_step) followed by the block commit (bha_state_commit);
+tokens per step = batch x B x 8 active-block tokens.  Inputs are resident in
+HBM; 14+ disjoint input sets rotate so the working set exceeds 4 x L2.  The
+timed loop replays CUDA graphs of the library's launches.
+
+Printed: one JSON line (rank 0) with the metric, the roofline of the
+dominant kernel, the CPU-oracle baseline, the end-to-end number through the
+C ABI with host buffers, the exact-prefix-softmax comparison on identical
+shapes and the SM clocks sampled during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+"""
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "hybrid-attn active-block tokens/s per layer at 1 B200; % of HBM roofline"
+DATA = ("synthetic: seeded Gaussian bf16 Q/K/V, N(0, std 1/sqrt(128)); prefix state from "
+        "the GPU prefill of a seeded 32768-token prompt (stands in for trained-model "
+        "activations; timing does not depend on values)")
+N_, HQ, HKV, B_, D_, P_ = 64, 16, 4, 32, 128, 32768
+DENOISE = 8
+UNIT_BYTES_STEP = (HQ // HKV) * B_ * D_ * 2 * 2 + 2 * B_ * D_ * 2 + D_ * D_ * 4  # Q+Y, K+V, S
+UNIT_BYTES_COMMIT = 2 * B_ * D_ * 2 + 2 * D_ * D_ * 4                           # K+V, S r+w
+WORKLOAD = ("long-prefix: batch 64, 16q/4kv heads, d=128, active block B=32, prefix 32768 "
+            "in fp32 state; step = 8 hybrid denoising steps + 1 block commit")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
+    ap.add_argument("--no-compare", action="store_true", help="skip the exact-path comparison")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def traffic_record(kernel, src_file):
+    """dram bytes per launch from the committed ncu summary, if the kernel's
+    source is unchanged since the capture (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec:
+        return None
+    with open(os.path.join(ROOT, "block_hybrid_linear_b200", "csrc", src_file), "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()
+    if rec.get("source_sha256") != sha:
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.QUERY,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return None
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- reference
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: the same metric on bounded samples
+    of the same workload, on the host cores."""
+    if rank != 0:
+        return
+    import numpy as np
+    import oracle
+    from block_hybrid_linear_b200 import inputs
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    std = 1.0 / math.sqrt(D_)
+    # a sample = a few (request, KV head) units through one block cycle
+    u_max = 64
+    Qb, Qv = inputs.normal_bf16_np(4000, inputs.TID_Q, (u_max // HKV, HQ, B_, D_), std)
+    Kb, Kv = inputs.normal_bf16_np(4000, inputs.TID_K, (u_max // HKV, HKV, B_, D_), std)
+    Vb, Vv = inputs.normal_bf16_np(4000, inputs.TID_V, (u_max // HKV, HKV, B_, D_), std)
+    Sv, zv = inputs.synthetic_state_np(4000, u_max // HKV, HKV, D_, P_, std)
+
+    def cycle(nreq):
+        S, z = Sv[:nreq], zv[:nreq]
+        for _ in range(DENOISE):
+            oracle.hybrid_step(Qv[:nreq], Kv[:nreq], Vv[:nreq], S, z)
+        oracle.state_commit(S, z, Kv[:nreq], Vv[:nreq])
+
+    t0 = time.perf_counter()
+    cycle(1)
+    t1 = time.perf_counter() - t0
+    budget = 90.0 / max(1, args.steps + args.warmup)
+    nreq = int(max(1, min(u_max // HKV, budget / max(t1, 1e-6))))
+    for _ in range(args.warmup):
+        cycle(nreq)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        cycle(nreq)
+    dt = time.perf_counter() - t0
+    tokens = nreq * B_ * DENOISE * args.steps
+    value = tokens / dt
+    sample = ("%d of 64 requests (all 4 KV heads each) through one block cycle per step: "
+              "8 oracle hybrid steps + 1 oracle commit, fp64" % nreq)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": DATA,
+        "config": {"workload": WORKLOAD, "sample": sample},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_native():
+    """Oracle timed on this host's cores on a bounded sample (~10-30 s)."""
+    import oracle
+    from block_hybrid_linear_b200 import inputs
+    cores = len(os.sched_getaffinity(0))
+    oracle.set_threads(cores)
+    std = 1.0 / math.sqrt(D_)
+    nreq = 16
+    Qb, Qv = inputs.normal_bf16_np(4000, inputs.TID_Q, (nreq, HQ, B_, D_), std)
+    Kb, Kv = inputs.normal_bf16_np(4000, inputs.TID_K, (nreq, HKV, B_, D_), std)
+    Vb, Vv = inputs.normal_bf16_np(4000, inputs.TID_V, (nreq, HKV, B_, D_), std)
+    Sv, zv = inputs.synthetic_state_np(4000, nreq, HKV, D_, P_, std)
+    t0 = time.perf_counter()
+    cycles = 0
+    while True:
+        for _ in range(DENOISE):
+            oracle.hybrid_step(Qv, Kv, Vv, Sv, zv)
+        oracle.state_commit(Sv, zv, Kv, Vv)
+        cycles += 1
+        if time.perf_counter() - t0 > 10.0 or cycles >= 50:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": nreq * B_ * DENOISE * cycles / dt, "unit": "tokens/s", "cores": cores,
+            "kind": "oracle",
+            "sample": "%d of 64 requests x %d block cycles (8 steps + commit), fp64 oracle, "
+                      "%.1f s" % (nreq, cycles, dt)}
+
+
+# ---------------------------------------------------------------- native
+
+def run_native(args, rank, world, local):
+    import torch
+    import block_hybrid_linear_b200 as bha
+    from block_hybrid_linear_b200 import build, inputs
+
+    build.build()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+    std = 1.0 / math.sqrt(D_)
+    seed = 4000 + 17 * rank
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+
+    # ---- prompt -> prefix state (prefill), timed as a side line
+    Kp = inputs.normal_bf16_torch(seed, inputs.TID_KP, (N_, HKV, P_, D_), std, dev)
+    Vp = inputs.normal_bf16_torch(seed, inputs.TID_VP, (N_, HKV, P_, D_), std, dev)
+    S0 = torch.empty(N_, HKV, D_, D_, device=dev)
+    z0 = torch.empty(N_, HKV, D_, device=dev)
+    need = bha.bha_state_prefill_workspace_size(N_, HKV, P_, D_)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    bha.bha_state_prefill(Kp, Vp, S0, z0, workspace=ws)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    reps = 5
+    e0.record()
+    for _ in range(reps):
+        bha.bha_state_prefill(Kp, Vp, S0, z0, workspace=ws)
+    e1.record()
+    torch.cuda.synchronize()
+    prefill_ms = e0.elapsed_time(e1) / reps
+    prefill_bytes = N_ * HKV * (2 * P_ * D_ * 2 + D_ * D_ * 4)
+
+    # ---- rotating input sets (disjoint memory, > 4 x L2 in total)
+    set_bytes = N_ * HKV * UNIT_BYTES_STEP
+    R = max(4, math.ceil(4 * l2 / set_bytes))
+    sets = []
+    for r in range(R):
+        sets.append(dict(
+            Q=inputs.normal_bf16_torch(seed + r, inputs.TID_Q, (N_, HQ, B_, D_), std, dev),
+            K=inputs.normal_bf16_torch(seed + r, inputs.TID_K, (N_, HKV, B_, D_), std, dev),
+            V=inputs.normal_bf16_torch(seed + r, inputs.TID_V, (N_, HKV, B_, D_), std, dev),
+            S=S0.clone(), z=z0.clone(),
+            Y=torch.empty(N_, HQ, B_, D_, dtype=torch.bfloat16, device=dev)))
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream(device=dev)
+
+    def cycle(c):
+        # one block: 8 denoising steps on 8 different sets, commit on the last
+        for s in range(DENOISE):
+            st = sets[(c * (DENOISE + 1) + s) % R]
+            bha.bha_hybrid_step(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"],
+                                stream=stream)
+        st = sets[(c * (DENOISE + 1) + DENOISE) % R]
+        bha.bha_state_commit(st["K"], st["V"], st["S"], st["z"], stream=stream)
+
+    # graph of R cycles: every set is touched in each role, rotation period R
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for c in range(2):
+            cycle(c)
+    stream.synchronize()
+    g_cycles = R
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for c in range(g_cycles):
+            cycle(c)
+    # kernel-only graphs for the per-launch durations of the two kernels
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=stream):
+        for k in range(4 * R):
+            st = sets[k % R]
+            bha.bha_hybrid_step(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"],
+                                stream=stream)
+    g_commit = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_commit, stream=stream):
+        for k in range(2 * R):
+            st = sets[k % R]
+            bha.bha_state_commit(st["K"], st["V"], st["S"], st["z"], stream=stream)
+    torch.cuda.synchronize()
+
+    reps = max(1, math.ceil(args.steps / g_cycles))
+    steps = reps * g_cycles
+    warm = max(1, math.ceil(args.warmup / g_cycles))
+    for _ in range(warm):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert bha.bha_device_error(True) == 0
+
+    clocks = ClockSampler(local)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ks0, ks1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kc0, kc1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    ev0.record(stream)
+    for _ in range(reps):
+        graph.replay()
+    ev1.record(stream)
+    # per-kernel durations, measured in the same run on the launching stream
+    ks0.record(stream)
+    for _ in range(max(1, reps // 4)):
+        g_step.replay()
+    ks1.record(stream)
+    kc0.record(stream)
+    for _ in range(max(1, reps // 4)):
+        g_commit.replay()
+    kc1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    t_ms = ev0.elapsed_time(ev1)
+    step_launch_ms = ks0.elapsed_time(ks1) / (max(1, reps // 4) * 4 * R)
+    commit_launch_ms = kc0.elapsed_time(kc1) / (max(1, reps // 4) * 2 * R)
+    assert bha.bha_device_error(True) == 0
+    if pg is not None:
+        t = torch.tensor([t_ms], device=dev)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        t_ms = float(t.item())
+    tokens = world * steps * N_ * B_ * DENOISE
+    value = tokens / (t_ms / 1e3)
+
+    peak, peak_kind = measured_peaks()
+    step_bytes = N_ * HKV * UNIT_BYTES_STEP
+    achieved = step_bytes / (step_launch_ms / 1e3) / 1e9
+    commit_bytes = N_ * HKV * UNIT_BYTES_COMMIT
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": steps, "warmup": warm * g_cycles, "ms_per_step": t_ms / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": DATA,
+        "config": {"workload": WORKLOAD, "batch": N_, "heads_q": HQ, "heads_kv": HKV,
+                   "head_dim": D_, "block": B_, "prefix": P_, "denoise_steps": DENOISE,
+                   "l2": "rotating %d disjoint input sets, %.0f MB > 4 x L2 (%.0f MB)"
+                         % (R, R * set_bytes / 1e6, l2 / 1e6),
+                   "parallelism": "replicas x%d (no collective)" % world},
+        "roofline": {"bound": "hbm", "kernel": "k_step_bf16", "achieved": achieved,
+                     "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "peak_kind": peak_kind,
+                     "traffic": traffic_record("k_step_bf16", "k_step.cu"),
+                     "algorithmic_bytes_per_launch": step_bytes,
+                     "launch_us": step_launch_ms * 1e3},
+        "hbm_roofline_frac": achieved / peak,
+        "commit": {"launch_us": commit_launch_ms * 1e3,
+                   "achieved_gbs": commit_bytes / (commit_launch_ms / 1e3) / 1e9,
+                   "algorithmic_bytes_per_launch": commit_bytes},
+        "prefill": {"ms": prefill_ms, "tokens": N_ * P_,
+                    "achieved_gbs": prefill_bytes / (prefill_ms / 1e3) / 1e9},
+        "gpu_launches": steps * (DENOISE + 1),
+        "clocks": clk,
+    }
+
+    # ---- exact prefix softmax on identical shapes (the comparison path)
+    if not args.no_compare:
+        del graph, g_step, g_commit
+        cap = P_ + B_
+        Kc = torch.empty(N_, HKV, cap, D_, dtype=torch.bfloat16, device=dev)
+        Vc = torch.empty_like(Kc)
+        Kc[:, :, :P_].copy_(Kp)
+        Vc[:, :, :P_].copy_(Vp)
+        st = sets[0]
+        Kc[:, :, P_:].copy_(st["K"])
+        Vc[:, :, P_:].copy_(st["V"])
+        del Kp, Vp
+        need = bha.bha_prefix_softmax_workspace_size(N_, HQ, HKV, B_, D_, P_)
+        wsp = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        Yx = torch.empty_like(st["Y"])
+        for _ in range(2):
+            bha.bha_prefix_softmax(st["Q"], Kc, Vc, P_, st["K"], st["V"], Yx, workspace=wsp)
+        torch.cuda.synchronize()
+        n_rep = 10
+        e0.record()
+        for _ in range(n_rep):
+            bha.bha_prefix_softmax(st["Q"], Kc, Vc, P_, st["K"], st["V"], Yx, workspace=wsp)
+        e1.record()
+        torch.cuda.synchronize()
+        px_ms = e0.elapsed_time(e1) / n_rep
+        px_bytes = N_ * HKV * (2 * (P_ + B_) * D_ * 2) + 2 * N_ * HQ * B_ * D_ * 2
+        comp = {"prefix_softmax": {"ms": px_ms, "tokens_per_s": N_ * B_ / (px_ms / 1e3),
+                                   "achieved_gbs": px_bytes / (px_ms / 1e3) / 1e9,
+                                   "frac_of_peak": px_bytes / (px_ms / 1e3) / 1e9 / peak}}
+        # library attention on the same shapes, as a sanity line for the exact path
+        try:
+            import torch.nn.functional as F
+            q = st["Q"]
+            for _ in range(2):
+                F.scaled_dot_product_attention(q, Kc, Vc, enable_gqa=True)
+            torch.cuda.synchronize()
+            e0.record()
+            for _ in range(n_rep):
+                F.scaled_dot_product_attention(q, Kc, Vc, enable_gqa=True)
+            e1.record()
+            torch.cuda.synchronize()
+            sd_ms = e0.elapsed_time(e1) / n_rep
+            comp["torch_sdpa"] = {"ms": sd_ms, "tokens_per_s": N_ * B_ / (sd_ms / 1e3)}
+        except Exception as exc:  # pragma: no cover
+            comp["torch_sdpa"] = {"error": str(exc)[:200]}
+        hybrid_step_ms = step_launch_ms
+        comp["hybrid_step_over_exact_speedup"] = px_ms / hybrid_step_ms
+        line["comparison"] = comp
+        del Kc, Vc
+
+    # ---- end to end through the C ABI with host buffers
+    if not args.no_e2e:
+        st = sets[0]
+        hQ = st["Q"].cpu().pin_memory()
+        hK = st["K"].cpu().pin_memory()
+        hV = st["V"].cpu().pin_memory()
+        hY = torch.empty(st["Y"].shape, dtype=torch.bfloat16).pin_memory()
+        dQ, dK, dV, dY = (torch.empty_like(st[k]) for k in ("Q", "K", "V", "Y"))
+        n_e2e = min(50, steps)
+
+        def e2e_cycle():
+            with torch.cuda.stream(stream):
+                for _ in range(DENOISE):
+                    dQ.copy_(hQ, non_blocking=True)
+                    dK.copy_(hK, non_blocking=True)
+                    dV.copy_(hV, non_blocking=True)
+                    bha.bha_hybrid_step(dQ, dK, dV, st["S"], dY, z=st["z"], stream=stream)
+                    hY.copy_(dY, non_blocking=True)
+                bha.bha_state_commit(dK, dV, st["S"], st["z"], stream=stream)
+
+        for _ in range(3):
+            e2e_cycle()
+        stream.synchronize()
+        barrier()
+        t0 = time.perf_counter()
+        ev0.record(stream)
+        for _ in range(n_e2e):
+            e2e_cycle()
+        ev1.record(stream)
+        stream.synchronize()
+        wall = time.perf_counter() - t0
+        e2e_ms = max(ev0.elapsed_time(ev1), wall * 1e3)
+        if pg is not None:
+            t = torch.tensor([e2e_ms], device=dev)
+            pg.all_reduce(t, op=pg.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = DENOISE * (hQ.numel() + hK.numel() + hV.numel()) * 2
+        d2h = DENOISE * hY.numel() * 2
+        line["e2e"] = {"value": world * n_e2e * N_ * B_ * DENOISE / (e2e_ms / 1e3),
+                       "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h}
+        line["gpu_launches_e2e"] = n_e2e * (DENOISE + 1)
+
+    if rank == 0 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline_native()
+    if pg is not None:
+        pg.barrier()
+        pg.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    run_native(args, rank, world, local)
+
+
+if __name__ == "__main__":
+    main()

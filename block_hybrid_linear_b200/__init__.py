@@ -1,1 +1,17 @@
-"""block_hybrid_linear_b200 -- block-hybrid attention on B200 (placeholder)."""
+"""block_hybrid_linear_b200 -- block-hybrid attention for blockwise
+semi-autoregressive diffusion-LM decoding, on NVIDIA B200 (sm_100a).
+
+Exact softmax inside the active denoising block plus ReLU-feature linear
+attention over all previous blocks through a per-KV-head fp32 prefix state
+("Retrofitting Linear Attention into Diffusion Language Models").  The
+compute lives in ``libbha.so`` (C ABI, ``include/bha.h``); this package is
+its binding (``_lib``) plus the seeded input generators (``inputs``).
+"""
+from ._lib import (  # noqa: F401
+    BHA_BF16, BHA_ERR_CUDA, BHA_ERR_DEVICE, BHA_ERR_INVALID_ARG,
+    BHA_ERR_MISALIGNED, BHA_ERR_TIMEOUT, BHA_ERR_UNSUPPORTED, BHA_ERR_WORKSPACE,
+    BHA_F32, BHA_FLAG_SHARED_DENOM, BHA_OK, BhaError, EXPORTED, LIB_PATH,
+    bha_block_partition, bha_device_error, bha_hybrid_step, bha_prefix_softmax,
+    bha_prefix_softmax_workspace_size, bha_state_commit, bha_state_prefill,
+    bha_state_prefill_workspace_size, bha_version, lib, status_string,
+)

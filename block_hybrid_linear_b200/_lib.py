@@ -1,0 +1,174 @@
+"""ctypes binding of ``libbha.so`` -- argument marshalling only.
+
+Each ``bha_*`` function here has the name and meaning of the C entry point
+declared in ``include/bha.h``: it reads sizes off the tensors' shapes,
+passes raw device pointers and the current CUDA stream, and raises
+``BhaError`` on a negative status.  All arithmetic runs in the library's
+CUDA kernels; there is no fallback.  PyTorch supplies device memory and
+streams only.
+"""
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbha.so")
+
+BHA_OK = 0
+BHA_ERR_INVALID_ARG = -1
+BHA_ERR_UNSUPPORTED = -2
+BHA_ERR_MISALIGNED = -3
+BHA_ERR_WORKSPACE = -4
+BHA_ERR_CUDA = -5
+BHA_ERR_TIMEOUT = -6
+BHA_ERR_DEVICE = -7
+BHA_BF16 = 0
+BHA_F32 = 1
+BHA_FLAG_SHARED_DENOM = 1
+
+# every symbol include/bha.h declares
+EXPORTED = [
+    "bha_status_string", "bha_version", "bha_state_prefill_workspace_size",
+    "bha_state_prefill", "bha_state_commit", "bha_hybrid_step",
+    "bha_prefix_softmax_workspace_size", "bha_prefix_softmax",
+    "bha_block_partition", "bha_device_error",
+]
+
+_lib = None
+
+
+class BhaError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__("%s failed: %s (%d)" % (where, status_string(status), status))
+
+
+def lib():
+    """Load libbha.so (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                "libbha.so is missing; build it with "
+                "`python -m block_hybrid_linear_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, sz, fl, u = (ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t,
+                            ctypes.c_float, ctypes.c_uint)
+        L.bha_status_string.argtypes = [i]
+        L.bha_status_string.restype = ctypes.c_char_p
+        L.bha_version.argtypes = []
+        L.bha_version.restype = i
+        L.bha_state_prefill_workspace_size.argtypes = [i, i, i, i, i]
+        L.bha_state_prefill_workspace_size.restype = sz
+        L.bha_state_prefill.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, sz, vp]
+        L.bha_state_prefill.restype = i
+        L.bha_state_commit.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp]
+        L.bha_state_commit.restype = i
+        L.bha_hybrid_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, fl, u,
+                                      i, vp]
+        L.bha_hybrid_step.restype = i
+        L.bha_prefix_softmax_workspace_size.argtypes = [i, i, i, i, i, i, i]
+        L.bha_prefix_softmax_workspace_size.restype = sz
+        L.bha_prefix_softmax.argtypes = [vp, vp, vp, i, i, vp, vp, vp, i, i, i, i,
+                                         i, fl, i, vp, sz, vp]
+        L.bha_prefix_softmax.restype = i
+        L.bha_block_partition.argtypes = [i, i, ctypes.POINTER(ctypes.c_int), i]
+        L.bha_block_partition.restype = i
+        L.bha_device_error.argtypes = [i]
+        L.bha_device_error.restype = i
+        _lib = L
+    return _lib
+
+
+def status_string(status):
+    return lib().bha_status_string(int(status)).decode()
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    handle = getattr(stream, "cuda_stream", stream)
+    return ctypes.c_void_p(int(handle))
+
+
+def _dtype(t):
+    import torch
+    if t.dtype == torch.bfloat16:
+        return BHA_BF16
+    if t.dtype == torch.float32:
+        return BHA_F32
+    raise TypeError("Q/K/V must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _check(status, where):
+    if status != BHA_OK:
+        raise BhaError(status, where)
+
+
+def bha_version():
+    return lib().bha_version()
+
+
+def bha_block_partition(L, B):
+    """Block boundaries [0, B, 2B, ..., L] of a length-L sequence."""
+    k = (L + B - 1) // B if B > 0 and L >= 0 else 0
+    buf = (ctypes.c_int * (k + 1))()
+    rc = lib().bha_block_partition(int(L), int(B), buf, k + 1)
+    if rc < 0:
+        raise BhaError(rc, "bha_block_partition")
+    return [int(buf[j]) for j in range(rc + 1)]
+
+
+def bha_device_error(reset=True):
+    """Synchronise and return the kernels' device error word (0 = none)."""
+    return lib().bha_device_error(1 if reset else 0)
+
+
+def bha_state_prefill_workspace_size(n, hkv, T, d, dtype=BHA_BF16):
+    return lib().bha_state_prefill_workspace_size(n, hkv, T, d, dtype)
+
+
+def bha_state_prefill(K, V, S, z=None, workspace=None, stream=None):
+    """S = phi(K)^T V, z = sum_t phi(k_t) over the prompt.  K, V: [n, hkv, T, d]."""
+    n, hkv, T, d = K.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().bha_state_prefill(_ptr(K), _ptr(V), n, hkv, T, d, _dtype(K), _ptr(S),
+                                   _ptr(z), _ptr(workspace), ws_bytes, _stream(stream)),
+           "bha_state_prefill")
+
+
+def bha_state_commit(Kb, Vb, S, z=None, stream=None):
+    """S += phi(Kb)^T Vb, z += sum_t phi(kb_t).  Kb, Vb: [n, hkv, b, d]."""
+    n, hkv, b, d = Kb.shape
+    _check(lib().bha_state_commit(_ptr(Kb), _ptr(Vb), n, hkv, b, d, _dtype(Kb), _ptr(S),
+                                  _ptr(z), _stream(stream)), "bha_state_commit")
+
+
+def bha_hybrid_step(Q, K, V, S, Y, z=None, scale=0.0, flags=0, stream=None):
+    """Y = softmax(Q K^T scale) V + phi(Q) S for the active block.
+
+    Q, Y: [n, hq, b, d]; K, V: [n, hkv, b, d]; S: [n, hkv, d, d] fp32."""
+    n, hq, b, d = Q.shape
+    hkv = K.shape[1]
+    _check(lib().bha_hybrid_step(_ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(z), _ptr(Y), n,
+                                 hq, hkv, b, d, float(scale), int(flags), _dtype(Q),
+                                 _stream(stream)), "bha_hybrid_step")
+
+
+def bha_prefix_softmax_workspace_size(n, hq, hkv, b, d, P, dtype=BHA_BF16):
+    return lib().bha_prefix_softmax_workspace_size(n, hq, hkv, b, d, P, dtype)
+
+
+def bha_prefix_softmax(Q, Kc, Vc, P, K, V, Y, scale=0.0, workspace=None, stream=None):
+    """Exact softmax over [Kc[:, :, :P] || K].  Kc, Vc: [n, hkv, cap, d]."""
+    n, hq, b, d = Q.shape
+    hkv, cap = Kc.shape[1], Kc.shape[2]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().bha_prefix_softmax(_ptr(Q), _ptr(Kc), _ptr(Vc), int(P), cap, _ptr(K),
+                                    _ptr(V), _ptr(Y), n, hq, hkv, b, d, float(scale),
+                                    _dtype(Q), _ptr(workspace), ws_bytes, _stream(stream)),
+           "bha_prefix_softmax")

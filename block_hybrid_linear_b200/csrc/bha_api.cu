@@ -1,0 +1,335 @@
+// C ABI of block-hybrid attention: argument validation, dispatch by dtype,
+// workspace queries, the device error word, the tensor-map encoder and the
+// host-side block partition.  Every check runs before any launch.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "../../include/bha.h"
+#include "bha_internal.h"
+
+namespace bha {
+
+// Kernel-reported error (BHA_OK / BHA_ERR_TIMEOUT / BHA_ERR_DEVICE), one per GPU.
+__device__ int g_dev_error = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  std::atomic<bool> ready{false};
+  int* dev_err = nullptr;
+  int sm_count = 0;
+  int cc_major = 0;
+  int cc_minor = 0;
+};
+DeviceInfo g_devices[kMaxDevices];
+std::mutex g_dev_mutex;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+int device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BHA_ERR_CUDA;
+  DeviceInfo& d = g_devices[dev];
+  if (!d.ready.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!d.ready.load(std::memory_order_relaxed)) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_dev_error) != cudaSuccess) return BHA_ERR_CUDA;
+      if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) !=
+              cudaSuccess ||
+          cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) !=
+              cudaSuccess ||
+          cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) !=
+              cudaSuccess)
+        return BHA_ERR_CUDA;
+      d.dev_err = static_cast<int*>(p);
+      d.ready.store(true, std::memory_order_release);
+    }
+  }
+  *out = &d;
+  return BHA_OK;
+}
+
+int make_ctx(bha_stream_t stream, bha_dtype dtype, Ctx* c) {
+  DeviceInfo* d = nullptr;
+  const int st = device_info(&d);
+  if (st != BHA_OK) return st;
+  // The tensor-core path is built for sm_100a only.
+  if (dtype == BHA_BF16 && d->cc_major != 10) return BHA_ERR_UNSUPPORTED;
+  c->stream = reinterpret_cast<cudaStream_t>(stream);
+  c->dev_err = d->dev_err;
+  c->sm_count = d->sm_count;
+  return BHA_OK;
+}
+
+bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
+
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + nb && b0 < a0 + na;
+}
+
+size_t esize(bha_dtype t) { return t == BHA_BF16 ? 2 : 4; }
+
+bool dtype_ok(bha_dtype t) { return t == BHA_BF16 || t == BHA_F32; }
+
+// d / b support: bf16 needs d = 128; fp32 any d <= 128 with d % 4 == 0.
+int check_dims(bha_dtype t, int d, int b_or_1) {
+  if (!dtype_ok(t)) return BHA_ERR_UNSUPPORTED;
+  if (d < 1 || b_or_1 < 1) return BHA_ERR_INVALID_ARG;
+  if (b_or_1 > 64) return BHA_ERR_UNSUPPORTED;
+  if (t == BHA_BF16 && d != 128) return BHA_ERR_UNSUPPORTED;
+  if (t == BHA_F32 && (d > 128 || d % 4 != 0)) return BHA_ERR_UNSUPPORTED;
+  return BHA_OK;
+}
+
+float resolve_scale(float scale, int d) {
+  return scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
+}
+
+int launch_status(int rc) {
+  if (rc == 0) return BHA_OK;
+  if (rc == -4) return BHA_ERR_WORKSPACE;
+  return BHA_ERR_CUDA;
+}
+
+}  // namespace
+
+bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* gaddr,
+                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                 CUtensorMapSwizzle swizzle) {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (g_encode == nullptr) return false;
+  cuuint64_t gd[5];
+  cuuint64_t gs[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) gs[i] = strides_bytes[i];
+  const CUresult r =
+      g_encode(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(gaddr), gd, gs, bx,
+               es, CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace bha
+
+using namespace bha;
+
+extern "C" {
+
+const char* bha_status_string(int status) {
+  switch (status) {
+    case BHA_OK: return "BHA_OK";
+    case BHA_ERR_INVALID_ARG: return "BHA_ERR_INVALID_ARG";
+    case BHA_ERR_UNSUPPORTED: return "BHA_ERR_UNSUPPORTED";
+    case BHA_ERR_MISALIGNED: return "BHA_ERR_MISALIGNED";
+    case BHA_ERR_WORKSPACE: return "BHA_ERR_WORKSPACE";
+    case BHA_ERR_CUDA: return "BHA_ERR_CUDA";
+    case BHA_ERR_TIMEOUT: return "BHA_ERR_TIMEOUT";
+    case BHA_ERR_DEVICE: return "BHA_ERR_DEVICE";
+    default: return "BHA_ERR_UNKNOWN";
+  }
+}
+
+int bha_version(void) { return 1; }
+
+int bha_block_partition(int L, int B, int* bounds, int max_bounds) {
+  if (L < 0 || B < 1 || bounds == nullptr) return BHA_ERR_INVALID_ARG;
+  const long long k = (static_cast<long long>(L) + B - 1) / B;
+  if (max_bounds < k + 1) return BHA_ERR_WORKSPACE;
+  bounds[0] = 0;
+  for (long long i = 1; i <= k; ++i) {
+    const long long e = i * B;
+    bounds[i] = static_cast<int>(e < L ? e : L);
+  }
+  return static_cast<int>(k);
+}
+
+int bha_device_error(int reset) {
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != BHA_OK) return BHA_ERR_CUDA;
+  if (cudaDeviceSynchronize() != cudaSuccess) return BHA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, d->dev_err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return BHA_ERR_CUDA;
+  if (reset) {
+    const int zero = 0;
+    if (cudaMemcpy(d->dev_err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return BHA_ERR_CUDA;
+  }
+  return v;
+}
+
+size_t bha_state_prefill_workspace_size(int n, int hkv, int T, int d, bha_dtype dtype) {
+  if (dtype != BHA_BF16 || n <= 0 || hkv <= 0 || T <= 0 || d != 128) return 0;
+  return prefill_bf16_workspace(n * hkv, T);
+}
+
+int bha_state_prefill(const void* K, const void* V, int n, int hkv, int T, int d,
+                      bha_dtype dtype, float* S, float* z, void* workspace,
+                      size_t workspace_bytes, bha_stream_t stream) {
+  int st = check_dims(dtype, d, 1);
+  if (st != BHA_OK) return st;
+  if (n < 0 || hkv < 1 || T < 0) return BHA_ERR_INVALID_ARG;
+  if (n == 0) return BHA_OK;
+  if (S == nullptr || (T > 0 && (K == nullptr || V == nullptr))) return BHA_ERR_INVALID_ARG;
+  if (misaligned(K) || misaligned(V) || misaligned(S) || misaligned(z) || misaligned(workspace))
+    return BHA_ERR_MISALIGNED;
+  const size_t units = static_cast<size_t>(n) * hkv;
+  const size_t kv_bytes = units * T * d * esize(dtype);
+  const size_t s_bytes = units * d * d * 4, z_bytes = units * d * 4;
+  if (overlap(S, s_bytes, K, kv_bytes) || overlap(S, s_bytes, V, kv_bytes) ||
+      overlap(z, z_bytes, K, kv_bytes) || overlap(z, z_bytes, V, kv_bytes) ||
+      overlap(z, z_bytes, S, s_bytes))
+    return BHA_ERR_INVALID_ARG;
+  const size_t need = bha_state_prefill_workspace_size(n, hkv, T, d, dtype);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BHA_ERR_WORKSPACE;
+  if (need > 0 && (overlap(workspace, need, S, s_bytes) || overlap(workspace, need, z, z_bytes) ||
+                   overlap(workspace, need, K, kv_bytes) || overlap(workspace, need, V, kv_bytes)))
+    return BHA_ERR_INVALID_ARG;
+  Ctx c;
+  st = make_ctx(stream, dtype, &c);
+  if (st != BHA_OK) return st;
+  if (dtype == BHA_F32)
+    return launch_status(launch_prefill_f32(c, static_cast<const float*>(K),
+                                            static_cast<const float*>(V), (int)units, T, d, S,
+                                            z));
+  return launch_status(launch_prefill_bf16(c, K, V, (int)units, T, S, z, workspace,
+                                           workspace_bytes));
+}
+
+int bha_state_commit(const void* Kb, const void* Vb, int n, int hkv, int b, int d,
+                     bha_dtype dtype, float* S, float* z, bha_stream_t stream) {
+  int st = check_dims(dtype, d, b);
+  if (st != BHA_OK) return st;
+  if (n < 0 || hkv < 1) return BHA_ERR_INVALID_ARG;
+  if (n == 0) return BHA_OK;
+  if (Kb == nullptr || Vb == nullptr || S == nullptr) return BHA_ERR_INVALID_ARG;
+  if (misaligned(Kb) || misaligned(Vb) || misaligned(S) || misaligned(z))
+    return BHA_ERR_MISALIGNED;
+  const size_t units = static_cast<size_t>(n) * hkv;
+  const size_t kv_bytes = units * b * d * esize(dtype);
+  const size_t s_bytes = units * d * d * 4, z_bytes = units * d * 4;
+  if (overlap(S, s_bytes, Kb, kv_bytes) || overlap(S, s_bytes, Vb, kv_bytes) ||
+      overlap(z, z_bytes, Kb, kv_bytes) || overlap(z, z_bytes, Vb, kv_bytes) ||
+      overlap(z, z_bytes, S, s_bytes))
+    return BHA_ERR_INVALID_ARG;
+  Ctx c;
+  st = make_ctx(stream, dtype, &c);
+  if (st != BHA_OK) return st;
+  if (dtype == BHA_F32)
+    return launch_status(launch_commit_f32(c, static_cast<const float*>(Kb),
+                                           static_cast<const float*>(Vb), (int)units, b, d, S,
+                                           z));
+  return launch_status(launch_commit_bf16(c, Kb, Vb, (int)units, b, S, z));
+}
+
+int bha_hybrid_step(const void* Qa, const void* Ka, const void* Va, const float* S,
+                    const float* z, void* Y, int n, int hq, int hkv, int b, int d, float scale,
+                    unsigned flags, bha_dtype dtype, bha_stream_t stream) {
+  int st = check_dims(dtype, d, b);
+  if (st != BHA_OK) return st;
+  if (n < 0 || hq < 1 || hkv < 1 || hq % hkv != 0) return BHA_ERR_INVALID_ARG;
+  if ((flags & ~BHA_FLAG_SHARED_DENOM) != 0) return BHA_ERR_INVALID_ARG;
+  const int shared = (flags & BHA_FLAG_SHARED_DENOM) ? 1 : 0;
+  if (n == 0) return BHA_OK;
+  if (Qa == nullptr || Ka == nullptr || Va == nullptr || S == nullptr || Y == nullptr)
+    return BHA_ERR_INVALID_ARG;
+  if (shared && z == nullptr) return BHA_ERR_INVALID_ARG;
+  if (misaligned(Qa) || misaligned(Ka) || misaligned(Va) || misaligned(S) || misaligned(z) ||
+      misaligned(Y))
+    return BHA_ERR_MISALIGNED;
+  const size_t es = esize(dtype);
+  const size_t q_bytes = static_cast<size_t>(n) * hq * b * d * es;
+  const size_t kv_bytes = static_cast<size_t>(n) * hkv * b * d * es;
+  const size_t s_bytes = static_cast<size_t>(n) * hkv * d * d * 4;
+  const size_t z_bytes = static_cast<size_t>(n) * hkv * d * 4;
+  if (overlap(Y, q_bytes, Qa, q_bytes) || overlap(Y, q_bytes, Ka, kv_bytes) ||
+      overlap(Y, q_bytes, Va, kv_bytes) || overlap(Y, q_bytes, S, s_bytes) ||
+      (shared && overlap(Y, q_bytes, z, z_bytes)))
+    return BHA_ERR_INVALID_ARG;
+  Ctx c;
+  st = make_ctx(stream, dtype, &c);
+  if (st != BHA_OK) return st;
+  const float sc = resolve_scale(scale, d);
+  if (dtype == BHA_F32)
+    return launch_status(launch_step_f32(
+        c, static_cast<const float*>(Qa), static_cast<const float*>(Ka),
+        static_cast<const float*>(Va), S, shared ? z : nullptr, static_cast<float*>(Y), n, hq,
+        hkv, b, d, sc, shared));
+  return launch_status(
+      launch_step_bf16(c, Qa, Ka, Va, S, shared ? z : nullptr, Y, n, hq, hkv, b, sc, shared));
+}
+
+size_t bha_prefix_softmax_workspace_size(int n, int hq, int hkv, int b, int d, int P,
+                                         bha_dtype dtype) {
+  if (dtype != BHA_BF16 || n <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0 || b < 1 || b > 64 ||
+      d != 128 || P < 0)
+    return 0;
+  return prefix_bf16_workspace(n, hq, hkv, b, P);
+}
+
+int bha_prefix_softmax(const void* Qa, const void* Kc, const void* Vc, int P, int cap,
+                       const void* Ka, const void* Va, void* Y, int n, int hq, int hkv, int b,
+                       int d, float scale, bha_dtype dtype, void* workspace,
+                       size_t workspace_bytes, bha_stream_t stream) {
+  int st = check_dims(dtype, d, b);
+  if (st != BHA_OK) return st;
+  if (n < 0 || hq < 1 || hkv < 1 || hq % hkv != 0 || P < 0 || cap < P)
+    return BHA_ERR_INVALID_ARG;
+  if (n == 0) return BHA_OK;
+  if (Qa == nullptr || Ka == nullptr || Va == nullptr || Y == nullptr ||
+      (P > 0 && (Kc == nullptr || Vc == nullptr)))
+    return BHA_ERR_INVALID_ARG;
+  if (misaligned(Qa) || misaligned(Kc) || misaligned(Vc) || misaligned(Ka) || misaligned(Va) ||
+      misaligned(Y) || misaligned(workspace))
+    return BHA_ERR_MISALIGNED;
+  const size_t es = esize(dtype);
+  const size_t q_bytes = static_cast<size_t>(n) * hq * b * d * es;
+  const size_t kv_bytes = static_cast<size_t>(n) * hkv * b * d * es;
+  const size_t c_bytes = static_cast<size_t>(n) * hkv * cap * d * es;
+  if (overlap(Y, q_bytes, Qa, q_bytes) || overlap(Y, q_bytes, Ka, kv_bytes) ||
+      overlap(Y, q_bytes, Va, kv_bytes) || overlap(Y, q_bytes, Kc, c_bytes) ||
+      overlap(Y, q_bytes, Vc, c_bytes))
+    return BHA_ERR_INVALID_ARG;
+  const size_t need = bha_prefix_softmax_workspace_size(n, hq, hkv, b, d, P, dtype);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BHA_ERR_WORKSPACE;
+  if (need > 0 && (overlap(workspace, need, Y, q_bytes) || overlap(workspace, need, Qa, q_bytes) ||
+                   overlap(workspace, need, Kc, c_bytes) || overlap(workspace, need, Vc, c_bytes)))
+    return BHA_ERR_INVALID_ARG;
+  Ctx c;
+  st = make_ctx(stream, dtype, &c);
+  if (st != BHA_OK) return st;
+  const float sc = resolve_scale(scale, d);
+  if (dtype == BHA_F32)
+    return launch_status(launch_prefix_f32(
+        c, static_cast<const float*>(Qa), static_cast<const float*>(Kc),
+        static_cast<const float*>(Vc), P, cap, static_cast<const float*>(Ka),
+        static_cast<const float*>(Va), static_cast<float*>(Y), n, hq, hkv, b, d, sc));
+  return launch_status(launch_prefix_bf16(c, Qa, Kc, Vc, P, cap, Ka, Va, Y, n, hq, hkv, b, sc,
+                                          workspace, workspace_bytes));
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// Internal host-side interface between the C ABI layer and the kernels.
+#pragma once
+
+#include <atomic>
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace bha {
+
+struct Ctx {
+  cudaStream_t stream;
+  int* dev_err;    // device error word of the current device
+  int sm_count;    // SMs of the current device
+};
+
+// Tensor-map encoder fetched from the driver at run time (no libcuda link).
+// Returns false if the driver entry point is unavailable or rejects the map.
+bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* gaddr,
+                 const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                 CUtensorMapSwizzle swizzle);
+
+// Sets a kernel's dynamic shared-memory limit and the maximum shared-memory
+// carveout once per device (bit `dev` of `done`), outside any hot path.
+template <typename Kernel>
+bool prepare_kernel(Kernel kern, int smem_bytes, std::atomic<uint64_t>& done) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  const uint64_t bit = 1ull << dev;
+  if (done.load(std::memory_order_acquire) & bit) return true;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
+      cudaSuccess)
+    return false;
+  cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  done.fetch_or(bit, std::memory_order_release);
+  return true;
+}
+
+// ---- fp32 reference mode (CUDA cores) ----
+int launch_step_f32(const Ctx& c, const float* Q, const float* K, const float* V,
+                    const float* S, const float* z, float* Y, int n, int hq, int hkv, int b,
+                    int d, float scale, int shared);
+int launch_commit_f32(const Ctx& c, const float* K, const float* V, int units, int b, int d,
+                      float* S, float* z);
+int launch_prefill_f32(const Ctx& c, const float* K, const float* V, int units, int T, int d,
+                       float* S, float* z);
+int launch_prefix_f32(const Ctx& c, const float* Q, const float* Kc, const float* Vc, int P,
+                      int cap, const float* K, const float* V, float* Y, int n, int hq, int hkv,
+                      int b, int d, float scale);
+
+// ---- bf16 tensor-core path (tcgen05, d = 128) ----
+int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, const float* S,
+                     const float* z, void* Y, int n, int hq, int hkv, int b, float scale,
+                     int shared);
+int launch_commit_bf16(const Ctx& c, const void* K, const void* V, int units, int b, float* S,
+                       float* z);
+size_t prefill_bf16_workspace(int units, int T);
+int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, int T, float* S,
+                        float* z, void* ws, size_t ws_bytes);
+size_t prefix_bf16_workspace(int n, int hq, int hkv, int b, int P);
+int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* Vc, int P,
+                       int cap, const void* K, const void* V, void* Y, int n, int hq, int hkv,
+                       int b, float scale, void* ws, size_t ws_bytes);
+
+}  // namespace bha

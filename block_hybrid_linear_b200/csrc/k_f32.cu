@@ -1,0 +1,231 @@
+// fp32 reference-mode kernels (CUDA cores, FFMA): the same operations as the
+// bf16 tensor-core path with fp32 Q/K/V/Y, any d <= 128 (d % 4 == 0) and
+// b <= 64.  Used for the worked example (d = 16) and tight-tolerance checks.
+// Simple one-row-at-a-time structure; not a performance path.
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "bha_internal.h"
+
+namespace bha {
+namespace {
+
+constexpr int kThreads = 128;
+
+__device__ __forceinline__ float relu(float x) { return x > 0.f ? x : 0.f; }
+
+__device__ float block_reduce_max(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float r = red[0];
+  for (int i = 1; i < kThreads / 32; ++i) r = fmaxf(r, red[i]);
+  return r;
+}
+
+__device__ float block_reduce_sum(float v, float* red) {
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  const int w = threadIdx.x / 32, l = threadIdx.x % 32;
+  __syncthreads();
+  if (l == 0) red[w] = v;
+  __syncthreads();
+  float r = 0.f;
+  for (int i = 0; i < kThreads / 32; ++i) r += red[i];
+  return r;
+}
+
+// One CTA per (request, query head).  Row by row: scores against the b block
+// keys, softmax, then each thread produces one output column
+//   y[c] = sum_j p_j v_j[c] + sum_r relu(q_r) S[r][c]      (default)
+//   y[c] = (sum_j e_j v_j[c] + e^{-m} lin[c]) / (l + e^{-m} relu(q).z)  (shared)
+__global__ void __launch_bounds__(kThreads) k_step_f32(const float* __restrict__ Q,
+                                                       const float* __restrict__ K,
+                                                       const float* __restrict__ V,
+                                                       const float* __restrict__ S,
+                                                       const float* __restrict__ z,
+                                                       float* __restrict__ Y, int hq, int hkv,
+                                                       int b, int d, float scale, int shared) {
+  extern __shared__ float sm[];
+  float* sK = sm;              // [b][d]
+  float* sV = sK + b * d;      // [b][d]
+  float* sq = sV + b * d;      // [d]
+  float* sp = sq + d;          // [b]
+  __shared__ float red[kThreads / 32];
+
+  const int nh = blockIdx.x;
+  const int ni = nh / hq, h = nh % hq, g = h / (hq / hkv);
+  const size_t kv_off = ((size_t)ni * hkv + g) * b * d;
+  for (int e = threadIdx.x; e < b * d; e += kThreads) {
+    sK[e] = K[kv_off + e];
+    sV[e] = V[kv_off + e];
+  }
+  const float* Sg = S + ((size_t)ni * hkv + g) * d * d;
+  const float* zg = z ? z + ((size_t)ni * hkv + g) * d : nullptr;
+  __syncthreads();
+
+  for (int i = 0; i < b; ++i) {
+    const size_t row = (((size_t)ni * hq + h) * b + i) * d;
+    for (int c = threadIdx.x; c < d; c += kThreads) sq[c] = Q[row + c];
+    __syncthreads();
+    float s = -INFINITY;
+    if (threadIdx.x < b) {
+      float acc = 0.f;
+      for (int c = 0; c < d; ++c) acc = fmaf(sq[c], sK[threadIdx.x * d + c], acc);
+      s = acc * scale;
+    }
+    const float m = block_reduce_max(s, red);
+    const float e = threadIdx.x < b ? expf(s - m) : 0.f;
+    const float l = block_reduce_sum(e, red);
+    if (threadIdx.x < b) sp[threadIdx.x] = e;
+    float qz = 0.f;
+    if (shared) {
+      float part = 0.f;
+      for (int r = threadIdx.x; r < d; r += kThreads) part = fmaf(relu(sq[r]), zg[r], part);
+      qz = block_reduce_sum(part, red);
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < d; c += kThreads) {
+      float soft = 0.f;
+      for (int j = 0; j < b; ++j) soft = fmaf(sp[j], sV[j * d + c], soft);
+      float lin = 0.f;
+      for (int r = 0; r < d; ++r) lin = fmaf(relu(sq[r]), Sg[(size_t)r * d + c], lin);
+      float y;
+      if (!shared) {
+        y = soft / l + lin;
+      } else {
+        const float em = expf(-m);
+        y = (soft + em * lin) / (l + em * qz);
+      }
+      Y[row + c] = y;
+    }
+    __syncthreads();
+  }
+}
+
+// S[u][r][c] (+)= sum_t relu(K[u][t][r]) V[u][t][c];  z[u][r] (+)= sum_t relu(K[u][t][r]).
+// One thread per (r, c) state element; accumulate != 0 adds to S (commit),
+// otherwise overwrites (prefill).
+__global__ void __launch_bounds__(kThreads) k_state_f32(const float* __restrict__ K,
+                                                        const float* __restrict__ V, int T,
+                                                        int d, float* __restrict__ S,
+                                                        float* __restrict__ z, int accumulate) {
+  const int u = blockIdx.y;
+  const int e = blockIdx.x * kThreads + threadIdx.x;
+  const float* Ku = K + (size_t)u * T * d;
+  const float* Vu = V + (size_t)u * T * d;
+  if (e < d * d) {
+    const int r = e / d, c = e % d;
+    float acc = 0.f;
+    for (int t = 0; t < T; ++t) acc = fmaf(relu(Ku[(size_t)t * d + r]), Vu[(size_t)t * d + c], acc);
+    float* dst = S + (size_t)u * d * d + e;
+    *dst = accumulate ? *dst + acc : acc;
+  }
+  if (z && e < d) {
+    float acc = 0.f;
+    for (int t = 0; t < T; ++t) acc += relu(Ku[(size_t)t * d + e]);
+    float* dst = z + (size_t)u * d + e;
+    *dst = accumulate ? *dst + acc : acc;
+  }
+}
+
+// Exact softmax over [cache[0:P] || block]: one CTA per (request, head, row);
+// keys are scored 128 at a time with an online max / sum rescale.
+__global__ void __launch_bounds__(kThreads) k_prefix_f32(
+    const float* __restrict__ Q, const float* __restrict__ Kc, const float* __restrict__ Vc,
+    int P, int cap, const float* __restrict__ K, const float* __restrict__ V,
+    float* __restrict__ Y, int hq, int hkv, int b, int d, float scale) {
+  extern __shared__ float sm[];
+  float* sq = sm;           // [d]
+  float* se = sq + d;       // [kThreads]
+  float* acc = se + kThreads;  // [d]
+  __shared__ float red[kThreads / 32];
+
+  const int id = blockIdx.x;
+  const int i = id % b, nh = id / b;
+  const int ni = nh / hq, h = nh % hq, g = h / (hq / hkv);
+  const size_t row = (((size_t)ni * hq + h) * b + i) * d;
+  const float* Kcg = Kc + ((size_t)ni * hkv + g) * cap * d;
+  const float* Vcg = Vc + ((size_t)ni * hkv + g) * cap * d;
+  const float* Kg = K + ((size_t)ni * hkv + g) * b * d;
+  const float* Vg = V + ((size_t)ni * hkv + g) * b * d;
+  for (int c = threadIdx.x; c < d; c += kThreads) {
+    sq[c] = Q[row + c];
+    acc[c] = 0.f;
+  }
+  __syncthreads();
+  const int L = P + b;
+  float m_run = -INFINITY, l_run = 0.f;
+  for (int j0 = 0; j0 < L; j0 += kThreads) {
+    const int j = j0 + threadIdx.x;
+    float s = -INFINITY;
+    if (j < L) {
+      const float* k = j < P ? Kcg + (size_t)j * d : Kg + (size_t)(j - P) * d;
+      float a = 0.f;
+      for (int c = 0; c < d; ++c) a = fmaf(sq[c], k[c], a);
+      s = a * scale;
+    }
+    const float m_new = fmaxf(m_run, block_reduce_max(s, red));
+    const float e = j < L ? expf(s - m_new) : 0.f;
+    const float corr = expf(m_run - m_new);  // 0 on the first chunk
+    se[threadIdx.x] = e;
+    l_run = l_run * corr + block_reduce_sum(e, red);
+    m_run = m_new;
+    __syncthreads();
+    const int cnt = min(kThreads, L - j0);
+    for (int c = threadIdx.x; c < d; c += kThreads) {
+      float a = acc[c] * corr;
+      for (int t = 0; t < cnt; ++t) {
+        const int jj = j0 + t;
+        const float* v = jj < P ? Vcg + (size_t)jj * d : Vg + (size_t)(jj - P) * d;
+        a = fmaf(se[t], v[c], a);
+      }
+      acc[c] = a;
+    }
+    __syncthreads();
+  }
+  for (int c = threadIdx.x; c < d; c += kThreads) Y[row + c] = acc[c] / l_run;
+}
+
+int finish_launch() {
+  return cudaGetLastError() == cudaSuccess ? 0 : -5;
+}
+
+}  // namespace
+
+int launch_step_f32(const Ctx& c, const float* Q, const float* K, const float* V,
+                    const float* S, const float* z, float* Y, int n, int hq, int hkv, int b,
+                    int d, float scale, int shared) {
+  const size_t smem = (size_t)(2 * b * d + d + b) * sizeof(float);
+  static std::atomic<uint64_t> prepared{0};
+  if (!prepare_kernel(k_step_f32, 2 * 64 * 128 * 4 + 4 * 128 + 4 * 64, prepared)) return -5;
+  k_step_f32<<<n * hq, kThreads, smem, c.stream>>>(Q, K, V, S, z, Y, hq, hkv, b, d, scale,
+                                                   shared);
+  return finish_launch();
+}
+
+int launch_commit_f32(const Ctx& c, const float* K, const float* V, int units, int b, int d,
+                      float* S, float* z) {
+  dim3 grid((d * d + kThreads - 1) / kThreads, units);
+  k_state_f32<<<grid, kThreads, 0, c.stream>>>(K, V, b, d, S, z, 1);
+  return finish_launch();
+}
+
+int launch_prefill_f32(const Ctx& c, const float* K, const float* V, int units, int T, int d,
+                       float* S, float* z) {
+  dim3 grid((d * d + kThreads - 1) / kThreads, units);
+  k_state_f32<<<grid, kThreads, 0, c.stream>>>(K, V, T, d, S, z, 0);
+  return finish_launch();
+}
+
+int launch_prefix_f32(const Ctx& c, const float* Q, const float* Kc, const float* Vc, int P,
+                      int cap, const float* K, const float* V, float* Y, int n, int hq, int hkv,
+                      int b, int d, float scale) {
+  const size_t smem = (size_t)(2 * d + kThreads) * sizeof(float);
+  k_prefix_f32<<<n * hq * b, kThreads, smem, c.stream>>>(Q, Kc, Vc, P, cap, K, V, Y, hq, hkv,
+                                                         b, d, scale);
+  return finish_launch();
+}
+
+}  // namespace bha

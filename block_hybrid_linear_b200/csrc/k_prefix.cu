@@ -1,0 +1,448 @@
+// bha_prefix_softmax, bf16 tensor-core path (d = 128): the comparison path.
+//
+// Exact softmax attention of the active block's queries over the whole KV
+// cache followed by the block itself -- the baseline of "Retrofitting Linear
+// Attention into Diffusion Language Models" (abstract: every denoising step
+// still attends to all previous blocks).  Flash-attention structure on
+// tcgen05:
+//   * one CTA per (request, KV head, 128-row tile of the G*b packed query
+//     rows, chunk of the key sequence); keys come in 128-token tiles, cache
+//     tiles first, the active block last;
+//   * a TMA warp streams K and V tiles through 2-stage rings, an MMA warp
+//     issues S = Q K^T into one of two TMEM buffers and O += P V into a TMEM
+//     accumulator, and four softmax warps (thread = query row = TMEM lane)
+//     run the online softmax in registers, rescaling O only when a row max
+//     grows by more than 2^8 (the stale max is exact for the final ratio);
+//   * chunks are combined by log-sum-exp in a second kernel, the way the
+//     LoSA page describes merging prefix and block attention with online
+//     softmax.  With one chunk the CTA normalises and stores Y itself.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+
+#include "bha_internal.h"
+#include "bha_ptx.cuh"
+
+namespace bha {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kTK = 128;             // keys per tile
+constexpr int kThreads = 256;
+constexpr uint32_t kTileBytes = kTK * kD * 2;   // 32 KB (K or V tile, Q, P)
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffK = kTileBytes;          // 2 stages
+constexpr uint32_t kOffV = 3 * kTileBytes;      // 2 stages
+constexpr uint32_t kOffP = 5 * kTileBytes;
+constexpr uint32_t kTiles = 6 * kTileBytes;     // 192 KB
+constexpr uint32_t kCtrlBytes = 256;
+constexpr uint32_t kSmem = kTiles + 1024;
+constexpr float kRescaleLog2 = 8.f;             // rescale O when max grows > 2^8
+constexpr int kTargetCtas = 592;                // four CTAs' worth per SM (148 SMs)
+constexpr int kMinTilesPerChunk = 8;
+
+struct PrefixArgs {
+  int* err;
+  float* wsO;        // [items][128][128] fp32 partial numerators (splits > 1)
+  float* wsML;       // [items][2][128] row max (log2 units) and row sum
+  int rows;          // G * b
+  int mtiles;
+  int P;             // cached tokens
+  int b;             // active-block tokens
+  int ncache_tiles;  // ceil(P / 128)
+  int splits;
+  int tiles_per;
+  float sl2;         // scale * log2(e)
+};
+
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
+      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
+      "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]),
+      "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]),
+      "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]),
+      "f"(v[29]), "f"(v[30]), "f"(v[31])
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    k_prefix_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
+                  const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKa,
+                  const __grid_constant__ CUtensorMap tmVa, const __grid_constant__ CUtensorMap tmY,
+                  const __grid_constant__ CUtensorMap tmO, const PrefixArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int item = blockIdx.x;
+  const int sp = item % a.splits;
+  const int umt = item / a.splits;
+  const int u = umt / a.mtiles, mt = umt % a.mtiles;
+  const int ntot = a.ncache_tiles + 1;
+  const int tile0 = sp * a.tiles_per;
+  const int nt = min(a.tiles_per, ntot - tile0);
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + kTiles;
+  uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
+  const uint32_t bar_q = ctrl, bar_kf = ctrl + 8, bar_ke = ctrl + 24, bar_vf = ctrl + 40,
+                 bar_ve = ctrl + 56, bar_sf = ctrl + 72, bar_pf = ctrl + 88, bar_pv = ctrl + 96;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 104);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 108);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_init(bar_q, 1);
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(bar_kf + 8 * s, 1);
+        mbar_init(bar_ke + 8 * s, 1);
+        mbar_init(bar_vf + 8 * s, 1);
+        mbar_init(bar_ve + 8 * s, 1);
+        mbar_init(bar_sf + 8 * s, 1);
+      }
+      mbar_init(bar_pf, 128);
+      mbar_init(bar_pv, 1);
+      *abort_flag = 0;
+      fence_mbar_init();
+    }
+    __syncwarp();
+    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_o = tmem + 256;
+
+  if (tid == 0) {
+    // ---------------- TMA producer
+    const int row0 = mt * 128;
+    mbar_arrive_expect_tx(bar_q, kTileBytes);
+    tma_load_3d(base + kOffQ, &tmQ, bar_q, 0, row0, u);
+    tma_load_3d(base + kOffQ + 16384, &tmQ, bar_q, 64, row0, u);
+    for (int i = 0; i < nt; ++i) {
+      const int st = i & 1;
+      const int gi = tile0 + i;
+      const bool cache = gi < a.ncache_tiles;
+      const CUtensorMap* mk = cache ? &tmKc : &tmKa;
+      const CUtensorMap* mv = cache ? &tmVc : &tmVa;
+      const int trow = cache ? gi * kTK : 0;
+      if (i >= 2 && !mbar_wait(bar_ke + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
+      mbar_arrive_expect_tx(bar_kf + 8 * st, kTileBytes);
+      tma_load_3d(base + kOffK + st * kTileBytes, mk, bar_kf + 8 * st, 0, trow, u);
+      tma_load_3d(base + kOffK + st * kTileBytes + 16384, mk, bar_kf + 8 * st, 64, trow, u);
+      if (i >= 2 && !mbar_wait(bar_ve + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
+      mbar_arrive_expect_tx(bar_vf + 8 * st, kTileBytes);
+      tma_load_3d(base + kOffV + st * kTileBytes, mv, bar_vf + 8 * st, 0, trow, u);
+      tma_load_3d(base + kOffV + st * kTileBytes + 16384, mv, bar_vf + 8 * st, 64, trow, u);
+    }
+  } else if (tid == 32) {
+    // ---------------- MMA issuer
+    constexpr uint32_t idesc_s = make_idesc_bf16(128, kTK, 0, 0);   // Q K^T, both K-major
+    constexpr uint32_t idesc_o = make_idesc_bf16(128, kD, 0, 1);    // P V, V MN-major
+    bool ok = mbar_wait(bar_q, 0, a.err, abort_flag);
+    auto issue_s = [&](int i) -> bool {
+      const int st = i & 1;
+      if (!mbar_wait(bar_kf + 8 * st, (i >> 1) & 1, a.err, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t kb = base + kOffK + st * kTileBytes;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t da =
+            make_sdesc(base + kOffQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128);
+        const uint64_t db = make_sdesc(kb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024,
+                                       kLayoutSW128);
+        mma_bf16_ss(tmem + st * 128, da, db, idesc_s, ks > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_sf + 8 * st);
+      mma_commit(bar_ke + 8 * st);
+      return true;
+    };
+    if (ok && nt > 0) ok = issue_s(0);
+    for (int i = 0; i < nt && ok; ++i) {
+      if (i + 1 < nt) ok = issue_s(i + 1);
+      if (!ok) break;
+      const int st = i & 1;
+      ok = mbar_wait(bar_pf, i & 1, a.err, abort_flag) &&
+           mbar_wait(bar_vf + 8 * st, (i >> 1) & 1, a.err, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t vb = base + kOffV + st * kTileBytes;
+#pragma unroll
+      for (int ks = 0; ks < kTK / 16; ++ks) {
+        const uint64_t da =
+            make_sdesc(base + kOffP + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128);
+        // V tile: [keys][d] as 2 boxes of 64 d-columns; keys are the K dim
+        const uint64_t db = make_sdesc(vb + ks * 2048, 16384, 1024, kLayoutSW128);
+        mma_bf16_ss(t_o, da, db, idesc_o, (i | ks) ? 1u : 0u);
+      }
+      mma_commit(bar_ve + 8 * st);
+      mma_commit(bar_pv);
+    }
+  }
+
+  // ---------------- softmax warps: thread = query row = TMEM lane
+  float mx = -INFINITY, l = 0.f;
+  const int r = (warp & 3) * 32 + lane;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  bool ok = true;
+  if (warp >= 4) {
+    for (int i = 0; i < nt; ++i) {
+      const int st = i & 1;
+      const int gi = tile0 + i;
+      const int valid = gi < a.ncache_tiles ? min(kTK, a.P - gi * kTK) : a.b;
+      ok = warp_all(ok && mbar_wait(bar_sf + 8 * st, (i >> 1) & 1, a.err, abort_flag));
+      if (!ok) break;
+      tc_fence_after();
+      float s[kTK];
+#pragma unroll
+      for (int c = 0; c < kTK; c += 32) {
+        float t[32];
+        tmem_ld32_sync(tmem + st * 128 + lane_base + c, t);
+#pragma unroll
+        for (int q = 0; q < 32; ++q) s[c + q] = t[q];
+      }
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kTK; ++j) {
+        if (j >= valid) s[j] = -INFINITY;
+        tmax = fmaxf(tmax, s[j]);
+      }
+      float corr = 1.f;
+      bool resc = false;
+      if (mx == -INFINITY) {
+        mx = tmax;
+      } else if ((tmax - mx) * a.sl2 > kRescaleLog2) {
+        corr = exp2f((mx - tmax) * a.sl2);
+        mx = tmax;
+        resc = true;
+      }
+      float ls = 0.f;
+#pragma unroll
+      for (int j = 0; j < kTK; ++j) {
+        s[j] = exp2f((s[j] - mx) * a.sl2);
+        ls += s[j];
+      }
+      l = l * corr + ls;
+      // P and O are free once P V of the previous tile has completed
+      if (i > 0) {
+        ok = warp_all(mbar_wait(bar_pv, (i - 1) & 1, a.err, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, resc)) {
+#pragma unroll 1
+          for (int c = 0; c < kD; c += 32) {
+            float o[32];
+            tmem_ld32_sync(t_o + lane_base + c, o);
+#pragma unroll
+            for (int q = 0; q < 32; ++q) o[q] *= corr;
+            tmem_st32(t_o + lane_base + c, o);
+          }
+        }
+      }
+#pragma unroll
+      for (int box = 0; box < 2; ++box) {
+        const uint32_t prow = base + kOffP + box * 16384 + r * 128;
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const float* e = s + box * 64 + jj * 8;
+          st_shared_v4(prow + ((jj ^ (r & 7)) << 4), pack_bf16x2(e[0], e[1]),
+                       pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_pf);
+    }
+    // final accumulator
+    if (ok && nt > 0) ok = warp_all(mbar_wait(bar_pv, (nt - 1) & 1, a.err, abort_flag));
+    tc_fence_after();
+    if (ok) {
+      if (a.splits == 1) {
+        const float inv = 1.f / l;
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+          float o[32];
+          tmem_ld32_sync(t_o + lane_base + cc * 32, o);
+          const uint32_t row = base + kOffQ + (cc >> 1) * 16384 + r * 128;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int j = (cc & 1) * 4 + q;
+            const float* e = o + 8 * q;
+            st_shared_v4(row + ((j ^ (r & 7)) << 4), pack_bf16x2(e[0] * inv, e[1] * inv),
+                         pack_bf16x2(e[2] * inv, e[3] * inv), pack_bf16x2(e[4] * inv, e[5] * inv),
+                         pack_bf16x2(e[6] * inv, e[7] * inv));
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int bx = 0; bx < 4; ++bx) {
+          float o[32];
+          tmem_ld32_sync(t_o + lane_base + bx * 32, o);
+          const uint32_t row = base + kOffK + bx * 16384 + r * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_f4(row + ((j ^ (r & 7)) << 4),
+                         make_float4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]));
+        }
+        float* ml = a.wsML + static_cast<size_t>(item) * 256;
+        ml[r] = mx * a.sl2;
+        ml[128 + r] = l;
+      }
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && !*abort_flag) {
+    if (a.splits == 1) {
+      tma_store_3d(&tmY, base + kOffQ, 0, mt * 128, u);
+      tma_store_3d(&tmY, base + kOffQ + 16384, 64, mt * 128, u);
+    } else {
+#pragma unroll
+      for (int bx = 0; bx < 4; ++bx) tma_store_3d(&tmO, base + kOffK + bx * 16384, 32 * bx, 0, item);
+    }
+    bulk_commit_group();
+    bulk_wait_group_read0();
+  }
+  __syncwarp();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// y[r][c] = sum_s 2^{m_s - M} O_s[r][c] / sum_s 2^{m_s - M} l_s,  M = max_s m_s
+__global__ void __launch_bounds__(256) k_prefix_merge(const float* __restrict__ wsO,
+                                                      const float* __restrict__ wsML,
+                                                      __nv_bfloat16* __restrict__ Y, int rows,
+                                                      int mtiles, int splits) {
+  const int umt = blockIdx.y;
+  const int u = umt / mtiles, mt = umt % mtiles;
+  const int e = blockIdx.x * 256 + threadIdx.x;      // float4 index in the 128 x 128 tile
+  const int r = e >> 5, c4 = e & 31;
+  const int grow = mt * 128 + r;
+  if (grow >= rows) return;
+  const size_t item0 = static_cast<size_t>(umt) * splits;
+  float M = -INFINITY;
+  for (int s = 0; s < splits; ++s) M = fmaxf(M, wsML[(item0 + s) * 256 + r]);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float den = 0.f;
+  for (int s = 0; s < splits; ++s) {
+    const float* ml = wsML + (item0 + s) * 256;
+    const float w = exp2f(ml[r] - M);
+    den = fmaf(w, ml[128 + r], den);
+    const float4 o = reinterpret_cast<const float4*>(wsO + (item0 + s) * kD * kD + r * kD)[c4];
+    acc.x = fmaf(w, o.x, acc.x);
+    acc.y = fmaf(w, o.y, acc.y);
+    acc.z = fmaf(w, o.z, acc.z);
+    acc.w = fmaf(w, o.w, acc.w);
+  }
+  const float inv = 1.f / den;
+  __nv_bfloat162* out = reinterpret_cast<__nv_bfloat162*>(
+      Y + (static_cast<size_t>(u) * rows + grow) * kD + c4 * 4);
+  out[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+  out[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+}
+
+void prefix_plan(int units, int mtiles, int P, int* splits, int* tiles_per) {
+  const int ntot = (P + kTK - 1) / kTK + 1;
+  const int items = units * mtiles;
+  int s = (kTargetCtas + items - 1) / items;
+  const int cap = (ntot + kMinTilesPerChunk - 1) / kMinTilesPerChunk;
+  if (s > cap) s = cap;
+  if (s < 1) s = 1;
+  const int tp = (ntot + s - 1) / s;
+  *splits = (ntot + tp - 1) / tp;
+  *tiles_per = tp;
+}
+
+bool bf16_rows_tmap(CUtensorMap* m, const void* X, uint64_t rows, uint64_t row_stride_elems,
+                    uint64_t units, uint32_t box_rows) {
+  const uint64_t dims[3] = {(uint64_t)kD, rows, units};
+  const uint64_t strides[2] = {kD * 2ull, row_stride_elems * kD * 2ull};
+  const uint32_t box[3] = {64, box_rows, 1};
+  return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+size_t prefix_bf16_workspace(int n, int hq, int hkv, int b, int P) {
+  const int units = n * hkv;
+  const int rows = (hq / hkv) * b;
+  const int mtiles = (rows + 127) / 128;
+  int splits, tp;
+  prefix_plan(units, mtiles, P, &splits, &tp);
+  if (splits <= 1) return 0;
+  return static_cast<size_t>(units) * mtiles * splits * (kD * kD + 256) * sizeof(float);
+}
+
+int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* Vc, int P,
+                       int cap, const void* K, const void* V, void* Y, int n, int hq, int hkv,
+                       int b, float scale, void* ws, size_t ws_bytes) {
+  const int units = n * hkv;
+  const int rows = (hq / hkv) * b;
+  const int mtiles = (rows + 127) / 128;
+  int splits, tp;
+  prefix_plan(units, mtiles, P, &splits, &tp);
+  const size_t need = prefix_bf16_workspace(n, hq, hkv, b, P);
+  if (need > ws_bytes) return -4;
+  const size_t items = static_cast<size_t>(units) * mtiles * splits;
+  float* wsO = splits > 1 ? static_cast<float*>(ws) : nullptr;
+  float* wsML = splits > 1 ? wsO + items * kD * kD : nullptr;
+
+  CUtensorMap tq, ty, tkc, tvc, tka, tva, to;
+  bool ok = bf16_rows_tmap(&tq, Q, rows, rows, units, 128) &&
+            bf16_rows_tmap(&ty, Y, rows, rows, units, 128) &&
+            bf16_rows_tmap(&tka, K, b, b, units, kTK) && bf16_rows_tmap(&tva, V, b, b, units, kTK);
+  if (P > 0) {
+    ok = ok && bf16_rows_tmap(&tkc, Kc, P, cap, units, kTK) &&
+         bf16_rows_tmap(&tvc, Vc, P, cap, units, kTK);
+  } else {
+    tkc = tka;   // never read: there are no cache tiles
+    tvc = tva;
+  }
+  if (splits > 1) {
+    const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)kD, items};
+    const uint64_t strides[2] = {kD * 4ull, (uint64_t)kD * kD * 4ull};
+    const uint32_t box[3] = {32, 128, 1};
+    ok = ok && encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, wsO, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+  } else {
+    to = ty;     // never used with one chunk
+  }
+  if (!ok) return -5;
+  PrefixArgs a;
+  a.err = c.dev_err;
+  a.wsO = wsO;
+  a.wsML = wsML;
+  a.rows = rows;
+  a.mtiles = mtiles;
+  a.P = P;
+  a.b = b;
+  a.ncache_tiles = (P + kTK - 1) / kTK;
+  a.splits = splits;
+  a.tiles_per = tp;
+  a.sl2 = scale * 1.4426950408889634f;
+  static std::atomic<uint64_t> prepared{0};
+  if (!prepare_kernel(k_prefix_bf16, (int)kSmem, prepared)) return -5;
+  k_prefix_bf16<<<(unsigned)items, kThreads, kSmem, c.stream>>>(tq, tkc, tvc, tka, tva, ty, to,
+                                                                 a);
+  if (cudaGetLastError() != cudaSuccess) return -5;
+  if (splits > 1) {
+    dim3 grid(kD * kD / 4 / 256, units * mtiles);
+    k_prefix_merge<<<grid, 256, 0, c.stream>>>(wsO, wsML, static_cast<__nv_bfloat16*>(Y), rows,
+                                               mtiles, splits);
+    if (cudaGetLastError() != cudaSuccess) return -5;
+  }
+  return 0;
+}
+
+}  // namespace bha

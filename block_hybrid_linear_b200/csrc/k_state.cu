@@ -1,0 +1,498 @@
+// bha_state_commit and bha_state_prefill, bf16 tensor-core path (d = 128).
+//
+// Both build the linear-attention prefix state of "Retrofitting Linear
+// Attention into Diffusion Language Models" (worked example: S_1 =
+// phi(K_1)^T V_1 and S_{1,2} = S_1 + phi(K_2)^T V_2, phi = ReLU):
+//     S[r][c] (+)= sum_t relu(k_t[r]) v_t[c],   z[r] (+)= sum_t relu(k_t[r]).
+// phi(K)^T V is an M=128 (feature r) x N=128 (value column c) contraction
+// over tokens t, run on tcgen05 with both operands MN-major: the K and V
+// tiles land by TMA exactly as they sit in memory ([t][128] rows, SW128),
+// phi is applied in place, and the fp32 accumulator lives in TMEM.
+//
+// Commit: one CTA per (request, KV head): one MMA chain over the b block
+// tokens, then S is read-modified-written through a swizzled fp32 tile
+// (thread = row r, conflict-free) and stored back by TMA.
+//
+// Prefill: one CTA per (unit, chunk of the prompt), a 3-stage TMA ring of
+// 64-token K/V tiles (32 KB per stage) feeding the MMA warp; the chunk's
+// partial state goes to the workspace (or straight to S when the prompt is
+// one chunk) and a second kernel adds the chunks in a fixed order.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "bha_internal.h"
+#include "bha_ptx.cuh"
+
+namespace bha {
+namespace {
+
+constexpr int kD = 128;
+constexpr int kThreads = 256;
+constexpr uint32_t kSBytes = kD * kD * 4;   // 64 KB fp32 state tile
+constexpr uint32_t kCtrlBytes = 128;
+
+__device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
+
+// Adds the TMEM accumulator (128 lanes x 128 fp32 columns) into / writes it
+// over the swizzled fp32 state tile at `tile` (4 SW128 boxes of 128 rows x
+// 32 columns).  Warp w handles rows 32*(w%4).., columns 64*(w/4)..
+__device__ __forceinline__ void accum_to_tile(uint32_t tmem, uint32_t tile, int warp, int lane,
+                                              bool add) {
+  const int r = (warp & 3) * 32 + lane;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+#pragma unroll 1
+  for (int bx = 2 * (warp >> 2); bx < 2 * (warp >> 2) + 2; ++bx) {
+    float acc[32];
+    tmem_ld32_sync(tmem + lane_base + bx * 32, acc);
+    const uint32_t row = tile + bx * 16384 + r * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t addr = row + ((j ^ (r & 7)) << 4);
+      float4 v = make_float4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+      if (add) {
+        const float4 s = ld_shared_f4(addr);
+        v.x += s.x;
+        v.y += s.y;
+        v.z += s.z;
+        v.w += s.w;
+      }
+      st_shared_f4(addr, v);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ commit
+
+struct CommitArgs {
+  float* z;   // [units][128] or null
+  int* err;
+  int b;
+};
+
+template <int BPAD>
+struct CommitLayout {
+  static constexpr uint32_t kKV = BPAD * 256;
+  static constexpr uint32_t kOffS = 0;
+  static constexpr uint32_t kOffK = kSBytes;
+  static constexpr uint32_t kOffV = kOffK + kKV;
+  static constexpr uint32_t kTiles = kOffV + kKV;
+  static constexpr uint32_t kSmem = kTiles + 1024;
+};
+
+template <int BPAD>
+__global__ void __launch_bounds__(kThreads, 2)
+    k_commit_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmS, const CommitArgs a) {
+  using Lay = CommitLayout<BPAD>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int u = blockIdx.x;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + Lay::kTiles;
+  uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
+  const uint32_t bar_kv = ctrl, bar_s = ctrl + 8, bar_done = ctrl + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 32);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 36);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_init(bar_kv, 1);
+      mbar_init(bar_s, 1);
+      mbar_init(bar_done, 1);
+      *abort_flag = 0;
+      fence_mbar_init();
+    }
+    __syncwarp();
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_kv, 2 * Lay::kKV);
+    tma_load_3d(base + Lay::kOffK, &tmK, bar_kv, 0, 0, u);
+    tma_load_3d(base + Lay::kOffK + BPAD * 128, &tmK, bar_kv, 64, 0, u);
+    tma_load_3d(base + Lay::kOffV, &tmV, bar_kv, 0, 0, u);
+    tma_load_3d(base + Lay::kOffV + BPAD * 128, &tmV, bar_kv, 64, 0, u);
+    mbar_arrive_expect_tx(bar_s, kSBytes);
+#pragma unroll
+    for (int bx = 0; bx < 4; ++bx)
+      tma_load_3d(base + Lay::kOffS + bx * 16384, &tmS, bar_s, 32 * bx, 0, u);
+  }
+
+  // phi(K) in place
+  bool ok = warp_all(mbar_wait(bar_kv, 0, a.err, abort_flag));
+  if (ok) {
+    for (uint32_t v = tid; v < Lay::kKV / 16; v += kThreads) {
+      const uint32_t addr = base + Lay::kOffK + v * 16;
+      uint4 x = ld_shared_v4(addr);
+      st_shared_v4(addr, relu_bf16x2(x.x), relu_bf16x2(x.y), relu_bf16x2(x.z),
+                   relu_bf16x2(x.w));
+    }
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+
+  if (tid == 32 && !*abort_flag) {
+    tc_fence_after();
+    constexpr uint32_t idesc = make_idesc_bf16(128, 128, 1, 1);
+#pragma unroll
+    for (int ks = 0; ks < BPAD / 16; ++ks) {
+      const uint64_t da = make_sdesc(base + Lay::kOffK + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
+      const uint64_t db = make_sdesc(base + Lay::kOffV + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
+      mma_bf16_ss(tmem, da, db, idesc, ks > 0 ? 1u : 0u);
+    }
+    mma_commit(bar_done);
+  }
+
+  // z += column sums of phi(K) (threads 0..127, one feature each)
+  if (a.z != nullptr && tid < kD && !*abort_flag) {
+    const int rr = tid;
+    const uint32_t col = base + Lay::kOffK + (rr >> 6) * (BPAD * 128) + (rr & 7) * 2;
+    float s = 0.f;
+    for (int t = 0; t < a.b; ++t) {
+      unsigned short hv;
+      const uint32_t addr = col + t * 128 + (((((rr & 63) >> 3) ^ (t & 7))) << 4);
+      asm volatile("ld.shared.u16 %0, [%1];" : "=h"(hv) : "r"(addr));
+      s += __uint_as_float(static_cast<uint32_t>(hv) << 16);
+    }
+    a.z[static_cast<size_t>(u) * kD + rr] += s;
+  }
+
+  ok = warp_all(mbar_wait(bar_s, 0, a.err, abort_flag) && mbar_wait(bar_done, 0, a.err, abort_flag));
+  tc_fence_after();
+  if (ok) accum_to_tile(tmem, base + Lay::kOffS, warp, lane, true);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && !*abort_flag) {
+#pragma unroll
+    for (int bx = 0; bx < 4; ++bx) tma_store_3d(&tmS, base + Lay::kOffS + bx * 16384, 32 * bx, 0, u);
+    bulk_commit_group();
+    bulk_wait_group_read0();
+  }
+  __syncwarp();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ------------------------------------------------------------------ prefill
+
+constexpr int kTok = 64;                  // tokens per pipeline stage
+constexpr int kStages = 3;
+constexpr uint32_t kStageBytes = 2 * kTok * kD * 2;   // K + V tile: 32 KB
+constexpr uint32_t kPrefTiles = kStages * kStageBytes; // 96 KB (>= 64 KB epilogue tile)
+constexpr uint32_t kPrefSmem = kPrefTiles + 1024;
+constexpr int kMaxTilesPerChunk = 64;     // 4096 tokens
+constexpr int kMinTilesPerChunk = 16;     // 1024 tokens
+constexpr int kTargetCtas = 296;          // two CTAs on each of 148 SMs
+
+struct PrefillArgs {
+  float* zdst;       // [items][128] or null (partial or final z)
+  int* err;
+  int T;             // prompt tokens
+  int splits;        // chunks per unit
+  int tiles_per;     // 64-token tiles per chunk
+};
+
+__global__ void __launch_bounds__(kThreads, 2)
+    k_prefill_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                   const __grid_constant__ CUtensorMap tmOut, const PrefillArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int item = blockIdx.x;                // = u * splits + s
+  const int u = item / a.splits, sp = item % a.splits;
+  const int ntiles_total = (a.T + kTok - 1) / kTok;
+  const int tile0 = sp * a.tiles_per;
+  const int ntile = min(a.tiles_per, ntiles_total - tile0);
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + kPrefTiles;
+  uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
+  const uint32_t bar_full = ctrl, bar_relu = ctrl + 24, bar_empty = ctrl + 48,
+                 bar_done = ctrl + 72;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 80);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 84);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < kStages; ++s) {
+        mbar_init(bar_full + 8 * s, 1);
+        mbar_init(bar_relu + 8 * s, 128);
+        mbar_init(bar_empty + 8 * s, 1);
+      }
+      mbar_init(bar_done, 1);
+      *abort_flag = 0;
+      fence_mbar_init();
+    }
+    __syncwarp();
+    tmem_alloc(smem_u32(tmem_slot), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  float zacc[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) zacc[q] = 0.f;
+
+  if (tid == 0) {
+    // producer
+    for (int i = 0; i < ntile; ++i) {
+      const int st = i % kStages;
+      if (i >= kStages &&
+          !mbar_wait(bar_empty + 8 * st, ((i / kStages) - 1) & 1, a.err, abort_flag))
+        break;
+      const uint32_t sbase = base + st * kStageBytes;
+      const uint32_t bf = bar_full + 8 * st;
+      const int t0 = (tile0 + i) * kTok;
+      mbar_arrive_expect_tx(bf, kStageBytes);
+      tma_load_3d(sbase, &tmK, bf, 0, t0, u);
+      tma_load_3d(sbase + 8192, &tmK, bf, 64, t0, u);
+      tma_load_3d(sbase + 16384, &tmV, bf, 0, t0, u);
+      tma_load_3d(sbase + 24576, &tmV, bf, 64, t0, u);
+    }
+  } else if (tid == 32) {
+    // MMA issuer: D[r][c] += sum_t phi(K)[t][r] V[t][c], both MN-major SW128
+    constexpr uint32_t idesc = make_idesc_bf16(128, 128, 1, 1);
+    bool ok = true;
+    for (int i = 0; i < ntile && ok; ++i) {
+      const int st = i % kStages;
+      ok = mbar_wait(bar_relu + 8 * st, (i / kStages) & 1, a.err, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t sbase = base + st * kStageBytes;
+#pragma unroll
+      for (int ks = 0; ks < kTok / 16; ++ks) {
+        const uint64_t da = make_sdesc(sbase + ks * 2048, 8192, 1024, kLayoutSW128);
+        const uint64_t db = make_sdesc(sbase + 16384 + ks * 2048, 8192, 1024, kLayoutSW128);
+        mma_bf16_ss(tmem, da, db, idesc, (i | ks) ? 1u : 0u);
+      }
+      mma_commit(bar_empty + 8 * st);
+    }
+    if (ok) mma_commit(bar_done);
+  } else if (warp >= 4) {
+    // phi(K) in place; thread owns logical 16-byte column chunk (box, j) of
+    // rows t_sub + 8k, so it can also accumulate z for those 8 features.
+    const int w = tid - 128;
+    const int box = w >> 6, j = (w >> 3) & 7, tsub = w & 7;
+    for (int i = 0; i < ntile; ++i) {
+      const int st = i % kStages;
+      if (!mbar_wait(bar_full + 8 * st, (i / kStages) & 1, a.err, abort_flag)) break;
+      const uint32_t kt = base + st * kStageBytes + box * 8192;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int t = tsub + 8 * k;
+        const uint32_t addr = kt + t * 128 + ((j ^ (t & 7)) << 4);
+        uint4 x = ld_shared_v4(addr);
+        x.x = relu_bf16x2(x.x);
+        x.y = relu_bf16x2(x.y);
+        x.z = relu_bf16x2(x.z);
+        x.w = relu_bf16x2(x.w);
+        st_shared_v4(addr, x.x, x.y, x.z, x.w);
+        const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          zacc[2 * q] += __uint_as_float(wv[q] << 16);
+          zacc[2 * q + 1] += __uint_as_float(wv[q] & 0xFFFF0000u);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(bar_relu + 8 * st);
+    }
+  }
+
+  // ---- epilogue: accumulator -> fp32 tile -> TMA store (partial or final)
+  __syncwarp();
+  const bool ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag));
+  tc_fence_after();
+  if (ok) accum_to_tile(tmem, base, warp, lane, false);
+  fence_proxy_async_smem();
+  if (warp >= 4 && a.zdst != nullptr) {
+    // reduce the 8 row-phases that share (box, j)
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      float v = zacc[q];
+      v += __shfl_xor_sync(0xffffffffu, v, 1);
+      v += __shfl_xor_sync(0xffffffffu, v, 2);
+      v += __shfl_xor_sync(0xffffffffu, v, 4);
+      zacc[q] = v;
+    }
+    const int w = tid - 128;
+    const int box = w >> 6, j = (w >> 3) & 7, tsub = w & 7;
+    if (tsub == 0 && ok) {
+      float* zd = a.zdst + static_cast<size_t>(item) * kD + box * 64 + j * 8;
+      reinterpret_cast<float4*>(zd)[0] = make_float4(zacc[0], zacc[1], zacc[2], zacc[3]);
+      reinterpret_cast<float4*>(zd)[1] = make_float4(zacc[4], zacc[5], zacc[6], zacc[7]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && !*abort_flag) {
+#pragma unroll
+    for (int bx = 0; bx < 4; ++bx) tma_store_3d(&tmOut, base + bx * 16384, 32 * bx, 0, item);
+    bulk_commit_group();
+    bulk_wait_group_read0();
+  }
+  __syncwarp();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// S[u] = sum over chunks s (in order) of ws_S[u][s];  same for z.
+__global__ void __launch_bounds__(256) k_prefill_reduce(const float4* __restrict__ wsS,
+                                                        const float4* __restrict__ wsZ,
+                                                        float4* __restrict__ S,
+                                                        float4* __restrict__ z, int splits) {
+  const int u = blockIdx.y;
+  const int e = blockIdx.x * 256 + threadIdx.x;    // float4 index within a unit
+  constexpr int kS4 = kD * kD / 4, kZ4 = kD / 4;
+  if (e < kS4) {
+    const float4* p = wsS + static_cast<size_t>(u) * splits * kS4 + e;
+    float4 acc = p[0];
+    for (int s = 1; s < splits; ++s) {
+      const float4 v = p[static_cast<size_t>(s) * kS4];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    S[static_cast<size_t>(u) * kS4 + e] = acc;
+  }
+  if (z != nullptr && e < kZ4) {
+    const float4* p = wsZ + static_cast<size_t>(u) * splits * kZ4 + e;
+    float4 acc = p[0];
+    for (int s = 1; s < splits; ++s) {
+      const float4 v = p[static_cast<size_t>(s) * kZ4];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    z[static_cast<size_t>(u) * kZ4 + e] = acc;
+  }
+}
+
+// Chunking of a T-token prompt: chunks of at most 64 tiles (4096 tokens),
+// split further (down to 16 tiles) while there are fewer than two CTAs per
+// SM of a 148-SM part.  Depends only on (units, T), so the workspace query
+// and the launch always agree.
+void prefill_plan(int units, int T, int* splits, int* tiles_per) {
+  const int tiles = (T + kTok - 1) / kTok;
+  int s = (tiles + kMaxTilesPerChunk - 1) / kMaxTilesPerChunk;
+  if (units * s < kTargetCtas) {
+    const int want = (kTargetCtas + units - 1) / units;
+    const int cap = (tiles + kMinTilesPerChunk - 1) / kMinTilesPerChunk;
+    const int more = want < cap ? want : cap;
+    if (more > s) s = more;
+  }
+  if (s < 1) s = 1;
+  const int tp = (tiles + s - 1) / s;
+  *splits = (tiles + tp - 1) / tp;   // no empty chunk
+  *tiles_per = tp;
+}
+
+bool state_tmap(CUtensorMap* m, const float* S, uint64_t items) {
+  const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)kD, items};
+  const uint64_t strides[2] = {kD * 4ull, (uint64_t)kD * kD * 4ull};
+  const uint32_t box[3] = {32, 128, 1};
+  return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, S, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool tokens_tmap(CUtensorMap* m, const void* X, int T, int units, uint32_t box_rows) {
+  const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)T, (uint64_t)units};
+  const uint64_t strides[2] = {kD * 2ull, (uint64_t)T * kD * 2ull};
+  const uint32_t box[3] = {64, box_rows, 1};
+  return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, X, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int BPAD>
+int launch_commit_bpad(const Ctx& c, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& ts, const CommitArgs& a, int units) {
+  using Lay = CommitLayout<BPAD>;
+  auto kern = k_commit_bf16<BPAD>;
+  static std::atomic<uint64_t> prepared{0};
+  if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
+  kern<<<units, kThreads, Lay::kSmem, c.stream>>>(tk, tv, ts, a);
+  return cudaGetLastError() == cudaSuccess ? 0 : -5;
+}
+
+}  // namespace
+
+int launch_commit_bf16(const Ctx& c, const void* K, const void* V, int units, int b, float* S,
+                       float* z) {
+  const int bpad = b <= 16 ? 16 : (b <= 32 ? 32 : 64);
+  CUtensorMap tk, tv, ts;
+  if (!tokens_tmap(&tk, K, b, units, bpad) || !tokens_tmap(&tv, V, b, units, bpad) ||
+      !state_tmap(&ts, S, units))
+    return -5;
+  CommitArgs a{z, c.dev_err, b};
+  switch (bpad) {
+    case 16: return launch_commit_bpad<16>(c, tk, tv, ts, a, units);
+    case 32: return launch_commit_bpad<32>(c, tk, tv, ts, a, units);
+    default: return launch_commit_bpad<64>(c, tk, tv, ts, a, units);
+  }
+}
+
+size_t prefill_bf16_workspace(int units, int T) {
+  if (T <= 0 || units <= 0) return 0;
+  int splits, tp;
+  prefill_plan(units, T, &splits, &tp);
+  if (splits <= 1) return 0;
+  return static_cast<size_t>(units) * splits * (kD * kD + kD) * sizeof(float);
+}
+
+int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, int T, float* S,
+                        float* z, void* ws, size_t ws_bytes) {
+  if (T == 0) {
+    if (cudaMemsetAsync(S, 0, static_cast<size_t>(units) * kD * kD * 4, c.stream) != cudaSuccess)
+      return -5;
+    if (z && cudaMemsetAsync(z, 0, static_cast<size_t>(units) * kD * 4, c.stream) != cudaSuccess)
+      return -5;
+    return 0;
+  }
+  int splits, tp;
+  prefill_plan(units, T, &splits, &tp);
+  const size_t need = prefill_bf16_workspace(units, T);
+  if (need > ws_bytes) return -4;
+  float* outS = S;
+  float* outZ = z;
+  if (splits > 1) {
+    outS = static_cast<float*>(ws);
+    outZ = z ? outS + static_cast<size_t>(units) * splits * kD * kD : nullptr;
+  }
+  CUtensorMap tk, tv, to;
+  if (!tokens_tmap(&tk, K, T, units, kTok) || !tokens_tmap(&tv, V, T, units, kTok) ||
+      !state_tmap(&to, outS, static_cast<uint64_t>(units) * splits))
+    return -5;
+  PrefillArgs a{outZ, c.dev_err, T, splits, tp};
+  static std::atomic<uint64_t> prepared{0};
+  if (!prepare_kernel(k_prefill_bf16, (int)kPrefSmem, prepared)) return -5;
+  k_prefill_bf16<<<units * splits, kThreads, kPrefSmem, c.stream>>>(tk, tv, to, a);
+  if (cudaGetLastError() != cudaSuccess) return -5;
+  if (splits > 1) {
+    dim3 grid((kD * kD / 4 + 255) / 256, units);
+    k_prefill_reduce<<<grid, 256, 0, c.stream>>>(
+        reinterpret_cast<const float4*>(outS), reinterpret_cast<const float4*>(outZ),
+        reinterpret_cast<float4*>(S), reinterpret_cast<float4*>(z), splits);
+    if (cudaGetLastError() != cudaSuccess) return -5;
+  }
+  return 0;
+}
+
+}  // namespace bha

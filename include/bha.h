@@ -1,0 +1,161 @@
+/*
+ * bha.h -- C ABI of block-hybrid attention on NVIDIA B200 (sm_100a).
+ *
+ * Method: "Retrofitting Linear Attention into Diffusion Language Models"
+ * (Kim, Roh, Kim; arXiv 2608.06628).  The paper-daily summary page gives the
+ * core formula (section 核心公式与算法) and a worked example (section
+ * 具体技术细节示例); the fugumt page carries the abstract.  During blockwise
+ * semi-autoregressive decoding, attention inside the active denoising block
+ * is exact softmax, and attention over all previous blocks is linear
+ * attention through a per-KV-head prefix state:
+ *
+ *     y   = softmax(Q_a K_a^T * scale) V_a + phi(Q_a) S_p
+ *     S_p = sum over committed tokens t of phi(k_t)^T v_t      (d x d)
+ *     phi = ReLU (elementwise; the worked example's kernel feature map)
+ *
+ * Tensors and layouts (row-major, contiguous, device memory):
+ *   Q_a, Y      [n][hq][b][d]         active-block queries / outputs
+ *   K_a, V_a    [n][hkv][b][d]        active-block keys / values
+ *   K_p, V_p    [n][hkv][T][d]        prompt keys / values (prefill)
+ *   K_c, V_c    [n][hkv][cap][d]      KV cache, first P tokens valid
+ *   S           [n][hkv][d][d] fp32   S[r][c] = sum_t phi(k_t)[r] v_t[c]
+ *   z           [n][hkv][d]    fp32   z[r]    = sum_t phi(k_t)[r]
+ * GQA: query head h reads KV head h / (hq / hkv) (contiguous grouping).
+ * Element type of Q/K/V/Y: bha_dtype (bf16, or fp32 for the reference mode);
+ * S and z are always fp32, and every path accumulates in fp32.
+ *
+ * Ownership: the caller allocates and owns every buffer, the workspace and
+ * the stream.  The library allocates no memory.  It holds one 4-byte device
+ * word per GPU that records a kernel-side error (read with
+ * bha_device_error), and a per-device host cache of that word's address.
+ *
+ * Behaviour: every compute call validates its arguments before any launch,
+ * returns a negative bha_status on failure (nothing launched), otherwise
+ * enqueues its kernels on `stream` and returns BHA_OK without waiting.  A
+ * launch failure reported by the runtime returns BHA_ERR_CUDA.  Kernels wait
+ * on their own asynchronous copies with a bounded spin; if a wait runs out
+ * they record BHA_ERR_TIMEOUT in the device error word and return.
+ * Pointers must be 16-byte aligned (BHA_ERR_MISALIGNED).  Outputs must not
+ * overlap inputs (BHA_ERR_INVALID_ARG).  n = 0 is a valid empty call.
+ *
+ * Supported shapes (else BHA_ERR_UNSUPPORTED):
+ *   BHA_BF16: d == 128, 1 <= b <= 64 (tensor-core paths, sm_100a).
+ *   BHA_F32 : 1 <= d <= 128, d % 4 == 0, 1 <= b <= 64 (CUDA-core reference
+ *             mode, used for the worked example and 1e-4 checks).
+ */
+#ifndef BHA_H
+#define BHA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream; identical to cudaStream_t (NULL = legacy default stream). */
+typedef struct CUstream_st *bha_stream_t;
+
+typedef enum {
+    BHA_OK = 0,
+    BHA_ERR_INVALID_ARG = -1, /* null pointer, bad count, aliasing, hq % hkv */
+    BHA_ERR_UNSUPPORTED = -2, /* shape/dtype outside the supported sets     */
+    BHA_ERR_MISALIGNED = -3,  /* a pointer is not 16-byte aligned           */
+    BHA_ERR_WORKSPACE = -4,   /* workspace NULL or smaller than required    */
+    BHA_ERR_CUDA = -5,        /* the CUDA runtime reported an error         */
+    BHA_ERR_TIMEOUT = -6,     /* a kernel's bounded wait ran out            */
+    BHA_ERR_DEVICE = -7       /* a kernel detected an internal fault        */
+} bha_status;
+
+typedef enum { BHA_BF16 = 0, BHA_F32 = 1 } bha_dtype;
+
+/* Normalise the two terms by one shared denominator (an engineer-added
+ * option; the pages add the terms unnormalised):
+ *   y = (sum_j e^{s_j - m} v_j + e^{-m} phi(q) S) /
+ *       (sum_j e^{s_j - m}     + e^{-m} phi(q) . z),   m = max_j s_j.
+ * Requires z.  The pages have no counterpart of this option. */
+#define BHA_FLAG_SHARED_DENOM 1u
+
+/* Human-readable name of a bha_status value (never NULL). */
+const char *bha_status_string(int status);
+
+/* ABI version, currently 1. */
+int bha_version(void);
+
+/*
+ * Prefill: fold a prompt into the prefix state (the prompt counts as the
+ * "previous blocks" of the first generated block; follows from the abstract's
+ * linear attention over previous blocks and the worked example's S_1).
+ *   S = phi(K_p)^T V_p,  z = sum_t phi(k_t)        (overwrites S and z)
+ * K, V: [n][hkv][T][d]; S: [n][hkv][d][d]; z: [n][hkv][d] or NULL.
+ * T = 0 writes S = 0 (and z = 0).  The bf16 path splits T into chunks
+ * reduced in a fixed order through `workspace` (deterministic result);
+ * workspace may be NULL when bha_state_prefill_workspace_size returns 0.
+ */
+size_t bha_state_prefill_workspace_size(int n, int hkv, int T, int d,
+                                        bha_dtype dtype);
+int bha_state_prefill(const void *K, const void *V, int n, int hkv, int T,
+                      int d, bha_dtype dtype, float *S, float *z,
+                      void *workspace, size_t workspace_bytes,
+                      bha_stream_t stream);
+
+/*
+ * Commit: add a finalised block to the prefix state (worked example:
+ * S_{1,2} = phi(K_1)^T V_1 + phi(K_2)^T V_2).
+ *   S += phi(K_blk)^T V_blk,  z += sum_t phi(k_t)     (in place)
+ * Kb, Vb: [n][hkv][b][d]; S: [n][hkv][d][d]; z: [n][hkv][d] or NULL.
+ */
+int bha_state_commit(const void *Kb, const void *Vb, int n, int hkv, int b,
+                     int d, bha_dtype dtype, float *S, float *z,
+                     bha_stream_t stream);
+
+/*
+ * One denoising step of block-hybrid attention (core formula): for every
+ * query row i of the active block,
+ *   y_i = sum_j softmax_j(scale q_i . k_j) v_j  +  phi(q_i) S
+ * with j over the b block tokens (bidirectional, no mask) and S the state
+ * of all previous blocks.  scale <= 0 selects 1/sqrt(d).  flags:
+ * BHA_FLAG_SHARED_DENOM (needs z).  Y must not overlap any input.
+ */
+int bha_hybrid_step(const void *Qa, const void *Ka, const void *Va,
+                    const float *S, const float *z, void *Y, int n, int hq,
+                    int hkv, int b, int d, float scale, unsigned flags,
+                    bha_dtype dtype, bha_stream_t stream);
+
+/*
+ * Comparison path: exact softmax attention of the active block over the
+ * whole KV cache plus the block itself (the abstract's baseline, where
+ * every denoising step attends to all previous blocks):
+ *   y_i = sum_j softmax_j(scale q_i . k_j) v_j,  j in [K_c[0:P] || K_a]
+ * Kc, Vc: [n][hkv][cap][d] with P <= cap valid tokens.  The bf16 path splits
+ * the P + b keys into chunks merged by log-sum-exp through `workspace`.
+ */
+size_t bha_prefix_softmax_workspace_size(int n, int hq, int hkv, int b,
+                                         int d, int P, bha_dtype dtype);
+int bha_prefix_softmax(const void *Qa, const void *Kc, const void *Vc, int P,
+                       int cap, const void *Ka, const void *Va, void *Y,
+                       int n, int hq, int hkv, int b, int d, float scale,
+                       bha_dtype dtype, void *workspace,
+                       size_t workspace_bytes, bha_stream_t stream);
+
+/*
+ * Block partition of a length-L sequence into blocks of B tokens, the last
+ * one possibly short (worked example: L=10, B=4 -> tokens 1-4, 5-8, 9-10).
+ * Host-only.  Writes bounds[0..k] = {0, B, 2B, ..., L} and returns k, the
+ * number of blocks; returns BHA_ERR_INVALID_ARG for L < 0, B < 1 or a NULL
+ * bounds, BHA_ERR_WORKSPACE if max_bounds < k + 1.
+ */
+int bha_block_partition(int L, int B, int *bounds, int max_bounds);
+
+/*
+ * Synchronises the current device and returns the device error word
+ * (BHA_OK, BHA_ERR_TIMEOUT or BHA_ERR_DEVICE) recorded by any kernel since
+ * the last reset; reset != 0 clears it.  Returns BHA_ERR_CUDA if the device
+ * cannot be read.
+ */
+int bha_device_error(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BHA_H */

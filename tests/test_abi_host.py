@@ -1,0 +1,157 @@
+"""Host-side checks of the C ABI (no GPU needed, no kernel launched).
+
+The library must load on a machine without a GPU driver, export every
+symbol include/bha.h declares, and reject bad arguments before touching the
+device.  Fake (never dereferenced) pointers stand in for device buffers.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from block_hybrid_linear_b200 import _lib
+from block_hybrid_linear_b200 import build as bha_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bha.h")
+
+GAP = 1 << 36  # 16-byte aligned fake device addresses, 64 GiB apart
+A, B, C, D, E, F = (GAP * k for k in range(1, 7))
+
+
+@pytest.fixture(scope="module")
+def L():
+    bha_build.build()
+    return _lib.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bha_\w+)\s*\(", text)))
+
+
+def test_header_and_binding_agree():
+    assert declared_symbols() == sorted(_lib.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, name in [(0, "BHA_OK"), (-1, "BHA_ERR_INVALID_ARG"), (-2, "BHA_ERR_UNSUPPORTED"),
+                       (-3, "BHA_ERR_MISALIGNED"), (-4, "BHA_ERR_WORKSPACE"),
+                       (-5, "BHA_ERR_CUDA"), (-6, "BHA_ERR_TIMEOUT"), (-7, "BHA_ERR_DEVICE")]:
+        assert _lib.status_string(code) == name
+    assert _lib.status_string(12345) == "BHA_ERR_UNKNOWN"
+    assert _lib.bha_version() == 1
+
+
+@pytest.mark.parametrize("L_", [0, 1, 2, 3, 4, 5, 10, 31, 32, 33, 64, 1000])
+@pytest.mark.parametrize("B_", [1, 2, 3, 4, 7, 32, 64])
+def test_block_partition_bit_exact_vs_oracle(L, L_, B_):
+    assert _lib.bha_block_partition(L_, B_) == oracle.block_partition(L_, B_)
+
+
+def test_block_partition_worked_example(L):
+    # paper-daily summary, worked example: L=10, B=4 -> tokens 1-4, 5-8, 9-10
+    assert _lib.bha_block_partition(10, 4) == [0, 4, 8, 10]
+
+
+def test_block_partition_errors(L):
+    buf = (ctypes.c_int * 2)()
+    assert L.bha_block_partition(10, 0, buf, 2) == _lib.BHA_ERR_INVALID_ARG
+    assert L.bha_block_partition(-1, 4, buf, 2) == _lib.BHA_ERR_INVALID_ARG
+    assert L.bha_block_partition(10, 4, None, 4) == _lib.BHA_ERR_INVALID_ARG
+    assert L.bha_block_partition(10, 4, buf, 2) == _lib.BHA_ERR_WORKSPACE
+
+
+def step(L, Q=A, K=B, V=C, S=D, z=None, Y=E, n=2, hq=16, hkv=4, b=32, d=128, scale=0.0,
+         flags=0, dtype=_lib.BHA_BF16):
+    return L.bha_hybrid_step(Q, K, V, S, z, Y, n, hq, hkv, b, d, scale, flags, dtype, None)
+
+
+def test_step_validation(L):
+    assert step(L, Q=None) == _lib.BHA_ERR_INVALID_ARG
+    assert step(L, S=None) == _lib.BHA_ERR_INVALID_ARG
+    assert step(L, Y=None) == _lib.BHA_ERR_INVALID_ARG
+    assert step(L, hq=6, hkv=4) == _lib.BHA_ERR_INVALID_ARG          # hq % hkv
+    assert step(L, hkv=0) == _lib.BHA_ERR_INVALID_ARG
+    assert step(L, n=-1) == _lib.BHA_ERR_INVALID_ARG
+    assert step(L, b=0) == _lib.BHA_ERR_INVALID_ARG
+    assert step(L, b=65) == _lib.BHA_ERR_UNSUPPORTED
+    assert step(L, d=64) == _lib.BHA_ERR_UNSUPPORTED                 # bf16 needs d=128
+    assert step(L, d=130, dtype=_lib.BHA_F32) == _lib.BHA_ERR_UNSUPPORTED
+    assert step(L, d=18, dtype=_lib.BHA_F32) == _lib.BHA_ERR_UNSUPPORTED
+    assert step(L, dtype=7) == _lib.BHA_ERR_UNSUPPORTED
+    assert step(L, flags=2) == _lib.BHA_ERR_INVALID_ARG
+    assert step(L, flags=_lib.BHA_FLAG_SHARED_DENOM) == _lib.BHA_ERR_INVALID_ARG  # no z
+    assert step(L, Q=A + 8) == _lib.BHA_ERR_MISALIGNED
+    assert step(L, Y=E + 2) == _lib.BHA_ERR_MISALIGNED
+    assert step(L, flags=1, z=F + 4) == _lib.BHA_ERR_MISALIGNED
+    assert step(L, Y=A) == _lib.BHA_ERR_INVALID_ARG                  # Y aliases Q
+    assert step(L, Y=B + 4096) == _lib.BHA_ERR_INVALID_ARG           # Y overlaps K
+    assert step(L, n=0) == _lib.BHA_OK                               # empty: no launch
+
+
+def test_valid_call_without_device_reports_cuda_error(L):
+    # Arguments are valid, so the call reaches the runtime, which has no GPU here.
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    assert step(L) == _lib.BHA_ERR_CUDA
+
+
+def test_commit_validation(L):
+    f = lambda **kw: L.bha_state_commit(kw.get("K", A), kw.get("V", B), kw.get("n", 2), 4,
+                                        kw.get("b", 32), kw.get("d", 128),
+                                        kw.get("dtype", _lib.BHA_BF16), kw.get("S", C),
+                                        kw.get("z", None), None)
+    assert f(K=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(S=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(b=65) == _lib.BHA_ERR_UNSUPPORTED
+    assert f(d=96) == _lib.BHA_ERR_UNSUPPORTED
+    assert f(S=C + 4) == _lib.BHA_ERR_MISALIGNED
+    assert f(S=A) == _lib.BHA_ERR_INVALID_ARG     # S overlaps K
+    assert f(z=C + 64) == _lib.BHA_ERR_INVALID_ARG  # z overlaps S
+    assert f(n=0) == _lib.BHA_OK
+
+
+def test_prefill_validation_and_workspace(L):
+    need = L.bha_state_prefill_workspace_size(64, 4, 32768, 128, _lib.BHA_BF16)
+    # 256 units x 8 chunks of 4096 tokens x (128 x 128 + 128) fp32
+    assert need == 256 * 8 * (128 * 128 + 128) * 4
+    assert L.bha_state_prefill_workspace_size(64, 4, 32768, 128, _lib.BHA_F32) == 0
+    assert L.bha_state_prefill_workspace_size(64, 4, 0, 128, _lib.BHA_BF16) == 0
+    big = GAP * 16
+    f = lambda **kw: L.bha_state_prefill(kw.get("K", A), kw.get("V", big), 64, 4,
+                                         kw.get("T", 32768), 128, _lib.BHA_BF16,
+                                         kw.get("S", 2 * big), None, kw.get("ws", 3 * big),
+                                         kw.get("ws_bytes", need), None)
+    assert f(ws=None) == _lib.BHA_ERR_WORKSPACE
+    assert f(ws_bytes=need - 16) == _lib.BHA_ERR_WORKSPACE
+    assert f(T=-1) == _lib.BHA_ERR_INVALID_ARG
+    assert f(K=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(ws=3 * big + 8) == _lib.BHA_ERR_MISALIGNED
+
+
+def test_prefix_validation_and_workspace(L):
+    need = L.bha_prefix_softmax_workspace_size(64, 16, 4, 32, 128, 32768, _lib.BHA_BF16)
+    assert need > 0 and need % 16 == 0
+    assert L.bha_prefix_softmax_workspace_size(64, 16, 4, 32, 128, 32768, _lib.BHA_F32) == 0
+    big = GAP * 16
+    f = lambda **kw: L.bha_prefix_softmax(A, kw.get("Kc", big), kw.get("Vc", 2 * big),
+                                          kw.get("P", 32768), kw.get("cap", 32768), B, C,
+                                          kw.get("Y", D), 64, 16, 4, 32, 128, 0.0,
+                                          _lib.BHA_BF16, kw.get("ws", 3 * big),
+                                          kw.get("ws_bytes", need), None)
+    assert f(cap=100) == _lib.BHA_ERR_INVALID_ARG    # P > cap
+    assert f(P=-1) == _lib.BHA_ERR_INVALID_ARG
+    assert f(Kc=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(ws=None) == _lib.BHA_ERR_WORKSPACE
+    assert f(Y=A) == _lib.BHA_ERR_INVALID_ARG        # Y aliases Q
+    assert f(Y=big + 64) == _lib.BHA_ERR_INVALID_ARG  # Y inside the cache
