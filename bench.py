@@ -45,12 +45,16 @@ WORKLOAD = ("long-prefix: batch 64, 16q/4kv heads, d=128, active block B=32, pre
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--no-compare", action="store_true", help="skip the exact-path comparison")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--only", choices=["step", "commit", "prefill", "prefix"],
+                    help="launch just this kernel warmup + steps times (small case for ncu)")
+    ap.add_argument("--prefix", type=int, default=8192,
+                    help="prompt / cache length used by --only prefill|prefix")
     return ap.parse_args()
 
 
@@ -140,43 +144,64 @@ class ClockSampler:
 
 def run_reference(args, rank, world):
     """The CPU oracle as the reference arm: the same metric on bounded samples
-    of the same workload, on the host cores."""
+    of the same workload, on the host cores.  A step's sample shrinks (whole
+    requests -> query heads x denoising steps) so that K + W steps stay
+    within about two minutes."""
     if rank != 0:
         return
-    import numpy as np
     import oracle
     from block_hybrid_linear_b200 import inputs
     cores = len(os.sched_getaffinity(0))
     oracle.set_threads(cores)
     std = 1.0 / math.sqrt(D_)
-    # a sample = a few (request, KV head) units through one block cycle
-    u_max = 64
-    Qb, Qv = inputs.normal_bf16_np(4000, inputs.TID_Q, (u_max // HKV, HQ, B_, D_), std)
-    Kb, Kv = inputs.normal_bf16_np(4000, inputs.TID_K, (u_max // HKV, HKV, B_, D_), std)
-    Vb, Vv = inputs.normal_bf16_np(4000, inputs.TID_V, (u_max // HKV, HKV, B_, D_), std)
-    Sv, zv = inputs.synthetic_state_np(4000, u_max // HKV, HKV, D_, P_, std)
+    nmax = 16
+    _, Qv = inputs.normal_bf16_np(4000, inputs.TID_Q, (nmax, HQ, B_, D_), std)
+    _, Kv = inputs.normal_bf16_np(4000, inputs.TID_K, (nmax, HKV, B_, D_), std)
+    _, Vv = inputs.normal_bf16_np(4000, inputs.TID_V, (nmax, HKV, B_, D_), std)
+    Sv, zv = inputs.synthetic_state_np(4000, nmax, HKV, D_, P_, std)
+    G = HQ // HKV
 
-    def cycle(nreq):
-        S, z = Sv[:nreq], zv[:nreq]
+    def full_cycle(nreq):
         for _ in range(DENOISE):
-            oracle.hybrid_step(Qv[:nreq], Kv[:nreq], Vv[:nreq], S, z)
-        oracle.state_commit(S, z, Kv[:nreq], Vv[:nreq])
+            oracle.hybrid_step(Qv[:nreq], Kv[:nreq], Vv[:nreq], Sv[:nreq], zv[:nreq])
+        oracle.state_commit(Sv[:nreq], zv[:nreq], Kv[:nreq], Vv[:nreq])
 
+    def head_steps(hs, ns):
+        # hs query heads of request 0 (sharing KV head 0 while hs <= G), ns steps
+        hkv = 1 if hs <= G else hs // G
+        for _ in range(ns):
+            oracle.hybrid_step(Qv[:1, :hs], Kv[:1, :hkv], Vv[:1, :hkv], Sv[:1, :hkv],
+                               zv[:1, :hkv])
+
+    budget = min(1.0, 120.0 / max(1, args.steps + args.warmup))
     t0 = time.perf_counter()
-    cycle(1)
-    t1 = time.perf_counter() - t0
-    budget = 90.0 / max(1, args.steps + args.warmup)
-    nreq = int(max(1, min(u_max // HKV, budget / max(t1, 1e-6))))
+    full_cycle(1)
+    t_req = time.perf_counter() - t0
+    if t_req <= budget:
+        nreq = int(min(nmax, max(1, budget // max(t_req, 1e-9))))
+        work = lambda: full_cycle(nreq)
+        tokens_per_step = nreq * B_ * DENOISE
+        sample = ("%d of 64 requests (16 query / 4 KV heads each) through one block cycle "
+                  "per step: 8 oracle hybrid steps + 1 oracle commit, fp64" % nreq)
+    else:
+        t0 = time.perf_counter()
+        head_steps(1, 1)
+        t_hs = max(time.perf_counter() - t0, 1e-9)
+        k = int(max(1, min(HQ * DENOISE, budget // t_hs)))
+        ns = min(DENOISE, k)
+        hs = max(1, min(G, k // ns))
+        work = lambda: head_steps(hs, ns)
+        tokens_per_step = hs / HQ * B_ * ns
+        sample = ("%d of 16 query heads of one request x %d of 8 denoising steps per step "
+                  "(oracle hybrid step, fp64; counted as %.3g active tokens)"
+                  % (hs, ns, tokens_per_step))
     for _ in range(args.warmup):
-        cycle(nreq)
+        work()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        cycle(nreq)
+        work()
     dt = time.perf_counter() - t0
-    tokens = nreq * B_ * DENOISE * args.steps
-    value = tokens / dt
-    sample = ("%d of 64 requests (all 4 KV heads each) through one block cycle per step: "
-              "8 oracle hybrid steps + 1 oracle commit, fp64" % nreq)
+    value = tokens_per_step * args.steps / dt
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
@@ -316,6 +341,7 @@ def run_native(args, rank, world, local):
     reps = max(1, math.ceil(args.steps / g_cycles))
     steps = reps * g_cycles
     warm = max(1, math.ceil(args.warmup / g_cycles))
+    torch.cuda.set_stream(stream)   # graph replays launch on the current stream
     for _ in range(warm):
         graph.replay()
     torch.cuda.synchronize()
@@ -488,9 +514,57 @@ def run_native(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def run_only(args):
+    """One kernel on the long-prefix shapes (prompt / cache length --prefix),
+    warmup + steps plain launches, for profiler captures."""
+    import torch
+    import block_hybrid_linear_b200 as bha
+    from block_hybrid_linear_b200 import build, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    std = 1.0 / math.sqrt(D_)
+    P = args.prefix
+    Q = inputs.normal_bf16_torch(1, inputs.TID_Q, (N_, HQ, B_, D_), std, dev)
+    K = inputs.normal_bf16_torch(1, inputs.TID_K, (N_, HKV, B_, D_), std, dev)
+    V = inputs.normal_bf16_torch(1, inputs.TID_V, (N_, HKV, B_, D_), std, dev)
+    Y = torch.empty_like(Q)
+    S = torch.randn(N_, HKV, D_, D_, device=dev)
+    z = torch.rand(N_, HKV, D_, device=dev)
+    if args.only in ("prefill", "prefix"):
+        Kp = inputs.normal_bf16_torch(1, inputs.TID_KP, (N_, HKV, P, D_), std, dev)
+        Vp = inputs.normal_bf16_torch(1, inputs.TID_VP, (N_, HKV, P, D_), std, dev)
+    if args.only == "prefill":
+        need = bha.bha_state_prefill_workspace_size(N_, HKV, P, D_)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        fn = lambda: bha.bha_state_prefill(Kp, Vp, S, z, workspace=ws)
+    elif args.only == "prefix":
+        need = bha.bha_prefix_softmax_workspace_size(N_, HQ, HKV, B_, D_, P)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        fn = lambda: bha.bha_prefix_softmax(Q, Kp, Vp, P, K, V, Y, workspace=ws)
+    elif args.only == "commit":
+        fn = lambda: bha.bha_state_commit(K, V, S, z)
+    else:
+        fn = lambda: bha.bha_hybrid_step(Q, K, V, S, Y, z=z)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    assert bha.bha_device_error(True) == 0
+    print(json.dumps({"only": args.only, "prefix": P, "launches": args.steps,
+                      "avg_ms": e0.elapsed_time(e1) / max(1, args.steps)}), flush=True)
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
+    if args.only:
+        run_only(args)
+        return
     if args.impl == "reference":
         run_reference(args, rank, world)
         return

@@ -7,6 +7,8 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <utility>
+
 namespace bha {
 
 struct Ctx {
@@ -35,6 +37,26 @@ bool prepare_kernel(Kernel kern, int smem_bytes, std::atomic<uint64_t>& done) {
   cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   done.fetch_or(bit, std::memory_order_release);
   return true;
+}
+
+// Launches `kern` with programmatic stream serialization: the kernel may be
+// scheduled while the previous kernel of the stream finishes; it must call
+// pdl_wait() before its first global-memory access.  Returns 0 or -5.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t smem,
+               cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...) != cudaSuccess) return -5;
+  return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
 
 // ---- fp32 reference mode (CUDA cores) ----

@@ -57,20 +57,6 @@ struct PrefixArgs {
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};\n\t"
-      "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
-      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]),
-      "f"(v[8]), "f"(v[9]), "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]),
-      "f"(v[15]), "f"(v[16]), "f"(v[17]), "f"(v[18]), "f"(v[19]), "f"(v[20]), "f"(v[21]),
-      "f"(v[22]), "f"(v[23]), "f"(v[24]), "f"(v[25]), "f"(v[26]), "f"(v[27]), "f"(v[28]),
-      "f"(v[29]), "f"(v[30]), "f"(v[31])
-      : "memory");
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
     k_prefix_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                   const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKa,
@@ -114,11 +100,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(smem_u32(tmem_slot), 512);
     tmem_relinquish();
   }
+  if (tid == 0) pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t t_o = tmem + 256;
+  pdl_wait();
 
   if (tid == 0) {
     // ---------------- TMA producer
@@ -242,7 +230,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld32_sync(t_o + lane_base + c, o);
 #pragma unroll
             for (int q = 0; q < 32; ++q) o[q] *= corr;
-            tmem_st32(t_o + lane_base + c, o);
+            tmem_st32_sync(t_o + lane_base + c, o);
           }
         }
       }
@@ -323,6 +311,8 @@ __global__ void __launch_bounds__(256) k_prefix_merge(const float* __restrict__ 
                                                       const float* __restrict__ wsML,
                                                       __nv_bfloat16* __restrict__ Y, int rows,
                                                       int mtiles, int splits) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int umt = blockIdx.y;
   const int u = umt / mtiles, mt = umt % mtiles;
   const int e = blockIdx.x * 256 + threadIdx.x;      // float4 index in the 128 x 128 tile
@@ -433,13 +423,23 @@ int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* 
   a.sl2 = scale * 1.4426950408889634f;
   static std::atomic<uint64_t> prepared{0};
   if (!prepare_kernel(k_prefix_bf16, (int)kSmem, prepared)) return -5;
-  k_prefix_bf16<<<(unsigned)items, kThreads, kSmem, c.stream>>>(tq, tkc, tvc, tka, tva, ty, to,
-                                                                 a);
-  if (cudaGetLastError() != cudaSuccess) return -5;
+  if (launch_pdl(k_prefix_bf16, (unsigned)items, kThreads, kSmem, c.stream, tq, tkc, tvc, tka,
+                 tva, ty, to, a))
+    return -5;
   if (splits > 1) {
-    dim3 grid(kD * kD / 4 / 256, units * mtiles);
-    k_prefix_merge<<<grid, 256, 0, c.stream>>>(wsO, wsML, static_cast<__nv_bfloat16*>(Y), rows,
-                                               mtiles, splits);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kD * kD / 4 / 256, units * mtiles);
+    cfg.blockDim = dim3(256);
+    cfg.stream = c.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_prefix_merge, static_cast<const float*>(wsO),
+                           static_cast<const float*>(wsML), static_cast<__nv_bfloat16*>(Y), rows,
+                           mtiles, splits) != cudaSuccess)
+      return -5;
     if (cudaGetLastError() != cudaSuccess) return -5;
   }
   return 0;

@@ -11,7 +11,9 @@
 //
 // Commit: one CTA per (request, KV head): one MMA chain over the b block
 // tokens, then S is read-modified-written through a swizzled fp32 tile
-// (thread = row r, conflict-free) and stored back by TMA.
+// (thread = row r, conflict-free) and stored back by TMA, one 64-column half
+// at a time.  Its operands are prefetched into L2 before the kernel waits
+// for the previous one.
 //
 // Prefill: one CTA per (unit, chunk of the prompt), a 3-stage TMA ring of
 // 64-token K/V tiles (32 KB per stage) feeding the MMA warp; the chunk's
@@ -103,15 +105,24 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_init(bar_done, 1);
       *abort_flag = 0;
       fence_mbar_init();
+      // warm L2 with this unit's operands while the previous kernel finishes
+      tma_prefetch_l2_3d(&tmK, 0, 0, u);
+      tma_prefetch_l2_3d(&tmK, 64, 0, u);
+      tma_prefetch_l2_3d(&tmV, 0, 0, u);
+      tma_prefetch_l2_3d(&tmV, 64, 0, u);
+#pragma unroll
+      for (int bx = 0; bx < 4; ++bx) tma_prefetch_l2_3d(&tmS, 32 * bx, 0, u);
     }
     __syncwarp();
     tmem_alloc(smem_u32(tmem_slot), 128);
     tmem_relinquish();
   }
+  if (tid == 0) pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
 
   if (tid == 0) {
     mbar_arrive_expect_tx(bar_kv, 2 * Lay::kKV);
@@ -140,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
 
   if (tid == 32 && !*abort_flag) {
+    // D[r][c] = sum_t phi(K)[t][r] V[t][c]: both operands MN-major SW128
     tc_fence_after();
     constexpr uint32_t idesc = make_idesc_bf16(128, 128, 1, 1);
 #pragma unroll
@@ -170,14 +182,16 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (ok) accum_to_tile(tmem, base + Lay::kOffS, warp, lane, true);
   fence_proxy_async_smem();
   tc_fence_before();
-  __syncthreads();
-  if (tid == 0 && !*abort_flag) {
-#pragma unroll
-    for (int bx = 0; bx < 4; ++bx) tma_store_3d(&tmS, base + Lay::kOffS + bx * 16384, 32 * bx, 0, u);
+  // each 64-column half is stored as soon as its four warps are done
+  const int hb = warp >> 2;
+  named_barrier_sync(1 + hb, 128);
+  if ((tid & 127) == 0 && !*abort_flag) {
+    tma_store_3d(&tmS, base + Lay::kOffS + (2 * hb) * 16384, 64 * hb, 0, u);
+    tma_store_3d(&tmS, base + Lay::kOffS + (2 * hb + 1) * 16384, 64 * hb + 32, 0, u);
     bulk_commit_group();
     bulk_wait_group_read0();
   }
-  __syncwarp();
+  __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 128);
@@ -238,10 +252,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_alloc(smem_u32(tmem_slot), 128);
     tmem_relinquish();
   }
+  if (tid == 0) pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();
 
   float zacc[8];
 #pragma unroll
@@ -357,6 +373,8 @@ __global__ void __launch_bounds__(256) k_prefill_reduce(const float4* __restrict
                                                         const float4* __restrict__ wsZ,
                                                         float4* __restrict__ S,
                                                         float4* __restrict__ z, int splits) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int u = blockIdx.y;
   const int e = blockIdx.x * 256 + threadIdx.x;    // float4 index within a unit
   constexpr int kS4 = kD * kD / 4, kZ4 = kD / 4;
@@ -428,8 +446,7 @@ int launch_commit_bpad(const Ctx& c, const CUtensorMap& tk, const CUtensorMap& t
   auto kern = k_commit_bf16<BPAD>;
   static std::atomic<uint64_t> prepared{0};
   if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
-  kern<<<units, kThreads, Lay::kSmem, c.stream>>>(tk, tv, ts, a);
-  return cudaGetLastError() == cudaSuccess ? 0 : -5;
+  return launch_pdl(kern, units, kThreads, Lay::kSmem, c.stream, tk, tv, ts, a);
 }
 
 }  // namespace
@@ -483,13 +500,22 @@ int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, i
   PrefillArgs a{outZ, c.dev_err, T, splits, tp};
   static std::atomic<uint64_t> prepared{0};
   if (!prepare_kernel(k_prefill_bf16, (int)kPrefSmem, prepared)) return -5;
-  k_prefill_bf16<<<units * splits, kThreads, kPrefSmem, c.stream>>>(tk, tv, to, a);
-  if (cudaGetLastError() != cudaSuccess) return -5;
+  if (launch_pdl(k_prefill_bf16, units * splits, kThreads, kPrefSmem, c.stream, tk, tv, to, a))
+    return -5;
   if (splits > 1) {
-    dim3 grid((kD * kD / 4 + 255) / 256, units);
-    k_prefill_reduce<<<grid, 256, 0, c.stream>>>(
-        reinterpret_cast<const float4*>(outS), reinterpret_cast<const float4*>(outZ),
-        reinterpret_cast<float4*>(S), reinterpret_cast<float4*>(z), splits);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((kD * kD / 4 + 255) / 256, units);
+    cfg.blockDim = dim3(256);
+    cfg.stream = c.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, k_prefill_reduce, reinterpret_cast<const float4*>(outS),
+                           reinterpret_cast<const float4*>(outZ), reinterpret_cast<float4*>(S),
+                           reinterpret_cast<float4*>(z), splits) != cudaSuccess)
+      return -5;
     if (cudaGetLastError() != cudaSuccess) return -5;
   }
   return 0;

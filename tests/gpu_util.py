@@ -65,15 +65,15 @@ class Guarded:
         numel = int(np.prod(shape))
         self.buf = torch.empty(numel + 2 * self.CANARY, dtype=dtype, device="cuda")
         self.buf.fill_(float("nan"))
-        self.buf[: self.CANARY].fill_(-12345.0)
-        self.buf[-self.CANARY:].fill_(-12345.0)
+        self.buf[: self.CANARY].fill_(-4096.0)
+        self.buf[-self.CANARY:].fill_(-4096.0)
         self.t = self.buf[self.CANARY: self.CANARY + numel].view(*shape)
 
     def intact(self):
         import torch
         lo = self.buf[: self.CANARY].float()
         hi = self.buf[-self.CANARY:].float()
-        return bool(torch.all(lo == -12345.0)) and bool(torch.all(hi == -12345.0))
+        return bool(torch.all(lo == -4096.0)) and bool(torch.all(hi == -4096.0))
 
     def no_nan(self):
         import torch
