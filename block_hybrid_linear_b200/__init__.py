@@ -13,5 +13,6 @@ from ._lib import (  # noqa: F401
     BHA_F32, BHA_FLAG_SHARED_DENOM, BHA_OK, BhaError, EXPORTED, LIB_PATH,
     bha_block_partition, bha_device_error, bha_hybrid_step, bha_prefix_softmax,
     bha_prefix_softmax_workspace_size, bha_state_commit, bha_state_prefill,
-    bha_state_prefill_workspace_size, bha_version, lib, status_string,
+    bha_state_prefill_noalloc, bha_state_prefill_workspace_size, bha_version, lib,
+    status_string,
 )

@@ -28,7 +28,7 @@ BHA_FLAG_SHARED_DENOM = 1
 # every symbol include/bha.h declares
 EXPORTED = [
     "bha_status_string", "bha_version", "bha_state_prefill_workspace_size",
-    "bha_state_prefill", "bha_state_commit", "bha_hybrid_step",
+    "bha_state_prefill", "bha_state_prefill_noalloc", "bha_state_commit", "bha_hybrid_step",
     "bha_prefix_softmax_workspace_size", "bha_prefix_softmax",
     "bha_block_partition", "bha_device_error",
 ]
@@ -61,6 +61,8 @@ def lib():
         L.bha_state_prefill_workspace_size.restype = sz
         L.bha_state_prefill.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp, sz, vp]
         L.bha_state_prefill.restype = i
+        L.bha_state_prefill_noalloc.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp]
+        L.bha_state_prefill_noalloc.restype = i
         L.bha_state_commit.argtypes = [vp, vp, i, i, i, i, i, vp, vp, vp]
         L.bha_state_commit.restype = i
         L.bha_hybrid_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, fl, u,
@@ -139,6 +141,15 @@ def bha_state_prefill(K, V, S, z=None, workspace=None, stream=None):
     _check(lib().bha_state_prefill(_ptr(K), _ptr(V), n, hkv, T, d, _dtype(K), _ptr(S),
                                    _ptr(z), _ptr(workspace), ws_bytes, _stream(stream)),
            "bha_state_prefill")
+
+
+def bha_state_prefill_noalloc(K, V, S, z=None, stream=None):
+    """bha_state_prefill with the library's fixed 32 MiB device scratch in
+    place of a caller workspace (for callers that cannot allocate)."""
+    n, hkv, T, d = K.shape
+    _check(lib().bha_state_prefill_noalloc(_ptr(K), _ptr(V), n, hkv, T, d, _dtype(K), _ptr(S),
+                                           _ptr(z), _stream(stream)),
+           "bha_state_prefill_noalloc")
 
 
 def bha_state_commit(Kb, Vb, S, z=None, stream=None):

@@ -27,7 +27,8 @@
  * Ownership: the caller allocates and owns every buffer, the workspace and
  * the stream.  The library allocates no memory.  It holds one 4-byte device
  * word per GPU that records a kernel-side error (read with
- * bha_device_error), and a per-device host cache of that word's address.
+ * bha_device_error), and a per-device host cache of that word's address;
+ * bha_state_prefill_noalloc also keeps a fixed 32 MiB device array per GPU.
  *
  * Behaviour: every compute call validates its arguments before any launch,
  * returns a negative bha_status on failure (nothing launched), otherwise
@@ -97,6 +98,24 @@ int bha_state_prefill(const void *K, const void *V, int n, int hkv, int T,
                       int d, bha_dtype dtype, float *S, float *z,
                       void *workspace, size_t workspace_bytes,
                       bha_stream_t stream);
+
+/*
+ * Allocation-free variant of bha_state_prefill (the paper has no counterpart:
+ * this is an interface for callers that cannot allocate device memory, such
+ * as plugins inside a host application that owns all device memory or
+ * runtimes that forbid allocation once serving has started).  Same
+ * arguments and result as bha_state_prefill without the workspace: the
+ * chunk partials go to a 32 MiB array held in the library's device memory
+ * on every GPU that uses it, until the process exits.  Returns
+ * BHA_ERR_WORKSPACE, launching nothing, when bha_state_prefill_workspace_size
+ * exceeds 32 MiB.  The array's device address is looked up on the first
+ * call made on each device (make that call before any stream capture).  All
+ * calls on a device share the array: calls whose kernels overlap on the GPU
+ * race on it.  It holds nothing that must start at zero.
+ */
+int bha_state_prefill_noalloc(const void *K, const void *V, int n, int hkv,
+                              int T, int d, bha_dtype dtype, float *S,
+                              float *z, bha_stream_t stream);
 
 /*
  * Commit: add a finalised block to the prefix state (worked example:
