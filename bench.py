@@ -140,6 +140,22 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def max_over_ranks(value, dist, device):
+    """Largest `value` across the process group (the job's time is the
+    slowest rank's); `dist` is torch.distributed or None for one process."""
+    if dist is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, time_ms):
+    """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
+    return tokens_per_rank * world / (time_ms / 1e3)
+
+
 # ---------------------------------------------------------------- reference
 
 def run_reference(args, rank, world):
@@ -375,12 +391,8 @@ def run_native(args, rank, world, local):
     step_launch_ms = ks0.elapsed_time(ks1) / (max(1, reps // 4) * 4 * R)
     commit_launch_ms = kc0.elapsed_time(kc1) / (max(1, reps // 4) * 2 * R)
     assert bha.bha_device_error(True) == 0
-    if pg is not None:
-        t = torch.tensor([t_ms], device=dev)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        t_ms = float(t.item())
-    tokens = world * steps * N_ * B_ * DENOISE
-    value = tokens / (t_ms / 1e3)
+    t_ms = max_over_ranks(t_ms, pg, dev)
+    value = job_throughput(steps * N_ * B_ * DENOISE, world, t_ms)
 
     peak, peak_kind = measured_peaks()
     step_bytes = N_ * HKV * UNIT_BYTES_STEP
@@ -494,13 +506,10 @@ def run_native(args, rank, world, local):
         stream.synchronize()
         wall = time.perf_counter() - t0
         e2e_ms = max(ev0.elapsed_time(ev1), wall * 1e3)
-        if pg is not None:
-            t = torch.tensor([e2e_ms], device=dev)
-            pg.all_reduce(t, op=pg.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(e2e_ms, pg, dev)
         h2d = DENOISE * (hQ.numel() + hK.numel() + hV.numel()) * 2
         d2h = DENOISE * hY.numel() * 2
-        line["e2e"] = {"value": world * n_e2e * N_ * B_ * DENOISE / (e2e_ms / 1e3),
+        line["e2e"] = {"value": job_throughput(n_e2e * N_ * B_ * DENOISE, world, e2e_ms),
                        "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h}
         line["gpu_launches_e2e"] = n_e2e * (DENOISE + 1)

@@ -30,7 +30,7 @@ EXPORTED = [
     "bha_status_string", "bha_version", "bha_state_prefill_workspace_size",
     "bha_state_prefill", "bha_state_prefill_noalloc", "bha_state_commit", "bha_hybrid_step",
     "bha_prefix_softmax_workspace_size", "bha_prefix_softmax",
-    "bha_block_partition", "bha_device_error",
+    "bha_block_partition", "bha_device_error", "bha_selftest_timeout",
 ]
 
 _lib = None
@@ -77,6 +77,8 @@ def lib():
         L.bha_block_partition.restype = i
         L.bha_device_error.argtypes = [i]
         L.bha_device_error.restype = i
+        L.bha_selftest_timeout.argtypes = [vp]
+        L.bha_selftest_timeout.restype = i
         _lib = L
     return _lib
 
@@ -128,6 +130,11 @@ def bha_block_partition(L, B):
 def bha_device_error(reset=True):
     """Synchronise and return the kernels' device error word (0 = none)."""
     return lib().bha_device_error(1 if reset else 0)
+
+
+def bha_selftest_timeout(stream=None):
+    """Launch the timeout self-test kernel (records BHA_ERR_TIMEOUT)."""
+    _check(lib().bha_selftest_timeout(_stream(stream)), "bha_selftest_timeout")
 
 
 def bha_state_prefill_workspace_size(n, hkv, T, d, dtype=BHA_BF16):

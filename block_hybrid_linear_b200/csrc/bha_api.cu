@@ -12,6 +12,7 @@
 
 #include "../../include/bha.h"
 #include "bha_internal.h"
+#include "bha_ptx.cuh"
 
 namespace bha {
 
@@ -103,6 +104,22 @@ int launch_status(int rc) {
   return BHA_ERR_CUDA;
 }
 
+// Waits on an mbarrier that nothing ever arrives at, with a short limit, to
+// exercise the kernels' timeout path: the wait gives up, records
+// BHA_ERR_TIMEOUT in the device error word and the kernel returns normally.
+__global__ void k_selftest_timeout(int* err, unsigned limit_us) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    mbar_wait(smem_u32(&bar), 0, err, &abort_flag, static_cast<uint64_t>(limit_us) * 1000ull);
+}
+
 }  // namespace
 
 bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* gaddr,
@@ -180,6 +197,13 @@ int bha_device_error(int reset) {
       return BHA_ERR_CUDA;
   }
   return v;
+}
+
+int bha_selftest_timeout(bha_stream_t stream) {
+  DeviceInfo* d = nullptr;
+  if (device_info(&d) != BHA_OK) return BHA_ERR_CUDA;
+  k_selftest_timeout<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(d->dev_err, 10000u);
+  return cudaGetLastError() == cudaSuccess ? BHA_OK : BHA_ERR_CUDA;
 }
 
 size_t bha_state_prefill_workspace_size(int n, int hkv, int T, int d, bha_dtype dtype) {

@@ -173,6 +173,15 @@ int bha_block_partition(int L, int B, int *bounds, int max_bounds);
  */
 int bha_device_error(int reset);
 
+/*
+ * Self-test of the timeout path (diagnostics; the pages have no counterpart):
+ * launches one small kernel that waits on a barrier nothing will complete,
+ * with a 10 ms limit instead of the kernels' 1 s.  The wait gives up, the
+ * kernel records BHA_ERR_TIMEOUT in the device error word and exits normally,
+ * so the context stays usable.  Returns BHA_OK once launched.
+ */
+int bha_selftest_timeout(bha_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif
