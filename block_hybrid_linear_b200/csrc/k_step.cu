@@ -71,6 +71,29 @@ struct StepLayout {
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
+// phi(q_r) * scale as fp32 into TMEM (this thread's lane, columns [0, 128)
+// from `tcol`), read from row r of the SW128 Q tile; one wait for all four
+// 32-column stores.
+__device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol, float scale) {
+#pragma unroll
+  for (int cg = 0; cg < 4; ++cg) {
+    float f[32];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int j = (cg & 1) * 4 + q;
+      const uint4 v = ld_shared_v4(qtile + (cg >> 1) * 16384 + r * 128 + ((j ^ (r & 7)) << 4));
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        f[8 * q + 2 * e] = fmaxf(__uint_as_float(w4[e] << 16), 0.f) * scale;
+        f[8 * q + 2 * e + 1] = fmaxf(__uint_as_float(w4[e] & 0xFFFF0000u), 0.f) * scale;
+      }
+    }
+    tmem_st32(tcol + cg * 32, f);
+  }
+  tmem_wait_st();
+}
+
 template <int BPAD, bool SHARED>
 __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     k_step_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -126,7 +149,12 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t t_d = tmem;           // [0, 128): the output accumulator
-  const uint32_t t_a = tmem + 128;     // [128, 256): scores, then phi(Q) as tf32
+  const uint32_t t_a = tmem + 128;     // [128, 256): phi(Q) as tf32 (the MMA's A)
+  // Scores: in the default mode they sit in the accumulator's first columns
+  // (P V overwrites them once read) so phi(Q) can be built in parallel; with
+  // the shared denominator phi(Q) needs the row max first, so the scores sit
+  // where phi(Q) will go.
+  const uint32_t t_sc = SHARED ? t_a : t_d;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   pdl_wait();   // inputs may come from the previous kernel of the stream
 
@@ -153,6 +181,14 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   }
 
   float beta = 1.f;   // per-row output scale (shared denominator only)
+  if (!SHARED && warp < 4) {
+    // phi(q) for row r = 32 w + lane into TMEM as soon as Q has landed, in
+    // parallel with the score MMA and the softmax
+    const bool okq = warp_all(mbar_wait(bar_q, 0, a.err, abort_flag));
+    if (okq) write_phiq(base + kOffQ, warp * 32 + lane, t_a + lane_base, 1.f);
+    tc_fence_before();
+    mbar_arrive(bar_a);
+  }
   if (warp >= 4) {
     // ---- row owners: thread = query row r of the tile = TMEM lane r
     const int r = (warp - 4) * 32 + lane;
@@ -166,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
                                          1024, kLayoutSW128);
           const uint64_t db = make_sdesc(base + kOffK + (ks >> 2) * (BPAD * 128) + (ks & 3) * 32,
                                          16, 1024, kLayoutSW128);
-          mma_bf16_ss(t_a, da, db, idesc, ks > 0 ? 1u : 0u);
+          mma_bf16_ss(t_sc, da, db, idesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(bar_sc);
       }
@@ -179,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
 #pragma unroll
       for (int j = 0; j < BPAD; j += 16) {
         float t[16];
-        tmem_ld16_sync(t_a + lane_base + j, t);
+        tmem_ld16_sync(t_sc + lane_base + j, t);
 #pragma unroll
         for (int q = 0; q < 16; ++q) sc[j + q] = t[q];
       }
@@ -247,29 +283,12 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     tc_fence_before();
     mbar_arrive(bar_p);
 
-    // phi(q) (times the row's scale) as fp32 into TMEM lane r, columns
-    // [128, 256), over the scores already read
-    if (ok) {
-#pragma unroll 1
-      for (int cg = 0; cg < 4; ++cg) {
-        float f[32];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int j = (cg & 1) * 4 + q;
-          const uint4 v = ld_shared_v4(base + kOffQ + (cg >> 1) * 16384 + r * 128 +
-                                       ((j ^ (r & 7)) << 4));
-          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            f[8 * q + 2 * e] = fmaxf(__uint_as_float(w4[e] << 16), 0.f) * ascale;
-            f[8 * q + 2 * e + 1] = fmaxf(__uint_as_float(w4[e] & 0xFFFF0000u), 0.f) * ascale;
-          }
-        }
-        tmem_st32_sync(t_a + lane_base + cg * 32, f);
-      }
+    if (SHARED) {
+      // phi(q) times the row's scale, over the scores already read
+      if (ok) write_phiq(base + kOffQ, r, t_a + lane_base, ascale);
+      tc_fence_before();
+      mbar_arrive(bar_a);
     }
-    tc_fence_before();
-    mbar_arrive(bar_a);
 
     if (tid == 128) {
       // MMA issuer for P V and the per-chunk phi(Q) S products
@@ -341,13 +360,14 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   if ((tid & 127) == 0 && !*abort_flag) {
     tma_store_3d(&tmY, base + kOffQ + hb * 16384, 64 * hb, mt * kMT, u);
     bulk_commit_group();
-    bulk_wait_group_read0();
   }
+  // every TMEM read is done once both halves passed their barrier
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
+  if ((tid & 127) == 0) bulk_wait_group_read0();   // shared memory stays until read
 }
 
 template <int BPAD, bool SHARED>
