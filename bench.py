@@ -55,6 +55,10 @@ def parse():
                     help="launch just this kernel warmup + steps times (small case for ncu)")
     ap.add_argument("--prefix", type=int, default=8192,
                     help="prompt / cache length used by --only prefill|prefix")
+    ap.add_argument("--workload", default="long-prefix",
+                    choices=["long-prefix", "single-step", "generation-loop", "stack"],
+                    help="long-prefix is the benchmark line; the others are the secondary "
+                         "workloads (one JSON line each)")
     return ap.parse_args()
 
 
@@ -568,11 +572,246 @@ def run_only(args):
                       "avg_ms": e0.elapsed_time(e1) / max(1, args.steps)}), flush=True)
 
 
+def _graph(fn, stream):
+    import torch
+    with torch.cuda.stream(stream):
+        fn()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def _time_graph(g, stream, reps):
+    import torch
+    torch.cuda.set_stream(stream)
+    g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps
+
+
+def run_single_step(args):
+    """Batch 8, 16q/4kv, B=32, prefix 4096 in the state: one denoising step
+    (launch-latency bound at this size), beside the exact path."""
+    import torch
+    import block_hybrid_linear_b200 as bha
+    from block_hybrid_linear_b200 import build, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    n, P = 8, 4096
+    std = 1.0 / math.sqrt(D_)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    Kp = inputs.normal_bf16_torch(2000, inputs.TID_KP, (n, HKV, P + B_, D_), std, dev)
+    Vp = inputs.normal_bf16_torch(2000, inputs.TID_VP, (n, HKV, P + B_, D_), std, dev)
+    S0 = torch.empty(n, HKV, D_, D_, device=dev)
+    z0 = torch.empty(n, HKV, D_, device=dev)
+    need = bha.bha_state_prefill_workspace_size(n, HKV, P, D_)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    bha.bha_state_prefill(Kp[:, :, :P].contiguous(), Vp[:, :, :P].contiguous(), S0, z0,
+                          workspace=ws)
+    R = max(4, math.ceil(4 * l2 / (n * HKV * UNIT_BYTES_STEP)))
+    sets = [dict(Q=inputs.normal_bf16_torch(r, inputs.TID_Q, (n, HQ, B_, D_), std, dev),
+                 K=inputs.normal_bf16_torch(r, inputs.TID_K, (n, HKV, B_, D_), std, dev),
+                 V=inputs.normal_bf16_torch(r, inputs.TID_V, (n, HKV, B_, D_), std, dev),
+                 S=S0.clone(), Y=torch.empty(n, HQ, B_, D_, dtype=torch.bfloat16, device=dev))
+            for r in range(R)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def steps():
+        for st in sets:
+            bha.bha_hybrid_step(st["Q"], st["K"], st["V"], st["S"], st["Y"], stream=stream)
+    g = _graph(steps, stream)
+    step_us = _time_graph(g, stream, 50) * 1e3 / R
+    needp = bha.bha_prefix_softmax_workspace_size(n, HQ, HKV, B_, D_, P)
+    wsp = torch.empty(max(needp, 16), dtype=torch.uint8, device=dev)
+    st = sets[0]
+
+    def exact():
+        bha.bha_prefix_softmax(st["Q"], Kp, Vp, P, st["K"], st["V"], st["Y"], workspace=wsp,
+                               stream=stream)
+    gx = _graph(exact, stream)
+    exact_us = _time_graph(gx, stream, 50) * 1e3
+    bytes_step = n * HKV * UNIT_BYTES_STEP
+    peak, _ = measured_peaks()
+    print(json.dumps({
+        "workload": "single-step: batch 8, 16q/4kv, d=128, B=32, prefix 4096 in the state",
+        "metric": METRIC, "unit": "tokens/s",
+        "hybrid_step": {"launch_us": step_us, "tokens_per_s": n * B_ / (step_us / 1e6),
+                        "achieved_gbs": bytes_step / (step_us / 1e6) / 1e9,
+                        "frac_of_peak": bytes_step / (step_us / 1e6) / 1e9 / peak,
+                        "algorithmic_bytes": bytes_step},
+        "prefix_softmax": {"launch_us": exact_us, "tokens_per_s": n * B_ / (exact_us / 1e6)},
+        "note": "4.7 MB per step: bound by launch latency, not by HBM"}), flush=True)
+
+
+def run_generation_loop(args):
+    """Batch 32, prompt 1024 -> state, 32 blocks x 8 denoising steps (one
+    commit per block), against exact attention over the growing KV cache
+    (appending each finished block).  Whole loops replayed as CUDA graphs."""
+    import torch
+    import block_hybrid_linear_b200 as bha
+    from block_hybrid_linear_b200 import build, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    n, T, nblk, nst = 32, 1024, 32, DENOISE
+    std = 1.0 / math.sqrt(D_)
+    cap = T + nblk * B_
+    Kc = inputs.normal_bf16_torch(3000, inputs.TID_KP, (n, HKV, cap, D_), std, dev)
+    Vc = inputs.normal_bf16_torch(3000, inputs.TID_VP, (n, HKV, cap, D_), std, dev)
+    Kp, Vp = Kc[:, :, :T].contiguous(), Vc[:, :, :T].contiguous()
+    Qs = inputs.normal_bf16_torch(3000, inputs.TID_Q, (nblk, nst, n, HQ, B_, D_), std, dev)
+    Ks = inputs.normal_bf16_torch(3000, inputs.TID_K, (nblk, nst, n, HKV, B_, D_), std, dev)
+    Vs = inputs.normal_bf16_torch(3000, inputs.TID_V, (nblk, nst, n, HKV, B_, D_), std, dev)
+    S = torch.empty(n, HKV, D_, D_, device=dev)
+    z = torch.empty(n, HKV, D_, device=dev)
+    Y = torch.empty(n, HQ, B_, D_, dtype=torch.bfloat16, device=dev)
+    need = bha.bha_state_prefill_workspace_size(n, HKV, T, D_)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    needp = max(bha.bha_prefix_softmax_workspace_size(n, HQ, HKV, B_, D_, T + blk * B_)
+                for blk in range(nblk))
+    wsp = torch.empty(max(needp, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def hybrid_loop():
+        bha.bha_state_prefill(Kp, Vp, S, z, workspace=ws, stream=stream)
+        for blk in range(nblk):
+            for st in range(nst):
+                bha.bha_hybrid_step(Qs[blk, st], Ks[blk, st], Vs[blk, st], S, Y, z=z,
+                                    stream=stream)
+            bha.bha_state_commit(Ks[blk, nst - 1], Vs[blk, nst - 1], S, z, stream=stream)
+
+    def exact_loop():
+        for blk in range(nblk):
+            P = T + blk * B_
+            for st in range(nst):
+                bha.bha_prefix_softmax(Qs[blk, st], Kc, Vc, P, Ks[blk, st], Vs[blk, st], Y,
+                                       workspace=wsp, stream=stream)
+            with torch.cuda.stream(stream):   # append the finished block to the cache
+                Kc[:, :, P:P + B_].copy_(Ks[blk, nst - 1])
+                Vc[:, :, P:P + B_].copy_(Vs[blk, nst - 1])
+
+    gh = _graph(hybrid_loop, stream)
+    gx = _graph(exact_loop, stream)
+    h_ms = _time_graph(gh, stream, 5)
+    x_ms = _time_graph(gx, stream, 5)
+    tokens = n * B_ * nblk * nst
+    print(json.dumps({
+        "workload": "generation-loop: batch 32, 16q/4kv, d=128, prompt 1024 prefilled, "
+                    "32 blocks x 8 denoising steps, B=32",
+        "metric": METRIC, "unit": "tokens/s",
+        "hybrid": {"loop_ms": h_ms, "tokens_per_s": tokens / (h_ms / 1e3),
+                   "launches": 2 + nblk * (nst + 1)},
+        "exact_prefix_softmax": {"loop_ms": x_ms, "tokens_per_s": tokens / (x_ms / 1e3)},
+        "speedup": x_ms / h_ms}), flush=True)
+
+
+def run_stack(args):
+    """20-layer attention stack (6 hybrid + 14 exact layers), prefix 8192:
+    one denoising step through the stack per batch size, the all-exact stack
+    beside it, device bytes per request, and the largest batch whose state
+    fits (searched by allocation, out-of-memory caught)."""
+    import torch
+    import block_hybrid_linear_b200 as bha
+    from block_hybrid_linear_b200 import build, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    P, layers, hyb = 8192, 20, 6
+    std = 1.0 / math.sqrt(D_)
+    kv_req = HKV * P * D_ * 2 * 2             # one exact layer, per request
+    st_req = HKV * (D_ * D_ + D_) * 4         # one hybrid layer, per request
+    hybrid_req = hyb * st_req + (layers - hyb) * kv_req
+    exact_req = layers * kv_req
+    stream = torch.cuda.Stream(device=dev)
+    rows = []
+    batches = [1, 2, 4, 8, 16, 32, 64, 128, 256]
+    nmax = batches[-1]
+    # one KV cache per exact layer and one state per hybrid layer, allocated
+    # once at the largest batch (distinct memory per layer); smaller batches
+    # use the leading requests
+    caches = [(inputs.normal_bf16_torch(5000 + l, inputs.TID_KC, (nmax, HKV, P, D_), std, dev),
+               inputs.normal_bf16_torch(5000 + l, inputs.TID_VC, (nmax, HKV, P, D_), std, dev))
+              for l in range(layers)]
+    states = [torch.randn(nmax, HKV, D_, D_, device=dev) for _ in range(hyb)]
+    Qa = inputs.normal_bf16_torch(5000, inputs.TID_Q, (nmax, HQ, B_, D_), std, dev)
+    Ka = inputs.normal_bf16_torch(5000, inputs.TID_K, (nmax, HKV, B_, D_), std, dev)
+    Va = inputs.normal_bf16_torch(5000, inputs.TID_V, (nmax, HKV, B_, D_), std, dev)
+    Ya = torch.empty_like(Qa)
+    for n in batches:
+        Q, K, V, Y = Qa[:n], Ka[:n], Va[:n], Ya[:n]
+        needp = bha.bha_prefix_softmax_workspace_size(n, HQ, HKV, B_, D_, P)
+        wsp = torch.empty(max(needp, 16), dtype=torch.uint8, device=dev)
+
+        def hybrid_stack():
+            for l in range(layers):
+                if l < hyb:
+                    bha.bha_hybrid_step(Q, K, V, states[l][:n], Y, stream=stream)
+                else:
+                    bha.bha_prefix_softmax(Q, caches[l][0][:n], caches[l][1][:n], P, K, V, Y,
+                                           workspace=wsp, stream=stream)
+
+        def exact_stack():
+            for l in range(layers):
+                bha.bha_prefix_softmax(Q, caches[l][0][:n], caches[l][1][:n], P, K, V, Y,
+                                       workspace=wsp, stream=stream)
+        gh, gx = _graph(hybrid_stack, stream), _graph(exact_stack, stream)
+        th = _time_graph(gh, stream, 10)
+        tx = _time_graph(gx, stream, 10)
+        rows.append({"batch": n, "hybrid_ms": th, "hybrid_tokens_per_s": n * B_ / (th / 1e3),
+                     "exact_ms": tx, "exact_tokens_per_s": n * B_ / (tx / 1e3),
+                     "speedup": tx / th})
+        del gh, gx, wsp
+    del caches, states, Qa, Ka, Va, Ya
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
+    def fits(per_req, n):
+        try:
+            buf = torch.empty(int(per_req) * n, dtype=torch.uint8, device=dev)
+            del buf
+            return True
+        except torch.OutOfMemoryError:
+            return False
+        finally:
+            torch.cuda.empty_cache()
+
+    def max_batch(per_req):
+        lo, hi = 0, 1
+        while hi <= 4096 and fits(per_req, hi):   # doubling until allocation fails
+            lo, hi = hi, hi * 2
+        while hi - lo > 1:                        # then bisect
+            mid = (lo + hi) // 2
+            lo, hi = (mid, hi) if fits(per_req, mid) else (lo, mid)
+        return lo
+    free, total = torch.cuda.mem_get_info(dev)
+    print(json.dumps({
+        "workload": "stack: 20 attention layers (6 hybrid + 14 exact), 16q/4kv, d=128, B=32, "
+                    "prefix 8192; one denoising step through the stack",
+        "metric": METRIC, "unit": "tokens/s", "sweep": rows,
+        "bytes_per_request": {"hybrid_layer_state": st_req, "exact_layer_kv": kv_req,
+                              "hybrid_stack": hybrid_req, "all_exact_stack": exact_req},
+        "max_batch_before_oom": {"hybrid_stack": max_batch(hybrid_req),
+                                 "all_exact_stack": max_batch(exact_req),
+                                 "device_free_bytes": free, "device_total_bytes": total}}),
+          flush=True)
+
+
 def main():
     args = parse()
     rank, world, local = dist_env()
     if args.only:
         run_only(args)
+        return
+    if args.workload != "long-prefix":
+        if rank == 0:
+            {"single-step": run_single_step, "generation-loop": run_generation_loop,
+             "stack": run_stack}[args.workload](args)
         return
     if args.impl == "reference":
         run_reference(args, rank, world)
