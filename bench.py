@@ -38,8 +38,10 @@ N_, HQ, HKV, B_, D_, P_ = 64, 16, 4, 32, 128, 32768
 DENOISE = 8
 UNIT_BYTES_STEP = (HQ // HKV) * B_ * D_ * 2 * 2 + 2 * B_ * D_ * 2 + D_ * D_ * 4  # Q+Y, K+V, S
 UNIT_BYTES_COMMIT = 2 * B_ * D_ * 2 + 2 * D_ * D_ * 4                           # K+V, S r+w
+UNIT_BYTES_FUSED = UNIT_BYTES_STEP + D_ * D_ * 4                                # + S write
 WORKLOAD = ("long-prefix: batch 64, 16q/4kv heads, d=128, active block B=32, prefix 32768 "
-            "in fp32 state; step = 8 hybrid denoising steps + 1 block commit")
+            "in fp32 state; step = one block: 8 hybrid denoising steps, the last fused with "
+            "the block commit")
 
 
 def parse():
@@ -51,7 +53,7 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--no-compare", action="store_true", help="skip the exact-path comparison")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["step", "commit", "prefill", "prefix"],
+    ap.add_argument("--only", choices=["step", "step_commit", "commit", "prefill", "prefix"],
                     help="launch just this kernel warmup + steps times (small case for ncu)")
     ap.add_argument("--prefix", type=int, default=8192,
                     help="prompt / cache length used by --only prefill|prefix")
@@ -325,13 +327,15 @@ def run_native(args, rank, world, local):
     stream = torch.cuda.Stream(device=dev)
 
     def cycle(c):
-        # one block: 8 denoising steps on 8 different sets, commit on the last
-        for s in range(DENOISE):
-            st = sets[(c * (DENOISE + 1) + s) % R]
+        # one block: 8 denoising steps on 8 different sets; the last one also
+        # commits the block (the fused step + commit kernel)
+        for s in range(DENOISE - 1):
+            st = sets[(c * DENOISE + s) % R]
             bha.bha_hybrid_step(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"],
                                 stream=stream)
-        st = sets[(c * (DENOISE + 1) + DENOISE) % R]
-        bha.bha_state_commit(st["K"], st["V"], st["S"], st["z"], stream=stream)
+        st = sets[(c * DENOISE + DENOISE - 1) % R]
+        bha.bha_hybrid_step_commit(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"],
+                                   stream=stream)
 
     # graph of R cycles: every set is touched in each role, rotation period R
     torch.cuda.synchronize()
@@ -355,7 +359,8 @@ def run_native(args, rank, world, local):
     with torch.cuda.graph(g_commit, stream=stream):
         for k in range(2 * R):
             st = sets[k % R]
-            bha.bha_state_commit(st["K"], st["V"], st["S"], st["z"], stream=stream)
+            bha.bha_hybrid_step_commit(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"],
+                                       stream=stream)
     torch.cuda.synchronize()
 
     reps = max(1, math.ceil(args.steps / g_cycles))
@@ -401,7 +406,7 @@ def run_native(args, rank, world, local):
     peak, peak_kind = measured_peaks()
     step_bytes = N_ * HKV * UNIT_BYTES_STEP
     achieved = step_bytes / (step_launch_ms / 1e3) / 1e9
-    commit_bytes = N_ * HKV * UNIT_BYTES_COMMIT
+    fused_bytes = N_ * HKV * UNIT_BYTES_FUSED
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": steps, "warmup": warm * g_cycles, "ms_per_step": t_ms / steps,
@@ -419,12 +424,14 @@ def run_native(args, rank, world, local):
                      "algorithmic_bytes_per_launch": step_bytes,
                      "launch_us": step_launch_ms * 1e3},
         "hbm_roofline_frac": achieved / peak,
-        "commit": {"launch_us": commit_launch_ms * 1e3,
-                   "achieved_gbs": commit_bytes / (commit_launch_ms / 1e3) / 1e9,
-                   "algorithmic_bytes_per_launch": commit_bytes},
+        "step_commit": {"kernel": "k_step_bf16 (fused commit)",
+                        "launch_us": commit_launch_ms * 1e3,
+                        "achieved_gbs": fused_bytes / (commit_launch_ms / 1e3) / 1e9,
+                        "frac_of_peak": fused_bytes / (commit_launch_ms / 1e3) / 1e9 / peak,
+                        "algorithmic_bytes_per_launch": fused_bytes},
         "prefill": {"ms": prefill_ms, "tokens": N_ * P_,
                     "achieved_gbs": prefill_bytes / (prefill_ms / 1e3) / 1e9},
-        "gpu_launches": steps * (DENOISE + 1),
+        "gpu_launches": steps * DENOISE,
         "clocks": clk,
     }
 
@@ -490,13 +497,13 @@ def run_native(args, rank, world, local):
 
         def e2e_cycle():
             with torch.cuda.stream(stream):
-                for _ in range(DENOISE):
+                for s in range(DENOISE):
                     dQ.copy_(hQ, non_blocking=True)
                     dK.copy_(hK, non_blocking=True)
                     dV.copy_(hV, non_blocking=True)
-                    bha.bha_hybrid_step(dQ, dK, dV, st["S"], dY, z=st["z"], stream=stream)
+                    call = bha.bha_hybrid_step_commit if s == DENOISE - 1 else bha.bha_hybrid_step
+                    call(dQ, dK, dV, st["S"], dY, z=st["z"], stream=stream)
                     hY.copy_(dY, non_blocking=True)
-                bha.bha_state_commit(dK, dV, st["S"], st["z"], stream=stream)
 
         for _ in range(3):
             e2e_cycle()
@@ -516,7 +523,7 @@ def run_native(args, rank, world, local):
         line["e2e"] = {"value": job_throughput(n_e2e * N_ * B_ * DENOISE, world, e2e_ms),
                        "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h}
-        line["gpu_launches_e2e"] = n_e2e * (DENOISE + 1)
+        line["gpu_launches_e2e"] = n_e2e * DENOISE
 
     if rank == 0 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline_native()
@@ -556,6 +563,8 @@ def run_only(args):
         fn = lambda: bha.bha_prefix_softmax(Q, Kp, Vp, P, K, V, Y, workspace=ws)
     elif args.only == "commit":
         fn = lambda: bha.bha_state_commit(K, V, S, z)
+    elif args.only == "step_commit":
+        fn = lambda: bha.bha_hybrid_step_commit(Q, K, V, S, Y, z=z)
     else:
         fn = lambda: bha.bha_hybrid_step(Q, K, V, S, Y, z=z)
     for _ in range(args.warmup):
@@ -682,10 +691,11 @@ def run_generation_loop(args):
     def hybrid_loop():
         bha.bha_state_prefill(Kp, Vp, S, z, workspace=ws, stream=stream)
         for blk in range(nblk):
-            for st in range(nst):
+            for st in range(nst - 1):
                 bha.bha_hybrid_step(Qs[blk, st], Ks[blk, st], Vs[blk, st], S, Y, z=z,
                                     stream=stream)
-            bha.bha_state_commit(Ks[blk, nst - 1], Vs[blk, nst - 1], S, z, stream=stream)
+            bha.bha_hybrid_step_commit(Qs[blk, nst - 1], Ks[blk, nst - 1], Vs[blk, nst - 1], S,
+                                       Y, z=z, stream=stream)
 
     def exact_loop():
         for blk in range(nblk):
@@ -707,7 +717,7 @@ def run_generation_loop(args):
                     "32 blocks x 8 denoising steps, B=32",
         "metric": METRIC, "unit": "tokens/s",
         "hybrid": {"loop_ms": h_ms, "tokens_per_s": tokens / (h_ms / 1e3),
-                   "launches": 2 + nblk * (nst + 1)},
+                   "launches": 2 + nblk * nst},
         "exact_prefix_softmax": {"loop_ms": x_ms, "tokens_per_s": tokens / (x_ms / 1e3)},
         "speedup": x_ms / h_ms}), flush=True)
 

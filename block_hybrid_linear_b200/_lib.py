@@ -29,6 +29,7 @@ BHA_FLAG_SHARED_DENOM = 1
 EXPORTED = [
     "bha_status_string", "bha_version", "bha_state_prefill_workspace_size",
     "bha_state_prefill", "bha_state_prefill_noalloc", "bha_state_commit", "bha_hybrid_step",
+    "bha_hybrid_step_commit",
     "bha_prefix_softmax_workspace_size", "bha_prefix_softmax",
     "bha_block_partition", "bha_device_error", "bha_selftest_timeout",
 ]
@@ -68,6 +69,9 @@ def lib():
         L.bha_hybrid_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, fl, u,
                                       i, vp]
         L.bha_hybrid_step.restype = i
+        L.bha_hybrid_step_commit.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, fl, u,
+                                             i, vp]
+        L.bha_hybrid_step_commit.restype = i
         L.bha_prefix_softmax_workspace_size.argtypes = [i, i, i, i, i, i, i]
         L.bha_prefix_softmax_workspace_size.restype = sz
         L.bha_prefix_softmax.argtypes = [vp, vp, vp, i, i, vp, vp, vp, i, i, i, i,
@@ -175,6 +179,15 @@ def bha_hybrid_step(Q, K, V, S, Y, z=None, scale=0.0, flags=0, stream=None):
     _check(lib().bha_hybrid_step(_ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(z), _ptr(Y), n,
                                  hq, hkv, b, d, float(scale), int(flags), _dtype(Q),
                                  _stream(stream)), "bha_hybrid_step")
+
+
+def bha_hybrid_step_commit(Q, K, V, S, Y, z=None, scale=0.0, flags=0, stream=None):
+    """bha_hybrid_step, then S += phi(K)^T V and z += sum phi(k) (in place)."""
+    n, hq, b, d = Q.shape
+    hkv = K.shape[1]
+    _check(lib().bha_hybrid_step_commit(_ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(z), _ptr(Y),
+                                        n, hq, hkv, b, d, float(scale), int(flags), _dtype(Q),
+                                        _stream(stream)), "bha_hybrid_step_commit")
 
 
 def bha_prefix_softmax_workspace_size(n, hq, hkv, b, d, P, dtype=BHA_BF16):

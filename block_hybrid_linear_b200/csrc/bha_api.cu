@@ -307,6 +307,56 @@ int bha_hybrid_step(const void* Qa, const void* Ka, const void* Va, const float*
       launch_step_bf16(c, Qa, Ka, Va, S, shared ? z : nullptr, Y, n, hq, hkv, b, sc, shared));
 }
 
+int bha_hybrid_step_commit(const void* Qa, const void* Ka, const void* Va, float* S, float* z,
+                           void* Y, int n, int hq, int hkv, int b, int d, float scale,
+                           unsigned flags, bha_dtype dtype, bha_stream_t stream) {
+  int st = check_dims(dtype, d, b);
+  if (st != BHA_OK) return st;
+  if (n < 0 || hq < 1 || hkv < 1 || hq % hkv != 0) return BHA_ERR_INVALID_ARG;
+  if ((flags & ~BHA_FLAG_SHARED_DENOM) != 0) return BHA_ERR_INVALID_ARG;
+  const int shared = (flags & BHA_FLAG_SHARED_DENOM) ? 1 : 0;
+  if (n == 0) return BHA_OK;
+  if (Qa == nullptr || Ka == nullptr || Va == nullptr || S == nullptr || Y == nullptr)
+    return BHA_ERR_INVALID_ARG;
+  if (shared && z == nullptr) return BHA_ERR_INVALID_ARG;
+  if (misaligned(Qa) || misaligned(Ka) || misaligned(Va) || misaligned(S) || misaligned(z) ||
+      misaligned(Y))
+    return BHA_ERR_MISALIGNED;
+  const size_t es = esize(dtype);
+  const size_t q_bytes = static_cast<size_t>(n) * hq * b * d * es;
+  const size_t kv_bytes = static_cast<size_t>(n) * hkv * b * d * es;
+  const size_t s_bytes = static_cast<size_t>(n) * hkv * d * d * 4;
+  const size_t z_bytes = static_cast<size_t>(n) * hkv * d * 4;
+  if (overlap(Y, q_bytes, Qa, q_bytes) || overlap(Y, q_bytes, Ka, kv_bytes) ||
+      overlap(Y, q_bytes, Va, kv_bytes) || overlap(Y, q_bytes, S, s_bytes) ||
+      overlap(Y, q_bytes, z, z_bytes) || overlap(S, s_bytes, Qa, q_bytes) ||
+      overlap(S, s_bytes, Ka, kv_bytes) || overlap(S, s_bytes, Va, kv_bytes) ||
+      overlap(z, z_bytes, Qa, q_bytes) || overlap(z, z_bytes, Ka, kv_bytes) ||
+      overlap(z, z_bytes, Va, kv_bytes) || overlap(z, z_bytes, S, s_bytes))
+    return BHA_ERR_INVALID_ARG;
+  Ctx c;
+  st = make_ctx(stream, dtype, &c);
+  if (st != BHA_OK) return st;
+  const float sc = resolve_scale(scale, d);
+  const int units = n * hkv;
+  if (dtype == BHA_F32) {
+    st = launch_status(launch_step_f32(
+        c, static_cast<const float*>(Qa), static_cast<const float*>(Ka),
+        static_cast<const float*>(Va), S, shared ? z : nullptr, static_cast<float*>(Y), n, hq,
+        hkv, b, d, sc, shared));
+    if (st != BHA_OK) return st;
+    return launch_status(launch_commit_f32(c, static_cast<const float*>(Ka),
+                                           static_cast<const float*>(Va), units, b, d, S, z));
+  }
+  if (!shared && (hq / hkv) * b <= 128)   // one kernel: step, then fold the block in
+    return launch_status(
+        launch_step_bf16(c, Qa, Ka, Va, S, nullptr, Y, n, hq, hkv, b, sc, 0, z, 1));
+  st = launch_status(
+      launch_step_bf16(c, Qa, Ka, Va, S, shared ? z : nullptr, Y, n, hq, hkv, b, sc, shared));
+  if (st != BHA_OK) return st;
+  return launch_status(launch_commit_bf16(c, Ka, Va, units, b, S, z));
+}
+
 size_t bha_prefix_softmax_workspace_size(int n, int hq, int hkv, int b, int d, int P,
                                          bha_dtype dtype) {
   if (dtype != BHA_BF16 || n <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0 || b < 1 || b > 64 ||

@@ -72,9 +72,11 @@ int launch_prefix_f32(const Ctx& c, const float* Q, const float* Kc, const float
                       int b, int d, float scale);
 
 // ---- bf16 tensor-core path (tcgen05, d = 128) ----
+// commit != 0 (default mode, G * b <= 128 only): also S += phi(K)^T V and
+// z += sum phi(k) (z = commit_z, may be null) after the step has used S.
 int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, const float* S,
                      const float* z, void* Y, int n, int hq, int hkv, int b, float scale,
-                     int shared);
+                     int shared, float* commit_z = nullptr, int commit = 0);
 int launch_commit_bf16(const Ctx& c, const void* K, const void* V, int units, int b, float* S,
                        float* z);
 size_t prefill_bf16_workspace(int units, int T);

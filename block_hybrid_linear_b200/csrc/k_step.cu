@@ -50,6 +50,7 @@ constexpr uint32_t kCtrlBytes = 128;
 
 struct StepArgs {
   const float* z;     // [units][128] (shared mode)
+  float* zc;          // [units][128] updated by the fused commit, or null
   int* err;           // device error word
   int rows;           // G * b query rows per unit
   int b;              // active block length
@@ -94,12 +95,22 @@ __device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol,
   tmem_wait_st();
 }
 
-template <int BPAD, bool SHARED>
+// COMMIT: also fold this step's block into the state after using it (the
+// block's last denoising step): S += phi(K)^T V, z += sum_t phi(k_t), with
+// the state tile already in shared memory updated in place and stored back.
+// P then lives in the consumed Q tile so that K survives for the commit MMA,
+// and phi(K)^T V accumulates in the TMEM columns phi(Q) used.  Default mode
+// and a single 128-row tile per unit only.
+template <int BPAD, bool SHARED, bool COMMIT>
 __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     k_step_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
                 const __grid_constant__ CUtensorMap tmY, const StepArgs a) {
+  static_assert(!(SHARED && COMMIT), "the fused commit runs in the default mode only");
   using Lay = StepLayout<BPAD>;
+  // P (the softmax weights, bf16, K-major) goes over the consumed K tile, or
+  // over the consumed Q tile when K is still needed by the commit
+  constexpr uint32_t kOffP = COMMIT ? kOffQ : kOffK;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -110,7 +121,8 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + Lay::kTiles;
   uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
   const uint32_t bar_q = ctrl, bar_k = ctrl + 8, bar_v = ctrl + 16, bar_s = ctrl + 24,
-                 bar_sc = ctrl + 56, bar_p = ctrl + 64, bar_a = ctrl + 72, bar_done = ctrl + 80;
+                 bar_sc = ctrl + 56, bar_p = ctrl + 64, bar_a = ctrl + 72, bar_done = ctrl + 80,
+                 bar_phik = ctrl + 96, bar_ds = ctrl + 104;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 88);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 92);
 
@@ -124,6 +136,10 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       mbar_init(bar_p, 128);
       mbar_init(bar_a, 128);
       mbar_init(bar_done, 1);
+      if (COMMIT) {
+        mbar_init(bar_phik, 128);
+        mbar_init(bar_ds, 1);
+      }
       *abort_flag = 0;
       fence_mbar_init();
       tma_prefetch_desc(&tmY);
@@ -188,6 +204,34 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     if (okq) write_phiq(base + kOffQ, warp * 32 + lane, t_a + lane_base, 1.f);
     tc_fence_before();
     mbar_arrive(bar_a);
+    if (COMMIT) {
+      // phi(K) in place once the score MMA has read K, and this block's
+      // column sums of phi(K) for z (thread = feature r)
+      const bool okk = warp_all(mbar_wait(bar_sc, 0, a.err, abort_flag));
+      if (okk) {
+        for (uint32_t v = tid; v < Lay::kKV / 16; v += 128) {
+          const uint32_t addr = base + kOffK + v * 16;
+          const uint4 x = ld_shared_v4(addr);
+          st_shared_v4(addr, relu_bf16x2(x.x), relu_bf16x2(x.y), relu_bf16x2(x.z),
+                       relu_bf16x2(x.w));
+        }
+      }
+      fence_proxy_async_smem();
+      named_barrier_sync(4, 128);   // the whole phi(K) tile is written
+      mbar_arrive(bar_phik);
+      if (okk && a.zc != nullptr) {
+        const int rr = tid;
+        const uint32_t col = base + kOffK + (rr >> 6) * (BPAD * 128) + (rr & 7) * 2;
+        float zs = 0.f;
+        for (int t = 0; t < a.b; ++t) {
+          unsigned short hv;
+          const uint32_t addr = col + t * 128 + ((((rr & 63) >> 3) ^ (t & 7)) << 4);
+          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(hv) : "r"(addr));
+          zs += __uint_as_float(static_cast<uint32_t>(hv) << 16);
+        }
+        a.zc[static_cast<size_t>(u) * kD + rr] += zs;
+      }
+    }
   }
   if (warp >= 4) {
     // ---- row owners: thread = query row r of the tile = TMEM lane r
@@ -266,8 +310,10 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       } else {
         pscale = 1.f / l;   // default: P is normalised, the terms add as they are
       }
-      // P row r -> K region (K-major, swizzle width = row bytes)
-      const uint32_t prow = base + kOffK + (r >> 3) * (8 * Lay::kRowB) + (r & 7) * Lay::kRowB;
+      // P row r (K-major, swizzle width = row bytes); over the Q tile only
+      // once phi(Q) has been read out of it
+      if (COMMIT) mbar_wait(bar_a, 0, a.err, abort_flag);
+      const uint32_t prow = base + kOffP + (r >> 3) * (8 * Lay::kRowB) + (r & 7) * Lay::kRowB;
       const uint32_t swz = Lay::kRowB == 128 ? (r & 7) : Lay::kRowB == 64 ? ((r & 7) >> 1)
                                                                           : ((r & 7) >> 2);
 #pragma unroll
@@ -298,7 +344,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         constexpr uint32_t idesc = make_idesc_bf16(128, 128, 0, 1);
 #pragma unroll
         for (int ks = 0; ks < BPAD / 16; ++ks) {
-          const uint64_t da = make_sdesc(base + kOffK + ks * 32, 16, 8 * Lay::kRowB, Lay::kPLayout);
+          const uint64_t da = make_sdesc(base + kOffP + ks * 32, 16, 8 * Lay::kRowB, Lay::kPLayout);
           const uint64_t db =
               make_sdesc(base + Lay::kOffV + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
           mma_bf16_ss(t_d, da, db, idesc, ks > 0 ? 1u : 0u);
@@ -320,6 +366,23 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         }
       }
       if (ok2) mma_commit(bar_done);
+      if (COMMIT && ok2) {
+        // phi(K)^T V over the block's tokens into the columns phi(Q) used,
+        // once the products that read them are complete
+        ok2 = mbar_wait(bar_done, 0, a.err, abort_flag) && mbar_wait(bar_phik, 0, a.err, abort_flag);
+        if (ok2) {
+          tc_fence_after();
+          constexpr uint32_t idesc = make_idesc_bf16(128, 128, 1, 1);
+#pragma unroll
+          for (int ks = 0; ks < BPAD / 16; ++ks) {
+            const uint64_t da = make_sdesc(base + kOffK + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
+            const uint64_t db =
+                make_sdesc(base + Lay::kOffV + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
+            mma_bf16_ss(t_a, da, db, idesc, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_ds);
+        }
+      }
     }
   }
 
@@ -361,6 +424,46 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     tma_store_3d(&tmY, base + kOffQ + hb * 16384, 64 * hb, mt * kMT, u);
     bulk_commit_group();
   }
+  if (COMMIT) {
+    // S += phi(K)^T V in the shared state tile (32-byte-chunk swizzle:
+    // chunk j of row rr of a 32 x 32 box sits at j ^ (rr % 4)), then store
+    const bool okc = warp_all(mbar_wait(bar_ds, 0, a.err, abort_flag));
+    tc_fence_after();
+    if (okc) {
+      const int rr = r & 31;
+      const uint32_t rowb = base + kOffS + (r >> 5) * 16384 + rr * 128;
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        float dsv[32];
+        tmem_ld32_sync(t_a + lane_base + hb * 64 + cc * 32, dsv);
+        const uint32_t box = rowb + (2 * hb + cc) * 4096;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t addr = box + ((j ^ (rr & 3)) << 5);
+          float4 s0 = ld_shared_f4(addr), s1 = ld_shared_f4(addr + 16);
+          s0.x += dsv[8 * j + 0];
+          s0.y += dsv[8 * j + 1];
+          s0.z += dsv[8 * j + 2];
+          s0.w += dsv[8 * j + 3];
+          s1.x += dsv[8 * j + 4];
+          s1.y += dsv[8 * j + 5];
+          s1.z += dsv[8 * j + 6];
+          s1.w += dsv[8 * j + 7];
+          st_shared_f4(addr, s0);
+          st_shared_f4(addr + 16, s1);
+        }
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && okc && !*abort_flag) {
+      for (int c = 0; c < 4; ++c)
+        for (int nb = 0; nb < 4; ++nb)
+          tma_store_3d(&tmS, base + kOffS + c * 16384 + nb * 4096, 32 * nb, 32 * c, u);
+      bulk_commit_group();
+    }
+  }
   // every TMEM read is done once both halves passed their barrier
   __syncthreads();
   if (warp == 0) {
@@ -370,11 +473,11 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   if ((tid & 127) == 0) bulk_wait_group_read0();   // shared memory stays until read
 }
 
-template <int BPAD, bool SHARED>
+template <int BPAD, bool SHARED, bool COMMIT>
 int launch_cfg(const Ctx& c, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                const CUtensorMap& ts, const CUtensorMap& ty, const StepArgs& a, int grid) {
   using Lay = StepLayout<BPAD>;
-  auto kern = k_step_bf16<BPAD, SHARED>;
+  auto kern = k_step_bf16<BPAD, SHARED, COMMIT>;
   static std::atomic<uint64_t> prepared{0};
   if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
   return launch_pdl(kern, grid, kThreads, Lay::kSmem, c.stream, tq, tk, tv, ts, ty, a);
@@ -383,16 +486,17 @@ int launch_cfg(const Ctx& c, const CUtensorMap& tq, const CUtensorMap& tk, const
 template <int BPAD>
 int launch_bpad(const Ctx& c, const CUtensorMap& tq, const CUtensorMap& tk,
                 const CUtensorMap& tv, const CUtensorMap& ts, const CUtensorMap& ty,
-                const StepArgs& a, int grid, int shared) {
-  return shared ? launch_cfg<BPAD, true>(c, tq, tk, tv, ts, ty, a, grid)
-                : launch_cfg<BPAD, false>(c, tq, tk, tv, ts, ty, a, grid);
+                const StepArgs& a, int grid, int shared, int commit) {
+  if (commit) return launch_cfg<BPAD, false, true>(c, tq, tk, tv, ts, ty, a, grid);
+  return shared ? launch_cfg<BPAD, true, false>(c, tq, tk, tv, ts, ty, a, grid)
+                : launch_cfg<BPAD, false, false>(c, tq, tk, tv, ts, ty, a, grid);
 }
 
 }  // namespace
 
 int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, const float* S,
                      const float* z, void* Y, int n, int hq, int hkv, int b, float scale,
-                     int shared) {
+                     int shared, float* commit_z, int commit) {
   const int G = hq / hkv;
   const int rows = G * b;
   const int units = n * hkv;
@@ -423,6 +527,7 @@ int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, 
 
   StepArgs a;
   a.z = z;
+  a.zc = commit ? commit_z : nullptr;
   a.err = c.dev_err;
   a.rows = rows;
   a.b = b;
@@ -431,9 +536,9 @@ int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, 
   a.scale_log2 = scale * 1.4426950408889634f;
   const int grid = units * mtiles;
   switch (bpad) {
-    case 16: return launch_bpad<16>(c, tq, tk, tv, ts, ty, a, grid, shared);
-    case 32: return launch_bpad<32>(c, tq, tk, tv, ts, ty, a, grid, shared);
-    default: return launch_bpad<64>(c, tq, tk, tv, ts, ty, a, grid, shared);
+    case 16: return launch_bpad<16>(c, tq, tk, tv, ts, ty, a, grid, shared, commit);
+    case 32: return launch_bpad<32>(c, tq, tk, tv, ts, ty, a, grid, shared, commit);
+    default: return launch_bpad<64>(c, tq, tk, tv, ts, ty, a, grid, shared, commit);
   }
 }
 

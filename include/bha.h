@@ -141,6 +141,21 @@ int bha_hybrid_step(const void *Qa, const void *Ka, const void *Va,
                     bha_dtype dtype, bha_stream_t stream);
 
 /*
+ * The block's last denoising step fused with its commit: the result of
+ * bha_hybrid_step on (Qa, Ka, Va, S, z), after which S += phi(Ka)^T Va and
+ * z += sum_t phi(ka_t) (z may be NULL in the default mode) -- the two steps
+ * the worked example takes when a block is finalised (block 2 uses S_1, then
+ * S_{1,2} = S_1 + phi(K_2)^T V_2).  In the default mode with G * b <= 128
+ * this is one kernel that reads the state once; otherwise it launches the
+ * step and the commit kernels back to back.  Y must not overlap any input,
+ * S or z; S and z must not overlap the inputs.
+ */
+int bha_hybrid_step_commit(const void *Qa, const void *Ka, const void *Va,
+                           float *S, float *z, void *Y, int n, int hq,
+                           int hkv, int b, int d, float scale, unsigned flags,
+                           bha_dtype dtype, bha_stream_t stream);
+
+/*
  * Comparison path: exact softmax attention of the active block over the
  * whole KV cache plus the block itself (the abstract's baseline, where
  * every denoising step attends to all previous blocks):

@@ -98,6 +98,19 @@ def test_step_validation(L):
     assert step(L, n=0) == _lib.BHA_OK                               # empty: no launch
 
 
+def test_step_commit_validation(L):
+    f = lambda **kw: L.bha_hybrid_step_commit(kw.get("Q", A), kw.get("K", B), kw.get("V", C),
+                                              kw.get("S", D), kw.get("z", None), kw.get("Y", E),
+                                              2, 16, 4, 32, 128, 0.0, kw.get("flags", 0),
+                                              _lib.BHA_BF16, None)
+    assert f(S=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(flags=1) == _lib.BHA_ERR_INVALID_ARG            # shared needs z
+    assert f(S=B) == _lib.BHA_ERR_INVALID_ARG                # S overlaps K
+    assert f(z=D + 64) == _lib.BHA_ERR_INVALID_ARG           # z overlaps S
+    assert f(Y=D) == _lib.BHA_ERR_INVALID_ARG                # Y overlaps S
+    assert f(S=D + 4) == _lib.BHA_ERR_MISALIGNED
+
+
 def test_valid_call_without_device_reports_cuda_error(L):
     # Arguments are valid, so the call reaches the runtime, which has no GPU here.
     import torch

@@ -286,3 +286,58 @@ def test_prefix_p0_equals_step_with_zero_state():
     bha.bha_hybrid_step(Q, K, V, torch.zeros(n, hkv, 128, 128, device="cuda"), Y2)
     torch.cuda.synchronize()
     assert rel_l2(host(Y1), host(Y2)) < 1e-2
+
+
+# ------------------------------------------------------------ fused last step + commit
+
+FUSED_CASES = [  # (n, hq, hkv, b): the first five run as one kernel in the default mode
+    (2, 16, 4, 32), (3, 4, 4, 32), (2, 8, 2, 17), (2, 8, 2, 10), (1, 4, 1, 1),
+    (2, 8, 1, 33),   # G*b = 264 rows: step + commit kernels
+    (1, 16, 4, 64),  # 256 rows
+]
+
+
+@pytest.mark.parametrize("mode", ["default", "default_noz", "shared"])
+@pytest.mark.parametrize("case", FUSED_CASES, ids=lambda c: "n%d_hq%d_hkv%d_b%d" % c)
+def test_step_commit_bf16(case, mode):
+    """Y from the state before the block, then S += phi(K)^T V, z += sum phi(k)
+    -- against the oracle's step followed by its commit."""
+    import torch
+    n, hq, hkv, b = case
+    seed = 600 + b
+    shared = mode == "shared"
+    Q, Qv = bf16_case((seed, 0), (n, hq, b, 128), STD)
+    K, Kv = bf16_case((seed, 1), (n, hkv, b, 128), STD)
+    V, Vv = bf16_case((seed, 2), (n, hkv, b, 128), STD)
+    Sv, zv = inputs.synthetic_state_np(seed, n, hkv, 128, 4096, STD)
+    S = dev_f32(Sv)
+    z = None if mode == "default_noz" else dev_f32(zv)
+    Y = Guarded((n, hq, b, 128), torch.bfloat16)
+    bha.bha_hybrid_step_commit(Q, K, V, S, Y.t, z=z,
+                               flags=bha.BHA_FLAG_SHARED_DENOM if shared else 0)
+    torch.cuda.synchronize()
+    assert Y.intact() and Y.no_nan()
+    check_bf16("step_commit_y", host(Y.t), oracle.hybrid_step(Qv, Kv, Vv, Sv, zv, shared=shared),
+               case=case, mode=mode)
+    rS, rz = oracle.state_commit(Sv, zv, Kv, Vv)
+    check_rel("step_commit_S", host(S), rS, TOL_STATE_REL, case=case, mode=mode)
+    if z is not None:
+        check_rel("step_commit_z", host(z), rz, TOL_STATE_REL, case=case, mode=mode)
+
+
+def test_step_commit_f32():
+    import torch
+    n, hq, hkv, b, d = 2, 4, 2, 7, 16
+    Qv = inputs.normal_f32_np(81, 0, (n, hq, b, d), 1.0)
+    Kv = inputs.normal_f32_np(81, 1, (n, hkv, b, d), 1.0)
+    Vv = inputs.normal_f32_np(81, 2, (n, hkv, b, d), 1.0)
+    Sv = inputs.normal_f32_np(81, 3, (n, hkv, d, d), 1.0)
+    zv = np.abs(inputs.normal_f32_np(81, 4, (n, hkv, d), 1.0))
+    S, z = dev_f32(Sv), dev_f32(zv)
+    Y = torch.empty(n, hq, b, d, device="cuda")
+    bha.bha_hybrid_step_commit(dev_f32(Qv), dev_f32(Kv), dev_f32(Vv), S, Y, z=z)
+    torch.cuda.synchronize()
+    check_rel("step_commit_f32_y", host(Y), oracle.hybrid_step(Qv, Kv, Vv, Sv, zv), TOL_F32_REL)
+    rS, rz = oracle.state_commit(Sv, zv, Kv, Vv)
+    check_rel("step_commit_f32_S", host(S), rS, TOL_F32_REL)
+    check_rel("step_commit_f32_z", host(z), rz, TOL_F32_REL)
