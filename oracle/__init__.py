@@ -46,12 +46,12 @@ def _load():
         lib.oracle_set_threads.restype = ctypes.c_int
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = ctypes.c_int
-        lib.oracle_state_prefill.argtypes = [dp, dp, L, L, L, dp, dp]
+        lib.oracle_state_prefill.argtypes = [dp, dp, L, L, L, dp, dp, ctypes.c_int, dp, L]
         lib.oracle_state_prefill.restype = None
-        lib.oracle_state_commit.argtypes = [dp, dp, dp, dp, L, L, L]
+        lib.oracle_state_commit.argtypes = [dp, dp, dp, dp, L, L, L, ctypes.c_int, dp, L]
         lib.oracle_state_commit.restype = None
         lib.oracle_hybrid_step.argtypes = [dp, dp, dp, dp, dp, dp, L, L, L, L,
-                                           L, ctypes.c_double, ctypes.c_int]
+                                           L, ctypes.c_double, ctypes.c_int, ctypes.c_int, dp]
         lib.oracle_hybrid_step.restype = None
         lib.oracle_prefix_softmax.argtypes = [dp, dp, dp, L, L, dp, dp, dp, L,
                                               L, L, L, L, ctypes.c_double]
@@ -81,10 +81,26 @@ def max_threads() -> int:
     return _load().oracle_max_threads()
 
 
-def state_prefill(K, V, with_z=True):
+FMAP_RELU, FMAP_ELU1, FMAP_RELU_PROJ = 0, 1, 2
+
+
+def _proj(fmap, W, d, hkv=None):
+    """(pointer array, number of projections) for the feature map; W must
+    hold one d x d projection per KV head of the tensors it is used with."""
+    if fmap != FMAP_RELU_PROJ:
+        return None, 1
+    W = _f64(W)
+    assert W.ndim == 3 and W.shape[1:] == (d, d)
+    assert hkv is None or W.shape[0] == hkv, "one projection per KV head"
+    return W, W.shape[0]
+
+
+def state_prefill(K, V, with_z=True, fmap=FMAP_RELU, W=None):
     """S = phi(K)^T V and z = sum_t phi(k_t) over a prompt.
 
-    K, V: [..., T, d] (leading dims are independent units, e.g. [n, hkv]).
+    K, V: [..., T, d] (leading dims are independent units, e.g. [n, hkv];
+    KV head fastest).  fmap / W: the feature map (W [hkv, d, d] for the
+    projected map; unit u uses W[u % hkv]).
     Returns (S [..., d, d], z [..., d] or None).
     """
     K = _f64(K)
@@ -94,15 +110,17 @@ def state_prefill(K, V, with_z=True):
     units = int(np.prod(lead)) if lead else 1
     S = np.zeros(lead + (d, d))
     z = np.zeros(lead + (d,)) if with_z else None
+    Wp, wu = _proj(fmap, W, d, K.shape[-3] if K.ndim >= 3 else 1)
     _load().oracle_state_prefill(_ptr(K), _ptr(V), units, T, d, _ptr(S),
-                                 _ptr(z))
+                                 _ptr(z), int(fmap), _ptr(Wp), wu)
     return S, z
 
 
-def state_commit(S, z, Kb, Vb):
+def state_commit(S, z, Kb, Vb, fmap=FMAP_RELU, W=None):
     """Return (S + phi(Kb)^T Vb, z + sum_t phi(kb_t)); inputs are not modified.
 
-    S [..., d, d], z [..., d] or None, Kb/Vb [..., b, d].
+    S [..., d, d], z [..., d] or None, Kb/Vb [..., b, d]; fmap / W as for
+    state_prefill.
     """
     S = _f64(S).copy()
     z = None if z is None else _f64(z).copy()
@@ -111,16 +129,19 @@ def state_commit(S, z, Kb, Vb):
     lead, (b, d) = Kb.shape[:-2], Kb.shape[-2:]
     assert S.shape == lead + (d, d)
     units = int(np.prod(lead)) if lead else 1
+    Wp, wu = _proj(fmap, W, d, Kb.shape[-3] if Kb.ndim >= 3 else 1)
     _load().oracle_state_commit(_ptr(S), _ptr(z), _ptr(Kb), _ptr(Vb), units,
-                                b, d)
+                                b, d, int(fmap), _ptr(Wp), wu)
     return S, z
 
 
-def hybrid_step(Q, K, V, S, z=None, scale=0.0, shared=False):
+def hybrid_step(Q, K, V, S, z=None, scale=0.0, shared=False, fmap=FMAP_RELU,
+                W=None):
     """Block-hybrid attention output for the active block.
 
     Q [n, hq, b, d]; K, V [n, hkv, b, d]; S [n, hkv, d, d]; z [n, hkv, d]
-    (required when shared).  scale <= 0 means 1/sqrt(d).
+    (required when shared).  scale <= 0 means 1/sqrt(d).  fmap / W: the
+    feature map (W [hkv, d, d]; query head h uses KV head h // G's W).
     Returns Y [n, hq, b, d] in float64.
     """
     Q, K, V, S = _f64(Q), _f64(K), _f64(V), _f64(S)
@@ -132,9 +153,10 @@ def hybrid_step(Q, K, V, S, z=None, scale=0.0, shared=False):
         assert z is not None
     zz = None if z is None else _f64(z)
     Y = np.zeros((n, hq, b, d))
+    Wp, _ = _proj(fmap, W, d, hkv)
     _load().oracle_hybrid_step(_ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(zz),
                                _ptr(Y), n, hq, hkv, b, d, float(scale),
-                               1 if shared else 0)
+                               1 if shared else 0, int(fmap), _ptr(Wp))
     return Y
 
 
@@ -166,7 +188,7 @@ def block_partition(L: int, B: int):
 
 
 def generate(Q_steps, K_steps, V_steps, K_prompt=None, V_prompt=None,
-             scale=0.0, shared=False):
+             scale=0.0, shared=False, fmap=FMAP_RELU, W=None):
     """Blockwise decoding loop of the worked example, on given inputs.
 
     Q_steps[blk][step] etc. hold the active block's tensors at each
@@ -178,7 +200,7 @@ def generate(Q_steps, K_steps, V_steps, K_prompt=None, V_prompt=None,
     first_k = K_steps[0][0]
     n, hkv, _, dd = first_k.shape
     if K_prompt is not None:
-        S, z = state_prefill(K_prompt, V_prompt)
+        S, z = state_prefill(K_prompt, V_prompt, fmap=fmap, W=W)
     else:
         S = np.zeros((n, hkv, dd, dd))
         z = np.zeros((n, hkv, dd))
@@ -187,7 +209,7 @@ def generate(Q_steps, K_steps, V_steps, K_prompt=None, V_prompt=None,
         ob = []
         for st in range(len(Q_steps[blk])):
             ob.append(hybrid_step(Q_steps[blk][st], K_steps[blk][st],
-                                  V_steps[blk][st], S, z, scale, shared))
+                                  V_steps[blk][st], S, z, scale, shared, fmap, W))
         outs.append(ob)
-        S, z = state_commit(S, z, K_steps[blk][-1], V_steps[blk][-1])
+        S, z = state_commit(S, z, K_steps[blk][-1], V_steps[blk][-1], fmap, W)
     return outs, S, z

@@ -41,6 +41,33 @@
 
 static double relu(double x) { return x > 0.0 ? x : 0.0; }
 
+/*
+ * Kernel feature maps phi.  The worked example (paper-daily summary page,
+ * 具体技术细节示例) takes phi = ReLU; the method details (技术方法详解) speak of
+ * kernel-function approximations in general and list better kernels as
+ * future work (未来研究方向), so two more maps are provided:
+ *   fmap 0  ReLU        phi(x)_c = max(x_c, 0)
+ *   fmap 1  ELU + 1     phi(x)_c = x_c + 1 if x_c > 0 else exp(x_c)
+ *   fmap 2  projected   phi(x)_c = max(sum_r x_r W[r][c], 0), W a d x d matrix
+ * out[c] = phi(x)_c for one d-vector x; W is the KV head's projection
+ * (ignored unless fmap = 2).
+ */
+static void phi_vec(const double *x, long d, int fmap, const double *W, double *out)
+{
+    for (long c = 0; c < d; ++c) {
+        if (fmap == 2) {
+            double acc = 0.0;
+            for (long r = 0; r < d; ++r)
+                acc += x[r] * W[r * d + c];
+            out[c] = relu(acc);
+        } else if (fmap == 1) {
+            out[c] = x[c] > 0.0 ? x[c] + 1.0 : exp(x[c]);
+        } else {
+            out[c] = relu(x[c]);
+        }
+    }
+}
+
 static int g_threads = 1;
 
 /* Number of OpenMP threads the routines below use (1 = single-threaded). */
@@ -62,34 +89,41 @@ int oracle_max_threads(void)
 
 /*
  * Prefix state of a prompt (the prompt counts as "previous blocks"):
- *   S[u][r][c] = sum_{t<T} relu(K[u][t][r]) * V[u][t][c]
- *   z[u][r]    = sum_{t<T} relu(K[u][t][r])
- * T = 0 gives S = 0, z = 0.  z may be NULL.
- * Worked example: S_1 = phi(K_1)^T V_1.
+ *   S[u][r][c] = sum_{t<T} phi(K[u][t])[r] * V[u][t][c]
+ *   z[u][r]    = sum_{t<T} phi(K[u][t])[r]
+ * T = 0 gives S = 0, z = 0.  z may be NULL.  W holds w_units projections
+ * (one per KV head); unit u uses W[u % w_units] (units are (n, kvh) pairs,
+ * KV head fastest).  Worked example: S_1 = phi(K_1)^T V_1.
  */
 void oracle_state_prefill(const double *K, const double *V, long units, long T,
-                          long d, double *S, double *z)
+                          long d, double *S, double *z, int fmap, const double *W,
+                          long w_units)
 {
     long u;
 #pragma omp parallel for num_threads(g_threads) schedule(static)
     for (u = 0; u < units; ++u) {
         const double *Ku = K + u * T * d;
         const double *Vu = V + u * T * d;
+        const double *Wu = W ? W + (u % w_units) * d * d : NULL;
         double *Su = S + u * d * d;
+        double *fk = (double *)malloc(sizeof(double) * (size_t)(T * d > 0 ? T * d : 1));
+        for (long t = 0; t < T; ++t)
+            phi_vec(Ku + t * d, d, fmap, Wu, fk + t * d);
         for (long r = 0; r < d; ++r) {
             for (long c = 0; c < d; ++c) {
                 double acc = 0.0;
                 for (long t = 0; t < T; ++t)
-                    acc += relu(Ku[t * d + r]) * Vu[t * d + c];
+                    acc += fk[t * d + r] * Vu[t * d + c];
                 Su[r * d + c] = acc;
             }
             if (z) {
                 double zs = 0.0;
                 for (long t = 0; t < T; ++t)
-                    zs += relu(Ku[t * d + r]);
+                    zs += fk[t * d + r];
                 z[u * d + r] = zs;
             }
         }
+        free(fk);
     }
 }
 
@@ -97,31 +131,37 @@ void oracle_state_prefill(const double *K, const double *V, long units, long T,
  * Block commit when a block is finalised:
  *   S[u] += phi(Kb[u])^T Vb[u],   z[u] += sum_t phi(Kb[u][t])
  * Worked example: S_{1,2} = phi(K_1)^T V_1 + phi(K_2)^T V_2.
- * Kb, Vb are [units][b][d].  z may be NULL.
+ * Kb, Vb are [units][b][d].  z may be NULL.  W as for the prefill.
  */
 void oracle_state_commit(double *S, double *z, const double *Kb,
-                         const double *Vb, long units, long b, long d)
+                         const double *Vb, long units, long b, long d, int fmap,
+                         const double *W, long w_units)
 {
     long u;
 #pragma omp parallel for num_threads(g_threads) schedule(static)
     for (u = 0; u < units; ++u) {
         const double *Ku = Kb + u * b * d;
         const double *Vu = Vb + u * b * d;
+        const double *Wu = W ? W + (u % w_units) * d * d : NULL;
         double *Su = S + u * d * d;
+        double *fk = (double *)malloc(sizeof(double) * (size_t)(b * d));
+        for (long t = 0; t < b; ++t)
+            phi_vec(Ku + t * d, d, fmap, Wu, fk + t * d);
         for (long r = 0; r < d; ++r) {
             for (long c = 0; c < d; ++c) {
                 double acc = 0.0;
                 for (long t = 0; t < b; ++t)
-                    acc += relu(Ku[t * d + r]) * Vu[t * d + c];
+                    acc += fk[t * d + r] * Vu[t * d + c];
                 Su[r * d + c] += acc;
             }
             if (z) {
                 double zs = 0.0;
                 for (long t = 0; t < b; ++t)
-                    zs += relu(Ku[t * d + r]);
+                    zs += fk[t * d + r];
                 z[u * d + r] += zs;
             }
         }
+        free(fk);
     }
 }
 
@@ -136,12 +176,13 @@ void oracle_state_commit(double *S, double *z, const double *Kb,
  *   default:  y_i = sum_j (e_j / l) v_{g,j} + lin
  *   shared :  y_i = (sum_j e_j v_{g,j} + e^{-m} lin) /
  *                   (l + e^{-m} phi(q_i) . z_g)
- * scale <= 0 selects 1/sqrt(d).  z is read only when shared != 0.
+ * scale <= 0 selects 1/sqrt(d).  z is read only when shared != 0.  phi is
+ * feature map fmap (W: [hkv][d][d], KV head g's projection, for fmap 2).
  */
 void oracle_hybrid_step(const double *Q, const double *K, const double *V,
                         const double *S, const double *z, double *Y, long n,
                         long hq, long hkv, long b, long d, double scale,
-                        int shared)
+                        int shared, int fmap, const double *W)
 {
     if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
     const long G = hq / hkv;
@@ -153,8 +194,10 @@ void oracle_hybrid_step(const double *Q, const double *K, const double *V,
         const double *Vg = V + (ni * hkv + g) * b * d;
         const double *Sg = S + (ni * hkv + g) * d * d;
         const double *zg = z ? z + (ni * hkv + g) * d : NULL;
+        const double *Wg = W ? W + g * d * d : NULL;
         double *s = (double *)malloc(sizeof(double) * (size_t)b);
         double *lin = (double *)malloc(sizeof(double) * (size_t)d);
+        double *fq = (double *)malloc(sizeof(double) * (size_t)d);
         for (long i = 0; i < b; ++i) {
             const double *q = Q + ((ni * hq + h) * b + i) * d;
             double *y = Y + ((ni * hq + h) * b + i) * d;
@@ -171,10 +214,11 @@ void oracle_hybrid_step(const double *Q, const double *K, const double *V,
                 s[j] = exp(s[j] - m); /* s now holds e_j */
                 l += s[j];
             }
+            phi_vec(q, d, fmap, Wg, fq);
             for (long c = 0; c < d; ++c) {
                 double acc = 0.0;
                 for (long r = 0; r < d; ++r)
-                    acc += relu(q[r]) * Sg[r * d + c];
+                    acc += fq[r] * Sg[r * d + c];
                 lin[c] = acc;
             }
             if (!shared) {
@@ -187,7 +231,7 @@ void oracle_hybrid_step(const double *Q, const double *K, const double *V,
             } else {
                 double qz = 0.0;
                 for (long r = 0; r < d; ++r)
-                    qz += relu(q[r]) * zg[r];
+                    qz += fq[r] * zg[r];
                 const double em = exp(-m);
                 const double den = l + em * qz;
                 for (long c = 0; c < d; ++c) {
@@ -200,6 +244,7 @@ void oracle_hybrid_step(const double *Q, const double *K, const double *V,
         }
         free(s);
         free(lin);
+        free(fq);
     }
 }
 

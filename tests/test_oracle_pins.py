@@ -406,3 +406,128 @@ def test_pins_catch_planted_mistake(name):
         except Exception:
             errs.append(float("inf"))
     assert max(errs) > 1e-3, (name, errs)
+
+
+# ------------------------------------------------------- other feature maps
+# The method details speak of kernel-function approximations and the future
+# work lists better kernels; these pins cover the two extra maps the oracle
+# provides: elu(x) + 1 and a learned projection relu(x W) (one W per KV head).
+
+def np_elu1(x):
+    return np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
+
+
+def np_relu_proj(x, W):
+    return np.maximum(x @ W, 0.0)
+
+
+def _bruteforce_linear(Q, Kp, Vp, phi):
+    """sum over prefix tokens t of (phi(q).phi(k_t)) v_t, token by token."""
+    n, hq, b, d = Q.shape
+    hkv = Kp.shape[1]
+    G = hq // hkv
+    out = np.zeros(Q.shape)
+    for ni in range(n):
+        for h in range(hq):
+            g = h // G
+            fk = phi(Kp[ni, g], g)
+            for i in range(b):
+                fq = phi(Q[ni, h, i][None], g)[0]
+                for t in range(Kp.shape[2]):
+                    out[ni, h, i] += float(fq @ fk[t]) * Vp[ni, g, t]
+    return out
+
+
+def pin_fmap_linear_bruteforce(impl_step, impl_prefill, fmap, W, phi):
+    n, hq, hkv, b, d, T = 1, 4, 2, 3, 8, 7
+    Q, K, V = rnd(151, (n, hq, b, d)), rnd(152, (n, hkv, b, d)), rnd(153, (n, hkv, b, d))
+    Kp, Vp = rnd(154, (n, hkv, T, d)), rnd(155, (n, hkv, T, d))
+    S, z = impl_prefill(Kp, Vp, fmap=fmap, W=W)
+    y = impl_step(Q, K, V, S, z, fmap=fmap, W=W)
+    soft = sdpa(Q, K, V, scale=1.0 / math.sqrt(d))
+    return relerr(y - soft, _bruteforce_linear(Q, Kp, Vp, phi))
+
+
+def test_elu1_linear_term_bruteforce():
+    e = pin_fmap_linear_bruteforce(oracle.hybrid_step, oracle.state_prefill,
+                                   oracle.FMAP_ELU1, None, lambda x, g: np_elu1(x))
+    assert e < TOL
+
+
+def test_relu_proj_linear_term_bruteforce():
+    W = rnd(160, (2, 8, 8), 0.5)
+    e = pin_fmap_linear_bruteforce(oracle.hybrid_step, oracle.state_prefill,
+                                   oracle.FMAP_RELU_PROJ, W, lambda x, g: np_relu_proj(x, W[g]))
+    assert e < TOL
+
+
+def test_relu_proj_identity_is_relu():
+    """W = I: the projected map is ReLU exactly."""
+    d = 8
+    W = np.broadcast_to(np.eye(d), (2, d, d)).copy()
+    Q, K, V = rnd(161, (2, 4, 5, d)), rnd(162, (2, 2, 5, d)), rnd(163, (2, 2, 5, d))
+    Kp, Vp = rnd(164, (2, 2, 9, d)), rnd(165, (2, 2, 9, d))
+    S1, z1 = oracle.state_prefill(Kp, Vp)
+    S2, z2 = oracle.state_prefill(Kp, Vp, fmap=oracle.FMAP_RELU_PROJ, W=W)
+    assert np.array_equal(S1, S2) and np.array_equal(z1, z2)
+    y1 = oracle.hybrid_step(Q, K, V, S1, z1, shared=True)
+    y2 = oracle.hybrid_step(Q, K, V, S2, z2, shared=True, fmap=oracle.FMAP_RELU_PROJ, W=W)
+    assert np.array_equal(y1, y2)
+
+
+def test_relu_proj_permutation_leaves_output_unchanged():
+    """W = a permutation P: phi(q) phi(K)^T = relu(q) P P^T relu(K)^T, so the
+    linear term (and y) equal the plain ReLU ones while S is permuted."""
+    d = 8
+    perm = np.random.default_rng(7).permutation(d)
+    P = np.eye(d)[:, perm]
+    W = np.stack([P, P])
+    Q, K, V = rnd(171, (1, 4, 5, d)), rnd(172, (1, 2, 5, d)), rnd(173, (1, 2, 5, d))
+    Kp, Vp = rnd(174, (1, 2, 9, d)), rnd(175, (1, 2, 9, d))
+    S1, _ = oracle.state_prefill(Kp, Vp)
+    S2, _ = oracle.state_prefill(Kp, Vp, fmap=oracle.FMAP_RELU_PROJ, W=W)
+    assert relerr(S2, S1[..., perm, :]) < TOL
+    y1 = oracle.hybrid_step(Q, K, V, S1)
+    y2 = oracle.hybrid_step(Q, K, V, S2, fmap=oracle.FMAP_RELU_PROJ, W=W)
+    assert relerr(y2, y1) < TOL
+
+
+def test_elu1_special_values():
+    """phi(0) = e^0 = 1, phi(x) = x + 1 for x > 0, phi(x) in (0, 1) for x < 0:
+    one token with k = (0, 2, -1, ...) gives S rows scaled by those values."""
+    d = 4
+    k = np.array([[[[0.0, 2.0, -1.0, 3.5]]]])
+    v = np.array([[[[1.0, -2.0, 0.5, 4.0]]]])
+    S, z = oracle.state_prefill(k, v, fmap=oracle.FMAP_ELU1)
+    phi = np.array([1.0, 3.0, math.exp(-1.0), 4.5])
+    assert np.allclose(S[0, 0], np.outer(phi, v[0, 0, 0]), rtol=0, atol=1e-15)
+    assert np.allclose(z[0, 0], phi, rtol=0, atol=1e-15)
+
+
+def test_fmap_prefill_equals_commits_and_order_invariance():
+    d, B = 8, 4
+    W = rnd(180, (1, d, d), 0.5)
+    Kp, Vp = rnd(181, (2, 1, 3 * B, d)), rnd(182, (2, 1, 3 * B, d))
+    for fmap, w in ((oracle.FMAP_ELU1, None), (oracle.FMAP_RELU_PROJ, W)):
+        S_all, z_all = oracle.state_prefill(Kp, Vp, fmap=fmap, W=w)
+        for order in ([0, 1, 2], [2, 1, 0]):
+            S = np.zeros((2, 1, d, d))
+            z = np.zeros((2, 1, d))
+            for blk in order:
+                sl = slice(blk * B, (blk + 1) * B)
+                S, z = oracle.state_commit(S, z, Kp[:, :, sl], Vp[:, :, sl], fmap, w)
+            assert relerr(S, S_all) < TOL and relerr(z, z_all) < TOL
+
+
+def test_fmap_pins_catch_planted_mistakes():
+    """Transposed projection, and ELU without the +1, fail the brute force."""
+    W = rnd(160, (2, 8, 8), 0.5)
+    wt = np.swapaxes(W, -1, -2).copy()
+    bad_step = lambda Q, K, V, S, z, fmap, W: oracle.hybrid_step(Q, K, V, S, z, fmap=fmap, W=wt)
+    e = pin_fmap_linear_bruteforce(bad_step, oracle.state_prefill, oracle.FMAP_RELU_PROJ, W,
+                                   lambda x, g: np_relu_proj(x, W[g]))
+    assert e > 1e-3
+    e2 = pin_fmap_linear_bruteforce(oracle.hybrid_step, oracle.state_prefill,
+                                    oracle.FMAP_ELU1, None,
+                                    lambda x, g: np_elu1(x) - 1.0)   # elu without +1
+    assert e2 > 1e-3
