@@ -58,7 +58,8 @@ def parse():
     ap.add_argument("--prefix", type=int, default=8192,
                     help="prompt / cache length used by --only prefill|prefix")
     ap.add_argument("--workload", default="long-prefix",
-                    choices=["long-prefix", "single-step", "generation-loop", "stack"],
+                    choices=["long-prefix", "single-step", "generation-loop", "stack",
+                             "feature-maps"],
                     help="long-prefix is the benchmark line; the others are the secondary "
                          "workloads (one JSON line each)")
     return ap.parse_args()
@@ -660,6 +661,79 @@ def run_single_step(args):
         "note": "4.7 MB per step: bound by launch latency, not by HBM"}), flush=True)
 
 
+def run_feature_maps(args):
+    """The long-prefix shapes (batch 64, 16q/4kv, d=128, B=32) under each
+    feature map (ReLU, elu + 1, ReLU after a per-KV-head projection W_g):
+    per-launch times of the step, the last step fused with the commit, the
+    commit, and a 32768-token prefill, as kernel-only CUDA graphs over
+    rotating input sets 4x the size of L2."""
+    import torch
+    import block_hybrid_linear_b200 as bha
+    from block_hybrid_linear_b200 import build, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    n, P = N_, 32768
+    std = 1.0 / math.sqrt(D_)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(4, math.ceil(4 * l2 / (n * HKV * UNIT_BYTES_STEP)))
+    W = inputs.normal_bf16_torch(4000, 90, (HKV, D_, D_), 1.0 / math.sqrt(D_), dev)  # N(0, 1/d)
+    sets = [dict(Q=inputs.normal_bf16_torch(r, inputs.TID_Q, (n, HQ, B_, D_), std, dev),
+                 K=inputs.normal_bf16_torch(r, inputs.TID_K, (n, HKV, B_, D_), std, dev),
+                 V=inputs.normal_bf16_torch(r, inputs.TID_V, (n, HKV, B_, D_), std, dev),
+                 S=torch.randn(n, HKV, D_, D_, device=dev), z=torch.rand(n, HKV, D_, device=dev),
+                 Y=torch.empty(n, HQ, B_, D_, dtype=torch.bfloat16, device=dev))
+            for r in range(R)]
+    Kp = inputs.normal_bf16_torch(4000, inputs.TID_KP, (n, HKV, P, D_), std, dev)
+    Vp = inputs.normal_bf16_torch(4000, inputs.TID_VP, (n, HKV, P, D_), std, dev)
+    need = bha.bha_state_prefill_workspace_size(n, HKV, P, D_)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    Sp = torch.empty(n, HKV, D_, D_, device=dev)
+    zp = torch.empty(n, HKV, D_, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    peak, _ = measured_peaks()
+    units = n * HKV
+    prefill_bytes = units * (2 * P * D_ * 2 + D_ * D_ * 4 + D_ * 4)
+    out = {}
+    for name, f in (("relu", bha.BHA_FMAP_RELU), ("elu1", bha.BHA_FMAP_ELU1),
+                    ("relu_proj", bha.BHA_FMAP_RELU_PROJ)):
+        Wf = W if f == bha.BHA_FMAP_RELU_PROJ else None
+        wbytes = 0 if Wf is None else HKV * D_ * D_ * 2
+
+        def per_launch(call, reps=50):
+            g = _graph(lambda: [call(st) for st in sets], stream)
+            return _time_graph(g, stream, reps) * 1e3 / R
+
+        res = {}
+        for op, call, ubytes in (
+                ("step", lambda st: bha.bha_hybrid_step_fm(
+                    st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"], fmap=f, W=Wf,
+                    stream=stream), UNIT_BYTES_STEP),
+                ("step_commit", lambda st: bha.bha_hybrid_step_commit_fm(
+                    st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"], fmap=f, W=Wf,
+                    stream=stream), UNIT_BYTES_FUSED),
+                ("commit", lambda st: bha.bha_state_commit_fm(
+                    st["K"], st["V"], st["S"], st["z"], fmap=f, W=Wf, stream=stream),
+                 UNIT_BYTES_COMMIT)):
+            us = per_launch(call)
+            nbytes = units * ubytes + wbytes
+            res[op] = {"launch_us": round(us, 3), "algorithmic_bytes": nbytes,
+                       "achieved_gbs": round(nbytes / (us / 1e6) / 1e9, 1),
+                       "frac_of_peak": round(nbytes / (us / 1e6) / 1e9 / peak, 4)}
+        gp = _graph(lambda: bha.bha_state_prefill_fm(Kp, Vp, Sp, zp, fmap=f, W=Wf, workspace=ws,
+                                                     stream=stream), stream)
+        us = _time_graph(gp, stream, 5) * 1e3
+        nbytes = prefill_bytes + wbytes
+        res["prefill_32768"] = {"launch_us": round(us, 1), "algorithmic_bytes": nbytes,
+                                "achieved_gbs": round(nbytes / (us / 1e6) / 1e9, 1),
+                                "frac_of_peak": round(nbytes / (us / 1e6) / 1e9 / peak, 4)}
+        out[name] = res
+    torch.cuda.synchronize()
+    assert bha.bha_device_error(True) == 0
+    print(json.dumps({
+        "workload": "feature-maps: batch 64, 16q/4kv, d=128, B=32; prefill of 32768 tokens",
+        "rotating_sets": R, "peak_gbs": peak, "maps": out}), flush=True)
+
+
 def run_generation_loop(args):
     """Batch 32, prompt 1024 -> state, 32 blocks x 8 denoising steps (one
     commit per block), against exact attention over the growing KV cache
@@ -821,7 +895,7 @@ def main():
     if args.workload != "long-prefix":
         if rank == 0:
             {"single-step": run_single_step, "generation-loop": run_generation_loop,
-             "stack": run_stack}[args.workload](args)
+             "stack": run_stack, "feature-maps": run_feature_maps}[args.workload](args)
         return
     if args.impl == "reference":
         run_reference(args, rank, world)

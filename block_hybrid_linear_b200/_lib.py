@@ -24,12 +24,16 @@ BHA_ERR_DEVICE = -7
 BHA_BF16 = 0
 BHA_F32 = 1
 BHA_FLAG_SHARED_DENOM = 1
+BHA_FMAP_RELU = 0
+BHA_FMAP_ELU1 = 1
+BHA_FMAP_RELU_PROJ = 2
 
 # every symbol include/bha.h declares
 EXPORTED = [
     "bha_status_string", "bha_version", "bha_state_prefill_workspace_size",
     "bha_state_prefill", "bha_state_prefill_noalloc", "bha_state_commit", "bha_hybrid_step",
-    "bha_hybrid_step_commit",
+    "bha_hybrid_step_commit", "bha_state_prefill_fm", "bha_state_commit_fm",
+    "bha_hybrid_step_fm", "bha_hybrid_step_commit_fm",
     "bha_prefix_softmax_workspace_size", "bha_prefix_softmax",
     "bha_block_partition", "bha_device_error", "bha_selftest_timeout",
 ]
@@ -72,6 +76,16 @@ def lib():
         L.bha_hybrid_step_commit.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, fl, u,
                                              i, vp]
         L.bha_hybrid_step_commit.restype = i
+        L.bha_state_prefill_fm.argtypes = [vp, vp, i, i, i, i, i, i, vp, vp, vp, vp, sz, vp]
+        L.bha_state_prefill_fm.restype = i
+        L.bha_state_commit_fm.argtypes = [vp, vp, i, i, i, i, i, i, vp, vp, vp, vp]
+        L.bha_state_commit_fm.restype = i
+        L.bha_hybrid_step_fm.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, fl, u, i, i,
+                                         vp, vp]
+        L.bha_hybrid_step_fm.restype = i
+        L.bha_hybrid_step_commit_fm.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, fl, u,
+                                                i, i, vp, vp]
+        L.bha_hybrid_step_commit_fm.restype = i
         L.bha_prefix_softmax_workspace_size.argtypes = [i, i, i, i, i, i, i]
         L.bha_prefix_softmax_workspace_size.restype = sz
         L.bha_prefix_softmax.argtypes = [vp, vp, vp, i, i, vp, vp, vp, i, i, i, i,
@@ -188,6 +202,46 @@ def bha_hybrid_step_commit(Q, K, V, S, Y, z=None, scale=0.0, flags=0, stream=Non
     _check(lib().bha_hybrid_step_commit(_ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(z), _ptr(Y),
                                         n, hq, hkv, b, d, float(scale), int(flags), _dtype(Q),
                                         _stream(stream)), "bha_hybrid_step_commit")
+
+
+def bha_state_prefill_fm(K, V, S, z=None, fmap=BHA_FMAP_RELU, W=None, workspace=None,
+                         stream=None):
+    """bha_state_prefill with feature map ``fmap``; W: [hkv, d, d] in K's dtype
+    for BHA_FMAP_RELU_PROJ, else None."""
+    n, hkv, T, d = K.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().bha_state_prefill_fm(_ptr(K), _ptr(V), n, hkv, T, d, _dtype(K), int(fmap),
+                                      _ptr(W), _ptr(S), _ptr(z), _ptr(workspace), ws_bytes,
+                                      _stream(stream)), "bha_state_prefill_fm")
+
+
+def bha_state_commit_fm(Kb, Vb, S, z=None, fmap=BHA_FMAP_RELU, W=None, stream=None):
+    """bha_state_commit with feature map ``fmap`` (W as for bha_state_prefill_fm)."""
+    n, hkv, b, d = Kb.shape
+    _check(lib().bha_state_commit_fm(_ptr(Kb), _ptr(Vb), n, hkv, b, d, _dtype(Kb), int(fmap),
+                                     _ptr(W), _ptr(S), _ptr(z), _stream(stream)),
+           "bha_state_commit_fm")
+
+
+def bha_hybrid_step_fm(Q, K, V, S, Y, z=None, scale=0.0, flags=0, fmap=BHA_FMAP_RELU, W=None,
+                       stream=None):
+    """bha_hybrid_step with feature map ``fmap`` (W as for bha_state_prefill_fm)."""
+    n, hq, b, d = Q.shape
+    hkv = K.shape[1]
+    _check(lib().bha_hybrid_step_fm(_ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(z), _ptr(Y), n,
+                                    hq, hkv, b, d, float(scale), int(flags), _dtype(Q),
+                                    int(fmap), _ptr(W), _stream(stream)), "bha_hybrid_step_fm")
+
+
+def bha_hybrid_step_commit_fm(Q, K, V, S, Y, z=None, scale=0.0, flags=0, fmap=BHA_FMAP_RELU,
+                              W=None, stream=None):
+    """bha_hybrid_step_commit with feature map ``fmap``."""
+    n, hq, b, d = Q.shape
+    hkv = K.shape[1]
+    _check(lib().bha_hybrid_step_commit_fm(_ptr(Q), _ptr(K), _ptr(V), _ptr(S), _ptr(z),
+                                           _ptr(Y), n, hq, hkv, b, d, float(scale), int(flags),
+                                           _dtype(Q), int(fmap), _ptr(W), _stream(stream)),
+           "bha_hybrid_step_commit_fm")
 
 
 def bha_prefix_softmax_workspace_size(n, hq, hkv, b, d, P, dtype=BHA_BF16):

@@ -94,6 +94,22 @@ int check_dims(bha_dtype t, int d, int b_or_1) {
   return BHA_OK;
 }
 
+// The map must be one of bha_fmap; W is required for the projected map and
+// only there.
+int check_fmap(bha_fmap fmap, const void* W) {
+  const int f = static_cast<int>(fmap);
+  if (f != BHA_FMAP_RELU && f != BHA_FMAP_ELU1 && f != BHA_FMAP_RELU_PROJ)
+    return BHA_ERR_INVALID_ARG;
+  if ((f == BHA_FMAP_RELU_PROJ) != (W != nullptr)) return BHA_ERR_INVALID_ARG;
+  if (misaligned(W)) return BHA_ERR_MISALIGNED;
+  return BHA_OK;
+}
+
+// Bytes of W ([hkv][d][d]); 0 when there is none.
+size_t w_bytes(const void* W, int hkv, int d, bha_dtype t) {
+  return W == nullptr ? 0 : static_cast<size_t>(hkv) * d * d * esize(t);
+}
+
 float resolve_scale(float scale, int d) {
   return scale > 0.f ? scale : 1.0f / std::sqrt(static_cast<float>(d));
 }
@@ -214,7 +230,16 @@ size_t bha_state_prefill_workspace_size(int n, int hkv, int T, int d, bha_dtype 
 int bha_state_prefill(const void* K, const void* V, int n, int hkv, int T, int d,
                       bha_dtype dtype, float* S, float* z, void* workspace,
                       size_t workspace_bytes, bha_stream_t stream) {
+  return bha_state_prefill_fm(K, V, n, hkv, T, d, dtype, BHA_FMAP_RELU, nullptr, S, z, workspace,
+                              workspace_bytes, stream);
+}
+
+int bha_state_prefill_fm(const void* K, const void* V, int n, int hkv, int T, int d,
+                         bha_dtype dtype, bha_fmap fmap, const void* W, float* S, float* z,
+                         void* workspace, size_t workspace_bytes, bha_stream_t stream) {
   int st = check_dims(dtype, d, 1);
+  if (st != BHA_OK) return st;
+  st = check_fmap(fmap, W);
   if (st != BHA_OK) return st;
   if (n < 0 || hkv < 1 || T < 0) return BHA_ERR_INVALID_ARG;
   if (n == 0) return BHA_OK;
@@ -224,29 +249,39 @@ int bha_state_prefill(const void* K, const void* V, int n, int hkv, int T, int d
   const size_t units = static_cast<size_t>(n) * hkv;
   const size_t kv_bytes = units * T * d * esize(dtype);
   const size_t s_bytes = units * d * d * 4, z_bytes = units * d * 4;
+  const size_t wb = w_bytes(W, hkv, d, dtype);
   if (overlap(S, s_bytes, K, kv_bytes) || overlap(S, s_bytes, V, kv_bytes) ||
       overlap(z, z_bytes, K, kv_bytes) || overlap(z, z_bytes, V, kv_bytes) ||
-      overlap(z, z_bytes, S, s_bytes))
+      overlap(z, z_bytes, S, s_bytes) || overlap(W, wb, S, s_bytes) || overlap(W, wb, z, z_bytes))
     return BHA_ERR_INVALID_ARG;
   const size_t need = bha_state_prefill_workspace_size(n, hkv, T, d, dtype);
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BHA_ERR_WORKSPACE;
   if (need > 0 && (overlap(workspace, need, S, s_bytes) || overlap(workspace, need, z, z_bytes) ||
-                   overlap(workspace, need, K, kv_bytes) || overlap(workspace, need, V, kv_bytes)))
+                   overlap(workspace, need, K, kv_bytes) || overlap(workspace, need, V, kv_bytes) ||
+                   overlap(workspace, need, W, wb)))
     return BHA_ERR_INVALID_ARG;
   Ctx c;
   st = make_ctx(stream, dtype, &c);
   if (st != BHA_OK) return st;
   if (dtype == BHA_F32)
     return launch_status(launch_prefill_f32(c, static_cast<const float*>(K),
-                                            static_cast<const float*>(V), (int)units, T, d, S,
-                                            z));
+                                            static_cast<const float*>(V), (int)units, T, d, S, z,
+                                            fmap, static_cast<const float*>(W), hkv));
   return launch_status(launch_prefill_bf16(c, K, V, (int)units, T, S, z, workspace,
-                                           workspace_bytes));
+                                           workspace_bytes, fmap, W, hkv));
 }
 
 int bha_state_commit(const void* Kb, const void* Vb, int n, int hkv, int b, int d,
                      bha_dtype dtype, float* S, float* z, bha_stream_t stream) {
+  return bha_state_commit_fm(Kb, Vb, n, hkv, b, d, dtype, BHA_FMAP_RELU, nullptr, S, z, stream);
+}
+
+int bha_state_commit_fm(const void* Kb, const void* Vb, int n, int hkv, int b, int d,
+                        bha_dtype dtype, bha_fmap fmap, const void* W, float* S, float* z,
+                        bha_stream_t stream) {
   int st = check_dims(dtype, d, b);
+  if (st != BHA_OK) return st;
+  st = check_fmap(fmap, W);
   if (st != BHA_OK) return st;
   if (n < 0 || hkv < 1) return BHA_ERR_INVALID_ARG;
   if (n == 0) return BHA_OK;
@@ -256,24 +291,35 @@ int bha_state_commit(const void* Kb, const void* Vb, int n, int hkv, int b, int 
   const size_t units = static_cast<size_t>(n) * hkv;
   const size_t kv_bytes = units * b * d * esize(dtype);
   const size_t s_bytes = units * d * d * 4, z_bytes = units * d * 4;
+  const size_t wb = w_bytes(W, hkv, d, dtype);
   if (overlap(S, s_bytes, Kb, kv_bytes) || overlap(S, s_bytes, Vb, kv_bytes) ||
       overlap(z, z_bytes, Kb, kv_bytes) || overlap(z, z_bytes, Vb, kv_bytes) ||
-      overlap(z, z_bytes, S, s_bytes))
+      overlap(z, z_bytes, S, s_bytes) || overlap(W, wb, S, s_bytes) || overlap(W, wb, z, z_bytes))
     return BHA_ERR_INVALID_ARG;
   Ctx c;
   st = make_ctx(stream, dtype, &c);
   if (st != BHA_OK) return st;
   if (dtype == BHA_F32)
     return launch_status(launch_commit_f32(c, static_cast<const float*>(Kb),
-                                           static_cast<const float*>(Vb), (int)units, b, d, S,
-                                           z));
-  return launch_status(launch_commit_bf16(c, Kb, Vb, (int)units, b, S, z));
+                                           static_cast<const float*>(Vb), (int)units, b, d, S, z,
+                                           fmap, static_cast<const float*>(W), hkv));
+  return launch_status(launch_commit_bf16(c, Kb, Vb, (int)units, b, S, z, fmap, W, hkv));
 }
 
 int bha_hybrid_step(const void* Qa, const void* Ka, const void* Va, const float* S,
                     const float* z, void* Y, int n, int hq, int hkv, int b, int d, float scale,
                     unsigned flags, bha_dtype dtype, bha_stream_t stream) {
+  return bha_hybrid_step_fm(Qa, Ka, Va, S, z, Y, n, hq, hkv, b, d, scale, flags, dtype,
+                            BHA_FMAP_RELU, nullptr, stream);
+}
+
+int bha_hybrid_step_fm(const void* Qa, const void* Ka, const void* Va, const float* S,
+                       const float* z, void* Y, int n, int hq, int hkv, int b, int d, float scale,
+                       unsigned flags, bha_dtype dtype, bha_fmap fmap, const void* W,
+                       bha_stream_t stream) {
   int st = check_dims(dtype, d, b);
+  if (st != BHA_OK) return st;
+  st = check_fmap(fmap, W);
   if (st != BHA_OK) return st;
   if (n < 0 || hq < 1 || hkv < 1 || hq % hkv != 0) return BHA_ERR_INVALID_ARG;
   if ((flags & ~BHA_FLAG_SHARED_DENOM) != 0) return BHA_ERR_INVALID_ARG;
@@ -290,9 +336,10 @@ int bha_hybrid_step(const void* Qa, const void* Ka, const void* Va, const float*
   const size_t kv_bytes = static_cast<size_t>(n) * hkv * b * d * es;
   const size_t s_bytes = static_cast<size_t>(n) * hkv * d * d * 4;
   const size_t z_bytes = static_cast<size_t>(n) * hkv * d * 4;
+  const size_t wb = w_bytes(W, hkv, d, dtype);
   if (overlap(Y, q_bytes, Qa, q_bytes) || overlap(Y, q_bytes, Ka, kv_bytes) ||
       overlap(Y, q_bytes, Va, kv_bytes) || overlap(Y, q_bytes, S, s_bytes) ||
-      (shared && overlap(Y, q_bytes, z, z_bytes)))
+      (shared && overlap(Y, q_bytes, z, z_bytes)) || overlap(Y, q_bytes, W, wb))
     return BHA_ERR_INVALID_ARG;
   Ctx c;
   st = make_ctx(stream, dtype, &c);
@@ -302,15 +349,25 @@ int bha_hybrid_step(const void* Qa, const void* Ka, const void* Va, const float*
     return launch_status(launch_step_f32(
         c, static_cast<const float*>(Qa), static_cast<const float*>(Ka),
         static_cast<const float*>(Va), S, shared ? z : nullptr, static_cast<float*>(Y), n, hq,
-        hkv, b, d, sc, shared));
-  return launch_status(
-      launch_step_bf16(c, Qa, Ka, Va, S, shared ? z : nullptr, Y, n, hq, hkv, b, sc, shared));
+        hkv, b, d, sc, shared, fmap, static_cast<const float*>(W)));
+  return launch_status(launch_step_bf16(c, Qa, Ka, Va, S, shared ? z : nullptr, Y, n, hq, hkv, b,
+                                        sc, shared, fmap, W));
 }
 
 int bha_hybrid_step_commit(const void* Qa, const void* Ka, const void* Va, float* S, float* z,
                            void* Y, int n, int hq, int hkv, int b, int d, float scale,
                            unsigned flags, bha_dtype dtype, bha_stream_t stream) {
+  return bha_hybrid_step_commit_fm(Qa, Ka, Va, S, z, Y, n, hq, hkv, b, d, scale, flags, dtype,
+                                   BHA_FMAP_RELU, nullptr, stream);
+}
+
+int bha_hybrid_step_commit_fm(const void* Qa, const void* Ka, const void* Va, float* S,
+                              float* z, void* Y, int n, int hq, int hkv, int b, int d,
+                              float scale, unsigned flags, bha_dtype dtype, bha_fmap fmap,
+                              const void* W, bha_stream_t stream) {
   int st = check_dims(dtype, d, b);
+  if (st != BHA_OK) return st;
+  st = check_fmap(fmap, W);
   if (st != BHA_OK) return st;
   if (n < 0 || hq < 1 || hkv < 1 || hq % hkv != 0) return BHA_ERR_INVALID_ARG;
   if ((flags & ~BHA_FLAG_SHARED_DENOM) != 0) return BHA_ERR_INVALID_ARG;
@@ -334,27 +391,34 @@ int bha_hybrid_step_commit(const void* Qa, const void* Ka, const void* Va, float
       overlap(z, z_bytes, Qa, q_bytes) || overlap(z, z_bytes, Ka, kv_bytes) ||
       overlap(z, z_bytes, Va, kv_bytes) || overlap(z, z_bytes, S, s_bytes))
     return BHA_ERR_INVALID_ARG;
+  const size_t wb = w_bytes(W, hkv, d, dtype);
+  if (overlap(W, wb, Y, q_bytes) || overlap(W, wb, S, s_bytes) || overlap(W, wb, z, z_bytes))
+    return BHA_ERR_INVALID_ARG;
   Ctx c;
   st = make_ctx(stream, dtype, &c);
   if (st != BHA_OK) return st;
   const float sc = resolve_scale(scale, d);
   const int units = n * hkv;
   if (dtype == BHA_F32) {
+    const float* Wf = static_cast<const float*>(W);
     st = launch_status(launch_step_f32(
         c, static_cast<const float*>(Qa), static_cast<const float*>(Ka),
         static_cast<const float*>(Va), S, shared ? z : nullptr, static_cast<float*>(Y), n, hq,
-        hkv, b, d, sc, shared));
+        hkv, b, d, sc, shared, fmap, Wf));
     if (st != BHA_OK) return st;
     return launch_status(launch_commit_f32(c, static_cast<const float*>(Ka),
-                                           static_cast<const float*>(Va), units, b, d, S, z));
+                                           static_cast<const float*>(Va), units, b, d, S, z,
+                                           fmap, Wf, hkv));
   }
-  if (!shared && (hq / hkv) * b <= 128)   // one kernel: step, then fold the block in
+  // one kernel (step, then fold the block in) in the default mode with one
+  // 128-row tile per unit and an elementwise map
+  if (!shared && (hq / hkv) * b <= 128 && fmap != BHA_FMAP_RELU_PROJ)
     return launch_status(
-        launch_step_bf16(c, Qa, Ka, Va, S, nullptr, Y, n, hq, hkv, b, sc, 0, z, 1));
-  st = launch_status(
-      launch_step_bf16(c, Qa, Ka, Va, S, shared ? z : nullptr, Y, n, hq, hkv, b, sc, shared));
+        launch_step_bf16(c, Qa, Ka, Va, S, nullptr, Y, n, hq, hkv, b, sc, 0, fmap, W, z, 1));
+  st = launch_status(launch_step_bf16(c, Qa, Ka, Va, S, shared ? z : nullptr, Y, n, hq, hkv, b,
+                                      sc, shared, fmap, W));
   if (st != BHA_OK) return st;
-  return launch_status(launch_commit_bf16(c, Ka, Va, units, b, S, z));
+  return launch_status(launch_commit_bf16(c, Ka, Va, units, b, S, z, fmap, W, hkv));
 }
 
 size_t bha_prefix_softmax_workspace_size(int n, int hq, int hkv, int b, int d, int P,

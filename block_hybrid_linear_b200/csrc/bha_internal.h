@@ -60,28 +60,32 @@ int launch_pdl(void (*kern)(KArgs...), unsigned grid, unsigned block, size_t sme
 }
 
 // ---- fp32 reference mode (CUDA cores) ----
+// fmap: the bha_fmap value; W: [hkv][d][d] (projected map) or null.
 int launch_step_f32(const Ctx& c, const float* Q, const float* K, const float* V,
                     const float* S, const float* z, float* Y, int n, int hq, int hkv, int b,
-                    int d, float scale, int shared);
+                    int d, float scale, int shared, int fmap, const float* W);
 int launch_commit_f32(const Ctx& c, const float* K, const float* V, int units, int b, int d,
-                      float* S, float* z);
+                      float* S, float* z, int fmap, const float* W, int hkv);
 int launch_prefill_f32(const Ctx& c, const float* K, const float* V, int units, int T, int d,
-                       float* S, float* z);
+                       float* S, float* z, int fmap, const float* W, int hkv);
 int launch_prefix_f32(const Ctx& c, const float* Q, const float* Kc, const float* Vc, int P,
                       int cap, const float* K, const float* V, float* Y, int n, int hq, int hkv,
                       int b, int d, float scale);
 
 // ---- bf16 tensor-core path (tcgen05, d = 128) ----
-// commit != 0 (default mode, G * b <= 128 only): also S += phi(K)^T V and
-// z += sum phi(k) (z = commit_z, may be null) after the step has used S.
+// fmap: the bha_fmap value; W: [hkv][128][128] bf16 (projected map) or null.
+// commit != 0 (default mode, G * b <= 128, elementwise maps only): also
+// S += phi(K)^T V and z += sum phi(k) (z = commit_z, may be null) after the
+// step has used S.
 int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, const float* S,
                      const float* z, void* Y, int n, int hq, int hkv, int b, float scale,
-                     int shared, float* commit_z = nullptr, int commit = 0);
+                     int shared, int fmap, const void* W, float* commit_z = nullptr,
+                     int commit = 0);
 int launch_commit_bf16(const Ctx& c, const void* K, const void* V, int units, int b, float* S,
-                       float* z);
+                       float* z, int fmap, const void* W, int hkv);
 size_t prefill_bf16_workspace(int units, int T);
 int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, int T, float* S,
-                        float* z, void* ws, size_t ws_bytes);
+                        float* z, void* ws, size_t ws_bytes, int fmap, const void* W, int hkv);
 size_t prefix_bf16_workspace(int n, int hq, int hkv, int b, int P);
 int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* Vc, int P,
                        int cap, const void* K, const void* V, void* Y, int n, int hq, int hkv,

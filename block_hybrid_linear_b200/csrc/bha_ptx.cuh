@@ -376,4 +376,50 @@ __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) {
   return lo | hi;
 }
 
+// ---------------------------------------------------------------- feature maps
+// The values match bha_fmap in bha.h.
+constexpr int kFmapRelu = 0;       // phi(x) = max(x, 0)
+constexpr int kFmapElu1 = 1;       // phi(x) = x + 1 (x > 0), exp(x) (x <= 0)
+constexpr int kFmapReluProj = 2;   // phi(x) = max(x W, 0)
+
+// phi of one element for the elementwise maps (the projected map applies
+// the ReLU part of it here, after the projection).
+template <int FMAP>
+__device__ __forceinline__ float phi_elem(float x) {
+  if (FMAP == kFmapElu1) return x > 0.f ? x + 1.f : __expf(x);
+  return fmaxf(x, 0.f);
+}
+
+// fp32 -> the nearest tf32 value (ties away from zero), in an fp32 register:
+// what the tensor core then reads from TMEM loses nothing more.
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// phi of both bf16 lanes of a packed pair, rounded back to bf16 (exact for
+// ReLU, round-to-nearest-even for elu + 1).
+template <int FMAP>
+__device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
+  if (FMAP == kFmapRelu) return relu_bf16x2(x);
+  return pack_bf16x2(phi_elem<FMAP>(__uint_as_float(x << 16)),
+                     phi_elem<FMAP>(__uint_as_float(x & 0xFFFF0000u)));
+}
+
+// Address of 16-byte chunk jj of row r in a K-major bf16 operand tile whose
+// rows are `ROWB` bytes (32, 64 or 128) with the swizzle of that width
+// (8-row groups of 8 * ROWB bytes; the tcgen05 descriptor takes SBO =
+// 8 * ROWB and the layout type of that swizzle).
+template <uint32_t ROWB>
+__device__ __forceinline__ uint32_t kmajor_chunk(uint32_t tile, int r, int jj) {
+  const uint32_t swz = ROWB == 128 ? (r & 7) : ROWB == 64 ? ((r & 7) >> 1) : ((r & 7) >> 2);
+  return tile + (r >> 3) * (8 * ROWB) + (r & 7) * ROWB + ((jj ^ swz) << 4);
+}
+
+template <uint32_t ROWB>
+constexpr uint32_t kmajor_layout() {
+  return ROWB == 32 ? kLayoutSW32 : ROWB == 64 ? kLayoutSW64 : kLayoutSW128;
+}
+
 }  // namespace bha

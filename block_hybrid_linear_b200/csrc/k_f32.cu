@@ -1,7 +1,8 @@
 // fp32 reference-mode kernels (CUDA cores, FFMA): the same operations as the
 // bf16 tensor-core path with fp32 Q/K/V/Y, any d <= 128 (d % 4 == 0) and
 // b <= 64.  Used for the worked example (d = 16) and tight-tolerance checks.
-// Simple one-row-at-a-time structure; not a performance path.
+// Simple one-row-at-a-time structure; not a performance path.  Feature
+// maps: 0 ReLU, 1 elu + 1, 2 ReLU(x W_g) with W [hkv][d][d] fp32.
 #include <cuda_runtime.h>
 #include <math.h>
 
@@ -13,6 +14,18 @@ namespace {
 constexpr int kThreads = 128;
 
 __device__ __forceinline__ float relu(float x) { return x > 0.f ? x : 0.f; }
+
+// Feature r of phi(x) for one d-vector x; Wg = W[g] for the projected map.
+__device__ __forceinline__ float phi_at(const float* x, int r, int d, int fmap, const float* Wg) {
+  if (fmap == 2) {
+    float acc = 0.f;
+    for (int i = 0; i < d; ++i) acc = fmaf(x[i], Wg[(size_t)i * d + r], acc);
+    return relu(acc);
+  }
+  const float v = x[r];
+  if (fmap == 1) return v > 0.f ? v + 1.f : expf(v);
+  return relu(v);
+}
 
 __device__ float block_reduce_max(float v, float* red) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
@@ -38,20 +51,22 @@ __device__ float block_reduce_sum(float v, float* red) {
 
 // One CTA per (request, query head).  Row by row: scores against the b block
 // keys, softmax, then each thread produces one output column
-//   y[c] = sum_j p_j v_j[c] + sum_r relu(q_r) S[r][c]      (default)
-//   y[c] = (sum_j e_j v_j[c] + e^{-m} lin[c]) / (l + e^{-m} relu(q).z)  (shared)
+//   y[c] = sum_j p_j v_j[c] + sum_r phi(q)_r S[r][c]      (default)
+//   y[c] = (sum_j e_j v_j[c] + e^{-m} lin[c]) / (l + e^{-m} phi(q).z)  (shared)
 __global__ void __launch_bounds__(kThreads) k_step_f32(const float* __restrict__ Q,
                                                        const float* __restrict__ K,
                                                        const float* __restrict__ V,
                                                        const float* __restrict__ S,
                                                        const float* __restrict__ z,
                                                        float* __restrict__ Y, int hq, int hkv,
-                                                       int b, int d, float scale, int shared) {
+                                                       int b, int d, float scale, int shared,
+                                                       int fmap, const float* __restrict__ W) {
   extern __shared__ float sm[];
   float* sK = sm;              // [b][d]
   float* sV = sK + b * d;      // [b][d]
   float* sq = sV + b * d;      // [d]
   float* sp = sq + d;          // [b]
+  float* sphi = sp + b;        // [d]  phi(q)
   __shared__ float red[kThreads / 32];
 
   const int nh = blockIdx.x;
@@ -63,12 +78,14 @@ __global__ void __launch_bounds__(kThreads) k_step_f32(const float* __restrict__
   }
   const float* Sg = S + ((size_t)ni * hkv + g) * d * d;
   const float* zg = z ? z + ((size_t)ni * hkv + g) * d : nullptr;
+  const float* Wg = W ? W + (size_t)g * d * d : nullptr;
   __syncthreads();
 
   for (int i = 0; i < b; ++i) {
     const size_t row = (((size_t)ni * hq + h) * b + i) * d;
     for (int c = threadIdx.x; c < d; c += kThreads) sq[c] = Q[row + c];
     __syncthreads();
+    for (int c = threadIdx.x; c < d; c += kThreads) sphi[c] = phi_at(sq, c, d, fmap, Wg);
     float s = -INFINITY;
     if (threadIdx.x < b) {
       float acc = 0.f;
@@ -82,7 +99,7 @@ __global__ void __launch_bounds__(kThreads) k_step_f32(const float* __restrict__
     float qz = 0.f;
     if (shared) {
       float part = 0.f;
-      for (int r = threadIdx.x; r < d; r += kThreads) part = fmaf(relu(sq[r]), zg[r], part);
+      for (int r = threadIdx.x; r < d; r += kThreads) part = fmaf(sphi[r], zg[r], part);
       qz = block_reduce_sum(part, red);
     }
     __syncthreads();
@@ -90,7 +107,7 @@ __global__ void __launch_bounds__(kThreads) k_step_f32(const float* __restrict__
       float soft = 0.f;
       for (int j = 0; j < b; ++j) soft = fmaf(sp[j], sV[j * d + c], soft);
       float lin = 0.f;
-      for (int r = 0; r < d; ++r) lin = fmaf(relu(sq[r]), Sg[(size_t)r * d + c], lin);
+      for (int r = 0; r < d; ++r) lin = fmaf(sphi[r], Sg[(size_t)r * d + c], lin);
       float y;
       if (!shared) {
         y = soft / l + lin;
@@ -104,27 +121,31 @@ __global__ void __launch_bounds__(kThreads) k_step_f32(const float* __restrict__
   }
 }
 
-// S[u][r][c] (+)= sum_t relu(K[u][t][r]) V[u][t][c];  z[u][r] (+)= sum_t relu(K[u][t][r]).
+// S[u][r][c] (+)= sum_t phi(k_t)[r] V[u][t][c];  z[u][r] (+)= sum_t phi(k_t)[r].
 // One thread per (r, c) state element; accumulate != 0 adds to S (commit),
 // otherwise overwrites (prefill).
 __global__ void __launch_bounds__(kThreads) k_state_f32(const float* __restrict__ K,
                                                         const float* __restrict__ V, int T,
                                                         int d, float* __restrict__ S,
-                                                        float* __restrict__ z, int accumulate) {
+                                                        float* __restrict__ z, int accumulate,
+                                                        int fmap, const float* __restrict__ W,
+                                                        int hkv) {
   const int u = blockIdx.y;
   const int e = blockIdx.x * kThreads + threadIdx.x;
   const float* Ku = K + (size_t)u * T * d;
   const float* Vu = V + (size_t)u * T * d;
+  const float* Wg = W ? W + (size_t)(u % hkv) * d * d : nullptr;
   if (e < d * d) {
     const int r = e / d, c = e % d;
     float acc = 0.f;
-    for (int t = 0; t < T; ++t) acc = fmaf(relu(Ku[(size_t)t * d + r]), Vu[(size_t)t * d + c], acc);
+    for (int t = 0; t < T; ++t)
+      acc = fmaf(phi_at(Ku + (size_t)t * d, r, d, fmap, Wg), Vu[(size_t)t * d + c], acc);
     float* dst = S + (size_t)u * d * d + e;
     *dst = accumulate ? *dst + acc : acc;
   }
   if (z && e < d) {
     float acc = 0.f;
-    for (int t = 0; t < T; ++t) acc += relu(Ku[(size_t)t * d + e]);
+    for (int t = 0; t < T; ++t) acc += phi_at(Ku + (size_t)t * d, e, d, fmap, Wg);
     float* dst = z + (size_t)u * d + e;
     *dst = accumulate ? *dst + acc : acc;
   }
@@ -196,26 +217,26 @@ int finish_launch() {
 
 int launch_step_f32(const Ctx& c, const float* Q, const float* K, const float* V,
                     const float* S, const float* z, float* Y, int n, int hq, int hkv, int b,
-                    int d, float scale, int shared) {
-  const size_t smem = (size_t)(2 * b * d + d + b) * sizeof(float);
+                    int d, float scale, int shared, int fmap, const float* W) {
+  const size_t smem = (size_t)(2 * b * d + 2 * d + b) * sizeof(float);
   static std::atomic<uint64_t> prepared{0};
-  if (!prepare_kernel(k_step_f32, 2 * 64 * 128 * 4 + 4 * 128 + 4 * 64, prepared)) return -5;
+  if (!prepare_kernel(k_step_f32, (2 * 64 * 128 + 2 * 128 + 64) * 4, prepared)) return -5;
   k_step_f32<<<n * hq, kThreads, smem, c.stream>>>(Q, K, V, S, z, Y, hq, hkv, b, d, scale,
-                                                   shared);
+                                                   shared, fmap, W);
   return finish_launch();
 }
 
 int launch_commit_f32(const Ctx& c, const float* K, const float* V, int units, int b, int d,
-                      float* S, float* z) {
+                      float* S, float* z, int fmap, const float* W, int hkv) {
   dim3 grid((d * d + kThreads - 1) / kThreads, units);
-  k_state_f32<<<grid, kThreads, 0, c.stream>>>(K, V, b, d, S, z, 1);
+  k_state_f32<<<grid, kThreads, 0, c.stream>>>(K, V, b, d, S, z, 1, fmap, W, hkv);
   return finish_launch();
 }
 
 int launch_prefill_f32(const Ctx& c, const float* K, const float* V, int units, int T, int d,
-                       float* S, float* z) {
+                       float* S, float* z, int fmap, const float* W, int hkv) {
   dim3 grid((d * d + kThreads - 1) / kThreads, units);
-  k_state_f32<<<grid, kThreads, 0, c.stream>>>(K, V, T, d, S, z, 0);
+  k_state_f32<<<grid, kThreads, 0, c.stream>>>(K, V, T, d, S, z, 0, fmap, W, hkv);
   return finish_launch();
 }
 

@@ -19,6 +19,15 @@
 // 64-token K/V tiles (32 KB per stage) feeding the MMA warp; the chunk's
 // partial state goes to the workspace (or straight to S when the prompt is
 // one chunk) and a second kernel adds the chunks in a fixed order.
+//
+// Feature maps (the method details' kernel-function approximation): elu + 1
+// is applied in place like ReLU (computed in fp32, rounded to bf16).  The
+// projected map phi(k) = ReLU(k W_g) takes one more MMA per K tile, the
+// transposed projection (K W_g)^T = W_g^T K^T (M = 128 features, N =
+// tokens, K = 128 inputs; A = W_g MN-major as it sits in memory, B = the K
+// tile K-major), into spare TMEM columns; one thread per feature applies the
+// ReLU, sums z, and writes phi(K)^T over the consumed K tile as a K-major
+// operand for phi(K)^T V.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -69,6 +78,7 @@ struct CommitArgs {
   float* z;   // [units][128] or null
   int* err;
   int b;
+  int hkv;    // unit u uses W[u % hkv] (projected map)
 };
 
 template <int BPAD>
@@ -81,7 +91,7 @@ struct CommitLayout {
   static constexpr uint32_t kSmem = kTiles + 1024;
 };
 
-template <int BPAD>
+template <int BPAD, int FMAP>
 __global__ void __launch_bounds__(kThreads, 2)
     k_commit_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                   const __grid_constant__ CUtensorMap tmS, const CommitArgs a) {
@@ -142,8 +152,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     for (uint32_t v = tid; v < Lay::kKV / 16; v += kThreads) {
       const uint32_t addr = base + Lay::kOffK + v * 16;
       uint4 x = ld_shared_v4(addr);
-      st_shared_v4(addr, relu_bf16x2(x.x), relu_bf16x2(x.y), relu_bf16x2(x.z),
-                   relu_bf16x2(x.w));
+      st_shared_v4(addr, phi_bf16x2<FMAP>(x.x), phi_bf16x2<FMAP>(x.y), phi_bf16x2<FMAP>(x.z),
+                   phi_bf16x2<FMAP>(x.w));
     }
   }
   fence_proxy_async_smem();
@@ -198,6 +208,167 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
+// Commit under the projected map.  TMEM: phi(K)^T V at [0, 128), the
+// projection (K W_g)^T at [128, 128 + BPAD).  Warps 0-3 (thread = feature r
+// = TMEM lane) turn row r of the projection into row r of phi(K)^T.
+template <int BPAD>
+struct CommitProjLayout {
+  static constexpr uint32_t kKV = BPAD * 256;
+  static constexpr uint32_t kOffS = 0;
+  static constexpr uint32_t kOffK = kSBytes;           // K, then phi(K)^T over it
+  static constexpr uint32_t kOffV = kOffK + kKV;
+  static constexpr uint32_t kOffW = kOffV + kKV;
+  static constexpr uint32_t kTiles = kOffW + 32768;
+  static constexpr uint32_t kSmem = kTiles + 1024;
+  static constexpr uint32_t kRowB = 2 * BPAD;          // one phi(K)^T row: BPAD tokens
+};
+
+template <int BPAD>
+__global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
+    k_commit_proj_bf16(const __grid_constant__ CUtensorMap tmK,
+                       const __grid_constant__ CUtensorMap tmV,
+                       const __grid_constant__ CUtensorMap tmS,
+                       const __grid_constant__ CUtensorMap tmW, const CommitArgs a) {
+  using Lay = CommitProjLayout<BPAD>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int u = blockIdx.x, g = u % a.hkv;
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + Lay::kTiles;
+  uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
+  const uint32_t bar_kv = ctrl, bar_s = ctrl + 8, bar_done = ctrl + 16, bar_w = ctrl + 24,
+                 bar_kw = ctrl + 40, bar_phik = ctrl + 48;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 32);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 36);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      mbar_init(bar_kv, 1);
+      mbar_init(bar_s, 1);
+      mbar_init(bar_done, 1);
+      mbar_init(bar_w, 1);
+      mbar_init(bar_kw, 1);
+      mbar_init(bar_phik, 128);
+      *abort_flag = 0;
+      fence_mbar_init();
+      tma_prefetch_l2_3d(&tmK, 0, 0, u);
+      tma_prefetch_l2_3d(&tmK, 64, 0, u);
+      tma_prefetch_l2_3d(&tmV, 0, 0, u);
+      tma_prefetch_l2_3d(&tmV, 64, 0, u);
+#pragma unroll
+      for (int bx = 0; bx < 4; ++bx) tma_prefetch_l2_3d(&tmS, 32 * bx, 0, u);
+      tma_prefetch_l2_3d(&tmW, 0, 0, g);
+      tma_prefetch_l2_3d(&tmW, 64, 0, g);
+    }
+    __syncwarp();
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) pdl_launch_dependents();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t t_kw = tmem + 128;
+  pdl_wait();
+
+  if (tid == 0) {
+    mbar_arrive_expect_tx(bar_kv, 2 * Lay::kKV);
+    tma_load_3d(base + Lay::kOffK, &tmK, bar_kv, 0, 0, u);
+    tma_load_3d(base + Lay::kOffK + BPAD * 128, &tmK, bar_kv, 64, 0, u);
+    tma_load_3d(base + Lay::kOffV, &tmV, bar_kv, 0, 0, u);
+    tma_load_3d(base + Lay::kOffV + BPAD * 128, &tmV, bar_kv, 64, 0, u);
+    mbar_arrive_expect_tx(bar_w, 32768);
+    tma_load_3d(base + Lay::kOffW, &tmW, bar_w, 0, 0, g);
+    tma_load_3d(base + Lay::kOffW + 16384, &tmW, bar_w, 64, 0, g);
+    mbar_arrive_expect_tx(bar_s, kSBytes);
+#pragma unroll
+    for (int bx = 0; bx < 4; ++bx)
+      tma_load_3d(base + Lay::kOffS + bx * 16384, &tmS, bar_s, 32 * bx, 0, u);
+  }
+  if (tid == 128) {
+    // (K W_g)^T[r][t] = sum_i W_g[i][r] K[t][i]: A = W_g MN-major, B = K K-major
+    if (mbar_wait(bar_kv, 0, a.err, abort_flag) && mbar_wait(bar_w, 0, a.err, abort_flag)) {
+      tc_fence_after();
+      constexpr uint32_t idesc = make_idesc_bf16(128, BPAD, 1, 0);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t da = make_sdesc(base + Lay::kOffW + ks * 2048, 16384, 1024, kLayoutSW128);
+        const uint64_t db = make_sdesc(base + Lay::kOffK + (ks >> 2) * (BPAD * 128) + (ks & 3) * 32,
+                                       16, 1024, kLayoutSW128);
+        mma_bf16_ss(t_kw, da, db, idesc, ks > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_kw);
+    }
+  }
+  if (warp < 4) {
+    // thread = feature r: ReLU, bf16, z, row r of phi(K)^T over the consumed K
+    const int r = tid;
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const bool okk = warp_all(mbar_wait(bar_kw, 0, a.err, abort_flag));
+    tc_fence_after();
+    if (okk) {
+      float zs = 0.f;
+#pragma unroll
+      for (int j0 = 0; j0 < BPAD; j0 += 16) {
+        float f[16];
+        tmem_ld16_sync(t_kw + lane_base + j0, f);
+        uint32_t w[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          w[q] = pack_bf16x2(fmaxf(f[2 * q], 0.f), fmaxf(f[2 * q + 1], 0.f));
+          // padded tokens are zero rows of K, so their features are 0
+          zs += __uint_as_float(w[q] << 16) + __uint_as_float(w[q] & 0xFFFF0000u);
+        }
+        st_shared_v4(kmajor_chunk<Lay::kRowB>(base + Lay::kOffK, r, j0 / 8), w[0], w[1], w[2], w[3]);
+        st_shared_v4(kmajor_chunk<Lay::kRowB>(base + Lay::kOffK, r, j0 / 8 + 1), w[4], w[5], w[6],
+                     w[7]);
+      }
+      if (a.z != nullptr) a.z[static_cast<size_t>(u) * kD + r] += zs;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    mbar_arrive(bar_phik);
+  }
+  if (tid == 128 && !*abort_flag) {
+    // D[r][c] = sum_t phi(K)^T[r][t] V[t][c]: A K-major, B = V MN-major
+    if (mbar_wait(bar_phik, 0, a.err, abort_flag)) {
+      tc_fence_after();
+      constexpr uint32_t idesc = make_idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+      for (int ks = 0; ks < BPAD / 16; ++ks) {
+        const uint64_t da = make_sdesc(base + Lay::kOffK + ks * 32, 16, 8 * Lay::kRowB,
+                                       kmajor_layout<Lay::kRowB>());
+        const uint64_t db = make_sdesc(base + Lay::kOffV + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
+        mma_bf16_ss(tmem, da, db, idesc, ks > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_done);
+    }
+  }
+
+  const bool ok =
+      warp_all(mbar_wait(bar_s, 0, a.err, abort_flag) && mbar_wait(bar_done, 0, a.err, abort_flag));
+  tc_fence_after();
+  if (ok) accum_to_tile(tmem, base + Lay::kOffS, warp, lane, true);
+  fence_proxy_async_smem();
+  tc_fence_before();
+  const int hb = warp >> 2;
+  named_barrier_sync(1 + hb, 128);
+  if ((tid & 127) == 0 && !*abort_flag) {
+    tma_store_3d(&tmS, base + Lay::kOffS + (2 * hb) * 16384, 64 * hb, 0, u);
+    tma_store_3d(&tmS, base + Lay::kOffS + (2 * hb + 1) * 16384, 64 * hb + 32, 0, u);
+    bulk_commit_group();
+    bulk_wait_group_read0();
+  }
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
 // ------------------------------------------------------------------ prefill
 
 constexpr int kTok = 64;                  // tokens per pipeline stage
@@ -215,8 +386,10 @@ struct PrefillArgs {
   int T;             // prompt tokens
   int splits;        // chunks per unit
   int tiles_per;     // 64-token tiles per chunk
+  int hkv;           // unit u uses W[u % hkv] (projected map)
 };
 
+template <int FMAP>
 __global__ void __launch_bounds__(kThreads, 2)
     k_prefill_bf16(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                    const __grid_constant__ CUtensorMap tmOut, const PrefillArgs a) {
@@ -307,15 +480,18 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int st = i % kStages;
       if (!mbar_wait(bar_full + 8 * st, (i / kStages) & 1, a.err, abort_flag)) break;
       const uint32_t kt = base + st * kStageBytes + box * 8192;
+      const int tvalid = a.T - (tile0 + i) * kTok;   // rows past the prompt are zero-filled
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const int t = tsub + 8 * k;
         const uint32_t addr = kt + t * 128 + ((j ^ (t & 7)) << 4);
         uint4 x = ld_shared_v4(addr);
-        x.x = relu_bf16x2(x.x);
-        x.y = relu_bf16x2(x.y);
-        x.z = relu_bf16x2(x.z);
-        x.w = relu_bf16x2(x.w);
+        x.x = phi_bf16x2<FMAP>(x.x);
+        x.y = phi_bf16x2<FMAP>(x.y);
+        x.z = phi_bf16x2<FMAP>(x.z);
+        x.w = phi_bf16x2<FMAP>(x.w);
+        // ReLU keeps them zero; elu + 1 would make them 1: clear them
+        if (FMAP != kFmapRelu && t >= tvalid) x = make_uint4(0u, 0u, 0u, 0u);
         st_shared_v4(addr, x.x, x.y, x.z, x.w);
         const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -365,6 +541,175 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(tmem, 128);
+  }
+}
+
+// Prefill under the projected map: a 2-stage ring (W_g takes the third
+// stage's room, keeping two CTAs per SM).  Per tile i: the MMA thread issues
+// (K W_g)^T into TMEM buffer i % 2 (columns 128 + 64 (i % 2)), then phi(K)^T
+// V of tile i - 1 once its features are written; warps 4-7 (thread =
+// feature r) read buffer i % 2, apply the ReLU, add to z and write row r of
+// phi(K)^T over the consumed K tile (K-major SW128, 64 tokens = 128 B).
+constexpr int kProjStages = 2;
+constexpr uint32_t kPrefProjOffW = kProjStages * kStageBytes;    // 64 KB (= epilogue tile)
+constexpr uint32_t kPrefProjTiles = kPrefProjOffW + 32768;
+constexpr uint32_t kPrefProjSmem = kPrefProjTiles + 1024;
+
+__global__ void __launch_bounds__(kThreads, 2)
+    k_prefill_proj_bf16(const __grid_constant__ CUtensorMap tmK,
+                        const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmOut,
+                        const __grid_constant__ CUtensorMap tmW, const PrefillArgs a) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int item = blockIdx.x;                // = u * splits + s
+  const int u = item / a.splits, sp = item % a.splits;
+  const int g = u % a.hkv;
+  const int ntiles_total = (a.T + kTok - 1) / kTok;
+  const int tile0 = sp * a.tiles_per;
+  const int ntile = min(a.tiles_per, ntiles_total - tile0);
+
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + kPrefProjTiles;
+  uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
+  const uint32_t bar_full = ctrl, bar_relu = ctrl + 16, bar_empty = ctrl + 32,
+                 bar_kw = ctrl + 48, bar_w = ctrl + 64, bar_done = ctrl + 72;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 80);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 84);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int s = 0; s < kProjStages; ++s) {
+        mbar_init(bar_full + 8 * s, 1);
+        mbar_init(bar_relu + 8 * s, 128);
+        mbar_init(bar_empty + 8 * s, 1);
+        mbar_init(bar_kw + 8 * s, 1);
+      }
+      mbar_init(bar_w, 1);
+      mbar_init(bar_done, 1);
+      *abort_flag = 0;
+      fence_mbar_init();
+    }
+    __syncwarp();
+    tmem_alloc(smem_u32(tmem_slot), 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) pdl_launch_dependents();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  pdl_wait();
+
+  float zacc = 0.f;
+  if (tid == 0) {
+    // producer: W_g once, then the K / V tiles
+    mbar_arrive_expect_tx(bar_w, 32768);
+    tma_load_3d(base + kPrefProjOffW, &tmW, bar_w, 0, 0, g);
+    tma_load_3d(base + kPrefProjOffW + 16384, &tmW, bar_w, 64, 0, g);
+    for (int i = 0; i < ntile; ++i) {
+      const int st = i % kProjStages;
+      if (i >= kProjStages &&
+          !mbar_wait(bar_empty + 8 * st, ((i / kProjStages) - 1) & 1, a.err, abort_flag))
+        break;
+      const uint32_t sbase = base + st * kStageBytes;
+      const uint32_t bf = bar_full + 8 * st;
+      const int t0 = (tile0 + i) * kTok;
+      mbar_arrive_expect_tx(bf, kStageBytes);
+      tma_load_3d(sbase, &tmK, bf, 0, t0, u);
+      tma_load_3d(sbase + 8192, &tmK, bf, 64, t0, u);
+      tma_load_3d(sbase + 16384, &tmV, bf, 0, t0, u);
+      tma_load_3d(sbase + 24576, &tmV, bf, 64, t0, u);
+    }
+  } else if (tid == 32) {
+    constexpr uint32_t id_kw = make_idesc_bf16(128, kTok, 1, 0);
+    constexpr uint32_t id_sv = make_idesc_bf16(128, 128, 0, 1);
+    // phi(K)^T V of tile j (stage j % 2) into the accumulator
+    auto issue_sv = [&](int j) -> bool {
+      const int sj = j % kProjStages;
+      if (!mbar_wait(bar_relu + 8 * sj, (j / kProjStages) & 1, a.err, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sb = base + sj * kStageBytes;
+#pragma unroll
+      for (int ks = 0; ks < kTok / 16; ++ks) {
+        const uint64_t da = make_sdesc(sb + ks * 32, 16, 1024, kLayoutSW128);
+        const uint64_t db = make_sdesc(sb + 16384 + ks * 2048, 8192, 1024, kLayoutSW128);
+        mma_bf16_ss(tmem, da, db, id_sv, (j | ks) ? 1u : 0u);
+      }
+      mma_commit(bar_empty + 8 * sj);
+      return true;
+    };
+    bool ok = mbar_wait(bar_w, 0, a.err, abort_flag);
+    for (int i = 0; i < ntile && ok; ++i) {
+      const int st = i % kProjStages;
+      ok = mbar_wait(bar_full + 8 * st, (i / kProjStages) & 1, a.err, abort_flag);
+      if (!ok) break;
+      tc_fence_after();
+      // (K W_g)^T of tile i: buffer st was last read for tile i - 2, whose
+      // features were waited for in the previous iteration
+      const uint32_t sbase = base + st * kStageBytes;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t da = make_sdesc(base + kPrefProjOffW + ks * 2048, 16384, 1024, kLayoutSW128);
+        const uint64_t db =
+            make_sdesc(sbase + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128);
+        mma_bf16_ss(tmem + 128 + 64 * st, da, db, id_kw, ks > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_kw + 8 * st);
+      if (i >= 1) ok = issue_sv(i - 1);
+    }
+    if (ok && ntile >= 1) ok = issue_sv(ntile - 1);
+    if (ok) mma_commit(bar_done);
+  } else if (warp >= 4) {
+    const int r = tid - 128;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    for (int i = 0; i < ntile; ++i) {
+      const int st = i % kProjStages;
+      if (!warp_all(mbar_wait(bar_kw + 8 * st, (i / kProjStages) & 1, a.err, abort_flag))) break;
+      tc_fence_after();
+      const uint32_t kt = base + st * kStageBytes;   // phi(K)^T over the consumed K tile
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float f[32];
+        tmem_ld32_sync(tmem + 128 + 64 * st + lane_base + 32 * h, f);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t w[4];
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            // tokens past the prompt are zero rows of K: their features are 0
+            w[q] = pack_bf16x2(fmaxf(f[8 * c + 2 * q], 0.f), fmaxf(f[8 * c + 2 * q + 1], 0.f));
+            zacc += __uint_as_float(w[q] << 16) + __uint_as_float(w[q] & 0xFFFF0000u);
+          }
+          st_shared_v4(kmajor_chunk<128>(kt, r, 4 * h + c), w[0], w[1], w[2], w[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar_relu + 8 * st);
+    }
+  }
+
+  // ---- epilogue: accumulator -> fp32 tile (over the two stages) -> TMA store
+  __syncwarp();
+  const bool ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag));
+  tc_fence_after();
+  if (ok) accum_to_tile(tmem, base, warp, lane, false);
+  fence_proxy_async_smem();
+  if (warp >= 4 && a.zdst != nullptr && ok) a.zdst[static_cast<size_t>(item) * kD + (tid - 128)] = zacc;
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && !*abort_flag) {
+#pragma unroll
+    for (int bx = 0; bx < 4; ++bx) tma_store_3d(&tmOut, base + bx * 16384, 32 * bx, 0, item);
+    bulk_commit_group();
+    bulk_wait_group_read0();
+  }
+  __syncwarp();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -439,30 +784,63 @@ bool tokens_tmap(CUtensorMap* m, const void* X, int T, int units, uint32_t box_r
                      CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+bool weights_tmap(CUtensorMap* m, const void* W, int hkv) {
+  const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)kD, (uint64_t)hkv};
+  const uint64_t strides[2] = {kD * 2ull, (uint64_t)kD * kD * 2ull};
+  const uint32_t box[3] = {64, (uint32_t)kD, 1};
+  return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, W, dims, strides, box,
+                     CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int BPAD, int FMAP>
+int launch_commit_cfg(const Ctx& c, const CUtensorMap& tk, const CUtensorMap& tv,
+                      const CUtensorMap& ts, const CUtensorMap& tw, const CommitArgs& a,
+                      int units) {
+  if constexpr (FMAP == kFmapReluProj) {
+    using Lay = CommitProjLayout<BPAD>;
+    auto kern = k_commit_proj_bf16<BPAD>;
+    static std::atomic<uint64_t> prepared{0};
+    if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
+    return launch_pdl(kern, units, kThreads, Lay::kSmem, c.stream, tk, tv, ts, tw, a);
+  } else {
+    using Lay = CommitLayout<BPAD>;
+    auto kern = k_commit_bf16<BPAD, FMAP>;
+    static std::atomic<uint64_t> prepared{0};
+    if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
+    return launch_pdl(kern, units, kThreads, Lay::kSmem, c.stream, tk, tv, ts, a);
+  }
+}
+
 template <int BPAD>
 int launch_commit_bpad(const Ctx& c, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& ts, const CommitArgs& a, int units) {
-  using Lay = CommitLayout<BPAD>;
-  auto kern = k_commit_bf16<BPAD>;
-  static std::atomic<uint64_t> prepared{0};
-  if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
-  return launch_pdl(kern, units, kThreads, Lay::kSmem, c.stream, tk, tv, ts, a);
+                       const CUtensorMap& ts, const CUtensorMap& tw, const CommitArgs& a,
+                       int units, int fmap) {
+  switch (fmap) {
+    case kFmapRelu: return launch_commit_cfg<BPAD, kFmapRelu>(c, tk, tv, ts, tw, a, units);
+    case kFmapElu1: return launch_commit_cfg<BPAD, kFmapElu1>(c, tk, tv, ts, tw, a, units);
+    default: return launch_commit_cfg<BPAD, kFmapReluProj>(c, tk, tv, ts, tw, a, units);
+  }
 }
 
 }  // namespace
 
 int launch_commit_bf16(const Ctx& c, const void* K, const void* V, int units, int b, float* S,
-                       float* z) {
+                       float* z, int fmap, const void* W, int hkv) {
   const int bpad = b <= 16 ? 16 : (b <= 32 ? 32 : 64);
-  CUtensorMap tk, tv, ts;
+  CUtensorMap tk, tv, ts, tw;
   if (!tokens_tmap(&tk, K, b, units, bpad) || !tokens_tmap(&tv, V, b, units, bpad) ||
       !state_tmap(&ts, S, units))
     return -5;
-  CommitArgs a{z, c.dev_err, b};
+  if (fmap == kFmapReluProj) {
+    if (!weights_tmap(&tw, W, hkv)) return -5;
+  } else {
+    tw = tk;
+  }
+  CommitArgs a{z, c.dev_err, b, hkv};
   switch (bpad) {
-    case 16: return launch_commit_bpad<16>(c, tk, tv, ts, a, units);
-    case 32: return launch_commit_bpad<32>(c, tk, tv, ts, a, units);
-    default: return launch_commit_bpad<64>(c, tk, tv, ts, a, units);
+    case 16: return launch_commit_bpad<16>(c, tk, tv, ts, tw, a, units, fmap);
+    case 32: return launch_commit_bpad<32>(c, tk, tv, ts, tw, a, units, fmap);
+    default: return launch_commit_bpad<64>(c, tk, tv, ts, tw, a, units, fmap);
   }
 }
 
@@ -475,7 +853,7 @@ size_t prefill_bf16_workspace(int units, int T) {
 }
 
 int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, int T, float* S,
-                        float* z, void* ws, size_t ws_bytes) {
+                        float* z, void* ws, size_t ws_bytes, int fmap, const void* W, int hkv) {
   if (T == 0) {
     if (cudaMemsetAsync(S, 0, static_cast<size_t>(units) * kD * kD * 4, c.stream) != cudaSuccess)
       return -5;
@@ -497,11 +875,27 @@ int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, i
   if (!tokens_tmap(&tk, K, T, units, kTok) || !tokens_tmap(&tv, V, T, units, kTok) ||
       !state_tmap(&to, outS, static_cast<uint64_t>(units) * splits))
     return -5;
-  PrefillArgs a{outZ, c.dev_err, T, splits, tp};
-  static std::atomic<uint64_t> prepared{0};
-  if (!prepare_kernel(k_prefill_bf16, (int)kPrefSmem, prepared)) return -5;
-  if (launch_pdl(k_prefill_bf16, units * splits, kThreads, kPrefSmem, c.stream, tk, tv, to, a))
-    return -5;
+  PrefillArgs a{outZ, c.dev_err, T, splits, tp, hkv};
+  int rc;
+  if (fmap == kFmapReluProj) {
+    CUtensorMap tw;
+    if (!weights_tmap(&tw, W, hkv)) return -5;
+    static std::atomic<uint64_t> prepared_p{0};
+    if (!prepare_kernel(k_prefill_proj_bf16, (int)kPrefProjSmem, prepared_p)) return -5;
+    rc = launch_pdl(k_prefill_proj_bf16, units * splits, kThreads, kPrefProjSmem, c.stream, tk, tv,
+                    to, tw, a);
+  } else if (fmap == kFmapElu1) {
+    static std::atomic<uint64_t> prepared_e{0};
+    if (!prepare_kernel(k_prefill_bf16<kFmapElu1>, (int)kPrefSmem, prepared_e)) return -5;
+    rc = launch_pdl(k_prefill_bf16<kFmapElu1>, units * splits, kThreads, kPrefSmem, c.stream, tk,
+                    tv, to, a);
+  } else {
+    static std::atomic<uint64_t> prepared_r{0};
+    if (!prepare_kernel(k_prefill_bf16<kFmapRelu>, (int)kPrefSmem, prepared_r)) return -5;
+    rc = launch_pdl(k_prefill_bf16<kFmapRelu>, units * splits, kThreads, kPrefSmem, c.stream, tk,
+                    tv, to, a);
+  }
+  if (rc) return -5;
   if (splits > 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((kD * kD / 4 + 255) / 256, units);

@@ -3,7 +3,9 @@
 // One denoising step of block-hybrid attention ("Retrofitting Linear
 // Attention into Diffusion Language Models", core formula; worked example,
 // blocks 2 and 3):
-//     y_i = sum_j softmax_j(scale q_i . k_j) v_j + phi(q_i) S,   phi = ReLU.
+//     y_i = sum_j softmax_j(scale q_i . k_j) v_j + phi(q_i) S,   phi = ReLU
+// (the worked example's map), elu + 1, or ReLU after a per-KV-head d x d
+// projection W_g (the method details' kernel-function approximation).
 //
 // One CTA per (request n, KV head g, 128-row tile of the G*b query rows that
 // share g).  Every operand of the unit is requested by TMA at once (Q, K, V
@@ -28,6 +30,13 @@
 // in flight from the start.  Launched with programmatic dependent launch: the
 // prologue, including L2 prefetches of all operands, overlaps the previous
 // kernel's tail.
+//
+// Projected map phi(q) = ReLU(q W_g): one more MMA (bf16) Q W_g -> TMEM,
+// M=128 N=128 K=128, into the columns phi(Q) occupies, then ReLU and tf32
+// rounding in TMEM.  W_g (32 KB, from L2: every unit of KV head g reads the
+// same W_g) lands where state chunks 2-3 go; those two chunks are loaded
+// once the Q W_g product has read it, so shared memory and the two CTAs per
+// SM stay as they are.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -46,12 +55,14 @@ constexpr uint32_t kSBytes = kD * kD * 4;    // 64 KB
 constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffS = kQBytes;
 constexpr uint32_t kOffK = kQBytes + kSBytes;
+constexpr uint32_t kOffW = kOffS + kSBytes / 2;   // projected map: over state chunks 2-3
 constexpr uint32_t kCtrlBytes = 128;
 
 struct StepArgs {
   const float* z;     // [units][128] (shared mode)
   float* zc;          // [units][128] updated by the fused commit, or null
   int* err;           // device error word
+  int hkv;            // KV heads (unit u uses W[u % hkv])
   int rows;           // G * b query rows per unit
   int b;              // active block length
   int mtiles;         // ceil(rows / 128)
@@ -74,7 +85,15 @@ __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu
 
 // phi(q_r) * scale as fp32 into TMEM (this thread's lane, columns [0, 128)
 // from `tcol`), read from row r of the SW128 Q tile; one wait for all four
-// 32-column stores.
+// 32-column stores.  Elementwise maps only.  Values are rounded to the
+// nearest tf32 unless they are tf32 already (ReLU of a bf16 value, unscaled).
+template <int FMAP, bool SCALED>
+__device__ __forceinline__ float phiq_tf32(float x, float scale) {
+  const float v = phi_elem<FMAP>(x) * scale;
+  return (FMAP == kFmapRelu && !SCALED) ? v : round_tf32(v);
+}
+
+template <int FMAP, bool SCALED>
 __device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol, float scale) {
 #pragma unroll
   for (int cg = 0; cg < 4; ++cg) {
@@ -86,8 +105,9 @@ __device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol,
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        f[8 * q + 2 * e] = fmaxf(__uint_as_float(w4[e] << 16), 0.f) * scale;
-        f[8 * q + 2 * e + 1] = fmaxf(__uint_as_float(w4[e] & 0xFFFF0000u), 0.f) * scale;
+        f[8 * q + 2 * e] = phiq_tf32<FMAP, SCALED>(__uint_as_float(w4[e] << 16), scale);
+        f[8 * q + 2 * e + 1] =
+            phiq_tf32<FMAP, SCALED>(__uint_as_float(w4[e] & 0xFFFF0000u), scale);
       }
     }
     tmem_st32(tcol + cg * 32, f);
@@ -95,18 +115,55 @@ __device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol,
   tmem_wait_st();
 }
 
+// Projected map: the Q W_g product sits in TMEM (this thread's lane, 128
+// columns from `tcol`); replace it by round_tf32(max(., 0) * scale).
+__device__ __forceinline__ void relu_tmem_phiq(uint32_t tcol, float scale) {
+#pragma unroll
+  for (int cg = 0; cg < 4; ++cg) {
+    float f[32];
+    tmem_ld32_sync(tcol + cg * 32, f);
+#pragma unroll
+    for (int q = 0; q < 32; ++q) f[q] = round_tf32(fmaxf(f[q], 0.f) * scale);
+    tmem_st32(tcol + cg * 32, f);
+  }
+  tmem_wait_st();
+}
+
+// Projected map, shared denominator: phi(q_r) . z_g from the Q W_g product
+// in TMEM.
+__device__ __forceinline__ float proj_qz(uint32_t tcol, const float* zu) {
+  float qz = 0.f;
+#pragma unroll
+  for (int cg = 0; cg < 4; ++cg) {
+    float f[32];
+    tmem_ld32_sync(tcol + cg * 32, f);
+#pragma unroll
+    for (int q = 0; q < 32; q += 4) {
+      const float4 zz = __ldg(reinterpret_cast<const float4*>(zu + cg * 32 + q));
+      qz = fmaf(round_tf32(fmaxf(f[q], 0.f)), zz.x, qz);
+      qz = fmaf(round_tf32(fmaxf(f[q + 1], 0.f)), zz.y, qz);
+      qz = fmaf(round_tf32(fmaxf(f[q + 2], 0.f)), zz.z, qz);
+      qz = fmaf(round_tf32(fmaxf(f[q + 3], 0.f)), zz.w, qz);
+    }
+  }
+  return qz;
+}
+
 // COMMIT: also fold this step's block into the state after using it (the
 // block's last denoising step): S += phi(K)^T V, z += sum_t phi(k_t), with
 // the state tile already in shared memory updated in place and stored back.
 // P then lives in the consumed Q tile so that K survives for the commit MMA,
 // and phi(K)^T V accumulates in the TMEM columns phi(Q) used.  Default mode
-// and a single 128-row tile per unit only.
-template <int BPAD, bool SHARED, bool COMMIT>
+// and a single 128-row tile per unit only; elementwise maps only.
+template <int BPAD, bool SHARED, bool COMMIT, int FMAP>
 __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     k_step_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
-                const __grid_constant__ CUtensorMap tmY, const StepArgs a) {
+                const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmW,
+                const StepArgs a) {
   static_assert(!(SHARED && COMMIT), "the fused commit runs in the default mode only");
+  static_assert(!(COMMIT && FMAP == kFmapReluProj), "the fused commit has no projected map");
+  constexpr bool PROJ = FMAP == kFmapReluProj;
   using Lay = StepLayout<BPAD>;
   // P (the softmax weights, bf16, K-major) goes over the consumed K tile, or
   // over the consumed Q tile when K is still needed by the commit
@@ -115,6 +172,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int u = blockIdx.x / a.mtiles, mt = blockIdx.x % a.mtiles;
+  const int g = u % a.hkv;
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -122,7 +180,8 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
   const uint32_t bar_q = ctrl, bar_k = ctrl + 8, bar_v = ctrl + 16, bar_s = ctrl + 24,
                  bar_sc = ctrl + 56, bar_p = ctrl + 64, bar_a = ctrl + 72, bar_done = ctrl + 80,
-                 bar_phik = ctrl + 96, bar_ds = ctrl + 104;
+                 bar_phik = ctrl + 96, bar_ds = ctrl + 104, bar_w = ctrl + 112,
+                 bar_qw = ctrl + 120;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 88);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 92);
 
@@ -140,6 +199,10 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         mbar_init(bar_phik, 128);
         mbar_init(bar_ds, 1);
       }
+      if (PROJ) {
+        mbar_init(bar_w, 1);
+        mbar_init(bar_qw, 1);
+      }
       *abort_flag = 0;
       fence_mbar_init();
       tma_prefetch_desc(&tmY);
@@ -154,6 +217,10 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       tma_prefetch_l2_3d(&tmV, 64, 0, u);
       for (int c = 0; c < 4; ++c)
         for (int nb = 0; nb < 4; ++nb) tma_prefetch_l2_3d(&tmS, 32 * nb, 32 * c, u);
+      if (PROJ) {
+        tma_prefetch_l2_3d(&tmW, 0, 0, g);
+        tma_prefetch_l2_3d(&tmW, 64, 0, g);
+      }
     }
     __syncwarp();
     tmem_alloc(smem_u32(tmem_slot), 256);
@@ -169,8 +236,9 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   // Scores: in the default mode they sit in the accumulator's first columns
   // (P V overwrites them once read) so phi(Q) can be built in parallel; with
   // the shared denominator phi(Q) needs the row max first, so the scores sit
-  // where phi(Q) will go.
-  const uint32_t t_sc = SHARED ? t_a : t_d;
+  // where phi(Q) will go -- except under the projected map, whose Q W_g
+  // product needs those columns from the start.
+  const uint32_t t_sc = (SHARED && !PROJ) ? t_a : t_d;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   pdl_wait();   // inputs may come from the previous kernel of the stream
 
@@ -186,8 +254,14 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     mbar_arrive_expect_tx(bar_v, Lay::kKV);
     tma_load_3d(base + Lay::kOffV, &tmV, bar_v, 0, 0, u);
     tma_load_3d(base + Lay::kOffV + BPAD * 128, &tmV, bar_v, 64, 0, u);
+    if (PROJ) {
+      mbar_arrive_expect_tx(bar_w, 2 * 16384);
+      tma_load_3d(base + kOffW, &tmW, bar_w, 0, 0, g);
+      tma_load_3d(base + kOffW + 16384, &tmW, bar_w, 64, 0, g);
+    }
     // chunk c = state rows 32c..32c+31; box (c, nb) = its columns 32nb..32nb+31
-    for (int c = 0; c < 4; ++c) {
+    // (the projected map loads chunks 2-3 later, over W_g)
+    for (int c = 0; c < (PROJ ? 2 : 4); ++c) {
       mbar_arrive_expect_tx(bar_s + 8 * c, 16384);
 #pragma unroll
       for (int nb = 0; nb < 4; ++nb)
@@ -196,12 +270,33 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     }
   }
 
+  // projected map: state chunks 2-3 over W_g once the Q W_g product is done
+  auto load_late_chunks = [&]() {
+    for (int c = 2; c < 4; ++c) {
+      mbar_arrive_expect_tx(bar_s + 8 * c, 16384);
+#pragma unroll
+      for (int nb = 0; nb < 4; ++nb)
+        tma_load_3d(base + kOffS + c * 16384 + nb * 4096, &tmS, bar_s + 8 * c, 32 * nb, 32 * c,
+                    u);
+    }
+  };
+  if (PROJ && SHARED && tid == 0) {
+    if (mbar_wait(bar_qw, 0, a.err, abort_flag)) load_late_chunks();
+  }
+
   float beta = 1.f;   // per-row output scale (shared denominator only)
   if (!SHARED && warp < 4) {
     // phi(q) for row r = 32 w + lane into TMEM as soon as Q has landed, in
     // parallel with the score MMA and the softmax
-    const bool okq = warp_all(mbar_wait(bar_q, 0, a.err, abort_flag));
-    if (okq) write_phiq(base + kOffQ, warp * 32 + lane, t_a + lane_base, 1.f);
+    if (PROJ) {
+      const bool okw = warp_all(mbar_wait(bar_qw, 0, a.err, abort_flag));
+      tc_fence_after();
+      if (okw && tid == 0) load_late_chunks();
+      if (okw) relu_tmem_phiq(t_a + lane_base, 1.f);
+    } else {
+      const bool okq = warp_all(mbar_wait(bar_q, 0, a.err, abort_flag));
+      if (okq) write_phiq<FMAP, false>(base + kOffQ, warp * 32 + lane, t_a + lane_base, 1.f);
+    }
     tc_fence_before();
     mbar_arrive(bar_a);
     if (COMMIT) {
@@ -212,8 +307,8 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         for (uint32_t v = tid; v < Lay::kKV / 16; v += 128) {
           const uint32_t addr = base + kOffK + v * 16;
           const uint4 x = ld_shared_v4(addr);
-          st_shared_v4(addr, relu_bf16x2(x.x), relu_bf16x2(x.y), relu_bf16x2(x.z),
-                       relu_bf16x2(x.w));
+          st_shared_v4(addr, phi_bf16x2<FMAP>(x.x), phi_bf16x2<FMAP>(x.y),
+                       phi_bf16x2<FMAP>(x.z), phi_bf16x2<FMAP>(x.w));
         }
       }
       fence_proxy_async_smem();
@@ -249,6 +344,19 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
           mma_bf16_ss(t_sc, da, db, idesc, ks > 0 ? 1u : 0u);
         }
         mma_commit(bar_sc);
+        if (PROJ && mbar_wait(bar_w, 0, a.err, abort_flag)) {
+          // Q W_g: A = Q (K-major), B = W_g [input i][feature j] (MN-major)
+          tc_fence_after();
+          constexpr uint32_t idw = make_idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t da = make_sdesc(base + kOffQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16,
+                                           1024, kLayoutSW128);
+            const uint64_t db = make_sdesc(base + kOffW + ks * 2048, 16384, 1024, kLayoutSW128);
+            mma_bf16_ss(t_a, da, db, idw, ks > 0 ? 1u : 0u);
+          }
+          mma_commit(bar_qw);
+        }
       }
     }
     const bool ok = warp_all(mbar_wait(bar_sc, 0, a.err, abort_flag));
@@ -278,21 +386,30 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       float pscale;
       float qz = 0.f;
       if (SHARED) {
-        const float* zu = a.z + static_cast<size_t>(u) * kD;
+        if (PROJ) {
+          const bool okw = warp_all(mbar_wait(bar_qw, 0, a.err, abort_flag));
+          tc_fence_after();
+          if (okw) qz = proj_qz(t_a + lane_base, a.z + static_cast<size_t>(u) * kD);
+        } else {
+          const float* zu = a.z + static_cast<size_t>(u) * kD;
 #pragma unroll
-        for (int box = 0; box < 2; ++box) {
+          for (int box = 0; box < 2; ++box) {
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint4 v = ld_shared_v4(base + kOffQ + box * 16384 + r * 128 +
-                                         ((j ^ (r & 7)) << 4));
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-            const float4 z0 = __ldg(reinterpret_cast<const float4*>(zu + box * 64 + j * 8));
-            const float4 z1 = __ldg(reinterpret_cast<const float4*>(zu + box * 64 + j * 8 + 4));
-            const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+            for (int j = 0; j < 8; ++j) {
+              const uint4 v = ld_shared_v4(base + kOffQ + box * 16384 + r * 128 +
+                                           ((j ^ (r & 7)) << 4));
+              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+              const float4 z0 = __ldg(reinterpret_cast<const float4*>(zu + box * 64 + j * 8));
+              const float4 z1 =
+                  __ldg(reinterpret_cast<const float4*>(zu + box * 64 + j * 8 + 4));
+              const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              qz = fmaf(fmaxf(__uint_as_float(w4[q] << 16), 0.f), zz[2 * q], qz);
-              qz = fmaf(fmaxf(__uint_as_float(w4[q] & 0xFFFF0000u), 0.f), zz[2 * q + 1], qz);
+              for (int q = 0; q < 4; ++q) {
+                qz = fmaf(phiq_tf32<FMAP, false>(__uint_as_float(w4[q] << 16), 1.f), zz[2 * q],
+                          qz);
+                qz = fmaf(phiq_tf32<FMAP, false>(__uint_as_float(w4[q] & 0xFFFF0000u), 1.f),
+                          zz[2 * q + 1], qz);
+              }
             }
           }
         }
@@ -330,8 +447,14 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     mbar_arrive(bar_p);
 
     if (SHARED) {
-      // phi(q) times the row's scale, over the scores already read
-      if (ok) write_phiq(base + kOffQ, r, t_a + lane_base, ascale);
+      // phi(q) times the row's scale, over the scores already read (or over
+      // the Q W_g product)
+      if (ok) {
+        if (PROJ)
+          relu_tmem_phiq(t_a + lane_base, ascale);
+        else
+          write_phiq<FMAP, true>(base + kOffQ, r, t_a + lane_base, ascale);
+      }
       tc_fence_before();
       mbar_arrive(bar_a);
     }
@@ -473,37 +596,51 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   if ((tid & 127) == 0) bulk_wait_group_read0();   // shared memory stays until read
 }
 
-template <int BPAD, bool SHARED, bool COMMIT>
-int launch_cfg(const Ctx& c, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-               const CUtensorMap& ts, const CUtensorMap& ty, const StepArgs& a, int grid) {
+template <int BPAD, bool SHARED, bool COMMIT, int FMAP>
+int launch_cfg(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int grid) {
   using Lay = StepLayout<BPAD>;
-  auto kern = k_step_bf16<BPAD, SHARED, COMMIT>;
+  auto kern = k_step_bf16<BPAD, SHARED, COMMIT, FMAP>;
   static std::atomic<uint64_t> prepared{0};
   if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
-  return launch_pdl(kern, grid, kThreads, Lay::kSmem, c.stream, tq, tk, tv, ts, ty, a);
+  return launch_pdl(kern, grid, kThreads, Lay::kSmem, c.stream, tm[0], tm[1], tm[2], tm[3], tm[4],
+                    tm[5], a);
+}
+
+template <int BPAD, int FMAP>
+int launch_fmap(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int grid, int shared,
+                int commit) {
+  if constexpr (FMAP != kFmapReluProj) {
+    if (commit) return launch_cfg<BPAD, false, true, FMAP>(c, tm, a, grid);
+  } else {
+    if (commit) return -5;
+  }
+  return shared ? launch_cfg<BPAD, true, false, FMAP>(c, tm, a, grid)
+                : launch_cfg<BPAD, false, false, FMAP>(c, tm, a, grid);
 }
 
 template <int BPAD>
-int launch_bpad(const Ctx& c, const CUtensorMap& tq, const CUtensorMap& tk,
-                const CUtensorMap& tv, const CUtensorMap& ts, const CUtensorMap& ty,
-                const StepArgs& a, int grid, int shared, int commit) {
-  if (commit) return launch_cfg<BPAD, false, true>(c, tq, tk, tv, ts, ty, a, grid);
-  return shared ? launch_cfg<BPAD, true, false>(c, tq, tk, tv, ts, ty, a, grid)
-                : launch_cfg<BPAD, false, false>(c, tq, tk, tv, ts, ty, a, grid);
+int launch_bpad(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int grid, int shared,
+                int commit, int fmap) {
+  switch (fmap) {
+    case kFmapRelu: return launch_fmap<BPAD, kFmapRelu>(c, tm, a, grid, shared, commit);
+    case kFmapElu1: return launch_fmap<BPAD, kFmapElu1>(c, tm, a, grid, shared, commit);
+    default: return launch_fmap<BPAD, kFmapReluProj>(c, tm, a, grid, shared, commit);
+  }
 }
 
 }  // namespace
 
 int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, const float* S,
                      const float* z, void* Y, int n, int hq, int hkv, int b, float scale,
-                     int shared, float* commit_z, int commit) {
+                     int shared, int fmap, const void* W, float* commit_z, int commit) {
   const int G = hq / hkv;
   const int rows = G * b;
   const int units = n * hkv;
   const int bpad = b <= 16 ? 16 : (b <= 32 ? 32 : 64);
   const int mtiles = (rows + kMT - 1) / kMT;
 
-  CUtensorMap tq, tk, tv, ts, ty;
+  // tm: Q, K, V, S, Y, W (Q's map stands in for W under the elementwise maps)
+  CUtensorMap tm[6];
   const uint64_t dq[3] = {(uint64_t)kD, (uint64_t)rows, (uint64_t)units};
   const uint64_t sq[2] = {kD * 2ull, (uint64_t)rows * kD * 2ull};
   const uint32_t bq[3] = {64, kMT, 1};
@@ -513,22 +650,33 @@ int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, 
   const uint64_t ds[3] = {(uint64_t)kD, (uint64_t)kD, (uint64_t)units};
   const uint64_t ss[2] = {kD * 4ull, (uint64_t)kD * kD * 4ull};
   const uint32_t bs[3] = {32, 32, 1};
-  if (!encode_tmap(&tq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dq, sq, bq,
+  const uint64_t dw[3] = {(uint64_t)kD, (uint64_t)kD, (uint64_t)hkv};
+  const uint64_t sw[2] = {kD * 2ull, (uint64_t)kD * kD * 2ull};
+  const uint32_t bw[3] = {64, (uint32_t)kD, 1};
+  if (!encode_tmap(&tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dq, sq, bq,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Y, dq, sq, bq,
+      !encode_tmap(&tm[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Y, dq, sq, bq,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap(&tk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, K, dk, sk, bk,
+      !encode_tmap(&tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, K, dk, sk, bk,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap(&tv, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dk, sk, bk,
+      !encode_tmap(&tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dk, sk, bk,
                    CU_TENSOR_MAP_SWIZZLE_128B) ||
-      !encode_tmap(&ts, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, S, ds, ss, bs,
+      !encode_tmap(&tm[3], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, S, ds, ss, bs,
                    CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B))
     return -5;
+  if (fmap == kFmapReluProj) {
+    if (!encode_tmap(&tm[5], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, W, dw, sw, bw,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+      return -5;
+  } else {
+    tm[5] = tm[0];
+  }
 
   StepArgs a;
   a.z = z;
   a.zc = commit ? commit_z : nullptr;
   a.err = c.dev_err;
+  a.hkv = hkv;
   a.rows = rows;
   a.b = b;
   a.mtiles = mtiles;
@@ -536,9 +684,9 @@ int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, 
   a.scale_log2 = scale * 1.4426950408889634f;
   const int grid = units * mtiles;
   switch (bpad) {
-    case 16: return launch_bpad<16>(c, tq, tk, tv, ts, ty, a, grid, shared, commit);
-    case 32: return launch_bpad<32>(c, tq, tk, tv, ts, ty, a, grid, shared, commit);
-    default: return launch_bpad<64>(c, tq, tk, tv, ts, ty, a, grid, shared, commit);
+    case 16: return launch_bpad<16>(c, tm, a, grid, shared, commit, fmap);
+    case 32: return launch_bpad<32>(c, tm, a, grid, shared, commit, fmap);
+    default: return launch_bpad<64>(c, tm, a, grid, shared, commit, fmap);
   }
 }
 

@@ -172,6 +172,57 @@ int bha_prefix_softmax(const void *Qa, const void *Kc, const void *Vc, int P,
                        size_t workspace_bytes, bha_stream_t stream);
 
 /*
+ * Feature maps.  The method-details section (技术方法详解) of the paper-daily
+ * summary page has the previous blocks go through a kernel-function
+ * approximation, and its future-work section (未来研究方向) names better
+ * kernel functions as the next step; the worked example uses ReLU.  Every
+ * call above uses BHA_FMAP_RELU.  The _fm variants below take the map:
+ *   BHA_FMAP_RELU       phi(x)_j = max(x_j, 0)
+ *   BHA_FMAP_ELU1       phi(x)_j = x_j + 1 if x_j > 0, else exp(x_j)
+ *   BHA_FMAP_RELU_PROJ  phi(x)_j = max(sum_i x_i W[g][i][j], 0)
+ * W: [hkv][d][d], row-major, element type = dtype; KV head g's queries and
+ * keys use W[g] (queries by the GQA map), so phi keeps d features and S
+ * stays d x d.  W must be non-NULL and 16-byte aligned for
+ * BHA_FMAP_RELU_PROJ and NULL otherwise (BHA_ERR_INVALID_ARG), and must not
+ * overlap an output.  The bf16 path applies phi in fp32 and rounds phi(k) to
+ * bf16 for the tensor core (as a bf16 model does); phi(q) enters the
+ * phi(q) S product as tf32 (10-bit mantissa, round to nearest).
+ */
+typedef enum {
+    BHA_FMAP_RELU = 0,
+    BHA_FMAP_ELU1 = 1,
+    BHA_FMAP_RELU_PROJ = 2
+} bha_fmap;
+
+/* bha_state_prefill with feature map `fmap` (workspace as for
+ * bha_state_prefill: the size does not depend on the map). */
+int bha_state_prefill_fm(const void *K, const void *V, int n, int hkv, int T,
+                         int d, bha_dtype dtype, bha_fmap fmap, const void *W,
+                         float *S, float *z, void *workspace,
+                         size_t workspace_bytes, bha_stream_t stream);
+
+/* bha_state_commit with feature map `fmap`. */
+int bha_state_commit_fm(const void *Kb, const void *Vb, int n, int hkv, int b,
+                        int d, bha_dtype dtype, bha_fmap fmap, const void *W,
+                        float *S, float *z, bha_stream_t stream);
+
+/* bha_hybrid_step with feature map `fmap` (phi of the queries; S and z
+ * must have been built with the same map). */
+int bha_hybrid_step_fm(const void *Qa, const void *Ka, const void *Va,
+                       const float *S, const float *z, void *Y, int n, int hq,
+                       int hkv, int b, int d, float scale, unsigned flags,
+                       bha_dtype dtype, bha_fmap fmap, const void *W,
+                       bha_stream_t stream);
+
+/* bha_hybrid_step_commit with feature map `fmap`.  BHA_FMAP_RELU_PROJ
+ * always runs the step and the commit as two kernels. */
+int bha_hybrid_step_commit_fm(const void *Qa, const void *Ka, const void *Va,
+                              float *S, float *z, void *Y, int n, int hq,
+                              int hkv, int b, int d, float scale,
+                              unsigned flags, bha_dtype dtype, bha_fmap fmap,
+                              const void *W, bha_stream_t stream);
+
+/*
  * Block partition of a length-L sequence into blocks of B tokens, the last
  * one possibly short (worked example: L=10, B=4 -> tokens 1-4, 5-8, 9-10).
  * Host-only.  Writes bounds[0..k] = {0, B, 2B, ..., L} and returns k, the

@@ -168,3 +168,45 @@ def test_prefix_validation_and_workspace(L):
     assert f(ws=None) == _lib.BHA_ERR_WORKSPACE
     assert f(Y=A) == _lib.BHA_ERR_INVALID_ARG        # Y aliases Q
     assert f(Y=big + 64) == _lib.BHA_ERR_INVALID_ARG  # Y inside the cache
+
+
+def test_feature_map_validation(L):
+    """The _fm entry points: unknown map, W present without the projected
+    map or missing with it, misaligned W, W overlapping an output."""
+    RELU, ELU1, PROJ = _lib.BHA_FMAP_RELU, _lib.BHA_FMAP_ELU1, _lib.BHA_FMAP_RELU_PROJ
+    W = F
+
+    def st(fmap, w, **kw):
+        return L.bha_hybrid_step_fm(A, B, C, D, None, kw.get("Y", E), 2, 16, 4, 32, 128, 0.0,
+                                    0, _lib.BHA_BF16, fmap, w, None)
+
+    def cm(fmap, w, **kw):
+        return L.bha_state_commit_fm(A, B, 2, 4, 32, 128, _lib.BHA_BF16, fmap, w,
+                                     kw.get("S", C), kw.get("z", None), None)
+
+    def pf(fmap, w, **kw):
+        return L.bha_state_prefill_fm(A, B, 2, 4, 64, 128, _lib.BHA_BF16, fmap, w,
+                                      kw.get("S", C), None, None, 0, None)
+
+    def sc(fmap, w, **kw):
+        return L.bha_hybrid_step_commit_fm(A, B, C, kw.get("S", D), None, E, 2, 16, 4, 32, 128,
+                                           0.0, 0, _lib.BHA_BF16, fmap, w, None)
+
+    for f in (st, cm, pf, sc):
+        assert f(3, None) == _lib.BHA_ERR_INVALID_ARG       # unknown map
+        assert f(-1, None) == _lib.BHA_ERR_INVALID_ARG
+        assert f(RELU, W) == _lib.BHA_ERR_INVALID_ARG       # W without the projected map
+        assert f(ELU1, W) == _lib.BHA_ERR_INVALID_ARG
+        assert f(PROJ, None) == _lib.BHA_ERR_INVALID_ARG    # projected map without W
+        assert f(PROJ, W + 8) == _lib.BHA_ERR_MISALIGNED
+    assert st(PROJ, W, Y=W + 4096) == _lib.BHA_ERR_INVALID_ARG   # Y overlaps W
+    assert cm(PROJ, W, S=W - 4096) == _lib.BHA_ERR_INVALID_ARG   # S overlaps W
+    assert cm(PROJ, W, z=W + 256) == _lib.BHA_ERR_INVALID_ARG    # z overlaps W
+    assert pf(PROJ, W, S=W + 16) == _lib.BHA_ERR_INVALID_ARG
+    assert sc(PROJ, W, S=W + 16) == _lib.BHA_ERR_INVALID_ARG
+    import torch
+    if not torch.cuda.is_available():
+        # valid arguments reach the runtime, which has no GPU here
+        for f in (st, cm, pf, sc):
+            for fmap, w in ((RELU, None), (ELU1, None), (PROJ, W)):
+                assert f(fmap, w) == _lib.BHA_ERR_CUDA

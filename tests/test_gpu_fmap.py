@@ -1,0 +1,300 @@
+"""GPU parity of the feature maps other than ReLU (elu + 1 and ReLU after a
+per-KV-head d x d projection W_g), through the C ABI's _fm entry points,
+against the fp64 oracle on the same seeded inputs.
+
+The method-details section of the paper-daily summary page has the
+previous blocks go through a kernel-function approximation, and its
+future-work section names better kernel functions; the worked example
+uses ReLU.  Prefix states for the step tests come from the oracle's own
+prefill under the same map (a 512-token prompt), so they carry that map's
+statistics.
+
+Tolerances: outputs use the bf16 contract bound (relative L2 1e-2, max-abs
+3e-2), the max-abs part scaled by the reference's largest magnitude where
+that exceeds 1: under elu + 1 every feature is near 1, so phi(q) S sums
+128 strongly correlated state rows and outputs reach the hundreds, where
+one bf16 step is already above 3e-2.  States built by the bf16
+path hold phi(k) rounded to bf16 before the fp32 contraction (one rounding,
+at most 2^-9 relative per feature, averaging out over tokens), so they are
+held to 5e-3 rather than the 1e-4 of ReLU, whose phi(k) is exact in bf16.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from block_hybrid_linear_b200 import inputs
+import block_hybrid_linear_b200 as bha
+
+from gpu_util import (TOL_F32_REL, Guarded, bf16_case, dev_bf16, dev_f32, host, log_parity,
+                      max_abs, rel_l2, TOL_BF16_ABS, TOL_BF16_REL)
+
+pytestmark = pytest.mark.gpu
+
+STD = 1.0 / math.sqrt(128)
+TOL_STATE_FMAP_REL = 5e-3
+FMAPS = {"elu1": bha.BHA_FMAP_ELU1, "proj": bha.BHA_FMAP_RELU_PROJ}
+TID_W = 90   # input-generator tensor id of the projections
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    import torch
+    from block_hybrid_linear_b200 import build
+    build.build()
+    oracle.set_threads(max(1, min(16, oracle.max_threads())))
+    torch.cuda.synchronize()
+    assert bha.bha_device_error(True) == 0
+    yield
+    assert bha.bha_device_error(True) == 0
+
+
+def weights(fmap, seed, hkv, d=128, dtype="bf16"):
+    """(device W or None, float64 W or None): W ~ N(0, 1/d) keeps q W at q's
+    scale."""
+    if fmap != bha.BHA_FMAP_RELU_PROJ:
+        return None, None
+    if dtype == "bf16":
+        bits, vals = inputs.normal_bf16_np(seed, TID_W, (hkv, d, d), 1.0 / math.sqrt(d))
+        return dev_bf16(bits), vals
+    vals = inputs.normal_f32_np(seed, TID_W, (hkv, d, d), 1.0 / math.sqrt(d))
+    return dev_f32(vals), vals
+
+
+def oracle_state(seed, n, hkv, fmap, Wv, d=128, T=512, std=STD):
+    """A prefix state under `fmap` from the oracle's prefill of a seeded prompt."""
+    Kp = inputs.normal_f32_np(seed, inputs.TID_KP, (n, hkv, T, d), std)
+    Vp = inputs.normal_f32_np(seed, inputs.TID_VP, (n, hkv, T, d), std)
+    S, z = oracle.state_prefill(Kp, Vp, fmap=fmap, W=Wv)
+    return S.astype(np.float32), z.astype(np.float32)
+
+
+def check(name, got, ref, tol_rel, tol_abs=None, **kw):
+    e_rel, e_abs = rel_l2(got, ref), max_abs(got, ref)
+    peak = float(np.max(np.abs(ref))) if np.size(ref) else 0.0
+    log_parity(name, rel_l2=e_rel, max_abs=e_abs, ref_peak=peak, **kw)
+    assert e_rel <= tol_rel, (name, e_rel)
+    if tol_abs is not None:
+        assert e_abs <= tol_abs * max(1.0, peak), (name, e_abs, peak)
+
+
+# ------------------------------------------------------------ hybrid step
+
+STEP_CASES = [  # (n, hq, hkv, b)
+    (2, 16, 4, 32),    # the model's shape
+    (2, 8, 2, 17),     # ragged b, BPAD 32
+    (2, 8, 2, 10),     # BPAD 16
+    (1, 4, 1, 1),      # one active token
+    (2, 8, 1, 33),     # BPAD 64, three M tiles with a ragged tail
+    (1, 16, 4, 64),    # two M tiles
+]
+
+
+@pytest.mark.parametrize("shared", [False, True], ids=["default", "shared"])
+@pytest.mark.parametrize("fmap", list(FMAPS), ids=list(FMAPS))
+@pytest.mark.parametrize("case", STEP_CASES, ids=lambda c: "n%d_hq%d_hkv%d_b%d" % c)
+def test_step_fmap_bf16(case, fmap, shared):
+    import torch
+    n, hq, hkv, b = case
+    f = FMAPS[fmap]
+    seed = 700 + b
+    Q, Qv = bf16_case((seed, 0), (n, hq, b, 128), STD)
+    K, Kv = bf16_case((seed, 1), (n, hkv, b, 128), STD)
+    V, Vv = bf16_case((seed, 2), (n, hkv, b, 128), STD)
+    W, Wv = weights(f, seed, hkv)
+    Sv, zv = oracle_state(seed, n, hkv, f, Wv)
+    Y = Guarded((n, hq, b, 128), torch.bfloat16)
+    bha.bha_hybrid_step_fm(Q, K, V, dev_f32(Sv), Y.t, z=dev_f32(zv),
+                           flags=bha.BHA_FLAG_SHARED_DENOM if shared else 0, fmap=f, W=W)
+    torch.cuda.synchronize()
+    assert Y.intact() and Y.no_nan()
+    ref = oracle.hybrid_step(Qv, Kv, Vv, Sv, zv, shared=shared, fmap=f, W=Wv)
+    check("step_fmap_bf16", host(Y.t), ref, TOL_BF16_REL, TOL_BF16_ABS, case=case, fmap=fmap,
+          shared=shared)
+
+
+def test_step_proj_identity_equals_relu():
+    """W_g = I makes the projected map ReLU: the projection of a bf16 q by I
+    is exact and both kernels round phi(q) (times e^{-m} in the shared mode)
+    to tf32 the same way, so the outputs are identical."""
+    import torch
+    n, hq, hkv, b = 2, 16, 4, 32
+    Q, _ = bf16_case((71, 0), (n, hq, b, 128), STD)
+    K, _ = bf16_case((71, 1), (n, hkv, b, 128), STD)
+    V, _ = bf16_case((71, 2), (n, hkv, b, 128), STD)
+    Sv, zv = inputs.synthetic_state_np(71, n, hkv, 128, 4096, STD)
+    S, z = dev_f32(Sv), dev_f32(zv)
+    W = torch.eye(128, dtype=torch.bfloat16, device="cuda").repeat(hkv, 1, 1).contiguous()
+    for flags in (0, bha.BHA_FLAG_SHARED_DENOM):
+        Yr = torch.empty(n, hq, b, 128, dtype=torch.bfloat16, device="cuda")
+        Yp = torch.empty_like(Yr)
+        bha.bha_hybrid_step(Q, K, V, S, Yr, z=z, flags=flags)
+        bha.bha_hybrid_step_fm(Q, K, V, S, Yp, z=z, flags=flags, fmap=bha.BHA_FMAP_RELU_PROJ, W=W)
+        torch.cuda.synchronize()
+        check("step_proj_identity", host(Yp), host(Yr), 0.0, flags=flags)
+
+
+@pytest.mark.parametrize("shared", [False, True], ids=["default", "shared"])
+@pytest.mark.parametrize("fmap", list(FMAPS), ids=list(FMAPS))
+@pytest.mark.parametrize("d", [16, 128])
+def test_step_fmap_f32(d, fmap, shared):
+    import torch
+    n, hq, hkv, b = 2, 4, 2, 13
+    f = FMAPS[fmap]
+    Qv = inputs.normal_f32_np(731, 0, (n, hq, b, d), 1.0)
+    Kv = inputs.normal_f32_np(731, 1, (n, hkv, b, d), 1.0)
+    Vv = inputs.normal_f32_np(731, 2, (n, hkv, b, d), 1.0)
+    W, Wv = weights(f, 731, hkv, d, "f32")
+    Sv, zv = oracle_state(731, n, hkv, f, Wv, d=d, T=64, std=1.0)
+    Y = Guarded((n, hq, b, d), torch.float32)
+    bha.bha_hybrid_step_fm(dev_f32(Qv), dev_f32(Kv), dev_f32(Vv), dev_f32(Sv), Y.t,
+                           z=dev_f32(zv), flags=bha.BHA_FLAG_SHARED_DENOM if shared else 0,
+                           fmap=f, W=W)
+    torch.cuda.synchronize()
+    assert Y.intact() and Y.no_nan()
+    ref = oracle.hybrid_step(Qv, Kv, Vv, Sv, zv, shared=shared, fmap=f, W=Wv)
+    check("step_fmap_f32", host(Y.t), ref, TOL_F32_REL, d=d, fmap=fmap, shared=shared)
+
+
+# ------------------------------------------------------------ commit
+
+@pytest.mark.parametrize("fmap", list(FMAPS), ids=list(FMAPS))
+@pytest.mark.parametrize("b", [1, 10, 16, 32, 33, 64])
+@pytest.mark.parametrize("with_z", [False, True])
+def test_commit_fmap_bf16(b, fmap, with_z):
+    import torch
+    n, hkv = 3, 4
+    f = FMAPS[fmap]
+    seed = 800 + b
+    K, Kv = bf16_case((seed, 1), (n, hkv, b, 128), STD)
+    V, Vv = bf16_case((seed, 2), (n, hkv, b, 128), STD)
+    W, Wv = weights(f, seed, hkv)
+    Sv, zv = oracle_state(seed, n, hkv, f, Wv, T=64)
+    S, z = dev_f32(Sv), dev_f32(zv) if with_z else None
+    bha.bha_state_commit_fm(K, V, S, z, fmap=f, W=W)
+    torch.cuda.synchronize()
+    rS, rz = oracle.state_commit(Sv, zv, Kv, Vv, fmap=f, W=Wv)
+    # the tolerance applies to what the block added (the old state is exact)
+    check("commit_fmap_bf16_dS", host(S) - Sv, rS - Sv, TOL_STATE_FMAP_REL, b=b, fmap=fmap)
+    if with_z:
+        check("commit_fmap_bf16_dz", host(z) - zv, rz - zv, TOL_STATE_FMAP_REL, b=b, fmap=fmap)
+
+
+@pytest.mark.parametrize("fmap", list(FMAPS), ids=list(FMAPS))
+@pytest.mark.parametrize("d", [16, 128])
+def test_commit_fmap_f32(d, fmap):
+    import torch
+    n, hkv, b = 2, 2, 9
+    f = FMAPS[fmap]
+    Kv = inputs.normal_f32_np(841, 1, (n, hkv, b, d), 1.0)
+    Vv = inputs.normal_f32_np(841, 2, (n, hkv, b, d), 1.0)
+    Sv = inputs.normal_f32_np(841, 3, (n, hkv, d, d), 1.0)
+    zv = np.abs(inputs.normal_f32_np(841, 4, (n, hkv, d), 1.0))
+    W, Wv = weights(f, 841, hkv, d, "f32")
+    S, z = dev_f32(Sv), dev_f32(zv)
+    bha.bha_state_commit_fm(dev_f32(Kv), dev_f32(Vv), S, z, fmap=f, W=W)
+    torch.cuda.synchronize()
+    rS, rz = oracle.state_commit(Sv, zv, Kv, Vv, fmap=f, W=Wv)
+    check("commit_fmap_f32_S", host(S), rS, TOL_F32_REL, d=d, fmap=fmap)
+    check("commit_fmap_f32_z", host(z), rz, TOL_F32_REL, d=d, fmap=fmap)
+
+
+# ------------------------------------------------------------ prefill
+
+@pytest.mark.parametrize("fmap", list(FMAPS), ids=list(FMAPS))
+@pytest.mark.parametrize("T", [0, 1, 63, 64, 65, 1000, 4113])
+def test_prefill_fmap_bf16(T, fmap):
+    import torch
+    n, hkv = 2, 2
+    f = FMAPS[fmap]
+    K, Kv = bf16_case((900 + T, 3), (n, hkv, T, 128), STD)
+    V, Vv = bf16_case((900 + T, 4), (n, hkv, T, 128), STD)
+    W, Wv = weights(f, 900 + T, hkv)
+    S = Guarded((n, hkv, 128, 128), torch.float32)
+    z = Guarded((n, hkv, 128), torch.float32)
+    need = bha.bha_state_prefill_workspace_size(n, hkv, T, 128)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda") if need else None
+    bha.bha_state_prefill_fm(K, V, S.t, z.t, fmap=f, W=W, workspace=ws)
+    torch.cuda.synchronize()
+    assert S.intact() and S.no_nan() and z.intact() and z.no_nan()
+    if T == 0:
+        assert np.all(host(S.t) == 0) and np.all(host(z.t) == 0)
+        return
+    rS, rz = oracle.state_prefill(Kv, Vv, fmap=f, W=Wv)
+    check("prefill_fmap_bf16_S", host(S.t), rS, TOL_STATE_FMAP_REL, T=T, fmap=fmap, ws=need)
+    check("prefill_fmap_bf16_z", host(z.t), rz, TOL_STATE_FMAP_REL, T=T, fmap=fmap)
+
+
+@pytest.mark.parametrize("fmap", list(FMAPS), ids=list(FMAPS))
+def test_prefill_fmap_f32(fmap):
+    import torch
+    n, hkv, T, d = 2, 2, 300, 16
+    f = FMAPS[fmap]
+    Kv = inputs.normal_f32_np(961, 3, (n, hkv, T, d), 1.0)
+    Vv = inputs.normal_f32_np(961, 4, (n, hkv, T, d), 1.0)
+    W, Wv = weights(f, 961, hkv, d, "f32")
+    S = torch.empty(n, hkv, d, d, device="cuda")
+    z = torch.empty(n, hkv, d, device="cuda")
+    bha.bha_state_prefill_fm(dev_f32(Kv), dev_f32(Vv), S, z, fmap=f, W=W)
+    torch.cuda.synchronize()
+    rS, rz = oracle.state_prefill(Kv, Vv, fmap=f, W=Wv)
+    check("prefill_fmap_f32_S", host(S), rS, TOL_F32_REL, fmap=fmap)
+    check("prefill_fmap_f32_z", host(z), rz, TOL_F32_REL, fmap=fmap)
+
+
+# ------------------------------------------------------------ last step + commit
+
+@pytest.mark.parametrize("mode", ["default", "shared"])
+@pytest.mark.parametrize("fmap", list(FMAPS), ids=list(FMAPS))
+@pytest.mark.parametrize("case", [(2, 16, 4, 32), (2, 8, 2, 17), (2, 8, 1, 33)],
+                         ids=lambda c: "n%d_hq%d_hkv%d_b%d" % c)
+def test_step_commit_fmap_bf16(case, fmap, mode):
+    """elu + 1 in the default mode with G*b <= 128 runs the fused kernel; the
+    projected map always runs step + commit."""
+    import torch
+    n, hq, hkv, b = case
+    f = FMAPS[fmap]
+    shared = mode == "shared"
+    seed = 1000 + b
+    Q, Qv = bf16_case((seed, 0), (n, hq, b, 128), STD)
+    K, Kv = bf16_case((seed, 1), (n, hkv, b, 128), STD)
+    V, Vv = bf16_case((seed, 2), (n, hkv, b, 128), STD)
+    W, Wv = weights(f, seed, hkv)
+    Sv, zv = oracle_state(seed, n, hkv, f, Wv)
+    S, z = dev_f32(Sv), dev_f32(zv)
+    Y = Guarded((n, hq, b, 128), torch.bfloat16)
+    bha.bha_hybrid_step_commit_fm(Q, K, V, S, Y.t, z=z,
+                                  flags=bha.BHA_FLAG_SHARED_DENOM if shared else 0, fmap=f, W=W)
+    torch.cuda.synchronize()
+    assert Y.intact() and Y.no_nan()
+    check("step_commit_fmap_y", host(Y.t),
+          oracle.hybrid_step(Qv, Kv, Vv, Sv, zv, shared=shared, fmap=f, W=Wv), TOL_BF16_REL,
+          TOL_BF16_ABS, case=case, fmap=fmap, mode=mode)
+    rS, rz = oracle.state_commit(Sv, zv, Kv, Vv, fmap=f, W=Wv)
+    check("step_commit_fmap_dS", host(S) - Sv, rS - Sv, TOL_STATE_FMAP_REL, case=case,
+          fmap=fmap, mode=mode)
+    check("step_commit_fmap_dz", host(z) - zv, rz - zv, TOL_STATE_FMAP_REL, case=case,
+          fmap=fmap, mode=mode)
+
+
+def test_step_commit_fmap_f32():
+    import torch
+    n, hq, hkv, b, d = 2, 4, 2, 7, 16
+    for f in FMAPS.values():
+        Qv = inputs.normal_f32_np(1081, 0, (n, hq, b, d), 1.0)
+        Kv = inputs.normal_f32_np(1081, 1, (n, hkv, b, d), 1.0)
+        Vv = inputs.normal_f32_np(1081, 2, (n, hkv, b, d), 1.0)
+        Sv = inputs.normal_f32_np(1081, 3, (n, hkv, d, d), 1.0)
+        zv = np.abs(inputs.normal_f32_np(1081, 4, (n, hkv, d), 1.0))
+        W, Wv = weights(f, 1081, hkv, d, "f32")
+        S, z = dev_f32(Sv), dev_f32(zv)
+        Y = torch.empty(n, hq, b, d, device="cuda")
+        bha.bha_hybrid_step_commit_fm(dev_f32(Qv), dev_f32(Kv), dev_f32(Vv), S, Y, z=z, fmap=f,
+                                      W=W)
+        torch.cuda.synchronize()
+        check("step_commit_fmap_f32_y", host(Y),
+              oracle.hybrid_step(Qv, Kv, Vv, Sv, zv, fmap=f, W=Wv), TOL_F32_REL, fmap=f)
+        rS, rz = oracle.state_commit(Sv, zv, Kv, Vv, fmap=f, W=Wv)
+        check("step_commit_fmap_f32_S", host(S), rS, TOL_F32_REL, fmap=f)
+        check("step_commit_fmap_f32_z", host(z), rz, TOL_F32_REL, fmap=f)
