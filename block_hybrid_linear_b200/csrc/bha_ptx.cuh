@@ -382,14 +382,6 @@ constexpr int kFmapRelu = 0;       // phi(x) = max(x, 0)
 constexpr int kFmapElu1 = 1;       // phi(x) = x + 1 (x > 0), exp(x) (x <= 0)
 constexpr int kFmapReluProj = 2;   // phi(x) = max(x W, 0)
 
-// phi of one element for the elementwise maps (the projected map applies
-// the ReLU part of it here, after the projection).
-template <int FMAP>
-__device__ __forceinline__ float phi_elem(float x) {
-  if (FMAP == kFmapElu1) return x > 0.f ? x + 1.f : __expf(x);
-  return fmaxf(x, 0.f);
-}
-
 // fp32 -> the nearest tf32 value (ties away from zero), in an fp32 register:
 // what the tensor core then reads from TMEM loses nothing more.
 __device__ __forceinline__ float round_tf32(float x) {
@@ -398,13 +390,30 @@ __device__ __forceinline__ float round_tf32(float x) {
   return __uint_as_float(r);
 }
 
-// phi of both bf16 lanes of a packed pair, rounded back to bf16 (exact for
-// ReLU, round-to-nearest-even for elu + 1).
+// elu + 1 of both lanes of a packed bf16 pair in packed bf16 arithmetic, as
+// a bf16 model evaluates it: max(1 + x, 2^(min(x, 0) * log2 e)).  For x <= 0
+// the exponential is the value (e^x >= 1 + x by convexity); for x > 0 it is
+// e^0 = 1 < 1 + x.  One two-lane ex2 per pair keeps the special-function
+// unit off the critical path.  log2 e enters as the bf16 1.4453125 (0.18%
+// high: a relative error below 0.0018 |x| in e^x, under the bf16 rounding of
+// the result for |x| < 1).  -inf -> 0, +inf -> +inf, +-0 -> 1.
+__device__ __forceinline__ uint32_t elu1_bf16x2(uint32_t w) {
+  const uint32_t zero = 0u, one = 0x3F803F80u, log2e = 0x3FB93FB9u;
+  uint32_t xm, t, e, p, r;
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(xm) : "r"(w), "r"(zero));
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(t) : "r"(xm), "r"(log2e));
+  asm("ex2.approx.ftz.bf16x2 %0, %1;" : "=r"(e) : "r"(t));
+  asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(p) : "r"(w), "r"(one));
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(p), "r"(e));
+  return r;
+}
+
+// phi of both bf16 lanes of a packed pair, as bf16 (elementwise maps; exact
+// for ReLU).
 template <int FMAP>
 __device__ __forceinline__ uint32_t phi_bf16x2(uint32_t x) {
   if (FMAP == kFmapRelu) return relu_bf16x2(x);
-  return pack_bf16x2(phi_elem<FMAP>(__uint_as_float(x << 16)),
-                     phi_elem<FMAP>(__uint_as_float(x & 0xFFFF0000u)));
+  return elu1_bf16x2(x);
 }
 
 // Address of 16-byte chunk jj of row r in a K-major bf16 operand tile whose

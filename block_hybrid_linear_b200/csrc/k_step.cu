@@ -85,12 +85,11 @@ __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu
 
 // phi(q_r) * scale as fp32 into TMEM (this thread's lane, columns [0, 128)
 // from `tcol`), read from row r of the SW128 Q tile; one wait for all four
-// 32-column stores.  Elementwise maps only.  Values are rounded to the
-// nearest tf32 unless they are tf32 already (ReLU of a bf16 value, unscaled).
-template <int FMAP, bool SCALED>
-__device__ __forceinline__ float phiq_tf32(float x, float scale) {
-  const float v = phi_elem<FMAP>(x) * scale;
-  return (FMAP == kFmapRelu && !SCALED) ? v : round_tf32(v);
+// 32-column stores.  Elementwise maps only: phi is a bf16 value (a tf32
+// value already); a scaled one is rounded to the nearest tf32.
+template <bool SCALED>
+__device__ __forceinline__ float phiq_tf32(float phi, float scale) {
+  return SCALED ? round_tf32(phi * scale) : phi;
 }
 
 template <int FMAP, bool SCALED>
@@ -105,9 +104,9 @@ __device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol,
       const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        f[8 * q + 2 * e] = phiq_tf32<FMAP, SCALED>(__uint_as_float(w4[e] << 16), scale);
-        f[8 * q + 2 * e + 1] =
-            phiq_tf32<FMAP, SCALED>(__uint_as_float(w4[e] & 0xFFFF0000u), scale);
+        const uint32_t p2 = phi_bf16x2<FMAP>(w4[e]);
+        f[8 * q + 2 * e] = phiq_tf32<SCALED>(__uint_as_float(p2 << 16), scale);
+        f[8 * q + 2 * e + 1] = phiq_tf32<SCALED>(__uint_as_float(p2 & 0xFFFF0000u), scale);
       }
     }
     tmem_st32(tcol + cg * 32, f);
@@ -405,10 +404,9 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
               const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
 #pragma unroll
               for (int q = 0; q < 4; ++q) {
-                qz = fmaf(phiq_tf32<FMAP, false>(__uint_as_float(w4[q] << 16), 1.f), zz[2 * q],
-                          qz);
-                qz = fmaf(phiq_tf32<FMAP, false>(__uint_as_float(w4[q] & 0xFFFF0000u), 1.f),
-                          zz[2 * q + 1], qz);
+                const uint32_t p2 = phi_bf16x2<FMAP>(w4[q]);
+                qz = fmaf(__uint_as_float(p2 << 16), zz[2 * q], qz);
+                qz = fmaf(__uint_as_float(p2 & 0xFFFF0000u), zz[2 * q + 1], qz);
               }
             }
           }
