@@ -544,22 +544,26 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-// Prefill under the projected map: a 2-stage ring (W_g takes the third
-// stage's room, keeping two CTAs per SM).  Per tile i: the MMA thread issues
-// (K W_g)^T into TMEM buffer i % 2 (columns 128 + 64 (i % 2)), then phi(K)^T
-// V of tile i - 1 once its features are written; warps 4-7 (thread =
-// feature r) read buffer i % 2, apply the ReLU, add to z and write row r of
-// phi(K)^T over the consumed K tile (K-major SW128, 64 tokens = 128 B).
-constexpr int kProjStages = 2;
-constexpr uint32_t kPrefProjOffW = kProjStages * kStageBytes;    // 64 KB (= epilogue tile)
-constexpr uint32_t kPrefProjTiles = kPrefProjOffW + 32768;
-constexpr uint32_t kPrefProjSmem = kPrefProjTiles + 1024;
+// Prefill under the projected map: the ReLU kernel's 3-stage ring and two
+// CTAs per SM, with W_g^T, the A operand of the projection, held in TMEM
+// (64 columns: lane = feature j, two bf16 inputs per column) so that shared
+// memory holds only the K / V tiles.  TMEM: phi(K)^T V at [0, 128), W_g^T at
+// [128, 192), one tile's projection (K W_g)^T at [192, 256).  The MMA thread
+// issues tile i's projection once the feature writers have read tile
+// i - 1's out of TMEM, and phi(K)^T V of tile i once its features are
+// written; warps 4-7 (thread = feature r) read the projection, release it,
+// apply the ReLU, add to z and write row r of phi(K)^T over the consumed K
+// tile (K-major SW128, 64 tokens = 128 B).
+struct PrefillProjArgs {
+  PrefillArgs p;
+  const uint16_t* W;   // [hkv][128][128] bf16 bits
+};
 
 __global__ void __launch_bounds__(kThreads, 2)
     k_prefill_proj_bf16(const __grid_constant__ CUtensorMap tmK,
                         const __grid_constant__ CUtensorMap tmV,
-                        const __grid_constant__ CUtensorMap tmOut,
-                        const __grid_constant__ CUtensorMap tmW, const PrefillArgs a) {
+                        const __grid_constant__ CUtensorMap tmOut, const PrefillProjArgs pa) {
+  const PrefillArgs& a = pa.p;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int item = blockIdx.x;                // = u * splits + s
@@ -571,23 +575,25 @@ __global__ void __launch_bounds__(kThreads, 2)
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + kPrefProjTiles;
+  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + kPrefTiles;
   uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
-  const uint32_t bar_full = ctrl, bar_relu = ctrl + 16, bar_empty = ctrl + 32,
-                 bar_kw = ctrl + 48, bar_w = ctrl + 64, bar_done = ctrl + 72;
+  const uint32_t bar_full = ctrl, bar_relu = ctrl + 24, bar_empty = ctrl + 48,
+                 bar_done = ctrl + 72, bar_kw = ctrl + 88, bar_kwfree = ctrl + 96,
+                 bar_wt = ctrl + 104;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 80);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 84);
 
   if (warp == 0) {
     if (lane == 0) {
-      for (int s = 0; s < kProjStages; ++s) {
+      for (int s = 0; s < kStages; ++s) {
         mbar_init(bar_full + 8 * s, 1);
         mbar_init(bar_relu + 8 * s, 128);
         mbar_init(bar_empty + 8 * s, 1);
-        mbar_init(bar_kw + 8 * s, 1);
       }
-      mbar_init(bar_w, 1);
       mbar_init(bar_done, 1);
+      mbar_init(bar_kw, 1);
+      mbar_init(bar_kwfree, 128);
+      mbar_init(bar_wt, 128);
       *abort_flag = 0;
       fence_mbar_init();
     }
@@ -600,18 +606,16 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const uint32_t t_w = tmem + 128, t_kw = tmem + 192;
   pdl_wait();
 
   float zacc = 0.f;
   if (tid == 0) {
-    // producer: W_g once, then the K / V tiles
-    mbar_arrive_expect_tx(bar_w, 32768);
-    tma_load_3d(base + kPrefProjOffW, &tmW, bar_w, 0, 0, g);
-    tma_load_3d(base + kPrefProjOffW + 16384, &tmW, bar_w, 64, 0, g);
+    // producer
     for (int i = 0; i < ntile; ++i) {
-      const int st = i % kProjStages;
-      if (i >= kProjStages &&
-          !mbar_wait(bar_empty + 8 * st, ((i / kProjStages) - 1) & 1, a.err, abort_flag))
+      const int st = i % kStages;
+      if (i >= kStages &&
+          !mbar_wait(bar_empty + 8 * st, ((i / kStages) - 1) & 1, a.err, abort_flag))
         break;
       const uint32_t sbase = base + st * kStageBytes;
       const uint32_t bf = bar_full + 8 * st;
@@ -623,12 +627,27 @@ __global__ void __launch_bounds__(kThreads, 2)
       tma_load_3d(sbase + 24576, &tmV, bf, 64, t0, u);
     }
   } else if (tid == 32) {
-    constexpr uint32_t id_kw = make_idesc_bf16(128, kTok, 1, 0);
+    // (K W_g)^T of tile i: A = W_g^T from TMEM, B = the K tile (K-major)
+    constexpr uint32_t id_kw = make_idesc_bf16(128, kTok, 0, 0);
     constexpr uint32_t id_sv = make_idesc_bf16(128, 128, 0, 1);
-    // phi(K)^T V of tile j (stage j % 2) into the accumulator
+    auto issue_kw = [&](int i) -> bool {
+      const int st = i % kStages;
+      if (!mbar_wait(bar_full + 8 * st, (i / kStages) & 1, a.err, abort_flag)) return false;
+      tc_fence_after();
+      const uint32_t sbase = base + st * kStageBytes;
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const uint64_t db =
+            make_sdesc(sbase + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128);
+        mma_bf16_ts(t_kw, t_w + 8 * ks, db, id_kw, ks > 0 ? 1u : 0u);
+      }
+      mma_commit(bar_kw);
+      return true;
+    };
+    // phi(K)^T V of tile j into the accumulator: A K-major, B = V MN-major
     auto issue_sv = [&](int j) -> bool {
-      const int sj = j % kProjStages;
-      if (!mbar_wait(bar_relu + 8 * sj, (j / kProjStages) & 1, a.err, abort_flag)) return false;
+      const int sj = j % kStages;
+      if (!mbar_wait(bar_relu + 8 * sj, (j / kStages) & 1, a.err, abort_flag)) return false;
       tc_fence_after();
       const uint32_t sb = base + sj * kStageBytes;
 #pragma unroll
@@ -640,64 +659,71 @@ __global__ void __launch_bounds__(kThreads, 2)
       mma_commit(bar_empty + 8 * sj);
       return true;
     };
-    bool ok = mbar_wait(bar_w, 0, a.err, abort_flag);
-    for (int i = 0; i < ntile && ok; ++i) {
-      const int st = i % kProjStages;
-      ok = mbar_wait(bar_full + 8 * st, (i / kProjStages) & 1, a.err, abort_flag);
-      if (!ok) break;
-      tc_fence_after();
-      // (K W_g)^T of tile i: buffer st was last read for tile i - 2, whose
-      // features were waited for in the previous iteration
-      const uint32_t sbase = base + st * kStageBytes;
-#pragma unroll
-      for (int ks = 0; ks < 8; ++ks) {
-        const uint64_t da = make_sdesc(base + kPrefProjOffW + ks * 2048, 16384, 1024, kLayoutSW128);
-        const uint64_t db =
-            make_sdesc(sbase + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024, kLayoutSW128);
-        mma_bf16_ss(tmem + 128 + 64 * st, da, db, id_kw, ks > 0 ? 1u : 0u);
+    bool ok = mbar_wait(bar_wt, 0, a.err, abort_flag) && (ntile < 1 || issue_kw(0));
+    for (int j = 0; j < ntile && ok; ++j) {
+      if (j + 1 < ntile) {
+        // the projection buffer is free once tile j's was read out of it
+        ok = mbar_wait(bar_kwfree, j & 1, a.err, abort_flag) && issue_kw(j + 1);
+        if (!ok) break;
       }
-      mma_commit(bar_kw + 8 * st);
-      if (i >= 1) ok = issue_sv(i - 1);
+      ok = issue_sv(j);
     }
-    if (ok && ntile >= 1) ok = issue_sv(ntile - 1);
     if (ok) mma_commit(bar_done);
   } else if (warp >= 4) {
     const int r = tid - 128;
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    for (int i = 0; i < ntile; ++i) {
-      const int st = i % kProjStages;
-      if (!warp_all(mbar_wait(bar_kw + 8 * st, (i / kProjStages) & 1, a.err, abort_flag))) break;
-      tc_fence_after();
-      const uint32_t kt = base + st * kStageBytes;   // phi(K)^T over the consumed K tile
-#pragma unroll
+    {
+      // W_g^T into TMEM: column c of lane r holds inputs 2c (low) and 2c + 1
+      const uint16_t* Wg = pa.W + static_cast<size_t>(g) * kD * kD + r;
+#pragma unroll 1
       for (int h = 0; h < 2; ++h) {
         float f[32];
-        tmem_ld32_sync(tmem + 128 + 64 * st + lane_base + 32 * h, f);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t w[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            // tokens past the prompt are zero rows of K: their features are 0
-            w[q] = pack_bf16x2(fmaxf(f[8 * c + 2 * q], 0.f), fmaxf(f[8 * c + 2 * q + 1], 0.f));
-            zacc += __uint_as_float(w[q] << 16) + __uint_as_float(w[q] & 0xFFFF0000u);
-          }
-          st_shared_v4(kmajor_chunk<128>(kt, r, 4 * h + c), w[0], w[1], w[2], w[3]);
+        for (int c = 0; c < 32; ++c) {
+          const int i0 = 2 * (32 * h + c);
+          const uint32_t lo = __ldg(Wg + i0 * kD), hi = __ldg(Wg + (i0 + 1) * kD);
+          f[c] = __uint_as_float(lo | (hi << 16));
         }
+        tmem_st32(t_w + lane_base + 32 * h, f);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar_wt);
+    }
+    for (int i = 0; i < ntile; ++i) {
+      const int st = i % kStages;
+      if (!warp_all(mbar_wait(bar_kw, i & 1, a.err, abort_flag))) break;
+      tc_fence_after();
+      float f[64];
+      tmem_ld32_sync(t_kw + lane_base, *reinterpret_cast<float(*)[32]>(f));
+      tmem_ld32_sync(t_kw + lane_base + 32, *reinterpret_cast<float(*)[32]>(f + 32));
+      tc_fence_before();
+      mbar_arrive(bar_kwfree);
+      const uint32_t kt = base + st * kStageBytes;   // phi(K)^T over the consumed K tile
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          // tokens past the prompt are zero rows of K: their features are 0
+          w[q] = pack_bf16x2(fmaxf(f[8 * c + 2 * q], 0.f), fmaxf(f[8 * c + 2 * q + 1], 0.f));
+          zacc += __uint_as_float(w[q] << 16) + __uint_as_float(w[q] & 0xFFFF0000u);
+        }
+        st_shared_v4(kmajor_chunk<128>(kt, r, c), w[0], w[1], w[2], w[3]);
       }
       fence_proxy_async_smem();
-      tc_fence_before();
       mbar_arrive(bar_relu + 8 * st);
     }
   }
 
-  // ---- epilogue: accumulator -> fp32 tile (over the two stages) -> TMA store
+  // ---- epilogue: accumulator -> fp32 tile -> TMA store (partial or final)
   __syncwarp();
   const bool ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag));
   tc_fence_after();
   if (ok) accum_to_tile(tmem, base, warp, lane, false);
   fence_proxy_async_smem();
-  if (warp >= 4 && a.zdst != nullptr && ok) a.zdst[static_cast<size_t>(item) * kD + (tid - 128)] = zacc;
+  if (warp >= 4 && a.zdst != nullptr && ok)
+    a.zdst[static_cast<size_t>(item) * kD + (tid - 128)] = zacc;
   tc_fence_before();
   __syncthreads();
   if (tid == 0 && !*abort_flag) {
@@ -878,12 +904,11 @@ int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, i
   PrefillArgs a{outZ, c.dev_err, T, splits, tp, hkv};
   int rc;
   if (fmap == kFmapReluProj) {
-    CUtensorMap tw;
-    if (!weights_tmap(&tw, W, hkv)) return -5;
     static std::atomic<uint64_t> prepared_p{0};
-    if (!prepare_kernel(k_prefill_proj_bf16, (int)kPrefProjSmem, prepared_p)) return -5;
-    rc = launch_pdl(k_prefill_proj_bf16, units * splits, kThreads, kPrefProjSmem, c.stream, tk, tv,
-                    to, tw, a);
+    if (!prepare_kernel(k_prefill_proj_bf16, (int)kPrefSmem, prepared_p)) return -5;
+    const PrefillProjArgs pa{a, static_cast<const uint16_t*>(W)};
+    rc = launch_pdl(k_prefill_proj_bf16, units * splits, kThreads, kPrefSmem, c.stream, tk, tv,
+                    to, pa);
   } else if (fmap == kFmapElu1) {
     static std::atomic<uint64_t> prepared_e{0};
     if (!prepare_kernel(k_prefill_bf16<kFmapElu1>, (int)kPrefSmem, prepared_e)) return -5;
