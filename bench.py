@@ -81,6 +81,15 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def source_sha256(src_file):
+    """sha256 over a kernel's source file and the device helpers it includes."""
+    h = hashlib.sha256()
+    for name in (src_file, "bha_ptx.cuh"):
+        with open(os.path.join(ROOT, "block_hybrid_linear_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def traffic_record(kernel, src_file):
     """dram bytes per launch from the committed ncu summary, if the kernel's
     source is unchanged since the capture (else None)."""
@@ -89,11 +98,7 @@ def traffic_record(kernel, src_file):
         return None
     with open(path) as f:
         rec = json.load(f).get(kernel)
-    if not rec:
-        return None
-    with open(os.path.join(ROOT, "block_hybrid_linear_b200", "csrc", src_file), "rb") as f:
-        sha = hashlib.sha256(f.read()).hexdigest()
-    if rec.get("source_sha256") != sha:
+    if not rec or rec.get("source_sha256") != source_sha256(src_file):
         return None
     return rec.get("dram_bytes_per_launch")
 

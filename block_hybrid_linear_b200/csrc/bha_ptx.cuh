@@ -138,6 +138,18 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, uint32_t src,
       : "memory");
 }
 
+// Global tile += shared tile (fp32 add, done at L2), same coordinates and
+// tensor map as tma_store_3d; the tile is read from shared memory
+// asynchronously (bulk group).
+__device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* m, uint32_t src, int c0,
+                                                  int c1, int c2) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.3d.global.shared::cta.add.tile.bulk_group"
+      " [%0, {%2, %3, %4}], [%1];" ::"l"(reinterpret_cast<uint64_t>(m)),
+      "r"(src), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_group() {
   asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
@@ -395,14 +407,6 @@ __device__ __forceinline__ uint32_t relu_bf16x2(uint32_t x) {
 constexpr int kFmapRelu = 0;       // phi(x) = max(x, 0)
 constexpr int kFmapElu1 = 1;       // phi(x) = x + 1 (x > 0), exp(x) (x <= 0)
 constexpr int kFmapReluProj = 2;   // phi(x) = max(x W, 0)
-
-// fp32 -> the nearest tf32 value (ties away from zero), in an fp32 register:
-// what the tensor core then reads from TMEM loses nothing more.
-__device__ __forceinline__ float round_tf32(float x) {
-  uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-  return __uint_as_float(r);
-}
 
 // elu + 1 of both lanes of a packed bf16 pair in packed bf16 arithmetic, as
 // a bf16 model evaluates it: max(1 + x, 2^(min(x, 0) * log2 e)).  For x <= 0

@@ -10,9 +10,10 @@
 // phi is applied in place, and the fp32 accumulator lives in TMEM.
 //
 // Commit: one CTA per (request, KV head): one MMA chain over the b block
-// tokens, then S is read-modified-written through a swizzled fp32 tile
-// (thread = row r, conflict-free) and stored back by TMA, one 64-column half
-// at a time.  Its operands are prefetched into L2 before the kernel waits
+// tokens gives phi(K)^T V in TMEM, which goes through a swizzled fp32 tile
+// (thread = row r, conflict-free) to a TMA reduce-add into S (the add is
+// done at L2, one 64-column half at a time): S never passes through the SM.
+// The operands, S included, are prefetched into L2 before the kernel waits
 // for the previous one.
 //
 // Prefill: one CTA per (unit, chunk of the prompt), a 3-stage TMA ring of
@@ -104,14 +105,13 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t base = (raw + 1023u) & ~1023u;
   const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + Lay::kTiles;
   uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
-  const uint32_t bar_kv = ctrl, bar_s = ctrl + 8, bar_done = ctrl + 16;
+  const uint32_t bar_kv = ctrl, bar_done = ctrl + 16;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 36);
 
   if (warp == 0) {
     if (lane == 0) {
       mbar_init(bar_kv, 1);
-      mbar_init(bar_s, 1);
       mbar_init(bar_done, 1);
       *abort_flag = 0;
       fence_mbar_init();
@@ -140,10 +140,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     tma_load_3d(base + Lay::kOffK + BPAD * 128, &tmK, bar_kv, 64, 0, u);
     tma_load_3d(base + Lay::kOffV, &tmV, bar_kv, 0, 0, u);
     tma_load_3d(base + Lay::kOffV + BPAD * 128, &tmV, bar_kv, 64, 0, u);
-    mbar_arrive_expect_tx(bar_s, kSBytes);
-#pragma unroll
-    for (int bx = 0; bx < 4; ++bx)
-      tma_load_3d(base + Lay::kOffS + bx * 16384, &tmS, bar_s, 32 * bx, 0, u);
   }
 
   // phi(K) in place
@@ -187,17 +183,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     a.z[static_cast<size_t>(u) * kD + rr] += s;
   }
 
-  ok = warp_all(mbar_wait(bar_s, 0, a.err, abort_flag) && mbar_wait(bar_done, 0, a.err, abort_flag));
+  ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag));
   tc_fence_after();
-  if (ok) accum_to_tile(tmem, base + Lay::kOffS, warp, lane, true);
+  if (ok) accum_to_tile(tmem, base + Lay::kOffS, warp, lane, false);
   fence_proxy_async_smem();
   tc_fence_before();
-  // each 64-column half is stored as soon as its four warps are done
+  // each 64-column half is added into S as soon as its four warps are done
   const int hb = warp >> 2;
   named_barrier_sync(1 + hb, 128);
-  if ((tid & 127) == 0 && !*abort_flag) {
-    tma_store_3d(&tmS, base + Lay::kOffS + (2 * hb) * 16384, 64 * hb, 0, u);
-    tma_store_3d(&tmS, base + Lay::kOffS + (2 * hb + 1) * 16384, 64 * hb + 32, 0, u);
+  if ((tid & 127) == 0 && ok && !*abort_flag) {
+    tma_reduce_add_3d(&tmS, base + Lay::kOffS + (2 * hb) * 16384, 64 * hb, 0, u);
+    tma_reduce_add_3d(&tmS, base + Lay::kOffS + (2 * hb + 1) * 16384, 64 * hb + 32, 0, u);
     bulk_commit_group();
     bulk_wait_group_read0();
   }
@@ -238,7 +234,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   const uint32_t base = (raw + 1023u) & ~1023u;
   const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + Lay::kTiles;
   uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
-  const uint32_t bar_kv = ctrl, bar_s = ctrl + 8, bar_done = ctrl + 16, bar_w = ctrl + 24,
+  const uint32_t bar_kv = ctrl, bar_done = ctrl + 16, bar_w = ctrl + 24,
                  bar_kw = ctrl + 40, bar_phik = ctrl + 48;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 32);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 36);
@@ -246,7 +242,6 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   if (warp == 0) {
     if (lane == 0) {
       mbar_init(bar_kv, 1);
-      mbar_init(bar_s, 1);
       mbar_init(bar_done, 1);
       mbar_init(bar_w, 1);
       mbar_init(bar_kw, 1);
@@ -283,10 +278,6 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     mbar_arrive_expect_tx(bar_w, 32768);
     tma_load_3d(base + Lay::kOffW, &tmW, bar_w, 0, 0, g);
     tma_load_3d(base + Lay::kOffW + 16384, &tmW, bar_w, 64, 0, g);
-    mbar_arrive_expect_tx(bar_s, kSBytes);
-#pragma unroll
-    for (int bx = 0; bx < 4; ++bx)
-      tma_load_3d(base + Lay::kOffS + bx * 16384, &tmS, bar_s, 32 * bx, 0, u);
   }
   if (tid == 128) {
     // (K W_g)^T[r][t] = sum_i W_g[i][r] K[t][i]: A = W_g MN-major, B = K K-major
@@ -348,17 +339,16 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     }
   }
 
-  const bool ok =
-      warp_all(mbar_wait(bar_s, 0, a.err, abort_flag) && mbar_wait(bar_done, 0, a.err, abort_flag));
+  const bool ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag));
   tc_fence_after();
-  if (ok) accum_to_tile(tmem, base + Lay::kOffS, warp, lane, true);
+  if (ok) accum_to_tile(tmem, base + Lay::kOffS, warp, lane, false);
   fence_proxy_async_smem();
   tc_fence_before();
   const int hb = warp >> 2;
   named_barrier_sync(1 + hb, 128);
-  if ((tid & 127) == 0 && !*abort_flag) {
-    tma_store_3d(&tmS, base + Lay::kOffS + (2 * hb) * 16384, 64 * hb, 0, u);
-    tma_store_3d(&tmS, base + Lay::kOffS + (2 * hb + 1) * 16384, 64 * hb + 32, 0, u);
+  if ((tid & 127) == 0 && ok && !*abort_flag) {
+    tma_reduce_add_3d(&tmS, base + Lay::kOffS + (2 * hb) * 16384, 64 * hb, 0, u);
+    tma_reduce_add_3d(&tmS, base + Lay::kOffS + (2 * hb + 1) * 16384, 64 * hb + 32, 0, u);
     bulk_commit_group();
     bulk_wait_group_read0();
   }

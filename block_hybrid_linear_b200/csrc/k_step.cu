@@ -32,8 +32,8 @@
 // kernel's tail.
 //
 // Projected map phi(q) = ReLU(q W_g): one more MMA (bf16) Q W_g -> TMEM,
-// M=128 N=128 K=128, into the columns phi(Q) occupies, then ReLU and tf32
-// rounding in TMEM.  W_g (32 KB, from L2: every unit of KV head g reads the
+// M=128 N=128 K=128, into the columns phi(Q) occupies, then the ReLU in
+// TMEM.  W_g (32 KB, from L2: every unit of KV head g reads the
 // same W_g) lands where state chunks 2-3 go; those two chunks are loaded
 // once the Q W_g product has read it, so shared memory and the two CTAs per
 // SM stay as they are.
@@ -85,14 +85,9 @@ __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu
 
 // phi(q_r) * scale as fp32 into TMEM (this thread's lane, columns [0, 128)
 // from `tcol`), read from row r of the SW128 Q tile; one wait for all four
-// 32-column stores.  Elementwise maps only: phi is a bf16 value (a tf32
-// value already); a scaled one is rounded to the nearest tf32.
-template <bool SCALED>
-__device__ __forceinline__ float phiq_tf32(float phi, float scale) {
-  return SCALED ? round_tf32(phi * scale) : phi;
-}
-
-template <int FMAP, bool SCALED>
+// 32-column stores.  Elementwise maps only (phi of a bf16 pair is a bf16
+// pair); the tensor core reads the values as tf32.
+template <int FMAP>
 __device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol, float scale) {
 #pragma unroll
   for (int cg = 0; cg < 4; ++cg) {
@@ -105,8 +100,8 @@ __device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol,
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const uint32_t p2 = phi_bf16x2<FMAP>(w4[e]);
-        f[8 * q + 2 * e] = phiq_tf32<SCALED>(__uint_as_float(p2 << 16), scale);
-        f[8 * q + 2 * e + 1] = phiq_tf32<SCALED>(__uint_as_float(p2 & 0xFFFF0000u), scale);
+        f[8 * q + 2 * e] = __uint_as_float(p2 << 16) * scale;
+        f[8 * q + 2 * e + 1] = __uint_as_float(p2 & 0xFFFF0000u) * scale;
       }
     }
     tmem_st32(tcol + cg * 32, f);
@@ -115,14 +110,14 @@ __device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol,
 }
 
 // Projected map: the Q W_g product sits in TMEM (this thread's lane, 128
-// columns from `tcol`); replace it by round_tf32(max(., 0) * scale).
+// columns from `tcol`); replace it by max(., 0) * scale.
 __device__ __forceinline__ void relu_tmem_phiq(uint32_t tcol, float scale) {
 #pragma unroll
   for (int cg = 0; cg < 4; ++cg) {
     float f[32];
     tmem_ld32_sync(tcol + cg * 32, f);
 #pragma unroll
-    for (int q = 0; q < 32; ++q) f[q] = round_tf32(fmaxf(f[q], 0.f) * scale);
+    for (int q = 0; q < 32; ++q) f[q] = fmaxf(f[q], 0.f) * scale;
     tmem_st32(tcol + cg * 32, f);
   }
   tmem_wait_st();
@@ -139,19 +134,19 @@ __device__ __forceinline__ float proj_qz(uint32_t tcol, const float* zu) {
 #pragma unroll
     for (int q = 0; q < 32; q += 4) {
       const float4 zz = __ldg(reinterpret_cast<const float4*>(zu + cg * 32 + q));
-      qz = fmaf(round_tf32(fmaxf(f[q], 0.f)), zz.x, qz);
-      qz = fmaf(round_tf32(fmaxf(f[q + 1], 0.f)), zz.y, qz);
-      qz = fmaf(round_tf32(fmaxf(f[q + 2], 0.f)), zz.z, qz);
-      qz = fmaf(round_tf32(fmaxf(f[q + 3], 0.f)), zz.w, qz);
+      qz = fmaf(fmaxf(f[q], 0.f), zz.x, qz);
+      qz = fmaf(fmaxf(f[q + 1], 0.f), zz.y, qz);
+      qz = fmaf(fmaxf(f[q + 2], 0.f), zz.z, qz);
+      qz = fmaf(fmaxf(f[q + 3], 0.f), zz.w, qz);
     }
   }
   return qz;
 }
 
 // COMMIT: also fold this step's block into the state after using it (the
-// block's last denoising step): S += phi(K)^T V, z += sum_t phi(k_t), with
-// the state tile already in shared memory updated in place and stored back.
-// P then lives in the consumed Q tile so that K survives for the commit MMA,
+// block's last denoising step): S += phi(K)^T V, z += sum_t phi(k_t); the
+// state is read once (the tile the step used) and phi(K)^T V goes over that
+// tile to a TMA reduce-add into S.  P then lives in the consumed Q tile so that K survives for the commit MMA,
 // and phi(K)^T V accumulates in the TMEM columns phi(Q) used.  Default mode
 // and a single 128-row tile per unit only; elementwise maps only.
 template <int BPAD, bool SHARED, bool COMMIT, int FMAP>
@@ -294,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       if (okw) relu_tmem_phiq(t_a + lane_base, 1.f);
     } else {
       const bool okq = warp_all(mbar_wait(bar_q, 0, a.err, abort_flag));
-      if (okq) write_phiq<FMAP, false>(base + kOffQ, warp * 32 + lane, t_a + lane_base, 1.f);
+      if (okq) write_phiq<FMAP>(base + kOffQ, warp * 32 + lane, t_a + lane_base, 1.f);
     }
     tc_fence_before();
     mbar_arrive(bar_a);
@@ -451,7 +446,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         if (PROJ)
           relu_tmem_phiq(t_a + lane_base, ascale);
         else
-          write_phiq<FMAP, true>(base + kOffQ, r, t_a + lane_base, ascale);
+          write_phiq<FMAP>(base + kOffQ, r, t_a + lane_base, ascale);
       }
       tc_fence_before();
       mbar_arrive(bar_a);
@@ -546,8 +541,9 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     bulk_commit_group();
   }
   if (COMMIT) {
-    // S += phi(K)^T V in the shared state tile (32-byte-chunk swizzle:
-    // chunk j of row rr of a 32 x 32 box sits at j ^ (rr % 4)), then store
+    // phi(K)^T V over the consumed state tile (32-byte-chunk swizzle: chunk
+    // j of row rr of a 32 x 32 box sits at j ^ (rr % 4)), then S += it by
+    // TMA reduce-add (the add is done at L2)
     const bool okc = warp_all(mbar_wait(bar_ds, 0, a.err, abort_flag));
     tc_fence_after();
     if (okc) {
@@ -561,17 +557,10 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint32_t addr = box + ((j ^ (rr & 3)) << 5);
-          float4 s0 = ld_shared_f4(addr), s1 = ld_shared_f4(addr + 16);
-          s0.x += dsv[8 * j + 0];
-          s0.y += dsv[8 * j + 1];
-          s0.z += dsv[8 * j + 2];
-          s0.w += dsv[8 * j + 3];
-          s1.x += dsv[8 * j + 4];
-          s1.y += dsv[8 * j + 5];
-          s1.z += dsv[8 * j + 6];
-          s1.w += dsv[8 * j + 7];
-          st_shared_f4(addr, s0);
-          st_shared_f4(addr + 16, s1);
+          st_shared_f4(addr, make_float4(dsv[8 * j], dsv[8 * j + 1], dsv[8 * j + 2],
+                                         dsv[8 * j + 3]));
+          st_shared_f4(addr + 16, make_float4(dsv[8 * j + 4], dsv[8 * j + 5], dsv[8 * j + 6],
+                                              dsv[8 * j + 7]));
         }
       }
     }
@@ -581,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     if (tid == 0 && okc && !*abort_flag) {
       for (int c = 0; c < 4; ++c)
         for (int nb = 0; nb < 4; ++nb)
-          tma_store_3d(&tmS, base + kOffS + c * 16384 + nb * 4096, 32 * nb, 32 * c, u);
+          tma_reduce_add_3d(&tmS, base + kOffS + c * 16384 + nb * 4096, 32 * nb, 32 * c, u);
       bulk_commit_group();
     }
   }

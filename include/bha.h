@@ -184,9 +184,10 @@ int bha_prefix_softmax(const void *Qa, const void *Kc, const void *Vc, int P,
  * keys use W[g] (queries by the GQA map), so phi keeps d features and S
  * stays d x d.  W must be non-NULL and 16-byte aligned for
  * BHA_FMAP_RELU_PROJ and NULL otherwise (BHA_ERR_INVALID_ARG), and must not
- * overlap an output.  The bf16 path applies phi in fp32 and rounds phi(k) to
- * bf16 for the tensor core (as a bf16 model does); phi(q) enters the
- * phi(q) S product as tf32 (10-bit mantissa, round to nearest).
+ * overlap an output.  The bf16 path evaluates elu + 1 in packed bf16
+ * arithmetic and rounds ReLU(x W_g) of keys to bf16 (phi(k) is a bf16 tensor-
+ * core operand, as in a bf16 model); phi(q) enters the phi(q) S product as
+ * tf32, like S.
  */
 typedef enum {
     BHA_FMAP_RELU = 0,

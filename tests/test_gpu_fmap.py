@@ -116,8 +116,8 @@ def test_step_fmap_bf16(case, fmap, shared):
 
 def test_step_proj_identity_equals_relu():
     """W_g = I makes the projected map ReLU: the projection of a bf16 q by I
-    is exact and both kernels round phi(q) (times e^{-m} in the shared mode)
-    to tf32 the same way, so the outputs are identical."""
+    is exact, so both kernels hand the tensor core the same phi(q) (times
+    e^{-m} in the shared mode) and the outputs are identical."""
     import torch
     n, hq, hkv, b = 2, 16, 4, 32
     Q, _ = bf16_case((71, 0), (n, hq, b, 128), STD)
