@@ -434,7 +434,8 @@ def run_native(args, rank, world, local):
                         "launch_us": commit_launch_ms * 1e3,
                         "achieved_gbs": fused_bytes / (commit_launch_ms / 1e3) / 1e9,
                         "frac_of_peak": fused_bytes / (commit_launch_ms / 1e3) / 1e9 / peak,
-                        "algorithmic_bytes_per_launch": fused_bytes},
+                        "algorithmic_bytes_per_launch": fused_bytes,
+                        "traffic": traffic_record("k_step_bf16_fused_commit", "k_step.cu")},
         "prefill": {"ms": prefill_ms, "tokens": N_ * P_,
                     "achieved_gbs": prefill_bytes / (prefill_ms / 1e3) / 1e9},
         "gpu_launches": steps * DENOISE,
