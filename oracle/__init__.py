@@ -177,6 +177,55 @@ def prefix_softmax(Q, Kc, Vc, P, K, V, scale=0.0):
     return Y
 
 
+def paged_cache(Kpool, Vpool, table, P_lens, page_size):
+    """The cache each request sees through its page table: token t of
+    request i is row t % page_size of page table[i][t // page_size] of the
+    pool ([num_pages, hkv, page_size, d]).  Returns per-request lists of
+    (Kc [hkv, P_i, d], Vc [hkv, P_i, d]) float64 arrays."""
+    Kpool, Vpool = _f64(Kpool), _f64(Vpool)
+    out = []
+    for i, P in enumerate(P_lens):
+        P = int(P)
+        pages = [int(table[i][t // page_size]) for t in range(P)]
+        rows = [t % page_size for t in range(P)]
+        Kc = np.stack([Kpool[p, :, r, :] for p, r in zip(pages, rows)], axis=1) if P else \
+            np.zeros((Kpool.shape[1], 0, Kpool.shape[3]))
+        Vc = np.stack([Vpool[p, :, r, :] for p, r in zip(pages, rows)], axis=1) if P else \
+            np.zeros((Vpool.shape[1], 0, Vpool.shape[3]))
+        out.append((Kc, Vc))
+    return out
+
+
+def prefix_softmax_paged(Q, Kpool, Vpool, table, P_lens, page_size, K, V, scale=0.0):
+    """Exact softmax attention of each request's active block over its own
+    cache (its first P_lens[i] tokens, read through its page table) followed
+    by the block.  Q [n, hq, b, d]; K, V [n, hkv, b, d].  Returns Y float64."""
+    Q, K, V = _f64(Q), _f64(K), _f64(V)
+    Y = np.zeros(Q.shape)
+    for i, (Kc, Vc) in enumerate(paged_cache(Kpool, Vpool, table, P_lens, page_size)):
+        P = Kc.shape[1]
+        Y[i:i + 1] = prefix_softmax(Q[i:i + 1], Kc[None], Vc[None], P, K[i:i + 1], V[i:i + 1],
+                                    scale)
+    return Y
+
+
+def state_prefill_ragged(K, V, T_lens, with_z=True, fmap=FMAP_RELU, W=None):
+    """Prefill of prompts of different lengths: request i folds its first
+    T_lens[i] tokens of K, V ([n, hkv, Tmax, d]; rows past T_lens[i] are
+    padding and ignored).  Returns (S [n, hkv, d, d], z [n, hkv, d] or None)."""
+    K, V = _f64(K), _f64(V)
+    n, hkv, _, d = K.shape
+    S = np.zeros((n, hkv, d, d))
+    z = np.zeros((n, hkv, d)) if with_z else None
+    for i, T in enumerate(T_lens):
+        T = int(T)
+        Si, zi = state_prefill(K[i:i + 1, :, :T], V[i:i + 1, :, :T], with_z, fmap, W)
+        S[i] = Si[0]
+        if with_z:
+            z[i] = zi[0]
+    return S, z
+
+
 def block_partition(L: int, B: int):
     """Block boundaries [0, B, 2B, ..., L] (last block may be short)."""
     k_max = (L + B - 1) // B if B > 0 else 0

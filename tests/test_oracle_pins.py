@@ -531,3 +531,114 @@ def test_fmap_pins_catch_planted_mistakes():
                                     oracle.FMAP_ELU1, None,
                                     lambda x, g: np_elu1(x) - 1.0)   # elu without +1
     assert e2 > 1e-3
+
+
+# ------------------------------------------------------------ ragged and paged batches
+# Per-request prefix lengths over a paged KV cache (the summary page pairs the
+# method with KV-cache management; its related work names PagedAttention) and
+# prompts of different lengths.
+
+def _scatter_pages(caches, page_size, num_pages, rng, fill=np.nan):
+    """Writes per-request contiguous caches [hkv, P_i, d] into a pool of pages
+    at random distinct page numbers; returns (pool, table)."""
+    hkv, d = caches[0].shape[0], caches[0].shape[2]
+    pool = np.full((num_pages, hkv, page_size, d), fill)
+    free = list(rng.permutation(num_pages))
+    max_pages = max(1, max((c.shape[1] + page_size - 1) // page_size for c in caches))
+    table = np.full((len(caches), max_pages), -1, dtype=np.int64)
+    for i, c in enumerate(caches):
+        for pg in range((c.shape[1] + page_size - 1) // page_size):
+            p = free.pop()
+            table[i, pg] = p
+            rows = c[:, pg * page_size:(pg + 1) * page_size, :]
+            pool[p, :, :rows.shape[1], :] = rows
+    return pool, table
+
+
+def _paged_case(seed, P_lens, page_size, n_extra_pages=5):
+    rng = np.random.default_rng(seed)
+    n, hq, hkv, b, d = len(P_lens), 4, 2, 5, 16
+    Kc = [rng.standard_normal((hkv, P, d)) for P in P_lens]
+    Vc = [rng.standard_normal((hkv, P, d)) for P in P_lens]
+    pages = sum((P + page_size - 1) // page_size for P in P_lens) + n_extra_pages
+    rng2 = np.random.default_rng(seed + 1)
+    Kpool, table = _scatter_pages(Kc, page_size, pages, rng2)
+    rng2 = np.random.default_rng(seed + 1)      # same page choice for V
+    Vpool, table_v = _scatter_pages(Vc, page_size, pages, rng2)
+    assert np.array_equal(table, table_v)
+    Q = rng.standard_normal((n, hq, b, d))
+    K = rng.standard_normal((n, hkv, b, d))
+    V = rng.standard_normal((n, hkv, b, d))
+    return Q, K, V, Kc, Vc, Kpool, Vpool, table
+
+
+@pytest.mark.parametrize("page_size", [1, 4, 16])
+def test_paged_prefix_equals_sdpa_per_request(page_size):
+    """Each request's output equals library softmax attention over its own
+    cache followed by its block; unused pool slots hold NaN and must not
+    matter."""
+    P_lens = [0, 7, 16, 33]
+    Q, K, V, Kc, Vc, Kpool, Vpool, table = _paged_case(11, P_lens, page_size)
+    Y = oracle.prefix_softmax_paged(Q, Kpool, Vpool, table, P_lens, page_size, K, V)
+    assert np.all(np.isfinite(Y))
+    for i, P in enumerate(P_lens):
+        ref = sdpa(Q[i:i + 1], np.concatenate([Kc[i][None], K[i:i + 1]], axis=2),
+                   np.concatenate([Vc[i][None], V[i:i + 1]], axis=2))
+        np.testing.assert_allclose(Y[i:i + 1], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_paged_prefix_page_order_invariance():
+    """Renumbering the pool's pages (and the table with them) changes nothing."""
+    P_lens = [5, 20, 13]
+    Q, K, V, _, _, Kpool, Vpool, table = _paged_case(12, P_lens, 4)
+    Y = oracle.prefix_softmax_paged(Q, Kpool, Vpool, table, P_lens, 4, K, V)
+    perm = np.random.default_rng(3).permutation(Kpool.shape[0])
+    inv = np.argsort(perm)
+    table2 = np.where(table >= 0, inv[np.maximum(table, 0)], -1)
+    Y2 = oracle.prefix_softmax_paged(Q, Kpool[perm], Vpool[perm], table2, P_lens, 4, K, V)
+    assert np.array_equal(Y, Y2)
+
+
+def test_paged_prefix_pins_catch_planted_mistakes():
+    """A gather reading the wrong row of a page, or every request through
+    request 0's table, fails the per-request SDPA pin."""
+    P_lens = [6, 11]
+    Q, K, V, Kc, Vc, Kpool, Vpool, table = _paged_case(13, P_lens, 4)
+
+    def check(gather):
+        for i, (kc, vc) in enumerate(gather):
+            ref = sdpa(Q[i:i + 1], np.concatenate([Kc[i][None], K[i:i + 1]], axis=2),
+                       np.concatenate([Vc[i][None], V[i:i + 1]], axis=2))
+            got = oracle.prefix_softmax(Q[i:i + 1], kc[None], vc[None], kc.shape[1],
+                                        K[i:i + 1], V[i:i + 1])
+            if not np.allclose(got, ref, rtol=1e-9, atol=1e-9):
+                return False
+        return True
+
+    good = oracle.paged_cache(Kpool, Vpool, table, P_lens, 4)
+    assert check(good)
+    shifted = [(np.stack([Kpool[table[i][t // 4], :, (t + 1) % 4] for t in range(P)], 1),
+                np.stack([Vpool[table[i][t // 4], :, (t + 1) % 4] for t in range(P)], 1))
+               for i, P in enumerate(P_lens)]
+    assert not check(shifted)
+    wrong_table = oracle.paged_cache(Kpool, Vpool, [table[0], table[0]], [6, 6], 4)
+    assert not check(wrong_table)
+
+
+def test_ragged_prefill_equals_per_request_numpy():
+    """Request i folds exactly its first T_i tokens; padding rows hold NaN."""
+    rng = np.random.default_rng(21)
+    n, hkv, Tmax, d = 4, 2, 40, 16
+    T_lens = [0, 1, 17, 40]
+    K = rng.standard_normal((n, hkv, Tmax, d))
+    V = rng.standard_normal((n, hkv, Tmax, d))
+    for i, T in enumerate(T_lens):
+        K[i, :, T:] = np.nan
+        V[i, :, T:] = np.nan
+    S, z = oracle.state_prefill_ragged(K, V, T_lens)
+    for i, T in enumerate(T_lens):
+        fk = np.maximum(K[i, :, :T], 0.0)
+        np.testing.assert_allclose(S[i], np.einsum("htr,htc->hrc", fk, V[i, :, :T]),
+                                   rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(z[i], fk.sum(axis=1), rtol=1e-12, atol=1e-12)
+    assert np.all(S[0] == 0) and np.all(z[0] == 0)
