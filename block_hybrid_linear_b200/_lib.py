@@ -33,7 +33,8 @@ EXPORTED = [
     "bha_status_string", "bha_version", "bha_state_prefill_workspace_size",
     "bha_state_prefill", "bha_state_prefill_noalloc", "bha_state_commit", "bha_hybrid_step",
     "bha_hybrid_step_commit", "bha_state_prefill_fm", "bha_state_commit_fm",
-    "bha_hybrid_step_fm", "bha_hybrid_step_commit_fm",
+    "bha_hybrid_step_fm", "bha_hybrid_step_commit_fm", "bha_prefix_softmax_paged_workspace_size",
+    "bha_prefix_softmax_paged", "bha_state_prefill_ragged",
     "bha_prefix_softmax_workspace_size", "bha_prefix_softmax",
     "bha_block_partition", "bha_device_error", "bha_selftest_timeout",
 ]
@@ -86,6 +87,14 @@ def lib():
         L.bha_hybrid_step_commit_fm.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, fl, u,
                                                 i, i, vp, vp]
         L.bha_hybrid_step_commit_fm.restype = i
+        L.bha_prefix_softmax_paged_workspace_size.argtypes = [i, i, i, i, i, i, i, i]
+        L.bha_prefix_softmax_paged_workspace_size.restype = sz
+        L.bha_prefix_softmax_paged.argtypes = [vp, vp, vp, i, i, vp, i, vp, vp, vp, vp, i, i, i,
+                                               i, i, fl, i, vp, sz, vp]
+        L.bha_prefix_softmax_paged.restype = i
+        L.bha_state_prefill_ragged.argtypes = [vp, vp, vp, i, i, i, i, i, i, vp, vp, vp, vp, sz,
+                                               vp]
+        L.bha_state_prefill_ragged.restype = i
         L.bha_prefix_softmax_workspace_size.argtypes = [i, i, i, i, i, i, i]
         L.bha_prefix_softmax_workspace_size.restype = sz
         L.bha_prefix_softmax.argtypes = [vp, vp, vp, i, i, vp, vp, vp, i, i, i, i,
@@ -257,3 +266,38 @@ def bha_prefix_softmax(Q, Kc, Vc, P, K, V, Y, scale=0.0, workspace=None, stream=
                                     _ptr(V), _ptr(Y), n, hq, hkv, b, d, float(scale),
                                     _dtype(Q), _ptr(workspace), ws_bytes, _stream(stream)),
            "bha_prefix_softmax")
+
+
+def bha_prefix_softmax_paged_workspace_size(n, hq, hkv, b, d, max_pages, page_size,
+                                            dtype=BHA_BF16):
+    return lib().bha_prefix_softmax_paged_workspace_size(n, hq, hkv, b, d, max_pages, page_size,
+                                                         dtype)
+
+
+def bha_prefix_softmax_paged(Q, Kpool, Vpool, block_table, P_lens, K, V, Y, scale=0.0,
+                             workspace=None, stream=None):
+    """Exact softmax of each request over its own paged cache, then its block.
+
+    Kpool, Vpool: [num_pages, hkv, page_size, d]; block_table: [n, max_pages]
+    int32 (device); P_lens: [n] int32 (device)."""
+    n, hq, b, d = Q.shape
+    num_pages, hkv, page_size, _ = Kpool.shape
+    max_pages = block_table.shape[1]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().bha_prefix_softmax_paged(_ptr(Q), _ptr(Kpool), _ptr(Vpool), num_pages,
+                                          page_size, _ptr(block_table), max_pages, _ptr(P_lens),
+                                          _ptr(K), _ptr(V), _ptr(Y), n, hq, hkv, b, d,
+                                          float(scale), _dtype(Q), _ptr(workspace), ws_bytes,
+                                          _stream(stream)), "bha_prefix_softmax_paged")
+
+
+def bha_state_prefill_ragged(K, V, T_lens, S, z=None, fmap=BHA_FMAP_RELU, W=None, workspace=None,
+                             stream=None):
+    """Prefill of prompts of different lengths: K, V [n, hkv, Tmax, d]; T_lens
+    [n] int32 (device)."""
+    n, hkv, T, d = K.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().bha_state_prefill_ragged(_ptr(K), _ptr(V), _ptr(T_lens), n, hkv, T, d,
+                                          _dtype(K), int(fmap), _ptr(W), _ptr(S), _ptr(z),
+                                          _ptr(workspace), ws_bytes, _stream(stream)),
+           "bha_state_prefill_ragged")

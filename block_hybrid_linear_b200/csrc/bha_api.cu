@@ -74,6 +74,8 @@ int make_ctx(bha_stream_t stream, bha_dtype dtype, Ctx* c) {
 
 bool misaligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) != 0; }
 
+bool misaligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) != 0; }
+
 bool overlap(const void* a, size_t na, const void* b, size_t nb) {
   if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
@@ -234,9 +236,14 @@ int bha_state_prefill(const void* K, const void* V, int n, int hkv, int T, int d
                               workspace_bytes, stream);
 }
 
-int bha_state_prefill_fm(const void* K, const void* V, int n, int hkv, int T, int d,
-                         bha_dtype dtype, bha_fmap fmap, const void* W, float* S, float* z,
-                         void* workspace, size_t workspace_bytes, bha_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// bha_state_prefill_fm with optional ragged prompt lengths (device, [n]).
+int prefill_impl(const void* K, const void* V, const int* T_lens, int n, int hkv, int T, int d,
+                 bha_dtype dtype, bha_fmap fmap, const void* W, float* S, float* z,
+                 void* workspace, size_t workspace_bytes, bha_stream_t stream) {
   int st = check_dims(dtype, d, 1);
   if (st != BHA_OK) return st;
   st = check_fmap(fmap, W);
@@ -258,7 +265,11 @@ int bha_state_prefill_fm(const void* K, const void* V, int n, int hkv, int T, in
   if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BHA_ERR_WORKSPACE;
   if (need > 0 && (overlap(workspace, need, S, s_bytes) || overlap(workspace, need, z, z_bytes) ||
                    overlap(workspace, need, K, kv_bytes) || overlap(workspace, need, V, kv_bytes) ||
-                   overlap(workspace, need, W, wb)))
+                   overlap(workspace, need, W, wb) ||
+                   overlap(workspace, need, T_lens, static_cast<size_t>(n) * 4)))
+    return BHA_ERR_INVALID_ARG;
+  if (overlap(T_lens, static_cast<size_t>(n) * 4, S, s_bytes) ||
+      overlap(T_lens, static_cast<size_t>(n) * 4, z, z_bytes))
     return BHA_ERR_INVALID_ARG;
   Ctx c;
   st = make_ctx(stream, dtype, &c);
@@ -266,9 +277,30 @@ int bha_state_prefill_fm(const void* K, const void* V, int n, int hkv, int T, in
   if (dtype == BHA_F32)
     return launch_status(launch_prefill_f32(c, static_cast<const float*>(K),
                                             static_cast<const float*>(V), (int)units, T, d, S, z,
-                                            fmap, static_cast<const float*>(W), hkv));
+                                            fmap, static_cast<const float*>(W), hkv, T_lens));
   return launch_status(launch_prefill_bf16(c, K, V, (int)units, T, S, z, workspace,
-                                           workspace_bytes, fmap, W, hkv));
+                                           workspace_bytes, fmap, W, hkv, T_lens));
+}
+
+}  // namespace
+
+extern "C" {
+
+int bha_state_prefill_fm(const void* K, const void* V, int n, int hkv, int T, int d,
+                         bha_dtype dtype, bha_fmap fmap, const void* W, float* S, float* z,
+                         void* workspace, size_t workspace_bytes, bha_stream_t stream) {
+  return prefill_impl(K, V, nullptr, n, hkv, T, d, dtype, fmap, W, S, z, workspace,
+                      workspace_bytes, stream);
+}
+
+int bha_state_prefill_ragged(const void* K, const void* V, const int* T_lens, int n, int hkv,
+                             int Tmax, int d, bha_dtype dtype, bha_fmap fmap, const void* W,
+                             float* S, float* z, void* workspace, size_t workspace_bytes,
+                             bha_stream_t stream) {
+  if (n > 0 && T_lens == nullptr) return BHA_ERR_INVALID_ARG;
+  if (misaligned4(T_lens)) return BHA_ERR_MISALIGNED;
+  return prefill_impl(K, V, T_lens, n, hkv, Tmax, d, dtype, fmap, W, S, z, workspace,
+                      workspace_bytes, stream);
 }
 
 int bha_state_commit(const void* Kb, const void* Vb, int n, int hkv, int b, int d,
@@ -468,6 +500,70 @@ int bha_prefix_softmax(const void* Qa, const void* Kc, const void* Vc, int P, in
         static_cast<const float*>(Va), static_cast<float*>(Y), n, hq, hkv, b, d, sc));
   return launch_status(launch_prefix_bf16(c, Qa, Kc, Vc, P, cap, Ka, Va, Y, n, hq, hkv, b, sc,
                                           workspace, workspace_bytes));
+}
+
+size_t bha_prefix_softmax_paged_workspace_size(int n, int hq, int hkv, int b, int d,
+                                               int max_pages, int page_size, bha_dtype dtype) {
+  if (max_pages < 1 || page_size < 1 || static_cast<long long>(max_pages) * page_size > (1 << 30))
+    return 0;
+  return bha_prefix_softmax_workspace_size(n, hq, hkv, b, d, max_pages * page_size, dtype);
+}
+
+int bha_prefix_softmax_paged(const void* Qa, const void* Kpool, const void* Vpool, int num_pages,
+                             int page_size, const int* block_table, int max_pages,
+                             const int* P_lens, const void* Ka, const void* Va, void* Y, int n,
+                             int hq, int hkv, int b, int d, float scale, bha_dtype dtype,
+                             void* workspace, size_t workspace_bytes, bha_stream_t stream) {
+  int st = check_dims(dtype, d, b);
+  if (st != BHA_OK) return st;
+  if (n < 0 || hq < 1 || hkv < 1 || hq % hkv != 0 || num_pages < 1 || max_pages < 1)
+    return BHA_ERR_INVALID_ARG;
+  int ps_log2 = 0;
+  while ((1 << ps_log2) < page_size && ps_log2 < 30) ++ps_log2;
+  if (page_size < 16 || page_size > 256 || (1 << ps_log2) != page_size)
+    return BHA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(max_pages) * page_size > (1 << 30) ||
+      static_cast<long long>(num_pages) * hkv > (1ll << 31) - 1)
+    return BHA_ERR_UNSUPPORTED;
+  if (n == 0) return BHA_OK;
+  if (Qa == nullptr || Kpool == nullptr || Vpool == nullptr || block_table == nullptr ||
+      P_lens == nullptr || Ka == nullptr || Va == nullptr || Y == nullptr)
+    return BHA_ERR_INVALID_ARG;
+  if (misaligned(Qa) || misaligned(Kpool) || misaligned(Vpool) || misaligned(Ka) ||
+      misaligned(Va) || misaligned(Y) || misaligned(workspace) || misaligned4(block_table) ||
+      misaligned4(P_lens))
+    return BHA_ERR_MISALIGNED;
+  const size_t es = esize(dtype);
+  const size_t q_bytes = static_cast<size_t>(n) * hq * b * d * es;
+  const size_t kv_bytes = static_cast<size_t>(n) * hkv * b * d * es;
+  const size_t pool_bytes = static_cast<size_t>(num_pages) * hkv * page_size * d * es;
+  const size_t t_bytes = static_cast<size_t>(n) * max_pages * 4;
+  const size_t p_bytes = static_cast<size_t>(n) * 4;
+  if (overlap(Y, q_bytes, Qa, q_bytes) || overlap(Y, q_bytes, Ka, kv_bytes) ||
+      overlap(Y, q_bytes, Va, kv_bytes) || overlap(Y, q_bytes, Kpool, pool_bytes) ||
+      overlap(Y, q_bytes, Vpool, pool_bytes) || overlap(Y, q_bytes, block_table, t_bytes) ||
+      overlap(Y, q_bytes, P_lens, p_bytes))
+    return BHA_ERR_INVALID_ARG;
+  const size_t need =
+      bha_prefix_softmax_paged_workspace_size(n, hq, hkv, b, d, max_pages, page_size, dtype);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BHA_ERR_WORKSPACE;
+  if (need > 0 &&
+      (overlap(workspace, need, Y, q_bytes) || overlap(workspace, need, Qa, q_bytes) ||
+       overlap(workspace, need, Kpool, pool_bytes) || overlap(workspace, need, Vpool, pool_bytes) ||
+       overlap(workspace, need, block_table, t_bytes) || overlap(workspace, need, P_lens, p_bytes)))
+    return BHA_ERR_INVALID_ARG;
+  Ctx c;
+  st = make_ctx(stream, dtype, &c);
+  if (st != BHA_OK) return st;
+  const float sc = resolve_scale(scale, d);
+  const PagedCache pg{block_table, P_lens, max_pages, ps_log2, num_pages};
+  if (dtype == BHA_F32)
+    return launch_status(launch_prefix_paged_f32(
+        c, static_cast<const float*>(Qa), static_cast<const float*>(Kpool),
+        static_cast<const float*>(Vpool), pg, static_cast<const float*>(Ka),
+        static_cast<const float*>(Va), static_cast<float*>(Y), n, hq, hkv, b, d, sc));
+  return launch_status(launch_prefix_paged_bf16(c, Qa, Kpool, Vpool, pg, Ka, Va, Y, n, hq, hkv,
+                                                b, sc, workspace, workspace_bytes));
 }
 
 }  // extern "C"

@@ -67,7 +67,8 @@ int launch_step_f32(const Ctx& c, const float* Q, const float* K, const float* V
 int launch_commit_f32(const Ctx& c, const float* K, const float* V, int units, int b, int d,
                       float* S, float* z, int fmap, const float* W, int hkv);
 int launch_prefill_f32(const Ctx& c, const float* K, const float* V, int units, int T, int d,
-                       float* S, float* z, int fmap, const float* W, int hkv);
+                       float* S, float* z, int fmap, const float* W, int hkv,
+                       const int* T_lens = nullptr);
 int launch_prefix_f32(const Ctx& c, const float* Q, const float* Kc, const float* Vc, int P,
                       int cap, const float* K, const float* V, float* Y, int n, int hq, int hkv,
                       int b, int d, float scale);
@@ -84,9 +85,27 @@ int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, 
 int launch_commit_bf16(const Ctx& c, const void* K, const void* V, int units, int b, float* S,
                        float* z, int fmap, const void* W, int hkv);
 size_t prefill_bf16_workspace(int units, int T);
+// T_lens (device, [n], or null): ragged prompts of at most T tokens each.
 int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, int T, float* S,
-                        float* z, void* ws, size_t ws_bytes, int fmap, const void* W, int hkv);
+                        float* z, void* ws, size_t ws_bytes, int fmap, const void* W, int hkv,
+                        const int* T_lens = nullptr);
 size_t prefix_bf16_workspace(int n, int hq, int hkv, int b, int P);
+// A paged KV cache: request i's token t at row t % 2^ps_log2 of page
+// table[i * max_pages + (t >> ps_log2)] of a pool of num_pages pages
+// [num_pages][hkv][page_size][d]; P_lens[i] cached tokens (device arrays).
+struct PagedCache {
+  const int* table;
+  const int* P_lens;
+  int max_pages;
+  int ps_log2;
+  int num_pages;
+};
+int launch_prefix_paged_bf16(const Ctx& c, const void* Q, const void* Kpool, const void* Vpool,
+                             const PagedCache& pg, const void* K, const void* V, void* Y, int n,
+                             int hq, int hkv, int b, float scale, void* ws, size_t ws_bytes);
+int launch_prefix_paged_f32(const Ctx& c, const float* Q, const float* Kpool, const float* Vpool,
+                            const PagedCache& pg, const float* K, const float* V, float* Y, int n,
+                            int hq, int hkv, int b, int d, float scale);
 int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* Vc, int P,
                        int cap, const void* K, const void* V, void* Y, int n, int hq, int hkv,
                        int b, float scale, void* ws, size_t ws_bytes);

@@ -129,34 +129,47 @@ __global__ void __launch_bounds__(kThreads) k_state_f32(const float* __restrict_
                                                         int d, float* __restrict__ S,
                                                         float* __restrict__ z, int accumulate,
                                                         int fmap, const float* __restrict__ W,
-                                                        int hkv) {
+                                                        int hkv, const int* __restrict__ T_lens) {
   const int u = blockIdx.y;
   const int e = blockIdx.x * kThreads + threadIdx.x;
   const float* Ku = K + (size_t)u * T * d;
   const float* Vu = V + (size_t)u * T * d;
+  // ragged prompts: this request's own length; rows past it are padding
+  const int Tu = T_lens ? min(max(T_lens[u / hkv], 0), T) : T;
   const float* Wg = W ? W + (size_t)(u % hkv) * d * d : nullptr;
   if (e < d * d) {
     const int r = e / d, c = e % d;
     float acc = 0.f;
-    for (int t = 0; t < T; ++t)
+    for (int t = 0; t < Tu; ++t)
       acc = fmaf(phi_at(Ku + (size_t)t * d, r, d, fmap, Wg), Vu[(size_t)t * d + c], acc);
     float* dst = S + (size_t)u * d * d + e;
     *dst = accumulate ? *dst + acc : acc;
   }
   if (z && e < d) {
     float acc = 0.f;
-    for (int t = 0; t < T; ++t) acc += phi_at(Ku + (size_t)t * d, e, d, fmap, Wg);
+    for (int t = 0; t < Tu; ++t) acc += phi_at(Ku + (size_t)t * d, e, d, fmap, Wg);
     float* dst = z + (size_t)u * d + e;
     *dst = accumulate ? *dst + acc : acc;
   }
 }
 
+// A paged cache for the exact path (null table: contiguous [n][hkv][cap][d]).
+struct PagedF32 {
+  const int* table;   // [n][max_pages]
+  const int* P_lens;  // [n]
+  int max_pages;
+  int ps_log2;
+  int num_pages;      // page numbers outside [0, num_pages) read as zero rows
+};
+
 // Exact softmax over [cache[0:P] || block]: one CTA per (request, head, row);
-// keys are scored 128 at a time with an online max / sum rescale.
+// keys are scored 128 at a time with an online max / sum rescale.  Paged:
+// request ni's cache is its first P_lens[ni] tokens, token j at row
+// j % page_size of page table[ni][j / page_size] of [pages][hkv][page_size][d].
 __global__ void __launch_bounds__(kThreads) k_prefix_f32(
     const float* __restrict__ Q, const float* __restrict__ Kc, const float* __restrict__ Vc,
     int P, int cap, const float* __restrict__ K, const float* __restrict__ V,
-    float* __restrict__ Y, int hq, int hkv, int b, int d, float scale) {
+    float* __restrict__ Y, int hq, int hkv, int b, int d, float scale, PagedF32 pg) {
   extern __shared__ float sm[];
   float* sq = sm;           // [d]
   float* se = sq + d;       // [kThreads]
@@ -167,8 +180,19 @@ __global__ void __launch_bounds__(kThreads) k_prefix_f32(
   const int i = id % b, nh = id / b;
   const int ni = nh / hq, h = nh % hq, g = h / (hq / hkv);
   const size_t row = (((size_t)ni * hq + h) * b + i) * d;
-  const float* Kcg = Kc + ((size_t)ni * hkv + g) * cap * d;
-  const float* Vcg = Vc + ((size_t)ni * hkv + g) * cap * d;
+  const float* Kcg = pg.table ? Kc : Kc + ((size_t)ni * hkv + g) * cap * d;
+  const float* Vcg = pg.table ? Vc : Vc + ((size_t)ni * hkv + g) * cap * d;
+  if (pg.table) P = min(max(pg.P_lens[ni], 0), pg.max_pages << pg.ps_log2);
+  const int ps_mask = (1 << pg.ps_log2) - 1;
+  __shared__ float zrow[128];   // the row of a page number out of range
+  for (int c = threadIdx.x; c < d; c += kThreads) zrow[c] = 0.f;
+  // cached token jj's row of the cache at cb (K or V)
+  auto cache_row = [&](const float* cb, int jj) -> const float* {
+    if (!pg.table) return cb + (size_t)jj * d;
+    const int page = pg.table[(size_t)ni * pg.max_pages + (jj >> pg.ps_log2)];
+    if (page < 0 || page >= pg.num_pages) return zrow;
+    return cb + (((size_t)page * hkv + g) * ((size_t)ps_mask + 1) + (jj & ps_mask)) * d;
+  };
   const float* Kg = K + ((size_t)ni * hkv + g) * b * d;
   const float* Vg = V + ((size_t)ni * hkv + g) * b * d;
   for (int c = threadIdx.x; c < d; c += kThreads) {
@@ -182,7 +206,7 @@ __global__ void __launch_bounds__(kThreads) k_prefix_f32(
     const int j = j0 + threadIdx.x;
     float s = -INFINITY;
     if (j < L) {
-      const float* k = j < P ? Kcg + (size_t)j * d : Kg + (size_t)(j - P) * d;
+      const float* k = j < P ? cache_row(Kcg, j) : Kg + (size_t)(j - P) * d;
       float a = 0.f;
       for (int c = 0; c < d; ++c) a = fmaf(sq[c], k[c], a);
       s = a * scale;
@@ -199,7 +223,7 @@ __global__ void __launch_bounds__(kThreads) k_prefix_f32(
       float a = acc[c] * corr;
       for (int t = 0; t < cnt; ++t) {
         const int jj = j0 + t;
-        const float* v = jj < P ? Vcg + (size_t)jj * d : Vg + (size_t)(jj - P) * d;
+        const float* v = jj < P ? cache_row(Vcg, jj) : Vg + (size_t)(jj - P) * d;
         a = fmaf(se[t], v[c], a);
       }
       acc[c] = a;
@@ -229,14 +253,15 @@ int launch_step_f32(const Ctx& c, const float* Q, const float* K, const float* V
 int launch_commit_f32(const Ctx& c, const float* K, const float* V, int units, int b, int d,
                       float* S, float* z, int fmap, const float* W, int hkv) {
   dim3 grid((d * d + kThreads - 1) / kThreads, units);
-  k_state_f32<<<grid, kThreads, 0, c.stream>>>(K, V, b, d, S, z, 1, fmap, W, hkv);
+  k_state_f32<<<grid, kThreads, 0, c.stream>>>(K, V, b, d, S, z, 1, fmap, W, hkv, nullptr);
   return finish_launch();
 }
 
 int launch_prefill_f32(const Ctx& c, const float* K, const float* V, int units, int T, int d,
-                       float* S, float* z, int fmap, const float* W, int hkv) {
+                       float* S, float* z, int fmap, const float* W, int hkv,
+                       const int* T_lens) {
   dim3 grid((d * d + kThreads - 1) / kThreads, units);
-  k_state_f32<<<grid, kThreads, 0, c.stream>>>(K, V, T, d, S, z, 0, fmap, W, hkv);
+  k_state_f32<<<grid, kThreads, 0, c.stream>>>(K, V, T, d, S, z, 0, fmap, W, hkv, T_lens);
   return finish_launch();
 }
 
@@ -245,7 +270,17 @@ int launch_prefix_f32(const Ctx& c, const float* Q, const float* Kc, const float
                       int b, int d, float scale) {
   const size_t smem = (size_t)(2 * d + kThreads) * sizeof(float);
   k_prefix_f32<<<n * hq * b, kThreads, smem, c.stream>>>(Q, Kc, Vc, P, cap, K, V, Y, hq, hkv,
-                                                         b, d, scale);
+                                                         b, d, scale, PagedF32{});
+  return finish_launch();
+}
+
+int launch_prefix_paged_f32(const Ctx& c, const float* Q, const float* Kpool, const float* Vpool,
+                            const PagedCache& pg, const float* K, const float* V, float* Y, int n,
+                            int hq, int hkv, int b, int d, float scale) {
+  const size_t smem = (size_t)(2 * d + kThreads) * sizeof(float);
+  const PagedF32 p{pg.table, pg.P_lens, pg.max_pages, pg.ps_log2, pg.num_pages};
+  k_prefix_f32<<<n * hq * b, kThreads, smem, c.stream>>>(Q, Kpool, Vpool, 0, 0, K, V, Y, hq, hkv,
+                                                         b, d, scale, p);
   return finish_launch();
 }
 

@@ -16,6 +16,16 @@
 //   * chunks are combined by log-sum-exp in a second kernel, the way the
 //     LoSA page describes merging prefix and block attention with online
 //     softmax.  With one chunk the CTA normalises and stores Y itself.
+// Paged variant (the summary page pairs the method with KV-cache management;
+// its related work names PagedAttention): the cache of request i is its first
+// P_lens[i] tokens, token t at row t % page_size of page block_table[i][t /
+// page_size] of a pool [pages][hkv][page_size][128].  A 128-key tile is one
+// TMA box per page (page_size < 128: 128 / page_size boxes, pages past the
+// request's cache not loaded; page_size >= 128: part of one page).  The plan
+// covers the longest possible cache; a chunk past a request's cache leaves a
+// neutral partial (row max -inf, sum 0) that the merge skips.  Rows past the
+// cache in its last tile hold stale pool data: their scores are masked and
+// their V rows zeroed before P V.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -43,6 +53,12 @@ constexpr int kMinTilesPerChunk = 8;
 
 struct PrefixArgs {
   int* err;
+  const int* table;  // paged: [n][max_pages] page numbers
+  const int* P_lens; // paged: [n] cached tokens per request
+  int max_pages;
+  int ps_log2;       // paged: log2(page_size)
+  int hkv;
+  int Pmax;          // paged: max_pages * page_size
   float* wsO;        // [items][128][128] fp32 partial numerators (splits > 1)
   float* wsML;       // [items][2][128] row max (log2 units) and row sum
   int rows;          // G * b
@@ -57,6 +73,7 @@ struct PrefixArgs {
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
+template <bool PAGED>
 __global__ void __launch_bounds__(kThreads, 1)
     k_prefix_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                   const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKa,
@@ -68,9 +85,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int sp = item % a.splits;
   const int umt = item / a.splits;
   const int u = umt / a.mtiles, mt = umt % a.mtiles;
-  const int ntot = a.ncache_tiles + 1;
   const int tile0 = sp * a.tiles_per;
-  const int nt = min(a.tiles_per, ntot - tile0);
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -108,27 +123,59 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t t_o = tmem + 256;
   pdl_wait();
 
+  // this request's cache length (per request when paged), tiles of this chunk
+  const int nreq = u / a.hkv, g = u % a.hkv;
+  const int P = PAGED ? min(max(__ldg(a.P_lens + nreq), 0), a.Pmax) : a.P;
+  const int ncache_tiles = PAGED ? (P + kTK - 1) / kTK : a.ncache_tiles;
+  const int nt = max(0, min(a.tiles_per, ncache_tiles + 1 - tile0));
+
   if (tid == 0) {
     // ---------------- TMA producer
     const int row0 = mt * 128;
     mbar_arrive_expect_tx(bar_q, kTileBytes);
     tma_load_3d(base + kOffQ, &tmQ, bar_q, 0, row0, u);
     tma_load_3d(base + kOffQ + 16384, &tmQ, bar_q, 64, row0, u);
+    // loads one K or V tile of the cache (through the page table) or of the block
+    auto load_tile = [&](const CUtensorMap* mc, const CUtensorMap* ma, uint32_t dst, uint32_t bar,
+                         int gi) {
+      if (gi >= ncache_tiles) {
+        mbar_arrive_expect_tx(bar, kTileBytes);
+        tma_load_3d(dst, ma, bar, 0, 0, u);
+        tma_load_3d(dst + 16384, ma, bar, 64, 0, u);
+      } else if (!PAGED) {
+        mbar_arrive_expect_tx(bar, kTileBytes);
+        tma_load_3d(dst, mc, bar, 0, gi * kTK, u);
+        tma_load_3d(dst + 16384, mc, bar, 64, gi * kTK, u);
+      } else {
+        const int t0 = gi * kTK;
+        const int* trow = a.table + static_cast<size_t>(nreq) * a.max_pages;
+        if (a.ps_log2 >= 7) {
+          // part of one page
+          const int pg = __ldg(trow + (t0 >> a.ps_log2));
+          const int row = t0 & ((1 << a.ps_log2) - 1);
+          mbar_arrive_expect_tx(bar, kTileBytes);
+          tma_load_3d(dst, mc, bar, 0, row, pg * a.hkv + g);
+          tma_load_3d(dst + 16384, mc, bar, 64, row, pg * a.hkv + g);
+        } else {
+          // 128 / page_size pages; only those holding cached tokens
+          const int ps = 1 << a.ps_log2;
+          const int npg = min(kTK >> a.ps_log2, (P - t0 + ps - 1) >> a.ps_log2);
+          mbar_arrive_expect_tx(bar, static_cast<uint32_t>(npg) * ps * 256);
+          for (int j = 0; j < npg; ++j) {
+            const int pg = __ldg(trow + (t0 >> a.ps_log2) + j);
+            tma_load_3d(dst + j * ps * 128, mc, bar, 0, 0, pg * a.hkv + g);
+            tma_load_3d(dst + 16384 + j * ps * 128, mc, bar, 64, 0, pg * a.hkv + g);
+          }
+        }
+      }
+    };
     for (int i = 0; i < nt; ++i) {
       const int st = i & 1;
       const int gi = tile0 + i;
-      const bool cache = gi < a.ncache_tiles;
-      const CUtensorMap* mk = cache ? &tmKc : &tmKa;
-      const CUtensorMap* mv = cache ? &tmVc : &tmVa;
-      const int trow = cache ? gi * kTK : 0;
       if (i >= 2 && !mbar_wait(bar_ke + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
-      mbar_arrive_expect_tx(bar_kf + 8 * st, kTileBytes);
-      tma_load_3d(base + kOffK + st * kTileBytes, mk, bar_kf + 8 * st, 0, trow, u);
-      tma_load_3d(base + kOffK + st * kTileBytes + 16384, mk, bar_kf + 8 * st, 64, trow, u);
+      load_tile(&tmKc, &tmKa, base + kOffK + st * kTileBytes, bar_kf + 8 * st, gi);
       if (i >= 2 && !mbar_wait(bar_ve + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
-      mbar_arrive_expect_tx(bar_vf + 8 * st, kTileBytes);
-      tma_load_3d(base + kOffV + st * kTileBytes, mv, bar_vf + 8 * st, 0, trow, u);
-      tma_load_3d(base + kOffV + st * kTileBytes + 16384, mv, bar_vf + 8 * st, 64, trow, u);
+      load_tile(&tmVc, &tmVa, base + kOffV + st * kTileBytes, bar_vf + 8 * st, gi);
     }
   } else if (tid == 32) {
     // ---------------- MMA issuer
@@ -184,7 +231,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < nt; ++i) {
       const int st = i & 1;
       const int gi = tile0 + i;
-      const int valid = gi < a.ncache_tiles ? min(kTK, a.P - gi * kTK) : a.b;
+      const int valid = gi < ncache_tiles ? min(kTK, P - gi * kTK) : a.b;
       ok = warp_all(ok && mbar_wait(bar_sf + 8 * st, (i >> 1) & 1, a.err, abort_flag));
       if (!ok) break;
       tc_fence_after();
@@ -231,6 +278,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int q = 0; q < 32; ++q) o[q] *= corr;
             tmem_st32_sync(t_o + lane_base + c, o);
+          }
+        }
+      }
+      if (PAGED && gi < ncache_tiles && valid < kTK) {
+        // rows past the cache hold stale pool data (or none was loaded):
+        // zero them in V so that P (0 there) times V stays finite
+        ok = warp_all(mbar_wait(bar_vf + 8 * st, (i >> 1) & 1, a.err, abort_flag));
+        if (!ok) break;
+        if (r >= valid) {
+          const uint32_t vrow = base + kOffV + st * kTileBytes + r * 128;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            st_shared_v4(vrow + q * 16, 0u, 0u, 0u, 0u);
+            st_shared_v4(vrow + 16384 + q * 16, 0u, 0u, 0u, 0u);
           }
         }
       }
@@ -327,6 +388,7 @@ __global__ void __launch_bounds__(256) k_prefix_merge(const float* __restrict__ 
   for (int s = 0; s < splits; ++s) {
     const float* ml = wsML + (item0 + s) * 256;
     const float w = exp2f(ml[r] - M);
+    if (w == 0.f) continue;   // a chunk past the request's cache (or negligible)
     den = fmaf(w, ml[128 + r], den);
     const float4 o = reinterpret_cast<const float4*>(wsO + (item0 + s) * kD * kD + r * kD)[c4];
     acc.x = fmaf(w, o.x, acc.x);
@@ -374,9 +436,13 @@ size_t prefix_bf16_workspace(int n, int hq, int hkv, int b, int P) {
   return static_cast<size_t>(units) * mtiles * splits * (kD * kD + 256) * sizeof(float);
 }
 
-int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* Vc, int P,
-                       int cap, const void* K, const void* V, void* Y, int n, int hq, int hkv,
-                       int b, float scale, void* ws, size_t ws_bytes) {
+namespace {
+
+// Shared by the contiguous and the paged launch; P is the cache length (the
+// longest possible one when paged).
+int launch_prefix_impl(const Ctx& c, const void* Q, const void* Kc, const void* Vc, int P, int cap,
+                       const PagedCache* pg, const void* K, const void* V, void* Y, int n, int hq,
+                       int hkv, int b, float scale, void* ws, size_t ws_bytes) {
   const int units = n * hkv;
   const int rows = (hq / hkv) * b;
   const int mtiles = (rows + 127) / 128;
@@ -392,7 +458,14 @@ int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* 
   bool ok = bf16_rows_tmap(&tq, Q, rows, rows, units, 128) &&
             bf16_rows_tmap(&ty, Y, rows, rows, units, 128) &&
             bf16_rows_tmap(&tka, K, b, b, units, kTK) && bf16_rows_tmap(&tva, V, b, b, units, kTK);
-  if (P > 0) {
+  if (pg != nullptr) {
+    // the pool as (128 columns, page rows, page * hkv + kv head)
+    const int ps = 1 << pg->ps_log2;
+    const uint32_t box_rows = ps < kTK ? ps : kTK;
+    const uint64_t units_pool = static_cast<uint64_t>(pg->num_pages) * hkv;
+    ok = ok && bf16_rows_tmap(&tkc, Kc, ps, ps, units_pool, box_rows) &&
+         bf16_rows_tmap(&tvc, Vc, ps, ps, units_pool, box_rows);
+  } else if (P > 0) {
     ok = ok && bf16_rows_tmap(&tkc, Kc, P, cap, units, kTK) &&
          bf16_rows_tmap(&tvc, Vc, P, cap, units, kTK);
   } else {
@@ -411,6 +484,12 @@ int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* 
   if (!ok) return -5;
   PrefixArgs a;
   a.err = c.dev_err;
+  a.table = pg ? pg->table : nullptr;
+  a.P_lens = pg ? pg->P_lens : nullptr;
+  a.max_pages = pg ? pg->max_pages : 0;
+  a.ps_log2 = pg ? pg->ps_log2 : 0;
+  a.hkv = hkv;
+  a.Pmax = P;
   a.wsO = wsO;
   a.wsML = wsML;
   a.rows = rows;
@@ -421,11 +500,19 @@ int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* 
   a.splits = splits;
   a.tiles_per = tp;
   a.sl2 = scale * 1.4426950408889634f;
-  static std::atomic<uint64_t> prepared{0};
-  if (!prepare_kernel(k_prefix_bf16, (int)kSmem, prepared)) return -5;
-  if (launch_pdl(k_prefix_bf16, (unsigned)items, kThreads, kSmem, c.stream, tq, tkc, tvc, tka,
-                 tva, ty, to, a))
-    return -5;
+  int rc;
+  if (pg != nullptr) {
+    static std::atomic<uint64_t> prepared{0};
+    if (!prepare_kernel(k_prefix_bf16<true>, (int)kSmem, prepared)) return -5;
+    rc = launch_pdl(k_prefix_bf16<true>, (unsigned)items, kThreads, kSmem, c.stream, tq, tkc, tvc,
+                    tka, tva, ty, to, a);
+  } else {
+    static std::atomic<uint64_t> prepared{0};
+    if (!prepare_kernel(k_prefix_bf16<false>, (int)kSmem, prepared)) return -5;
+    rc = launch_pdl(k_prefix_bf16<false>, (unsigned)items, kThreads, kSmem, c.stream, tq, tkc,
+                    tvc, tka, tva, ty, to, a);
+  }
+  if (rc) return -5;
   if (splits > 1) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(kD * kD / 4 / 256, units * mtiles);
@@ -443,6 +530,23 @@ int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* 
     if (cudaGetLastError() != cudaSuccess) return -5;
   }
   return 0;
+}
+
+}  // namespace
+
+int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* Vc, int P,
+                       int cap, const void* K, const void* V, void* Y, int n, int hq, int hkv,
+                       int b, float scale, void* ws, size_t ws_bytes) {
+  return launch_prefix_impl(c, Q, Kc, Vc, P, cap, nullptr, K, V, Y, n, hq, hkv, b, scale, ws,
+                            ws_bytes);
+}
+
+int launch_prefix_paged_bf16(const Ctx& c, const void* Q, const void* Kpool, const void* Vpool,
+                             const PagedCache& pg, const void* K, const void* V, void* Y, int n,
+                             int hq, int hkv, int b, float scale, void* ws, size_t ws_bytes) {
+  const int Pmax = pg.max_pages << pg.ps_log2;
+  return launch_prefix_impl(c, Q, Kpool, Vpool, Pmax, Pmax, &pg, K, V, Y, n, hq, hkv, b, scale,
+                            ws, ws_bytes);
 }
 
 }  // namespace bha

@@ -73,6 +73,18 @@ __device__ __forceinline__ void accum_to_tile(uint32_t tmem, uint32_t tile, int 
   }
 }
 
+// Zeros in place of the accumulator (a chunk with no tokens): same tile
+// addressing as accum_to_tile.
+__device__ __forceinline__ void zero_tile(uint32_t tile, int warp, int lane) {
+  const int r = (warp & 3) * 32 + lane;
+#pragma unroll 1
+  for (int bx = 2 * (warp >> 2); bx < 2 * (warp >> 2) + 2; ++bx) {
+    const uint32_t row = tile + bx * 16384 + r * 128;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) st_shared_f4(row + (j << 4), make_float4(0.f, 0.f, 0.f, 0.f));
+  }
+}
+
 // ------------------------------------------------------------------ commit
 
 struct CommitArgs {
@@ -373,11 +385,19 @@ constexpr int kTargetCtas = 296;          // two CTAs on each of 148 SMs
 struct PrefillArgs {
   float* zdst;       // [items][128] or null (partial or final z)
   int* err;
-  int T;             // prompt tokens
+  int T;             // prompt tokens (the longest, for ragged prompts)
   int splits;        // chunks per unit
   int tiles_per;     // 64-token tiles per chunk
   int hkv;           // unit u uses W[u % hkv] (projected map)
+  const int* T_lens; // ragged prompts: [n] tokens per request (device), else null
 };
+
+// Prompt length of unit u's request: T, or its own length (clamped to
+// [0, T]) for ragged prompts, whose rows past it are padding.  Reads device
+// memory: call after pdl_wait.
+__device__ __forceinline__ int unit_tokens(const PrefillArgs& a, int u) {
+  return a.T_lens ? min(max(__ldg(a.T_lens + u / a.hkv), 0), a.T) : a.T;
+}
 
 template <int FMAP>
 __global__ void __launch_bounds__(kThreads, 2)
@@ -387,9 +407,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int item = blockIdx.x;                // = u * splits + s
   const int u = item / a.splits, sp = item % a.splits;
-  const int ntiles_total = (a.T + kTok - 1) / kTok;
   const int tile0 = sp * a.tiles_per;
-  const int ntile = min(a.tiles_per, ntiles_total - tile0);
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -421,6 +439,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   pdl_wait();
+  const int Tu = unit_tokens(a, u);
+  const int ntile = max(0, min(a.tiles_per, (Tu + kTok - 1) / kTok - tile0));
 
   float zacc[8];
 #pragma unroll
@@ -470,7 +490,11 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int st = i % kStages;
       if (!mbar_wait(bar_full + 8 * st, (i / kStages) & 1, a.err, abort_flag)) break;
       const uint32_t kt = base + st * kStageBytes + box * 8192;
-      const int tvalid = a.T - (tile0 + i) * kTok;   // rows past the prompt are zero-filled
+      // rows past the prompt: zero-filled past the buffer (ReLU keeps them
+      // zero, elu + 1 would make them 1), padding of a ragged prompt inside
+      // it (K and V cleared, so that 0 times V stays finite)
+      const int tvalid = Tu - (tile0 + i) * kTok;
+      const bool clear = FMAP != kFmapRelu || a.T_lens != nullptr;
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
         const int t = tsub + 8 * k;
@@ -480,8 +504,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         x.y = phi_bf16x2<FMAP>(x.y);
         x.z = phi_bf16x2<FMAP>(x.z);
         x.w = phi_bf16x2<FMAP>(x.w);
-        // ReLU keeps them zero; elu + 1 would make them 1: clear them
-        if (FMAP != kFmapRelu && t >= tvalid) x = make_uint4(0u, 0u, 0u, 0u);
+        if (clear && t >= tvalid) {
+          x = make_uint4(0u, 0u, 0u, 0u);
+          if (a.T_lens != nullptr) st_shared_v4(addr + 16384, 0u, 0u, 0u, 0u);   // V row
+        }
         st_shared_v4(addr, x.x, x.y, x.z, x.w);
         const uint32_t wv[4] = {x.x, x.y, x.z, x.w};
 #pragma unroll
@@ -495,11 +521,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
 
-  // ---- epilogue: accumulator -> fp32 tile -> TMA store (partial or final)
+  // ---- epilogue: accumulator -> fp32 tile -> TMA store (partial or final);
+  // a chunk past a ragged prompt's end stores zeros
   __syncwarp();
   const bool ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag));
   tc_fence_after();
-  if (ok) accum_to_tile(tmem, base, warp, lane, false);
+  if (ok) {
+    if (ntile > 0)
+      accum_to_tile(tmem, base, warp, lane, false);
+    else
+      zero_tile(base, warp, lane);
+  }
   fence_proxy_async_smem();
   if (warp >= 4 && a.zdst != nullptr) {
     // reduce the 8 row-phases that share (box, j)
@@ -559,9 +591,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int item = blockIdx.x;                // = u * splits + s
   const int u = item / a.splits, sp = item % a.splits;
   const int g = u % a.hkv;
-  const int ntiles_total = (a.T + kTok - 1) / kTok;
   const int tile0 = sp * a.tiles_per;
-  const int ntile = min(a.tiles_per, ntiles_total - tile0);
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -598,6 +628,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const uint32_t tmem = *tmem_slot;
   const uint32_t t_w = tmem + 128, t_kw = tmem + 192;
   pdl_wait();
+  const int Tu = unit_tokens(a, u);
+  const int ntile = max(0, min(a.tiles_per, (Tu + kTok - 1) / kTok - tile0));
 
   float zacc = 0.f;
   if (tid == 0) {
@@ -690,16 +722,24 @@ __global__ void __launch_bounds__(kThreads, 2)
       tc_fence_before();
       mbar_arrive(bar_kwfree);
       const uint32_t kt = base + st * kStageBytes;   // phi(K)^T over the consumed K tile
+      // tokens past the prompt: zero rows of K past the buffer (features 0);
+      // padding of a ragged prompt inside it: features and V rows cleared
+      const int tvalid = a.T_lens != nullptr ? Tu - (tile0 + i) * kTok : kTok;
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         uint32_t w[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          // tokens past the prompt are zero rows of K: their features are 0
-          w[q] = pack_bf16x2(fmaxf(f[8 * c + 2 * q], 0.f), fmaxf(f[8 * c + 2 * q + 1], 0.f));
+          const int t = 8 * c + 2 * q;
+          w[q] = pack_bf16x2(t < tvalid ? fmaxf(f[t], 0.f) : 0.f,
+                             t + 1 < tvalid ? fmaxf(f[t + 1], 0.f) : 0.f);
           zacc += __uint_as_float(w[q] << 16) + __uint_as_float(w[q] & 0xFFFF0000u);
         }
         st_shared_v4(kmajor_chunk<128>(kt, r, c), w[0], w[1], w[2], w[3]);
+      }
+      for (int idx = r; idx < (kTok - max(tvalid, 0)) * 16; idx += 128) {
+        const int row = tvalid + (idx >> 4), ch = idx & 15;
+        st_shared_v4(kt + 16384 + (ch >> 3) * 8192 + row * 128 + (ch & 7) * 16, 0u, 0u, 0u, 0u);
       }
       fence_proxy_async_smem();
       mbar_arrive(bar_relu + 8 * st);
@@ -710,7 +750,12 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncwarp();
   const bool ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag));
   tc_fence_after();
-  if (ok) accum_to_tile(tmem, base, warp, lane, false);
+  if (ok) {
+    if (ntile > 0)
+      accum_to_tile(tmem, base, warp, lane, false);
+    else
+      zero_tile(base, warp, lane);
+  }
   fence_proxy_async_smem();
   if (warp >= 4 && a.zdst != nullptr && ok)
     a.zdst[static_cast<size_t>(item) * kD + (tid - 128)] = zacc;
@@ -869,7 +914,8 @@ size_t prefill_bf16_workspace(int units, int T) {
 }
 
 int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, int T, float* S,
-                        float* z, void* ws, size_t ws_bytes, int fmap, const void* W, int hkv) {
+                        float* z, void* ws, size_t ws_bytes, int fmap, const void* W, int hkv,
+                        const int* T_lens) {
   if (T == 0) {
     if (cudaMemsetAsync(S, 0, static_cast<size_t>(units) * kD * kD * 4, c.stream) != cudaSuccess)
       return -5;
@@ -891,7 +937,7 @@ int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, i
   if (!tokens_tmap(&tk, K, T, units, kTok) || !tokens_tmap(&tv, V, T, units, kTok) ||
       !state_tmap(&to, outS, static_cast<uint64_t>(units) * splits))
     return -5;
-  PrefillArgs a{outZ, c.dev_err, T, splits, tp, hkv};
+  PrefillArgs a{outZ, c.dev_err, T, splits, tp, hkv, T_lens};
   int rc;
   if (fmap == kFmapReluProj) {
     static std::atomic<uint64_t> prepared_p{0};

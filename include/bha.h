@@ -224,6 +224,53 @@ int bha_hybrid_step_commit_fm(const void *Qa, const void *Ka, const void *Va,
                               const void *W, bha_stream_t stream);
 
 /*
+ * Ragged and paged batches.  The method-details section (技术方法详解) of the
+ * summary page pairs the method with KV-cache management and its related
+ * work (相关工作) names PagedAttention: requests of one batch carry caches
+ * and prompts of their own lengths.
+ */
+
+/*
+ * Exact path over a paged KV cache with per-request cache lengths: for each
+ * request i, the result of bha_prefix_softmax with its own cache, its first
+ * P_lens[i] tokens, token t at row t % page_size of page
+ * block_table[i][t / page_size].
+ *   Kpool, Vpool  [num_pages][hkv][page_size][d]   pages of keys / values
+ *   block_table   [n][max_pages] int32, device memory
+ *   P_lens        [n] int32, device memory; clamped to [0, max_pages * page_size]
+ * page_size is a power of two from 16 to 256 (else BHA_ERR_UNSUPPORTED).
+ * Pool slots past a request's cache may hold anything; a page number outside
+ * [0, num_pages) reads as zero rows.  block_table and P_lens must be 4-byte
+ * aligned.  The workspace is sized for the longest cache,
+ * max_pages * page_size tokens.
+ */
+size_t bha_prefix_softmax_paged_workspace_size(int n, int hq, int hkv, int b,
+                                               int d, int max_pages,
+                                               int page_size, bha_dtype dtype);
+int bha_prefix_softmax_paged(const void *Qa, const void *Kpool,
+                             const void *Vpool, int num_pages, int page_size,
+                             const int *block_table, int max_pages,
+                             const int *P_lens, const void *Ka,
+                             const void *Va, void *Y, int n, int hq, int hkv,
+                             int b, int d, float scale, bha_dtype dtype,
+                             void *workspace, size_t workspace_bytes,
+                             bha_stream_t stream);
+
+/*
+ * Prefill of prompts of different lengths: request i folds its first
+ * T_lens[i] tokens of K, V [n][hkv][Tmax][d] (T_lens: [n] int32 in device
+ * memory, 4-byte aligned, clamped to [0, Tmax]); rows past T_lens[i] are
+ * padding and may hold anything.  Overwrites S and z as bha_state_prefill
+ * does; feature map as for the _fm calls; the workspace is that of
+ * bha_state_prefill for Tmax tokens.
+ */
+int bha_state_prefill_ragged(const void *K, const void *V, const int *T_lens,
+                             int n, int hkv, int Tmax, int d, bha_dtype dtype,
+                             bha_fmap fmap, const void *W, float *S, float *z,
+                             void *workspace, size_t workspace_bytes,
+                             bha_stream_t stream);
+
+/*
  * Block partition of a length-L sequence into blocks of B tokens, the last
  * one possibly short (worked example: L=10, B=4 -> tokens 1-4, 5-8, 9-10).
  * Host-only.  Writes bounds[0..k] = {0, B, 2B, ..., L} and returns k, the

@@ -210,3 +210,58 @@ def test_feature_map_validation(L):
         for f in (st, cm, pf, sc):
             for fmap, w in ((RELU, None), (ELU1, None), (PROJ, W)):
                 assert f(fmap, w) == _lib.BHA_ERR_CUDA
+
+
+def test_paged_prefix_validation(L):
+    """bha_prefix_softmax_paged: page sizes, counts, alignment, aliasing and
+    the workspace (sized for the longest cache)."""
+    n, hq, hkv, b, d, maxp, ps = 4, 16, 4, 32, 128, 64, 128
+    need = L.bha_prefix_softmax_paged_workspace_size(n, hq, hkv, b, d, maxp, ps, _lib.BHA_BF16)
+    assert need == L.bha_prefix_softmax_workspace_size(n, hq, hkv, b, d, maxp * ps,
+                                                       _lib.BHA_BF16)
+    assert need > 0
+    big = GAP * 16
+
+    def f(**kw):
+        return L.bha_prefix_softmax_paged(
+            A, kw.get("Kp", big), kw.get("Vp", 2 * big), kw.get("num_pages", 1000),
+            kw.get("ps", ps), kw.get("table", C), kw.get("maxp", maxp), kw.get("plens", D),
+            B, E, kw.get("Y", F), kw.get("n", n), hq, hkv, b, d, 0.0,
+            kw.get("dtype", _lib.BHA_BF16), kw.get("ws", 3 * big), kw.get("ws_bytes", need), None)
+
+    for bad in (8, 48, 512, 0):
+        assert f(ps=bad) == _lib.BHA_ERR_UNSUPPORTED, bad
+    assert f(maxp=0) == _lib.BHA_ERR_INVALID_ARG
+    assert f(num_pages=0) == _lib.BHA_ERR_INVALID_ARG
+    assert f(table=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(plens=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(table=C + 2) == _lib.BHA_ERR_MISALIGNED
+    assert f(plens=D + 1) == _lib.BHA_ERR_MISALIGNED
+    assert f(Kp=big + 8) == _lib.BHA_ERR_MISALIGNED
+    assert f(ws=None) == _lib.BHA_ERR_WORKSPACE
+    assert f(ws_bytes=need - 16) == _lib.BHA_ERR_WORKSPACE
+    assert f(Y=big + 4096) == _lib.BHA_ERR_INVALID_ARG      # Y inside the pool
+    assert f(Y=C) == _lib.BHA_ERR_INVALID_ARG               # Y over the page table
+    assert f(n=0) == _lib.BHA_OK
+    import torch
+    if not torch.cuda.is_available():
+        assert f() == _lib.BHA_ERR_CUDA
+        assert f(ps=16, dtype=_lib.BHA_F32) == _lib.BHA_ERR_CUDA
+
+
+def test_ragged_prefill_validation(L):
+    need = L.bha_state_prefill_workspace_size(4, 4, 4096, 128, _lib.BHA_BF16)
+    big = GAP * 16
+
+    def f(**kw):
+        return L.bha_state_prefill_ragged(A, big, kw.get("tl", C), kw.get("n", 4), 4, 4096, 128,
+                                          _lib.BHA_BF16, 0, None, kw.get("S", 2 * big), None,
+                                          3 * big if need else None, need, None)
+
+    assert f(tl=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(tl=C + 2) == _lib.BHA_ERR_MISALIGNED
+    assert f(S=C) == _lib.BHA_ERR_INVALID_ARG               # S over the lengths
+    assert f(n=0, tl=None) == _lib.BHA_OK
+    import torch
+    if not torch.cuda.is_available():
+        assert f() == _lib.BHA_ERR_CUDA
