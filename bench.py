@@ -59,7 +59,7 @@ def parse():
                     help="prompt / cache length used by --only prefill|prefix")
     ap.add_argument("--workload", default="long-prefix",
                     choices=["long-prefix", "single-step", "generation-loop", "stack",
-                             "feature-maps"],
+                             "feature-maps", "ragged"],
                     help="long-prefix is the benchmark line; the others are the secondary "
                          "workloads (one JSON line each)")
     return ap.parse_args()
@@ -740,6 +740,124 @@ def run_feature_maps(args):
         "rotating_sets": R, "peak_gbs": peak, "maps": out}), flush=True)
 
 
+def run_ragged(args):
+    """Batch 64, 16q/4kv, d=128, B=32 with per-request prefix lengths drawn
+    uniformly from [1, 16384] (mean about 8192, seeded): the exact path over a
+    paged KV cache (pages of 128 tokens) against the same path padded to the
+    longest cache, the hybrid step, the ragged prefill of the same prompts, and
+    the 20-layer stack (6 hybrid + 14 exact layers) memory per request and
+    largest batch before out-of-memory with paged and with padded caches."""
+    import numpy as np
+    import torch
+    import block_hybrid_linear_b200 as bha
+    from block_hybrid_linear_b200 import build, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    n, ps, Lmax, layers, hyb = N_, 128, 16384, 20, 6
+    std = 1.0 / math.sqrt(D_)
+    lengths = np.random.default_rng(6000).integers(1, Lmax + 1, size=8192)
+    P_lens = lengths[:n]
+    pages = (P_lens + ps - 1) // ps
+    num_pages, max_pages = int(pages.sum()), int(pages.max())
+    order = np.random.default_rng(6001).permutation(num_pages)
+    table = np.full((n, max_pages), -1, dtype=np.int32)
+    k = 0
+    for i in range(n):
+        table[i, :pages[i]] = order[k:k + pages[i]]
+        k += pages[i]
+    Kpool = inputs.normal_bf16_torch(6000, inputs.TID_KC, (num_pages, HKV, ps, D_), std, dev)
+    Vpool = inputs.normal_bf16_torch(6000, inputs.TID_VC, (num_pages, HKV, ps, D_), std, dev)
+    tab = torch.from_numpy(table).to(dev)
+    plen = torch.from_numpy(P_lens.astype(np.int32)).to(dev)
+    Q = inputs.normal_bf16_torch(6000, inputs.TID_Q, (n, HQ, B_, D_), std, dev)
+    K = inputs.normal_bf16_torch(6000, inputs.TID_K, (n, HKV, B_, D_), std, dev)
+    V = inputs.normal_bf16_torch(6000, inputs.TID_V, (n, HKV, B_, D_), std, dev)
+    Y = torch.empty_like(Q)
+    S = torch.randn(n, HKV, D_, D_, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    peak, _ = measured_peaks()
+    units = n * HKV
+    # exact path, paged, each request over its own cache
+    need = bha.bha_prefix_softmax_paged_workspace_size(n, HQ, HKV, B_, D_, max_pages, ps)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    g = _graph(lambda: bha.bha_prefix_softmax_paged(Q, Kpool, Vpool, tab, plen, K, V, Y,
+                                                    workspace=ws, stream=stream), stream)
+    paged_ms = _time_graph(g, stream, 20)
+    paged_bytes = int(HKV * (P_lens.sum() + n * B_) * D_ * 4 + units * 65536)
+    del g
+    # the same path over caches padded to the longest one
+    Pmax = int(P_lens.max())
+    Kc = inputs.normal_bf16_torch(6002, inputs.TID_KC, (n, HKV, Pmax, D_), std, dev)
+    Vc = inputs.normal_bf16_torch(6002, inputs.TID_VC, (n, HKV, Pmax, D_), std, dev)
+    needc = bha.bha_prefix_softmax_workspace_size(n, HQ, HKV, B_, D_, Pmax)
+    wsc = torch.empty(max(needc, 16), dtype=torch.uint8, device=dev)
+    g = _graph(lambda: bha.bha_prefix_softmax(Q, Kc, Vc, Pmax, K, V, Y, workspace=wsc,
+                                              stream=stream), stream)
+    padded_ms = _time_graph(g, stream, 20)
+    del g
+    g = _graph(lambda: bha.bha_hybrid_step(Q, K, V, S, Y, stream=stream), stream)
+    step_us = _time_graph(g, stream, 200) * 1e3
+    del g
+    # ragged prefill of the same prompt lengths from the padded buffers
+    needp = bha.bha_state_prefill_workspace_size(n, HKV, Pmax, D_)
+    wsp = torch.empty(max(needp, 16), dtype=torch.uint8, device=dev)
+    z = torch.empty(n, HKV, D_, device=dev)
+    g = _graph(lambda: bha.bha_state_prefill_ragged(Kc, Vc, plen, S, z, workspace=wsp,
+                                                    stream=stream), stream)
+    prefill_ms = _time_graph(g, stream, 10)
+    prefill_bytes = int(HKV * P_lens.sum() * D_ * 4 + units * (D_ * D_ + D_) * 4)
+    del g, Kc, Vc, Kpool, Vpool, wsc, ws, wsp
+    torch.cuda.synchronize()
+    assert bha.bha_device_error(True) == 0
+    torch.cuda.empty_cache()
+    # memory of the 20-layer stack per request, and the largest batch that fits
+    kv_tok = HKV * D_ * 2 * 2                     # K and V bytes per cached token, one layer
+    st_req = HKV * (D_ * D_ + D_) * 4
+    pg_all = ((lengths + ps - 1) // ps) * ps
+    hybrid_paged = hyb * st_req + (layers - hyb) * kv_tok * pg_all
+    exact_paged = layers * kv_tok * pg_all
+    exact_padded = np.full_like(lengths, layers * kv_tok * Lmax)
+
+    def fits(nbytes):
+        try:
+            buf = torch.empty(int(nbytes), dtype=torch.uint8, device=dev)
+            del buf
+            return True
+        except torch.OutOfMemoryError:
+            return False
+        finally:
+            torch.cuda.empty_cache()
+
+    def max_batch(per_req):
+        cum = np.cumsum(per_req.astype(np.float64))
+        lo, hi = 0, len(cum)
+        while hi - lo > 1:
+            mid = (lo + hi) // 2
+            lo, hi = (mid, hi) if fits(cum[mid - 1]) else (lo, mid)
+        return lo
+    print(json.dumps({
+        "workload": "ragged: batch 64, 16q/4kv, d=128, B=32, prefix lengths uniform in "
+                    "[1, 16384] (seeded), paged KV cache with 128-token pages",
+        "metric": METRIC, "unit": "tokens/s",
+        "prefix_tokens": {"sum": int(P_lens.sum()), "max": Pmax, "mean": float(P_lens.mean())},
+        "exact_paged": {"ms": paged_ms, "tokens_per_s": n * B_ / (paged_ms / 1e3),
+                        "algorithmic_bytes": paged_bytes,
+                        "achieved_gbs": paged_bytes / (paged_ms / 1e3) / 1e9,
+                        "frac_of_peak": paged_bytes / (paged_ms / 1e3) / 1e9 / peak},
+        "exact_padded_to_longest": {"ms": padded_ms, "tokens_per_s": n * B_ / (padded_ms / 1e3)},
+        "hybrid_step": {"us": step_us, "tokens_per_s": n * B_ / (step_us / 1e6)},
+        "ragged_prefill": {"ms": prefill_ms, "algorithmic_bytes": prefill_bytes,
+                           "achieved_gbs": prefill_bytes / (prefill_ms / 1e3) / 1e9,
+                           "frac_of_peak": prefill_bytes / (prefill_ms / 1e3) / 1e9 / peak},
+        "stack_bytes_per_request_mean": {"hybrid_paged": float(hybrid_paged.mean()),
+                                         "all_exact_paged": float(exact_paged.mean()),
+                                         "all_exact_padded_16384": float(exact_padded.mean())},
+        "stack_max_batch_before_oom": {"hybrid_paged": max_batch(hybrid_paged),
+                                       "all_exact_paged": max_batch(exact_paged),
+                                       "all_exact_padded_16384": max_batch(exact_padded)}}),
+          flush=True)
+
+
 def run_generation_loop(args):
     """Batch 32, prompt 1024 -> state, 32 blocks x 8 denoising steps (one
     commit per block), against exact attention over the growing KV cache
@@ -901,7 +1019,8 @@ def main():
     if args.workload != "long-prefix":
         if rank == 0:
             {"single-step": run_single_step, "generation-loop": run_generation_loop,
-             "stack": run_stack, "feature-maps": run_feature_maps}[args.workload](args)
+             "stack": run_stack, "feature-maps": run_feature_maps,
+             "ragged": run_ragged}[args.workload](args)
         return
     if args.impl == "reference":
         run_reference(args, rank, world)

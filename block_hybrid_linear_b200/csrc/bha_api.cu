@@ -504,9 +504,11 @@ int bha_prefix_softmax(const void* Qa, const void* Kc, const void* Vc, int P, in
 
 size_t bha_prefix_softmax_paged_workspace_size(int n, int hq, int hkv, int b, int d,
                                                int max_pages, int page_size, bha_dtype dtype) {
-  if (max_pages < 1 || page_size < 1 || static_cast<long long>(max_pages) * page_size > (1 << 30))
+  if (dtype != BHA_BF16 || n <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0 || b < 1 || b > 64 ||
+      d != 128 || max_pages < 1 || page_size < 1 ||
+      static_cast<long long>(max_pages) * page_size > (1 << 30))
     return 0;
-  return bha_prefix_softmax_workspace_size(n, hq, hkv, b, d, max_pages * page_size, dtype);
+  return prefix_paged_bf16_workspace(n, hq, hkv, b, max_pages * page_size);
 }
 
 int bha_prefix_softmax_paged(const void* Qa, const void* Kpool, const void* Vpool, int num_pages,

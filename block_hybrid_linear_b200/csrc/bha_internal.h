@@ -90,6 +90,7 @@ int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, i
                         float* z, void* ws, size_t ws_bytes, int fmap, const void* W, int hkv,
                         const int* T_lens = nullptr);
 size_t prefix_bf16_workspace(int n, int hq, int hkv, int b, int P);
+size_t prefix_paged_bf16_workspace(int n, int hq, int hkv, int b, int Pmax);
 // A paged KV cache: request i's token t at row t % 2^ps_log2 of page
 // table[i * max_pages + (t >> ps_log2)] of a pool of num_pages pages
 // [num_pages][hkv][page_size][d]; P_lens[i] cached tokens (device arrays).

@@ -22,10 +22,11 @@
 // page_size] of a pool [pages][hkv][page_size][128].  A 128-key tile is one
 // TMA box per page (page_size < 128: 128 / page_size boxes, pages past the
 // request's cache not loaded; page_size >= 128: part of one page).  The plan
-// covers the longest possible cache; a chunk past a request's cache leaves a
-// neutral partial (row max -inf, sum 0) that the merge skips.  Rows past the
-// cache in its last tile hold stale pool data: their scores are masked and
-// their V rows zeroed before P V.
+// covers the longest possible cache in chunks of 16 tiles (2048 keys) so
+// that short and long requests balance over the SMs; a chunk past a
+// request's cache does nothing, and the merge reads only the chunks its
+// request has.  Rows past the cache in its last tile hold stale pool data:
+// their scores are masked and their V rows zeroed before P V.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>
@@ -45,11 +46,14 @@ constexpr uint32_t kOffK = kTileBytes;          // 2 stages
 constexpr uint32_t kOffV = 3 * kTileBytes;      // 2 stages
 constexpr uint32_t kOffP = 5 * kTileBytes;
 constexpr uint32_t kTiles = 6 * kTileBytes;     // 192 KB
+constexpr int kMaxChunkPages = 128;               // paged: a chunk's page numbers (16 tiles of 16-token pages)
+constexpr uint32_t kPageList = kMaxChunkPages * 4;
 constexpr uint32_t kCtrlBytes = 256;
-constexpr uint32_t kSmem = kTiles + 1024;
+constexpr uint32_t kSmem = kTiles + kPageList + 1024;
 constexpr float kRescaleLog2 = 8.f;             // rescale O when max grows > 2^8
 constexpr int kTargetCtas = 592;                // four CTAs' worth per SM (148 SMs)
 constexpr int kMinTilesPerChunk = 8;
+constexpr int kPagedTilesPerChunk = 16;
 
 struct PrefixArgs {
   int* err;
@@ -89,7 +93,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + kTiles;
+  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + kTiles + kPageList;
+  int* page_list = reinterpret_cast<int*>(smem_raw + (base - raw) + kTiles);
   uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
   const uint32_t bar_q = ctrl, bar_kf = ctrl + 8, bar_ke = ctrl + 24, bar_vf = ctrl + 40,
                  bar_ve = ctrl + 56, bar_sf = ctrl + 72, bar_pf = ctrl + 88, bar_pv = ctrl + 96;
@@ -128,8 +133,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int P = PAGED ? min(max(__ldg(a.P_lens + nreq), 0), a.Pmax) : a.P;
   const int ncache_tiles = PAGED ? (P + kTK - 1) / kTK : a.ncache_tiles;
   const int nt = max(0, min(a.tiles_per, ncache_tiles + 1 - tile0));
+  const bool live = nt > 0;   // false only for a chunk past a paged request's cache
+  if (PAGED && warp == 0 && live) {
+    // this chunk's page numbers into shared memory at once, so that the
+    // producer never waits on a table read before a tile's copy
+    const int t_first = tile0 * kTK;
+    const int t_end = min((tile0 + nt) * kTK, P);
+    const int pg0 = t_first >> a.ps_log2;
+    const int npg = t_end > t_first ? ((t_end - 1) >> a.ps_log2) - pg0 + 1 : 0;
+    const int* trow = a.table + static_cast<size_t>(nreq) * a.max_pages + pg0;
+    for (int k = lane; k < npg; k += 32) page_list[k] = __ldg(trow + k);
+    __syncwarp();
+  }
 
-  if (tid == 0) {
+  if (tid == 0 && live) {
     // ---------------- TMA producer
     const int row0 = mt * 128;
     mbar_arrive_expect_tx(bar_q, kTileBytes);
@@ -147,11 +164,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_3d(dst, mc, bar, 0, gi * kTK, u);
         tma_load_3d(dst + 16384, mc, bar, 64, gi * kTK, u);
       } else {
+        // page numbers from the chunk's list (entry 0 = the chunk's first page)
         const int t0 = gi * kTK;
-        const int* trow = a.table + static_cast<size_t>(nreq) * a.max_pages;
+        const int pbase = (tile0 * kTK) >> a.ps_log2;
         if (a.ps_log2 >= 7) {
           // part of one page
-          const int pg = __ldg(trow + (t0 >> a.ps_log2));
+          const int pg = page_list[(t0 >> a.ps_log2) - pbase];
           const int row = t0 & ((1 << a.ps_log2) - 1);
           mbar_arrive_expect_tx(bar, kTileBytes);
           tma_load_3d(dst, mc, bar, 0, row, pg * a.hkv + g);
@@ -162,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int npg = min(kTK >> a.ps_log2, (P - t0 + ps - 1) >> a.ps_log2);
           mbar_arrive_expect_tx(bar, static_cast<uint32_t>(npg) * ps * 256);
           for (int j = 0; j < npg; ++j) {
-            const int pg = __ldg(trow + (t0 >> a.ps_log2) + j);
+            const int pg = page_list[(t0 >> a.ps_log2) - pbase + j];
             tma_load_3d(dst + j * ps * 128, mc, bar, 0, 0, pg * a.hkv + g);
             tma_load_3d(dst + 16384 + j * ps * 128, mc, bar, 64, 0, pg * a.hkv + g);
           }
@@ -177,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (i >= 2 && !mbar_wait(bar_ve + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
       load_tile(&tmVc, &tmVa, base + kOffV + st * kTileBytes, bar_vf + 8 * st, gi);
     }
-  } else if (tid == 32) {
+  } else if (tid == 32 && live) {
     // ---------------- MMA issuer
     constexpr uint32_t idesc_s = make_idesc_bf16(128, kTK, 0, 0);   // Q K^T, both K-major
     constexpr uint32_t idesc_o = make_idesc_bf16(128, kD, 0, 1);    // P V, V MN-major
@@ -227,7 +245,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int r = (warp & 3) * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   bool ok = true;
-  if (warp >= 4) {
+  if (warp >= 4 && live) {
     for (int i = 0; i < nt; ++i) {
       const int st = i & 1;
       const int gi = tile0 + i;
@@ -349,7 +367,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (tid == 0 && !*abort_flag) {
+  if (tid == 0 && live && !*abort_flag) {
     if (a.splits == 1) {
       tma_store_3d(&tmY, base + kOffQ, 0, mt * 128, u);
       tma_store_3d(&tmY, base + kOffQ + 16384, 64, mt * 128, u);
@@ -367,20 +385,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// y[r][c] = sum_s 2^{m_s - M} O_s[r][c] / sum_s 2^{m_s - M} l_s,  M = max_s m_s
+// y[r][c] = sum_s 2^{m_s - M} O_s[r][c] / sum_s 2^{m_s - M} l_s,  M = max_s m_s,
+// over the chunks the request has (all of them, unless paged).
+struct MergeArgs {
+  int rows, mtiles, splits;
+  const int* P_lens;   // paged: [n] cached tokens, else null
+  int hkv, Pmax, tiles_per;
+};
+
 __global__ void __launch_bounds__(256) k_prefix_merge(const float* __restrict__ wsO,
                                                       const float* __restrict__ wsML,
-                                                      __nv_bfloat16* __restrict__ Y, int rows,
-                                                      int mtiles, int splits) {
+                                                      __nv_bfloat16* __restrict__ Y,
+                                                      const MergeArgs ma) {
   pdl_launch_dependents();
   pdl_wait();
+  const int rows = ma.rows, mtiles = ma.mtiles;
   const int umt = blockIdx.y;
   const int u = umt / mtiles, mt = umt % mtiles;
+  int splits = ma.splits;
+  if (ma.P_lens != nullptr) {
+    const int P = min(max(__ldg(ma.P_lens + u / ma.hkv), 0), ma.Pmax);
+    splits = min(splits, ((P + kTK - 1) / kTK + 1 + ma.tiles_per - 1) / ma.tiles_per);
+  }
   const int e = blockIdx.x * 256 + threadIdx.x;      // float4 index in the 128 x 128 tile
   const int r = e >> 5, c4 = e & 31;
   const int grow = mt * 128 + r;
   if (grow >= rows) return;
-  const size_t item0 = static_cast<size_t>(umt) * splits;
+  const size_t item0 = static_cast<size_t>(umt) * ma.splits;
   float M = -INFINITY;
   for (int s = 0; s < splits; ++s) M = fmaxf(M, wsML[(item0 + s) * 256 + r]);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -388,7 +419,7 @@ __global__ void __launch_bounds__(256) k_prefix_merge(const float* __restrict__ 
   for (int s = 0; s < splits; ++s) {
     const float* ml = wsML + (item0 + s) * 256;
     const float w = exp2f(ml[r] - M);
-    if (w == 0.f) continue;   // a chunk past the request's cache (or negligible)
+    if (w == 0.f) continue;   // no weight (a row underflow): skip the read
     den = fmaf(w, ml[128 + r], den);
     const float4 o = reinterpret_cast<const float4*>(wsO + (item0 + s) * kD * kD + r * kD)[c4];
     acc.x = fmaf(w, o.x, acc.x);
@@ -401,6 +432,14 @@ __global__ void __launch_bounds__(256) k_prefix_merge(const float* __restrict__ 
       Y + (static_cast<size_t>(u) * rows + grow) * kD + c4 * 4);
   out[0] = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
   out[1] = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+}
+
+// Paged: chunks of kPagedTilesPerChunk tiles over the longest cache.
+void prefix_plan_paged(int P, int* splits, int* tiles_per) {
+  const int ntot = (P + kTK - 1) / kTK + 1;
+  const int tp = ntot < kPagedTilesPerChunk ? ntot : kPagedTilesPerChunk;
+  *splits = (ntot + tp - 1) / tp;
+  *tiles_per = tp;
 }
 
 void prefix_plan(int units, int mtiles, int P, int* splits, int* tiles_per) {
@@ -426,14 +465,29 @@ bool bf16_rows_tmap(CUtensorMap* m, const void* X, uint64_t rows, uint64_t row_s
 
 }  // namespace
 
-size_t prefix_bf16_workspace(int n, int hq, int hkv, int b, int P) {
+namespace {
+
+size_t workspace_for(int n, int hq, int hkv, int b, int P, bool paged) {
   const int units = n * hkv;
   const int rows = (hq / hkv) * b;
   const int mtiles = (rows + 127) / 128;
   int splits, tp;
-  prefix_plan(units, mtiles, P, &splits, &tp);
+  if (paged)
+    prefix_plan_paged(P, &splits, &tp);
+  else
+    prefix_plan(units, mtiles, P, &splits, &tp);
   if (splits <= 1) return 0;
   return static_cast<size_t>(units) * mtiles * splits * (kD * kD + 256) * sizeof(float);
+}
+
+}  // namespace
+
+size_t prefix_bf16_workspace(int n, int hq, int hkv, int b, int P) {
+  return workspace_for(n, hq, hkv, b, P, false);
+}
+
+size_t prefix_paged_bf16_workspace(int n, int hq, int hkv, int b, int Pmax) {
+  return workspace_for(n, hq, hkv, b, Pmax, true);
 }
 
 namespace {
@@ -447,8 +501,11 @@ int launch_prefix_impl(const Ctx& c, const void* Q, const void* Kc, const void* 
   const int rows = (hq / hkv) * b;
   const int mtiles = (rows + 127) / 128;
   int splits, tp;
-  prefix_plan(units, mtiles, P, &splits, &tp);
-  const size_t need = prefix_bf16_workspace(n, hq, hkv, b, P);
+  if (pg != nullptr)
+    prefix_plan_paged(P, &splits, &tp);
+  else
+    prefix_plan(units, mtiles, P, &splits, &tp);
+  const size_t need = workspace_for(n, hq, hkv, b, P, pg != nullptr);
   if (need > ws_bytes) return -4;
   const size_t items = static_cast<size_t>(units) * mtiles * splits;
   float* wsO = splits > 1 ? static_cast<float*>(ws) : nullptr;
@@ -523,9 +580,10 @@ int launch_prefix_impl(const Ctx& c, const void* Q, const void* Kc, const void* 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    const MergeArgs ma{rows, mtiles, splits, pg ? pg->P_lens : nullptr, hkv, P, tp};
     if (cudaLaunchKernelEx(&cfg, k_prefix_merge, static_cast<const float*>(wsO),
-                           static_cast<const float*>(wsML), static_cast<__nv_bfloat16*>(Y), rows,
-                           mtiles, splits) != cudaSuccess)
+                           static_cast<const float*>(wsML), static_cast<__nv_bfloat16*>(Y),
+                           ma) != cudaSuccess)
       return -5;
     if (cudaGetLastError() != cudaSuccess) return -5;
   }

@@ -521,10 +521,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
 
-  // ---- epilogue: accumulator -> fp32 tile -> TMA store (partial or final);
-  // a chunk past a ragged prompt's end stores zeros
+  // ---- epilogue: accumulator -> fp32 tile -> TMA store (partial or final).
+  // A chunk past a ragged prompt's end stores nothing (the reduce reads only
+  // the chunks its request has), or zeros when it is the unit's only chunk.
   __syncwarp();
-  const bool ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag));
+  const bool store = ntile > 0 || a.splits == 1;
+  const bool ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag)) && store;
   tc_fence_after();
   if (ok) {
     if (ntile > 0)
@@ -553,7 +555,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
   tc_fence_before();
   __syncthreads();
-  if (tid == 0 && !*abort_flag) {
+  if (tid == 0 && ok && !*abort_flag) {
 #pragma unroll
     for (int bx = 0; bx < 4; ++bx) tma_store_3d(&tmOut, base + bx * 16384, 32 * bx, 0, item);
     bulk_commit_group();
@@ -746,9 +748,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
   }
 
-  // ---- epilogue: accumulator -> fp32 tile -> TMA store (partial or final)
+  // ---- epilogue: accumulator -> fp32 tile -> TMA store (partial or final);
+  // nothing for a chunk past a ragged prompt's end unless it is the only one
   __syncwarp();
-  const bool ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag));
+  const bool store = ntile > 0 || a.splits == 1;
+  const bool ok = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag)) && store;
   tc_fence_after();
   if (ok) {
     if (ntile > 0)
@@ -761,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     a.zdst[static_cast<size_t>(item) * kD + (tid - 128)] = zacc;
   tc_fence_before();
   __syncthreads();
-  if (tid == 0 && !*abort_flag) {
+  if (tid == 0 && ok && !*abort_flag) {
 #pragma unroll
     for (int bx = 0; bx < 4; ++bx) tma_store_3d(&tmOut, base + bx * 16384, 32 * bx, 0, item);
     bulk_commit_group();
@@ -774,20 +778,34 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 }
 
-// S[u] = sum over chunks s (in order) of ws_S[u][s];  same for z.
+// S[u] = sum over chunks s (in order) of ws_S[u][s];  same for z.  Ragged
+// prompts: only the chunks the request's prompt reaches (none: S = z = 0).
+struct ReduceArgs {
+  int splits;
+  const int* T_lens;   // ragged: [n] prompt tokens, else null
+  int hkv, T, tiles_per;
+};
+
 __global__ void __launch_bounds__(256) k_prefill_reduce(const float4* __restrict__ wsS,
                                                         const float4* __restrict__ wsZ,
                                                         float4* __restrict__ S,
-                                                        float4* __restrict__ z, int splits) {
+                                                        float4* __restrict__ z,
+                                                        const ReduceArgs ra) {
   pdl_launch_dependents();
   pdl_wait();
   const int u = blockIdx.y;
   const int e = blockIdx.x * 256 + threadIdx.x;    // float4 index within a unit
   constexpr int kS4 = kD * kD / 4, kZ4 = kD / 4;
+  const int splits = ra.splits;
+  int nvalid = splits;
+  if (ra.T_lens != nullptr) {
+    const int Tu = min(max(__ldg(ra.T_lens + u / ra.hkv), 0), ra.T);
+    nvalid = min(splits, ((Tu + kTok - 1) / kTok + ra.tiles_per - 1) / ra.tiles_per);
+  }
   if (e < kS4) {
     const float4* p = wsS + static_cast<size_t>(u) * splits * kS4 + e;
-    float4 acc = p[0];
-    for (int s = 1; s < splits; ++s) {
+    float4 acc = nvalid > 0 ? p[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 1; s < nvalid; ++s) {
       const float4 v = p[static_cast<size_t>(s) * kS4];
       acc.x += v.x;
       acc.y += v.y;
@@ -798,8 +816,8 @@ __global__ void __launch_bounds__(256) k_prefill_reduce(const float4* __restrict
   }
   if (z != nullptr && e < kZ4) {
     const float4* p = wsZ + static_cast<size_t>(u) * splits * kZ4 + e;
-    float4 acc = p[0];
-    for (int s = 1; s < splits; ++s) {
+    float4 acc = nvalid > 0 ? p[0] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int s = 1; s < nvalid; ++s) {
       const float4 v = p[static_cast<size_t>(s) * kZ4];
       acc.x += v.x;
       acc.y += v.y;
@@ -967,9 +985,10 @@ int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, i
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    const ReduceArgs ra{splits, T_lens, hkv, T, tp};
     if (cudaLaunchKernelEx(&cfg, k_prefill_reduce, reinterpret_cast<const float4*>(outS),
                            reinterpret_cast<const float4*>(outZ), reinterpret_cast<float4*>(S),
-                           reinterpret_cast<float4*>(z), splits) != cudaSuccess)
+                           reinterpret_cast<float4*>(z), ra) != cudaSuccess)
       return -5;
     if (cudaGetLastError() != cudaSuccess) return -5;
   }

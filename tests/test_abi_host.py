@@ -217,9 +217,10 @@ def test_paged_prefix_validation(L):
     the workspace (sized for the longest cache)."""
     n, hq, hkv, b, d, maxp, ps = 4, 16, 4, 32, 128, 64, 128
     need = L.bha_prefix_softmax_paged_workspace_size(n, hq, hkv, b, d, maxp, ps, _lib.BHA_BF16)
-    assert need == L.bha_prefix_softmax_workspace_size(n, hq, hkv, b, d, maxp * ps,
-                                                       _lib.BHA_BF16)
-    assert need > 0
+    # chunks of 16 key tiles over the longest cache (8192 keys + the block: 65 tiles -> 5)
+    assert need == n * hkv * 5 * (128 * 128 + 256) * 4
+    assert L.bha_prefix_softmax_paged_workspace_size(n, hq, hkv, b, d, maxp, ps,
+                                                     _lib.BHA_F32) == 0
     big = GAP * 16
 
     def f(**kw):
