@@ -8,11 +8,13 @@
 //   * one CTA per (request, KV head, 128-row tile of the G*b packed query
 //     rows, chunk of the key sequence); keys come in 128-token tiles, cache
 //     tiles first, the active block last;
-//   * a TMA warp streams K and V tiles through 2-stage rings, an MMA warp
-//     issues S = Q K^T into one of two TMEM buffers and O += P V into a TMEM
-//     accumulator, and four softmax warps (thread = query row = TMEM lane)
-//     run the online softmax in registers, rescaling O only when a row max
-//     grows by more than 2^8 (the stale max is exact for the final ratio);
+//   * a TMA thread streams K and V tiles through 3-stage rings, an MMA
+//     thread issues S = Q K^T into one of two TMEM buffers and O += P V into
+//     a TMEM accumulator, and four softmax warps (thread = query row = TMEM
+//     lane) run the online softmax in registers, rescaling O only when a row
+//     max grows by more than 2^8 (the stale max is exact for the final
+//     ratio).  P goes back into TMEM (bf16 pairs, two buffers) as the A
+//     operand of P V, so shared memory holds only Q and the K / V rings;
 //   * chunks are combined by log-sum-exp in a second kernel, the way the
 //     LoSA page describes merging prefix and block attention with online
 //     softmax.  With one chunk the CTA normalises and stores Y itself.
@@ -40,12 +42,15 @@ namespace {
 constexpr int kD = 128;
 constexpr int kTK = 128;             // keys per tile
 constexpr int kThreads = 256;
-constexpr uint32_t kTileBytes = kTK * kD * 2;   // 32 KB (K or V tile, Q, P)
+constexpr uint32_t kTileBytes = kTK * kD * 2;   // 32 KB (K or V tile, Q)
+constexpr int kStages = 3;
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kTileBytes;          // 2 stages
-constexpr uint32_t kOffV = 3 * kTileBytes;      // 2 stages
-constexpr uint32_t kOffP = 5 * kTileBytes;
-constexpr uint32_t kTiles = 6 * kTileBytes;     // 192 KB
+constexpr uint32_t kOffK = kTileBytes;                      // 3 stages
+constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;    // 3 stages
+constexpr uint32_t kTiles = kOffV + kStages * kTileBytes;   // 224 KB
+// TMEM columns: S buffers [0, 128) and [128, 256), O [256, 384), P buffers
+// [384, 448) and [448, 512) (128 bf16 keys = 64 columns per row)
+constexpr uint32_t kColO = 256, kColP = 384;
 constexpr int kMaxChunkPages = 128;               // paged: a chunk's page numbers (16 tiles of 16-token pages)
 constexpr uint32_t kPageList = kMaxChunkPages * 4;
 constexpr uint32_t kCtrlBytes = 256;
@@ -96,23 +101,28 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + kTiles + kPageList;
   int* page_list = reinterpret_cast<int*>(smem_raw + (base - raw) + kTiles);
   uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
-  const uint32_t bar_q = ctrl, bar_kf = ctrl + 8, bar_ke = ctrl + 24, bar_vf = ctrl + 40,
-                 bar_ve = ctrl + 56, bar_sf = ctrl + 72, bar_pf = ctrl + 88, bar_pv = ctrl + 96;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 104);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 108);
+  // per stage: K / V landed (kf, vf), K / V consumed (ke, ve); per S buffer:
+  // scores ready (sf); per P buffer: P written (pf), P V done (pvb)
+  const uint32_t bar_q = ctrl, bar_kf = ctrl + 8, bar_ke = ctrl + 32, bar_vf = ctrl + 56,
+                 bar_ve = ctrl + 80, bar_sf = ctrl + 104, bar_pf = ctrl + 120,
+                 bar_pvb = ctrl + 136;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 152);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 156);
 
   if (warp == 0) {
     if (lane == 0) {
       mbar_init(bar_q, 1);
-      for (int s = 0; s < 2; ++s) {
+      for (int s = 0; s < kStages; ++s) {
         mbar_init(bar_kf + 8 * s, 1);
         mbar_init(bar_ke + 8 * s, 1);
         mbar_init(bar_vf + 8 * s, 1);
         mbar_init(bar_ve + 8 * s, 1);
-        mbar_init(bar_sf + 8 * s, 1);
       }
-      mbar_init(bar_pf, 128);
-      mbar_init(bar_pv, 1);
+      for (int s = 0; s < 2; ++s) {
+        mbar_init(bar_sf + 8 * s, 1);
+        mbar_init(bar_pf + 8 * s, 128);
+        mbar_init(bar_pvb + 8 * s, 1);
+      }
       *abort_flag = 0;
       fence_mbar_init();
     }
@@ -125,7 +135,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t t_o = tmem + 256;
+  const uint32_t t_o = tmem + kColO;
   pdl_wait();
 
   // this request's cache length (per request when paged), tiles of this chunk
@@ -188,11 +198,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     for (int i = 0; i < nt; ++i) {
-      const int st = i & 1;
+      const int st = i % kStages, ph = ((i / kStages) - 1) & 1;
       const int gi = tile0 + i;
-      if (i >= 2 && !mbar_wait(bar_ke + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
+      if (i >= kStages && !mbar_wait(bar_ke + 8 * st, ph, a.err, abort_flag)) break;
       load_tile(&tmKc, &tmKa, base + kOffK + st * kTileBytes, bar_kf + 8 * st, gi);
-      if (i >= 2 && !mbar_wait(bar_ve + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
+      if (i >= kStages && !mbar_wait(bar_ve + 8 * st, ph, a.err, abort_flag)) break;
       load_tile(&tmVc, &tmVa, base + kOffV + st * kTileBytes, bar_vf + 8 * st, gi);
     }
   } else if (tid == 32 && live) {
@@ -200,9 +210,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t idesc_s = make_idesc_bf16(128, kTK, 0, 0);   // Q K^T, both K-major
     constexpr uint32_t idesc_o = make_idesc_bf16(128, kD, 0, 1);    // P V, V MN-major
     bool ok = mbar_wait(bar_q, 0, a.err, abort_flag);
+    // S(i) into S buffer i % 2 (its last reader, tile i - 2, wrote P before
+    // the previous iteration's P V was issued)
     auto issue_s = [&](int i) -> bool {
-      const int st = i & 1;
-      if (!mbar_wait(bar_kf + 8 * st, (i >> 1) & 1, a.err, abort_flag)) return false;
+      const int st = i % kStages;
+      if (!mbar_wait(bar_kf + 8 * st, (i / kStages) & 1, a.err, abort_flag)) return false;
       tc_fence_after();
       const uint32_t kb = base + kOffK + st * kTileBytes;
 #pragma unroll
@@ -211,9 +223,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             make_sdesc(base + kOffQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128);
         const uint64_t db = make_sdesc(kb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024,
                                        kLayoutSW128);
-        mma_bf16_ss(tmem + st * 128, da, db, idesc_s, ks > 0 ? 1u : 0u);
+        mma_bf16_ss(tmem + (i & 1) * 128, da, db, idesc_s, ks > 0 ? 1u : 0u);
       }
-      mma_commit(bar_sf + 8 * st);
+      mma_commit(bar_sf + 8 * (i & 1));
       mma_commit(bar_ke + 8 * st);
       return true;
     };
@@ -221,22 +233,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < nt && ok; ++i) {
       if (i + 1 < nt) ok = issue_s(i + 1);
       if (!ok) break;
-      const int st = i & 1;
-      ok = mbar_wait(bar_pf, i & 1, a.err, abort_flag) &&
-           mbar_wait(bar_vf + 8 * st, (i >> 1) & 1, a.err, abort_flag);
+      const int st = i % kStages, pb = i & 1;
+      ok = mbar_wait(bar_pf + 8 * pb, (i >> 1) & 1, a.err, abort_flag) &&
+           mbar_wait(bar_vf + 8 * st, (i / kStages) & 1, a.err, abort_flag);
       if (!ok) break;
       tc_fence_after();
       const uint32_t vb = base + kOffV + st * kTileBytes;
 #pragma unroll
       for (int ks = 0; ks < kTK / 16; ++ks) {
-        const uint64_t da =
-            make_sdesc(base + kOffP + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128);
-        // V tile: [keys][d] as 2 boxes of 64 d-columns; keys are the K dim
+        // P from TMEM (8 columns per 16 keys); V tile: [keys][d] as 2 boxes
+        // of 64 d-columns, keys the K dim (MN-major)
         const uint64_t db = make_sdesc(vb + ks * 2048, 16384, 1024, kLayoutSW128);
-        mma_bf16_ss(t_o, da, db, idesc_o, (i | ks) ? 1u : 0u);
+        mma_bf16_ts(t_o, tmem + kColP + 64 * pb + 8 * ks, db, idesc_o, (i | ks) ? 1u : 0u);
       }
       mma_commit(bar_ve + 8 * st);
-      mma_commit(bar_pv);
+      mma_commit(bar_pvb + 8 * pb);
     }
   }
 
@@ -247,17 +258,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool ok = true;
   if (warp >= 4 && live) {
     for (int i = 0; i < nt; ++i) {
-      const int st = i & 1;
+      const int st = i % kStages, sb = i & 1;
       const int gi = tile0 + i;
       const int valid = gi < ncache_tiles ? min(kTK, P - gi * kTK) : a.b;
-      ok = warp_all(ok && mbar_wait(bar_sf + 8 * st, (i >> 1) & 1, a.err, abort_flag));
+      ok = warp_all(ok && mbar_wait(bar_sf + 8 * sb, (i >> 1) & 1, a.err, abort_flag));
       if (!ok) break;
       tc_fence_after();
       float s[kTK];
 #pragma unroll
       for (int c = 0; c < kTK; c += 32) {
         float t[32];
-        tmem_ld32_sync(tmem + st * 128 + lane_base + c, t);
+        tmem_ld32_sync(tmem + sb * 128 + lane_base + c, t);
 #pragma unroll
         for (int q = 0; q < 32; ++q) s[c + q] = t[q];
       }
@@ -283,12 +294,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         ls += s[j];
       }
       l = l * corr + ls;
-      // P and O are free once P V of the previous tile has completed
-      if (i > 0) {
-        ok = warp_all(mbar_wait(bar_pv, (i - 1) & 1, a.err, abort_flag));
+      // O is stable once P V of the previous tile has completed (only a
+      // rescale needs it); P buffer sb once P V of tile i - 2 has
+      if (i > 0 && __any_sync(0xffffffffu, resc)) {
+        ok = warp_all(mbar_wait(bar_pvb + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1, a.err,
+                                abort_flag));
         if (!ok) break;
         tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
+        {
 #pragma unroll 1
           for (int c = 0; c < kD; c += 32) {
             float o[32];
@@ -302,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (PAGED && gi < ncache_tiles && valid < kTK) {
         // rows past the cache hold stale pool data (or none was loaded):
         // zero them in V so that P (0 there) times V stays finite
-        ok = warp_all(mbar_wait(bar_vf + 8 * st, (i >> 1) & 1, a.err, abort_flag));
+        ok = warp_all(mbar_wait(bar_vf + 8 * st, (i / kStages) & 1, a.err, abort_flag));
         if (!ok) break;
         if (r >= valid) {
           const uint32_t vrow = base + kOffV + st * kTileBytes + r * 128;
@@ -313,22 +326,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-#pragma unroll
-      for (int box = 0; box < 2; ++box) {
-        const uint32_t prow = base + kOffP + box * 16384 + r * 128;
-#pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const float* e = s + box * 64 + jj * 8;
-          st_shared_v4(prow + ((jj ^ (r & 7)) << 4), pack_bf16x2(e[0], e[1]),
-                       pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
-        }
+      if (i >= 2) {
+        ok = warp_all(mbar_wait(bar_pvb + 8 * sb, ((i >> 1) - 1) & 1, a.err, abort_flag));
+        if (!ok) break;
+        tc_fence_after();
       }
-      fence_proxy_async_smem();
+      // P row r as bf16 pairs into TMEM (column c = keys 2c, 2c + 1)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c)
+          pk[c] = __uint_as_float(pack_bf16x2(s[64 * h + 2 * c], s[64 * h + 2 * c + 1]));
+        tmem_st32(tmem + kColP + 64 * sb + lane_base + 32 * h, pk);
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();   // the zeroed V rows, if any
       tc_fence_before();
-      mbar_arrive(bar_pf);
+      mbar_arrive(bar_pf + 8 * sb);
     }
     // final accumulator
-    if (ok && nt > 0) ok = warp_all(mbar_wait(bar_pv, (nt - 1) & 1, a.err, abort_flag));
+    if (ok && nt > 0)
+      ok = warp_all(mbar_wait(bar_pvb + 8 * ((nt - 1) & 1), ((nt - 1) >> 1) & 1, a.err,
+                              abort_flag));
     tc_fence_after();
     if (ok) {
       if (a.splits == 1) {
