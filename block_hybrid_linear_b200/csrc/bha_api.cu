@@ -443,8 +443,8 @@ int bha_hybrid_step_commit_fm(const void* Qa, const void* Ka, const void* Va, fl
                                            fmap, Wf, hkv));
   }
   // one kernel (step, then fold the block in) in the default mode with one
-  // 128-row tile per unit and an elementwise map
-  if (!shared && (hq / hkv) * b <= 128 && fmap != BHA_FMAP_RELU_PROJ)
+  // 128-row tile per unit
+  if (!shared && (hq / hkv) * b <= 128)
     return launch_status(
         launch_step_bf16(c, Qa, Ka, Va, S, nullptr, Y, n, hq, hkv, b, sc, 0, fmap, W, z, 1));
   st = launch_status(launch_step_bf16(c, Qa, Ka, Va, S, shared ? z : nullptr, Y, n, hq, hkv, b,

@@ -75,7 +75,7 @@ int launch_prefix_f32(const Ctx& c, const float* Q, const float* Kc, const float
 
 // ---- bf16 tensor-core path (tcgen05, d = 128) ----
 // fmap: the bha_fmap value; W: [hkv][128][128] bf16 (projected map) or null.
-// commit != 0 (default mode, G * b <= 128, elementwise maps only): also
+// commit != 0 (default mode, G * b <= 128): also
 // S += phi(K)^T V and z += sum phi(k) (z = commit_z, may be null) after the
 // step has used S.
 int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, const float* S,

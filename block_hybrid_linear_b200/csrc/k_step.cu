@@ -56,7 +56,7 @@ constexpr uint32_t kOffQ = 0;
 constexpr uint32_t kOffS = kQBytes;
 constexpr uint32_t kOffK = kQBytes + kSBytes;
 constexpr uint32_t kOffW = kOffS + kSBytes / 2;   // projected map: over state chunks 2-3
-constexpr uint32_t kCtrlBytes = 128;
+constexpr uint32_t kCtrlBytes = 256;
 
 struct StepArgs {
   const float* z;     // [units][128] (shared mode)
@@ -143,12 +143,18 @@ __device__ __forceinline__ float proj_qz(uint32_t tcol, const float* zu) {
   return qz;
 }
 
+// COMMIT with the projected map: the transposed projection (K W_g)^T =
+// W_g^T K^T (A = W_g MN-major, B = K K-major, M = 128 features, N = BPAD
+// tokens) is issued with Q W_g into the accumulator's columns [BPAD,
+// 2 BPAD), which P V overwrites only after warps 0-3 (thread = feature)
+// have read it; they write phi(K)^T as a K-major operand over the consumed
+// K tile.
 // COMMIT: also fold this step's block into the state after using it (the
 // block's last denoising step): S += phi(K)^T V, z += sum_t phi(k_t); the
 // state is read once (the tile the step used) and phi(K)^T V goes over that
 // tile to a TMA reduce-add into S.  P then lives in the consumed Q tile so that K survives for the commit MMA,
 // and phi(K)^T V accumulates in the TMEM columns phi(Q) used.  Default mode
-// and a single 128-row tile per unit only; elementwise maps only.
+// and a single 128-row tile per unit only.
 template <int BPAD, bool SHARED, bool COMMIT, int FMAP>
 __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     k_step_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -156,7 +162,6 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmW,
                 const StepArgs a) {
   static_assert(!(SHARED && COMMIT), "the fused commit runs in the default mode only");
-  static_assert(!(COMMIT && FMAP == kFmapReluProj), "the fused commit has no projected map");
   constexpr bool PROJ = FMAP == kFmapReluProj;
   using Lay = StepLayout<BPAD>;
   // P (the softmax weights, bf16, K-major) goes over the consumed K tile, or
@@ -175,7 +180,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   const uint32_t bar_q = ctrl, bar_k = ctrl + 8, bar_v = ctrl + 16, bar_s = ctrl + 24,
                  bar_sc = ctrl + 56, bar_p = ctrl + 64, bar_a = ctrl + 72, bar_done = ctrl + 80,
                  bar_phik = ctrl + 96, bar_ds = ctrl + 104, bar_w = ctrl + 112,
-                 bar_qw = ctrl + 120;
+                 bar_qw = ctrl + 120, bar_kwr = ctrl + 128;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 88);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 92);
 
@@ -196,6 +201,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       if (PROJ) {
         mbar_init(bar_w, 1);
         mbar_init(bar_qw, 1);
+        if (COMMIT) mbar_init(bar_kwr, 128);
       }
       *abort_flag = 0;
       fence_mbar_init();
@@ -293,7 +299,36 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     }
     tc_fence_before();
     mbar_arrive(bar_a);
-    if (COMMIT) {
+    if (COMMIT && PROJ) {
+      // thread = feature r: row r of (K W_g)^T (landed with Q W_g) out of
+      // TMEM, which P V may then overwrite; ReLU, bf16, z, and row r of
+      // phi(K)^T over the consumed K tile
+      constexpr uint32_t kRowB = 2 * BPAD;
+      const int rr = tid;
+      uint32_t wv[BPAD / 2];
+      float zs = 0.f;
+#pragma unroll
+      for (int j0 = 0; j0 < BPAD; j0 += 16) {
+        float f[16];
+        tmem_ld16_sync(t_d + BPAD + lane_base + j0, f);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          // padded tokens are zero rows of K, so their features are 0
+          wv[j0 / 2 + q] = pack_bf16x2(fmaxf(f[2 * q], 0.f), fmaxf(f[2 * q + 1], 0.f));
+          zs += __uint_as_float(wv[j0 / 2 + q] << 16) +
+                __uint_as_float(wv[j0 / 2 + q] & 0xFFFF0000u);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_kwr);
+#pragma unroll
+      for (int jj = 0; jj < BPAD / 8; ++jj)
+        st_shared_v4(kmajor_chunk<kRowB>(base + kOffK, rr, jj), wv[4 * jj], wv[4 * jj + 1],
+                     wv[4 * jj + 2], wv[4 * jj + 3]);
+      fence_proxy_async_smem();
+      mbar_arrive(bar_phik);
+      if (a.zc != nullptr) a.zc[static_cast<size_t>(u) * kD + rr] += zs;
+    } else if (COMMIT) {
       // phi(K) in place once the score MMA has read K, and this block's
       // column sums of phi(K) for z (thread = feature r)
       const bool okk = warp_all(mbar_wait(bar_sc, 0, a.err, abort_flag));
@@ -348,6 +383,17 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
                                            1024, kLayoutSW128);
             const uint64_t db = make_sdesc(base + kOffW + ks * 2048, 16384, 1024, kLayoutSW128);
             mma_bf16_ss(t_a, da, db, idw, ks > 0 ? 1u : 0u);
+          }
+          if (COMMIT) {
+            // (K W_g)^T: A = W_g MN-major, B = K K-major
+            constexpr uint32_t idk = make_idesc_bf16(128, BPAD, 1, 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+              const uint64_t da = make_sdesc(base + kOffW + ks * 2048, 16384, 1024, kLayoutSW128);
+              const uint64_t db = make_sdesc(
+                  base + kOffK + (ks >> 2) * (BPAD * 128) + (ks & 3) * 32, 16, 1024, kLayoutSW128);
+              mma_bf16_ss(t_d + BPAD, da, db, idk, ks > 0 ? 1u : 0u);
+            }
           }
           mma_commit(bar_qw);
         }
@@ -454,7 +500,8 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
 
     if (tid == 128) {
       // MMA issuer for P V and the per-chunk phi(Q) S products
-      bool ok2 = mbar_wait(bar_p, 0, a.err, abort_flag) && mbar_wait(bar_v, 0, a.err, abort_flag);
+      bool ok2 = mbar_wait(bar_p, 0, a.err, abort_flag) && mbar_wait(bar_v, 0, a.err, abort_flag) &&
+                 (!(COMMIT && PROJ) || mbar_wait(bar_kwr, 0, a.err, abort_flag));
       if (ok2) {
         tc_fence_after();
         constexpr uint32_t idesc = make_idesc_bf16(128, 128, 0, 1);
@@ -488,10 +535,15 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         ok2 = mbar_wait(bar_done, 0, a.err, abort_flag) && mbar_wait(bar_phik, 0, a.err, abort_flag);
         if (ok2) {
           tc_fence_after();
-          constexpr uint32_t idesc = make_idesc_bf16(128, 128, 1, 1);
+          // A = phi(K)^T: MN-major phi(K) in place, or K-major rows of the
+          // projected map's features
+          constexpr uint32_t idesc = make_idesc_bf16(128, 128, PROJ ? 0 : 1, 1);
 #pragma unroll
           for (int ks = 0; ks < BPAD / 16; ++ks) {
-            const uint64_t da = make_sdesc(base + kOffK + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
+            const uint64_t da =
+                PROJ ? make_sdesc(base + kOffK + ks * 32, 16, 16 * BPAD,
+                                  kmajor_layout<2 * BPAD>())
+                     : make_sdesc(base + kOffK + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
             const uint64_t db =
                 make_sdesc(base + Lay::kOffV + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
             mma_bf16_ss(t_a, da, db, idesc, ks > 0 ? 1u : 0u);
@@ -596,11 +648,7 @@ int launch_cfg(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int 
 template <int BPAD, int FMAP>
 int launch_fmap(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int grid, int shared,
                 int commit) {
-  if constexpr (FMAP != kFmapReluProj) {
-    if (commit) return launch_cfg<BPAD, false, true, FMAP>(c, tm, a, grid);
-  } else {
-    if (commit) return -5;
-  }
+  if (commit) return launch_cfg<BPAD, false, true, FMAP>(c, tm, a, grid);
   return shared ? launch_cfg<BPAD, true, false, FMAP>(c, tm, a, grid)
                 : launch_cfg<BPAD, false, false, FMAP>(c, tm, a, grid);
 }

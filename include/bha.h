@@ -215,8 +215,8 @@ int bha_hybrid_step_fm(const void *Qa, const void *Ka, const void *Va,
                        bha_dtype dtype, bha_fmap fmap, const void *W,
                        bha_stream_t stream);
 
-/* bha_hybrid_step_commit with feature map `fmap`.  BHA_FMAP_RELU_PROJ
- * always runs the step and the commit as two kernels. */
+/* bha_hybrid_step_commit with feature map `fmap` (one kernel in the same
+ * cases as bha_hybrid_step_commit, for every map). */
 int bha_hybrid_step_commit_fm(const void *Qa, const void *Ka, const void *Va,
                               float *S, float *z, void *Y, int n, int hq,
                               int hkv, int b, int d, float scale,

@@ -250,8 +250,9 @@ def test_prefill_fmap_f32(fmap):
 @pytest.mark.parametrize("case", [(2, 16, 4, 32), (2, 8, 2, 17), (2, 8, 1, 33)],
                          ids=lambda c: "n%d_hq%d_hkv%d_b%d" % c)
 def test_step_commit_fmap_bf16(case, fmap, mode):
-    """elu + 1 in the default mode with G*b <= 128 runs the fused kernel; the
-    projected map always runs step + commit."""
+    """In the default mode with G*b <= 128 both maps run the fused kernel
+    (the projected one computes (K W_g)^T beside Q W_g); otherwise step +
+    commit kernels."""
     import torch
     n, hq, hkv, b = case
     f = FMAPS[fmap]
