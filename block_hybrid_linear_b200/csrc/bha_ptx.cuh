@@ -239,6 +239,24 @@ __device__ __forceinline__ void mma_commit(uint32_t bar) {
 // receives TMEM lane (base lane + t), columns [col, col + N).  The load and
 // its completion wait are one asm statement, so the destination registers
 // are valid (and cannot be read early) once the statement has executed.
+// One 32-bit column of this warp's 32 lanes (ld: with its completion wait).
+__device__ __forceinline__ float tmem_ld1_sync(uint32_t taddr) {
+  uint32_t r;
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r)
+      : "r"(taddr)
+      : "memory");
+  return __uint_as_float(r);
+}
+
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr),
+               "r"(__float_as_uint(v))
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, float (&v)[16]) {
   uint32_t r[16];
   asm volatile(

@@ -83,12 +83,14 @@ struct StepLayout {
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
-// phi(q_r) * scale as fp32 into TMEM (this thread's lane, columns [0, 128)
-// from `tcol`), read from row r of the SW128 Q tile; one wait for all four
+// phi(q_r) as fp32 into TMEM (this thread's lane, columns [0, 128) from
+// `tcol`), read from row r of the SW128 Q tile; one wait for all four
 // 32-column stores.  Elementwise maps only (phi of a bf16 pair is a bf16
-// pair); the tensor core reads the values as tf32.
-template <int FMAP>
-__device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol, float scale) {
+// pair; the tensor core reads the values as tf32).  QZ: also returns
+// phi(q_r) . z (the shared denominator's term), z from global memory.
+template <int FMAP, bool QZ>
+__device__ __forceinline__ float write_phiq(uint32_t qtile, int r, uint32_t tcol, const float* zu) {
+  float qz = 0.f;
 #pragma unroll
   for (int cg = 0; cg < 4; ++cg) {
     float f[32];
@@ -100,47 +102,63 @@ __device__ __forceinline__ void write_phiq(uint32_t qtile, int r, uint32_t tcol,
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const uint32_t p2 = phi_bf16x2<FMAP>(w4[e]);
-        f[8 * q + 2 * e] = __uint_as_float(p2 << 16) * scale;
-        f[8 * q + 2 * e + 1] = __uint_as_float(p2 & 0xFFFF0000u) * scale;
+        f[8 * q + 2 * e] = __uint_as_float(p2 << 16);
+        f[8 * q + 2 * e + 1] = __uint_as_float(p2 & 0xFFFF0000u);
+      }
+      if (QZ) {
+        // columns cg * 32 + 8 q .. + 7
+        const float4 z0 = __ldg(reinterpret_cast<const float4*>(zu + cg * 32 + 8 * q));
+        const float4 z1 = __ldg(reinterpret_cast<const float4*>(zu + cg * 32 + 8 * q + 4));
+        const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qz = fmaf(f[8 * q + e], zz[e], qz);
       }
     }
     tmem_st32(tcol + cg * 32, f);
   }
   tmem_wait_st();
+  return qz;
 }
 
 // Projected map: the Q W_g product sits in TMEM (this thread's lane, 128
-// columns from `tcol`); replace it by max(., 0) * scale.
-__device__ __forceinline__ void relu_tmem_phiq(uint32_t tcol, float scale) {
-#pragma unroll
-  for (int cg = 0; cg < 4; ++cg) {
-    float f[32];
-    tmem_ld32_sync(tcol + cg * 32, f);
-#pragma unroll
-    for (int q = 0; q < 32; ++q) f[q] = fmaxf(f[q], 0.f) * scale;
-    tmem_st32(tcol + cg * 32, f);
-  }
-  tmem_wait_st();
-}
-
-// Projected map, shared denominator: phi(q_r) . z_g from the Q W_g product
-// in TMEM.
-__device__ __forceinline__ float proj_qz(uint32_t tcol, const float* zu) {
+// columns from `tcol`); replace it by max(., 0).  QZ: also returns
+// phi(q_r) . z.
+template <bool QZ>
+__device__ __forceinline__ float relu_tmem_phiq(uint32_t tcol, const float* zu) {
   float qz = 0.f;
 #pragma unroll
   for (int cg = 0; cg < 4; ++cg) {
     float f[32];
     tmem_ld32_sync(tcol + cg * 32, f);
 #pragma unroll
-    for (int q = 0; q < 32; q += 4) {
-      const float4 zz = __ldg(reinterpret_cast<const float4*>(zu + cg * 32 + q));
-      qz = fmaf(fmaxf(f[q], 0.f), zz.x, qz);
-      qz = fmaf(fmaxf(f[q + 1], 0.f), zz.y, qz);
-      qz = fmaf(fmaxf(f[q + 2], 0.f), zz.z, qz);
-      qz = fmaf(fmaxf(f[q + 3], 0.f), zz.w, qz);
+    for (int q = 0; q < 32; ++q) f[q] = fmaxf(f[q], 0.f);
+    if (QZ) {
+#pragma unroll
+      for (int q = 0; q < 32; q += 4) {
+        const float4 zz = __ldg(reinterpret_cast<const float4*>(zu + cg * 32 + q));
+        qz = fmaf(f[q], zz.x, qz);
+        qz = fmaf(f[q + 1], zz.y, qz);
+        qz = fmaf(f[q + 2], zz.z, qz);
+        qz = fmaf(f[q + 3], zz.w, qz);
+      }
     }
+    tmem_st32(tcol + cg * 32, f);
   }
+  tmem_wait_st();
   return qz;
+}
+
+// Shared denominator: this thread's row of phi(Q) in TMEM times s.
+__device__ __forceinline__ void scale_tmem_row(uint32_t tcol, float s) {
+#pragma unroll
+  for (int cg = 0; cg < 4; ++cg) {
+    float f[32];
+    tmem_ld32_sync(tcol + cg * 32, f);
+#pragma unroll
+    for (int q = 0; q < 32; ++q) f[q] *= s;
+    tmem_st32(tcol + cg * 32, f);
+  }
+  tmem_wait_st();
 }
 
 // COMMIT with the projected map: the transposed projection (K W_g)^T =
@@ -180,7 +198,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   const uint32_t bar_q = ctrl, bar_k = ctrl + 8, bar_v = ctrl + 16, bar_s = ctrl + 24,
                  bar_sc = ctrl + 56, bar_p = ctrl + 64, bar_a = ctrl + 72, bar_done = ctrl + 80,
                  bar_phik = ctrl + 96, bar_ds = ctrl + 104, bar_w = ctrl + 112,
-                 bar_qw = ctrl + 120, bar_kwr = ctrl + 128;
+                 bar_qw = ctrl + 120, bar_kwr = ctrl + 128, bar_a2 = ctrl + 136;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 88);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 92);
 
@@ -193,6 +211,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       mbar_init(bar_sc, 1);
       mbar_init(bar_p, 128);
       mbar_init(bar_a, 128);
+      if (SHARED) mbar_init(bar_a2, 128);
       mbar_init(bar_done, 1);
       if (COMMIT) {
         mbar_init(bar_phik, 128);
@@ -233,12 +252,12 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   const uint32_t tmem = *tmem_slot;
   const uint32_t t_d = tmem;           // [0, 128): the output accumulator
   const uint32_t t_a = tmem + 128;     // [128, 256): phi(Q) as tf32 (the MMA's A)
-  // Scores: in the default mode they sit in the accumulator's first columns
-  // (P V overwrites them once read) so phi(Q) can be built in parallel; with
-  // the shared denominator phi(Q) needs the row max first, so the scores sit
-  // where phi(Q) will go -- except under the projected map, whose Q W_g
-  // product needs those columns from the start.
-  const uint32_t t_sc = (SHARED && !PROJ) ? t_a : t_d;
+  // Scores sit in the accumulator's first columns (P V overwrites them once
+  // read), so phi(Q) is built in parallel.  With the shared denominator,
+  // warps 0-3 also hand each row's phi(q) . z to the row owners through the
+  // accumulator's last column, which P V overwrites only after it is read.
+  const uint32_t t_sc = t_d;
+  const uint32_t t_qz = t_d + kD - 1;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   pdl_wait();   // inputs may come from the previous kernel of the stream
 
@@ -280,22 +299,25 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
                     u);
     }
   };
-  if (PROJ && SHARED && tid == 0) {
-    if (mbar_wait(bar_qw, 0, a.err, abort_flag)) load_late_chunks();
-  }
-
   float beta = 1.f;   // per-row output scale (shared denominator only)
-  if (!SHARED && warp < 4) {
+  if (warp < 4) {
     // phi(q) for row r = 32 w + lane into TMEM as soon as Q has landed, in
-    // parallel with the score MMA and the softmax
+    // parallel with the score MMA and the softmax (and phi(q) . z)
+    const float* zu = SHARED ? a.z + static_cast<size_t>(u) * kD : nullptr;
+    float qz = 0.f;
+    bool okf;
     if (PROJ) {
-      const bool okw = warp_all(mbar_wait(bar_qw, 0, a.err, abort_flag));
+      okf = warp_all(mbar_wait(bar_qw, 0, a.err, abort_flag));
       tc_fence_after();
-      if (okw && tid == 0) load_late_chunks();
-      if (okw) relu_tmem_phiq(t_a + lane_base, 1.f);
+      if (okf && tid == 0) load_late_chunks();
+      if (okf) qz = relu_tmem_phiq<SHARED>(t_a + lane_base, zu);
     } else {
-      const bool okq = warp_all(mbar_wait(bar_q, 0, a.err, abort_flag));
-      if (okq) write_phiq<FMAP>(base + kOffQ, warp * 32 + lane, t_a + lane_base, 1.f);
+      okf = warp_all(mbar_wait(bar_q, 0, a.err, abort_flag));
+      if (okf) qz = write_phiq<FMAP, SHARED>(base + kOffQ, warp * 32 + lane, t_a + lane_base, zu);
+    }
+    if (SHARED && okf) {
+      tmem_st1(t_qz + lane_base, qz);
+      tmem_wait_st();
     }
     tc_fence_before();
     mbar_arrive(bar_a);
@@ -424,34 +446,11 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         l += sc[j];
       }
       float pscale;
-      float qz = 0.f;
       if (SHARED) {
-        if (PROJ) {
-          const bool okw = warp_all(mbar_wait(bar_qw, 0, a.err, abort_flag));
-          tc_fence_after();
-          if (okw) qz = proj_qz(t_a + lane_base, a.z + static_cast<size_t>(u) * kD);
-        } else {
-          const float* zu = a.z + static_cast<size_t>(u) * kD;
-#pragma unroll
-          for (int box = 0; box < 2; ++box) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const uint4 v = ld_shared_v4(base + kOffQ + box * 16384 + r * 128 +
-                                           ((j ^ (r & 7)) << 4));
-              const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-              const float4 z0 = __ldg(reinterpret_cast<const float4*>(zu + box * 64 + j * 8));
-              const float4 z1 =
-                  __ldg(reinterpret_cast<const float4*>(zu + box * 64 + j * 8 + 4));
-              const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-#pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                const uint32_t p2 = phi_bf16x2<FMAP>(w4[q]);
-                qz = fmaf(__uint_as_float(p2 << 16), zz[2 * q], qz);
-                qz = fmaf(__uint_as_float(p2 & 0xFFFF0000u), zz[2 * q + 1], qz);
-              }
-            }
-          }
-        }
+        // phi(q) . z from warps 0-3 (with phi(Q), unscaled, in TMEM)
+        const bool oka = warp_all(mbar_wait(bar_a, 0, a.err, abort_flag));
+        tc_fence_after();
+        const float qz = oka ? tmem_ld1_sync(t_qz + lane_base) : 0.f;
         // y = (sum_j e_j v_j + e^{-m_s} phi(q) S) / (l + e^{-m_s} phi(q).z),
         // m_s = scale * m; the factor that stays <= 1 is applied to phi(q)
         // (m_s >= 0) or to P (m_s < 0), so nothing overflows.
@@ -486,16 +485,11 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     mbar_arrive(bar_p);
 
     if (SHARED) {
-      // phi(q) times the row's scale, over the scores already read (or over
-      // the Q W_g product)
-      if (ok) {
-        if (PROJ)
-          relu_tmem_phiq(t_a + lane_base, ascale);
-        else
-          write_phiq<FMAP>(base + kOffQ, r, t_a + lane_base, ascale);
-      }
+      // the row's factor e^{-m_s} into its phi(q) (rows with m_s < 0 put
+      // theirs into P instead)
+      if (ok && __any_sync(0xffffffffu, ascale != 1.f)) scale_tmem_row(t_a + lane_base, ascale);
       tc_fence_before();
-      mbar_arrive(bar_a);
+      mbar_arrive(bar_a2);
     }
 
     if (tid == 128) {
@@ -512,7 +506,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
               make_sdesc(base + Lay::kOffV + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
           mma_bf16_ss(t_d, da, db, idesc, ks > 0 ? 1u : 0u);
         }
-        ok2 = mbar_wait(bar_a, 0, a.err, abort_flag);
+        ok2 = mbar_wait(SHARED ? bar_a2 : bar_a, 0, a.err, abort_flag);
       }
       for (int c = 0; c < 4 && ok2; ++c) {
         ok2 = mbar_wait(bar_s + 8 * c, 0, a.err, abort_flag);

@@ -8,7 +8,9 @@
 * long prefix (batch 64, prefix 32768): the step and the commit on all 256
   units; the 32k prefill and the exact prefix softmax on sampled units (the
   oracle's cost per unit is ~1 s there), in the launch configuration the
-  benchmark times.
+  benchmark times;
+* stack (prefix 8192) at its largest swept batch, 256: one exact and one
+  hybrid layer on sampled units; and the longest prompt, 131072 tokens.
 Plus the timeout self-test of the bounded waits.
 """
 import math
@@ -203,6 +205,61 @@ def test_long_prefix_prefill_and_exact_path_sampled():
         ref = oracle.prefix_softmax(qh, kp, vp, P, host(K[ni:ni + 1, g:g + 1]),
                                     host(V[ni:ni + 1, g:g + 1]))
         check_bf16("config4_prefix", host(Y[ni:ni + 1, g * G:(g + 1) * G]), ref, unit=u)
+
+
+def test_stack_config_exact_and_hybrid_layers_largest_batch_sampled():
+    """The stack workload at its largest swept batch (256 requests, prefix
+    8192): one exact layer (the contiguous exact path) and one hybrid layer
+    (prefill of the same prefix, then a step), checked on units {first,
+    middle, last} against the oracle."""
+    import torch
+    n, hq, hkv, b, P, seed = 256, 16, 4, 32, 8192, 5000
+    Kc = inputs.normal_bf16_torch(seed, inputs.TID_KC, (n, hkv, P, 128), STD, "cuda")
+    Vc = inputs.normal_bf16_torch(seed, inputs.TID_VC, (n, hkv, P, 128), STD, "cuda")
+    Q = inputs.normal_bf16_torch(seed, inputs.TID_Q, (n, hq, b, 128), STD, "cuda")
+    K = inputs.normal_bf16_torch(seed, inputs.TID_K, (n, hkv, b, 128), STD, "cuda")
+    V = inputs.normal_bf16_torch(seed, inputs.TID_V, (n, hkv, b, 128), STD, "cuda")
+    Yx = torch.empty(n, hq, b, 128, dtype=torch.bfloat16, device="cuda")
+    Yh = torch.empty_like(Yx)
+    needp = bha.bha_prefix_softmax_workspace_size(n, hq, hkv, b, 128, P)
+    wsp = torch.empty(max(needp, 16), dtype=torch.uint8, device="cuda")
+    bha.bha_prefix_softmax(Q, Kc, Vc, P, K, V, Yx, workspace=wsp)
+    S = torch.empty(n, hkv, 128, 128, device="cuda")
+    need = bha.bha_state_prefill_workspace_size(n, hkv, P, 128)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+    bha.bha_state_prefill(Kc, Vc, S, None, workspace=ws)
+    bha.bha_hybrid_step(Q, K, V, S, Yh)
+    torch.cuda.synchronize()
+    G = hq // hkv
+    for u in (0, (n * hkv) // 2 + 3, n * hkv - 1):
+        ni, g = divmod(u, hkv)
+        kc, vc = host(Kc[ni:ni + 1, g:g + 1]), host(Vc[ni:ni + 1, g:g + 1])
+        qh = host(Q[ni:ni + 1, g * G:(g + 1) * G])
+        kh, vh = host(K[ni:ni + 1, g:g + 1]), host(V[ni:ni + 1, g:g + 1])
+        check_bf16("config5_exact", host(Yx[ni:ni + 1, g * G:(g + 1) * G]),
+                   oracle.prefix_softmax(qh, kc, vc, P, kh, vh), unit=u)
+        rS, _ = oracle.state_prefill(kc, vc, with_z=False)
+        check_rel("config5_prefill_S", host(S[ni:ni + 1, g:g + 1]), rS, TOL_STATE_REL, unit=u)
+        check_bf16("config5_hybrid", host(Yh[ni:ni + 1, g * G:(g + 1) * G]),
+                   oracle.hybrid_step(qh, kh, vh, rS), unit=u)
+
+
+def test_prefill_longest_prompt_sampled():
+    """A 131072-token prompt (32 chunks per unit, reduced in order) for one
+    request: every KV head against the oracle."""
+    import torch
+    n, hkv, T = 1, 4, 131072
+    Kp = inputs.normal_bf16_torch(7000, inputs.TID_KP, (n, hkv, T, 128), STD, "cuda")
+    Vp = inputs.normal_bf16_torch(7000, inputs.TID_VP, (n, hkv, T, 128), STD, "cuda")
+    S = torch.empty(n, hkv, 128, 128, device="cuda")
+    z = torch.empty(n, hkv, 128, device="cuda")
+    need = bha.bha_state_prefill_workspace_size(n, hkv, T, 128)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+    bha.bha_state_prefill(Kp, Vp, S, z, workspace=ws)
+    torch.cuda.synchronize()
+    rS, rz = oracle.state_prefill(host(Kp), host(Vp))
+    check_rel("prefill_131072_S", host(S), rS, TOL_STATE_REL, ws=need)
+    check_rel("prefill_131072_z", host(z), rz, TOL_STATE_REL)
 
 
 def test_bounded_wait_timeout_is_reported_and_context_survives():
