@@ -6,25 +6,25 @@
 // still attends to all previous blocks).  Flash-attention structure on
 // tcgen05:
 //   * one CTA per (request, KV head, 128-row tile of the G*b packed query
-//     rows, chunk of the key sequence); keys come in 128-token tiles, cache
-//     tiles first, the active block last;
-//   * a TMA thread streams K and V tiles through 3-stage rings, an MMA
+//     rows, chunk of the key sequence); keys come in 64-token tiles, cache
+//     tiles first, the active block last; 113 KB of shared memory and 256
+//     TMEM columns, so two CTAs share an SM and one's prologue, pipeline
+//     fill and epilogue overlap the other's stream;
+//   * a TMA thread streams K and V tiles through 2-stage rings, an MMA
 //     thread issues S = Q K^T into one of two TMEM buffers and O += P V into
 //     a TMEM accumulator, and four softmax warps (thread = query row = TMEM
 //     lane) run the online softmax in registers, rescaling O only when a row
-//     max grows by more than 2^8 (the stale max is exact for the final
-//     ratio).  P goes back into TMEM (bf16 pairs, two buffers) as the A
-//     operand of P V, so shared memory holds only Q and the K / V rings;
+//     max grows by more than 2^8 (the stale max is exact for the final ratio);
 //   * chunks are combined by log-sum-exp in a second kernel, the way the
 //     LoSA page describes merging prefix and block attention with online
 //     softmax.  With one chunk the CTA normalises and stores Y itself.
 // Paged variant (the summary page pairs the method with KV-cache management;
 // its related work names PagedAttention): the cache of request i is its first
 // P_lens[i] tokens, token t at row t % page_size of page block_table[i][t /
-// page_size] of a pool [pages][hkv][page_size][128].  A 128-key tile is one
-// TMA box per page (page_size < 128: 128 / page_size boxes, pages past the
-// request's cache not loaded; page_size >= 128: part of one page).  The plan
-// covers the longest possible cache in chunks of 16 tiles (2048 keys) so
+// page_size] of a pool [pages][hkv][page_size][128].  A 64-key tile is one
+// TMA box per page (page_size < 64: 64 / page_size boxes, pages past the
+// request's cache not loaded; page_size >= 64: part of one page).  The plan
+// covers the longest possible cache in chunks of 32 tiles (2048 keys) so
 // that short and long requests balance over the SMs; a chunk past a
 // request's cache does nothing, and the merge reads only the chunks its
 // request has.  Rows past the cache in its last tile hold stale pool data:
@@ -33,6 +33,8 @@
 #include <cuda_runtime.h>
 #include <math.h>
 
+#include <cmath>
+
 #include "bha_internal.h"
 #include "bha_ptx.cuh"
 
@@ -40,25 +42,23 @@ namespace bha {
 namespace {
 
 constexpr int kD = 128;
-constexpr int kTK = 128;             // keys per tile
+constexpr int kTK = 64;              // keys per tile
 constexpr int kThreads = 256;
-constexpr uint32_t kTileBytes = kTK * kD * 2;   // 32 KB (K or V tile, Q)
-constexpr int kStages = 3;
+constexpr uint32_t kQBytes = 128 * kD * 2;      // 32 KB: 2 boxes of 64 columns
+constexpr uint32_t kTileBytes = kTK * kD * 2;   // 16 KB K or V tile: 2 boxes of 8 KB
+constexpr uint32_t kBox = kTK * 128;            // one 64-column box of a K / V tile
 constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffK = kTileBytes;                      // 3 stages
-constexpr uint32_t kOffV = kOffK + kStages * kTileBytes;    // 3 stages
-constexpr uint32_t kTiles = kOffV + kStages * kTileBytes;   // 224 KB
-// TMEM columns: S buffers [0, 128) and [128, 256), O [256, 384), P buffers
-// [384, 448) and [448, 512) (128 bf16 keys = 64 columns per row)
-constexpr uint32_t kColO = 256, kColP = 384;
-constexpr int kMaxChunkPages = 128;               // paged: a chunk's page numbers (16 tiles of 16-token pages)
-constexpr uint32_t kPageList = kMaxChunkPages * 4;
+constexpr uint32_t kOffK = kQBytes;                     // 2 stages
+constexpr uint32_t kOffV = kOffK + 2 * kTileBytes;      // 2 stages
+constexpr uint32_t kOffP = kOffV + 2 * kTileBytes;      // 128 rows x 64 keys bf16
+constexpr uint32_t kTiles = kOffP + 128 * kTK * 2;      // 112 KB
 constexpr uint32_t kCtrlBytes = 256;
-constexpr uint32_t kSmem = kTiles + kPageList + 1024;
+constexpr uint32_t kSmem = kTiles + 1024;
+constexpr uint32_t kTmemCols = 256;   // S buffers [0, 64), [64, 128); O [128, 256)
+constexpr uint32_t kColO = 128;
 constexpr float kRescaleLog2 = 8.f;             // rescale O when max grows > 2^8
-constexpr int kTargetCtas = 592;                // four CTAs' worth per SM (148 SMs)
-constexpr int kMinTilesPerChunk = 8;
-constexpr int kPagedTilesPerChunk = 16;
+constexpr int kMinTilesPerChunk = 16;           // 1024 keys
+constexpr int kPagedTilesPerChunk = 32;         // 2048 keys
 
 struct PrefixArgs {
   int* err;
@@ -83,7 +83,7 @@ struct PrefixArgs {
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
 template <bool PAGED>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     k_prefix_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmKc,
                   const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmKa,
                   const __grid_constant__ CUtensorMap tmVa, const __grid_constant__ CUtensorMap tmY,
@@ -98,36 +98,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + kTiles + kPageList;
-  int* page_list = reinterpret_cast<int*>(smem_raw + (base - raw) + kTiles);
+  const uint32_t ctrl = (base - raw >= kCtrlBytes) ? raw : base + kTiles;
   uint8_t* ctrl_ptr = smem_raw + (ctrl - raw);
-  // per stage: K / V landed (kf, vf), K / V consumed (ke, ve); per S buffer:
-  // scores ready (sf); per P buffer: P written (pf), P V done (pvb)
-  const uint32_t bar_q = ctrl, bar_kf = ctrl + 8, bar_ke = ctrl + 32, bar_vf = ctrl + 56,
-                 bar_ve = ctrl + 80, bar_sf = ctrl + 104, bar_pf = ctrl + 120,
-                 bar_pvb = ctrl + 136;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 152);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 156);
+  const uint32_t bar_q = ctrl, bar_kf = ctrl + 8, bar_ke = ctrl + 24, bar_vf = ctrl + 40,
+                 bar_ve = ctrl + 56, bar_sf = ctrl + 72, bar_pf = ctrl + 88, bar_pv = ctrl + 96;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 104);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 108);
 
   if (warp == 0) {
     if (lane == 0) {
       mbar_init(bar_q, 1);
-      for (int s = 0; s < kStages; ++s) {
+      for (int s = 0; s < 2; ++s) {
         mbar_init(bar_kf + 8 * s, 1);
         mbar_init(bar_ke + 8 * s, 1);
         mbar_init(bar_vf + 8 * s, 1);
         mbar_init(bar_ve + 8 * s, 1);
-      }
-      for (int s = 0; s < 2; ++s) {
         mbar_init(bar_sf + 8 * s, 1);
-        mbar_init(bar_pf + 8 * s, 128);
-        mbar_init(bar_pvb + 8 * s, 1);
       }
+      mbar_init(bar_pf, 128);
+      mbar_init(bar_pv, 1);
       *abort_flag = 0;
       fence_mbar_init();
     }
     __syncwarp();
-    tmem_alloc(smem_u32(tmem_slot), 512);
+    tmem_alloc(smem_u32(tmem_slot), kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) pdl_launch_dependents();
@@ -144,22 +138,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int ncache_tiles = PAGED ? (P + kTK - 1) / kTK : a.ncache_tiles;
   const int nt = max(0, min(a.tiles_per, ncache_tiles + 1 - tile0));
   const bool live = nt > 0;   // false only for a chunk past a paged request's cache
-  if (PAGED && warp == 0 && live) {
-    // this chunk's page numbers into shared memory at once, so that the
-    // producer never waits on a table read before a tile's copy
-    const int t_first = tile0 * kTK;
-    const int t_end = min((tile0 + nt) * kTK, P);
-    const int pg0 = t_first >> a.ps_log2;
-    const int npg = t_end > t_first ? ((t_end - 1) >> a.ps_log2) - pg0 + 1 : 0;
-    const int* trow = a.table + static_cast<size_t>(nreq) * a.max_pages + pg0;
-    for (int k = lane; k < npg; k += 32) page_list[k] = __ldg(trow + k);
-    __syncwarp();
-  }
 
   if (tid == 0 && live) {
     // ---------------- TMA producer
     const int row0 = mt * 128;
-    mbar_arrive_expect_tx(bar_q, kTileBytes);
+    mbar_arrive_expect_tx(bar_q, kQBytes);
     tma_load_3d(base + kOffQ, &tmQ, bar_q, 0, row0, u);
     tma_load_3d(base + kOffQ + 16384, &tmQ, bar_q, 64, row0, u);
     // loads one K or V tile of the cache (through the page table) or of the block
@@ -168,41 +151,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (gi >= ncache_tiles) {
         mbar_arrive_expect_tx(bar, kTileBytes);
         tma_load_3d(dst, ma, bar, 0, 0, u);
-        tma_load_3d(dst + 16384, ma, bar, 64, 0, u);
+        tma_load_3d(dst + kBox, ma, bar, 64, 0, u);
       } else if (!PAGED) {
         mbar_arrive_expect_tx(bar, kTileBytes);
         tma_load_3d(dst, mc, bar, 0, gi * kTK, u);
-        tma_load_3d(dst + 16384, mc, bar, 64, gi * kTK, u);
+        tma_load_3d(dst + kBox, mc, bar, 64, gi * kTK, u);
       } else {
-        // page numbers from the chunk's list (entry 0 = the chunk's first page)
         const int t0 = gi * kTK;
-        const int pbase = (tile0 * kTK) >> a.ps_log2;
-        if (a.ps_log2 >= 7) {
+        const int* trow = a.table + static_cast<size_t>(nreq) * a.max_pages;
+        if (a.ps_log2 >= 6) {
           // part of one page
-          const int pg = page_list[(t0 >> a.ps_log2) - pbase];
+          const int pg = __ldg(trow + (t0 >> a.ps_log2));
           const int row = t0 & ((1 << a.ps_log2) - 1);
           mbar_arrive_expect_tx(bar, kTileBytes);
           tma_load_3d(dst, mc, bar, 0, row, pg * a.hkv + g);
-          tma_load_3d(dst + 16384, mc, bar, 64, row, pg * a.hkv + g);
+          tma_load_3d(dst + kBox, mc, bar, 64, row, pg * a.hkv + g);
         } else {
-          // 128 / page_size pages; only those holding cached tokens
+          // 64 / page_size pages; only those holding cached tokens
           const int ps = 1 << a.ps_log2;
           const int npg = min(kTK >> a.ps_log2, (P - t0 + ps - 1) >> a.ps_log2);
           mbar_arrive_expect_tx(bar, static_cast<uint32_t>(npg) * ps * 256);
           for (int j = 0; j < npg; ++j) {
-            const int pg = page_list[(t0 >> a.ps_log2) - pbase + j];
+            const int pg = __ldg(trow + (t0 >> a.ps_log2) + j);
             tma_load_3d(dst + j * ps * 128, mc, bar, 0, 0, pg * a.hkv + g);
-            tma_load_3d(dst + 16384 + j * ps * 128, mc, bar, 64, 0, pg * a.hkv + g);
+            tma_load_3d(dst + kBox + j * ps * 128, mc, bar, 64, 0, pg * a.hkv + g);
           }
         }
       }
     };
     for (int i = 0; i < nt; ++i) {
-      const int st = i % kStages, ph = ((i / kStages) - 1) & 1;
+      const int st = i & 1;
       const int gi = tile0 + i;
-      if (i >= kStages && !mbar_wait(bar_ke + 8 * st, ph, a.err, abort_flag)) break;
+      if (i >= 2 && !mbar_wait(bar_ke + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
       load_tile(&tmKc, &tmKa, base + kOffK + st * kTileBytes, bar_kf + 8 * st, gi);
-      if (i >= kStages && !mbar_wait(bar_ve + 8 * st, ph, a.err, abort_flag)) break;
+      if (i >= 2 && !mbar_wait(bar_ve + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
       load_tile(&tmVc, &tmVa, base + kOffV + st * kTileBytes, bar_vf + 8 * st, gi);
     }
   } else if (tid == 32 && live) {
@@ -210,22 +192,20 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr uint32_t idesc_s = make_idesc_bf16(128, kTK, 0, 0);   // Q K^T, both K-major
     constexpr uint32_t idesc_o = make_idesc_bf16(128, kD, 0, 1);    // P V, V MN-major
     bool ok = mbar_wait(bar_q, 0, a.err, abort_flag);
-    // S(i) into S buffer i % 2 (its last reader, tile i - 2, wrote P before
-    // the previous iteration's P V was issued)
     auto issue_s = [&](int i) -> bool {
-      const int st = i % kStages;
-      if (!mbar_wait(bar_kf + 8 * st, (i / kStages) & 1, a.err, abort_flag)) return false;
+      const int st = i & 1;
+      if (!mbar_wait(bar_kf + 8 * st, (i >> 1) & 1, a.err, abort_flag)) return false;
       tc_fence_after();
       const uint32_t kb = base + kOffK + st * kTileBytes;
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         const uint64_t da =
             make_sdesc(base + kOffQ + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024, kLayoutSW128);
-        const uint64_t db = make_sdesc(kb + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024,
+        const uint64_t db = make_sdesc(kb + (ks >> 2) * kBox + (ks & 3) * 32, 16, 1024,
                                        kLayoutSW128);
-        mma_bf16_ss(tmem + (i & 1) * 128, da, db, idesc_s, ks > 0 ? 1u : 0u);
+        mma_bf16_ss(tmem + st * kTK, da, db, idesc_s, ks > 0 ? 1u : 0u);
       }
-      mma_commit(bar_sf + 8 * (i & 1));
+      mma_commit(bar_sf + 8 * st);
       mma_commit(bar_ke + 8 * st);
       return true;
     };
@@ -233,21 +213,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = 0; i < nt && ok; ++i) {
       if (i + 1 < nt) ok = issue_s(i + 1);
       if (!ok) break;
-      const int st = i % kStages, pb = i & 1;
-      ok = mbar_wait(bar_pf + 8 * pb, (i >> 1) & 1, a.err, abort_flag) &&
-           mbar_wait(bar_vf + 8 * st, (i / kStages) & 1, a.err, abort_flag);
+      const int st = i & 1;
+      ok = mbar_wait(bar_pf, i & 1, a.err, abort_flag) &&
+           mbar_wait(bar_vf + 8 * st, (i >> 1) & 1, a.err, abort_flag);
       if (!ok) break;
       tc_fence_after();
       const uint32_t vb = base + kOffV + st * kTileBytes;
 #pragma unroll
       for (int ks = 0; ks < kTK / 16; ++ks) {
-        // P from TMEM (8 columns per 16 keys); V tile: [keys][d] as 2 boxes
-        // of 64 d-columns, keys the K dim (MN-major)
-        const uint64_t db = make_sdesc(vb + ks * 2048, 16384, 1024, kLayoutSW128);
-        mma_bf16_ts(t_o, tmem + kColP + 64 * pb + 8 * ks, db, idesc_o, (i | ks) ? 1u : 0u);
+        // P: 128 rows of 64 keys (K-major, SW128)
+        const uint64_t da = make_sdesc(base + kOffP + ks * 32, 16, 1024, kLayoutSW128);
+        // V tile: [keys][d] as 2 boxes of 64 d-columns; keys are the K dim
+        const uint64_t db = make_sdesc(vb + ks * 2048, kBox, 1024, kLayoutSW128);
+        mma_bf16_ss(t_o, da, db, idesc_o, (i | ks) ? 1u : 0u);
       }
       mma_commit(bar_ve + 8 * st);
-      mma_commit(bar_pvb + 8 * pb);
+      mma_commit(bar_pv);
     }
   }
 
@@ -258,17 +239,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   bool ok = true;
   if (warp >= 4 && live) {
     for (int i = 0; i < nt; ++i) {
-      const int st = i % kStages, sb = i & 1;
+      const int st = i & 1;
       const int gi = tile0 + i;
       const int valid = gi < ncache_tiles ? min(kTK, P - gi * kTK) : a.b;
-      ok = warp_all(ok && mbar_wait(bar_sf + 8 * sb, (i >> 1) & 1, a.err, abort_flag));
+      ok = warp_all(ok && mbar_wait(bar_sf + 8 * st, (i >> 1) & 1, a.err, abort_flag));
       if (!ok) break;
       tc_fence_after();
       float s[kTK];
 #pragma unroll
       for (int c = 0; c < kTK; c += 32) {
         float t[32];
-        tmem_ld32_sync(tmem + sb * 128 + lane_base + c, t);
+        tmem_ld32_sync(tmem + st * kTK + lane_base + c, t);
 #pragma unroll
         for (int q = 0; q < 32; ++q) s[c + q] = t[q];
       }
@@ -294,14 +275,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         ls += s[j];
       }
       l = l * corr + ls;
-      // O is stable once P V of the previous tile has completed (only a
-      // rescale needs it); P buffer sb once P V of tile i - 2 has
-      if (i > 0 && __any_sync(0xffffffffu, resc)) {
-        ok = warp_all(mbar_wait(bar_pvb + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1, a.err,
-                                abort_flag));
+      // P and O are free once P V of the previous tile has completed
+      if (i > 0) {
+        ok = warp_all(mbar_wait(bar_pv, (i - 1) & 1, a.err, abort_flag));
         if (!ok) break;
         tc_fence_after();
-        {
+        if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll 1
           for (int c = 0; c < kD; c += 32) {
             float o[32];
@@ -315,40 +294,32 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (PAGED && gi < ncache_tiles && valid < kTK) {
         // rows past the cache hold stale pool data (or none was loaded):
         // zero them in V so that P (0 there) times V stays finite
-        ok = warp_all(mbar_wait(bar_vf + 8 * st, (i / kStages) & 1, a.err, abort_flag));
+        ok = warp_all(mbar_wait(bar_vf + 8 * st, (i >> 1) & 1, a.err, abort_flag));
         if (!ok) break;
-        if (r >= valid) {
+        if (r >= valid && r < kTK) {
           const uint32_t vrow = base + kOffV + st * kTileBytes + r * 128;
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
             st_shared_v4(vrow + q * 16, 0u, 0u, 0u, 0u);
-            st_shared_v4(vrow + 16384 + q * 16, 0u, 0u, 0u, 0u);
+            st_shared_v4(vrow + kBox + q * 16, 0u, 0u, 0u, 0u);
           }
         }
       }
-      if (i >= 2) {
-        ok = warp_all(mbar_wait(bar_pvb + 8 * sb, ((i >> 1) - 1) & 1, a.err, abort_flag));
-        if (!ok) break;
-        tc_fence_after();
-      }
-      // P row r as bf16 pairs into TMEM (column c = keys 2c, 2c + 1)
+      {
+        const uint32_t prow = base + kOffP + r * 128;
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        float pk[32];
-#pragma unroll
-        for (int c = 0; c < 32; ++c)
-          pk[c] = __uint_as_float(pack_bf16x2(s[64 * h + 2 * c], s[64 * h + 2 * c + 1]));
-        tmem_st32(tmem + kColP + 64 * sb + lane_base + 32 * h, pk);
+        for (int jj = 0; jj < 8; ++jj) {
+          const float* e = s + jj * 8;
+          st_shared_v4(prow + ((jj ^ (r & 7)) << 4), pack_bf16x2(e[0], e[1]),
+                       pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]), pack_bf16x2(e[6], e[7]));
+        }
       }
-      tmem_wait_st();
-      fence_proxy_async_smem();   // the zeroed V rows, if any
+      fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(bar_pf + 8 * sb);
+      mbar_arrive(bar_pf);
     }
     // final accumulator
-    if (ok && nt > 0)
-      ok = warp_all(mbar_wait(bar_pvb + 8 * ((nt - 1) & 1), ((nt - 1) >> 1) & 1, a.err,
-                              abort_flag));
+    if (ok && nt > 0) ok = warp_all(mbar_wait(bar_pv, (nt - 1) & 1, a.err, abort_flag));
     tc_fence_after();
     if (ok) {
       if (a.splits == 1) {
@@ -401,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncwarp();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kTmemCols);
   }
 }
 
@@ -462,14 +433,31 @@ void prefix_plan_paged(int P, int* splits, int* tiles_per) {
   *tiles_per = tp;
 }
 
+// Chunking of the keys: the chunk count s (chunks of at least 16 tiles)
+// that maximises the expected use of the machine -- the filled fraction of
+// the last wave of CTAs (two per SM on 148 SMs) times the share of traffic
+// that is not chunk partials (64 KB numerator + row statistics, written and
+// read back, per chunk).  Depends only on the shapes, so the workspace query
+// and the launch agree.
 void prefix_plan(int units, int mtiles, int P, int* splits, int* tiles_per) {
+  constexpr double kSlots = 296.0;
   const int ntot = (P + kTK - 1) / kTK + 1;
   const int items = units * mtiles;
-  int s = (kTargetCtas + items - 1) / items;
   const int cap = (ntot + kMinTilesPerChunk - 1) / kMinTilesPerChunk;
-  if (s > cap) s = cap;
-  if (s < 1) s = 1;
-  const int tp = (ntot + s - 1) / s;
+  const double unit_bytes = static_cast<double>(ntot) * kTK * kD * 2 * 2;   // K and V
+  int best = 1;
+  double best_score = -1.0;
+  for (int s = 1; s <= cap && s <= 64; ++s) {
+    const double waves = items * s / kSlots;
+    const double fill = waves / std::ceil(waves);
+    const double partial = s > 1 ? s * 2.0 * (kD * kD + 256) * 4 / unit_bytes : 0.0;
+    const double score = fill * (1.0 - partial);
+    if (score > best_score + 1e-9) {
+      best_score = score;
+      best = s;
+    }
+  }
+  const int tp = (ntot + best - 1) / best;
   *splits = (ntot + tp - 1) / tp;
   *tiles_per = tp;
 }
