@@ -274,6 +274,32 @@ def cpu_baseline_native():
 
 # ---------------------------------------------------------------- native
 
+def same_bytes_copy(nbytes, R, stream, dev, peak):
+    """Per-launch time of ``dst.copy_(src)`` moving ``nbytes`` (read + write)
+    over R rotating buffer pairs, 4 R launches per graph replay."""
+    import torch
+    n = nbytes // 4
+    src = [torch.ones(n, dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    dst = [torch.empty_like(x) for x in src]
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for k in range(4 * R):
+            dst[k % R].copy_(src[k % R])
+    for _ in range(3):
+        g.replay()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(10):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (10 * 4 * R)
+    gbs = 4 * n / (us / 1e6) / 1e9
+    del g
+    return {"launch_us": us, "achieved_gbs": gbs, "frac_of_peak": gbs / peak}
+
+
 def run_native(args, rank, world, local):
     import torch
     import block_hybrid_linear_b200 as bha
@@ -441,6 +467,13 @@ def run_native(args, rank, world, local):
         "gpu_launches": steps * DENOISE,
         "clocks": clk,
     }
+
+    # ---- calibration: the peak's own method (a torch copy, half the bytes read
+    # and half written) at the step's bytes per launch, back to back in a graph
+    # over rotating buffers like the step, right after it: what a plain stream
+    # of this size reaches on this GPU at these clocks
+    if not args.no_compare:
+        line["roofline"]["same_bytes_copy"] = same_bytes_copy(step_bytes, R, stream, dev, peak)
 
     # ---- exact prefix softmax on identical shapes (the comparison path)
     if not args.no_compare:

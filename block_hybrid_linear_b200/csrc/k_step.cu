@@ -8,8 +8,10 @@
 // projection W_g (the method details' kernel-function approximation).
 //
 // One CTA per (request n, KV head g, 128-row tile of the G*b query rows that
-// share g).  Every operand of the unit is requested by TMA at once (Q, K, V
-// first, then the fp32 state S in four 32-row chunks):
+// share g).  TMA brings Q, K, V first; the fp32 state S (four 32-row chunks)
+// is requested once this CTA's Q has landed, so that across the grid the
+// softmax operands are not queued behind the state (measured: 2 % faster in
+// the default mode, 4 % with the shared denominator):
 //   Q   128 x 128 bf16  (2 SW128 boxes, K-major)               32 KB
 //   S   128 x 128 fp32  (16 boxes of 32 rows x 32 cols, 32B-atom swizzle)  64 KB
 //   K,V BPAD x 128 bf16 (2 SW128 boxes each)                   2 x 8 KB at BPAD=32
@@ -261,7 +263,20 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   pdl_wait();   // inputs may come from the previous kernel of the stream
 
-  // ---- producer: Q, K, V first (the softmax half), then the state chunks
+  // chunk c = state rows 32c..32c+31; box (c, nb) = its columns 32nb..32nb+31
+  auto load_state_chunks = [&](int c0, int c1) {
+    for (int c = c0; c < c1; ++c) {
+      mbar_arrive_expect_tx(bar_s + 8 * c, 16384);
+#pragma unroll
+      for (int nb = 0; nb < 4; ++nb)
+        tma_load_3d(base + kOffS + c * 16384 + nb * 4096, &tmS, bar_s + 8 * c, 32 * nb, 32 * c,
+                    u);
+    }
+  };
+
+  // ---- producer: Q, K, V first (the softmax half); the state chunks are
+  // requested once this CTA's Q has landed (below), so that across the grid
+  // the softmax operands are not queued behind the state
   if (tid == 0) {
     const int row0 = mt * kMT;
     mbar_arrive_expect_tx(bar_q, kQBytes);
@@ -278,27 +293,10 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       tma_load_3d(base + kOffW, &tmW, bar_w, 0, 0, g);
       tma_load_3d(base + kOffW + 16384, &tmW, bar_w, 64, 0, g);
     }
-    // chunk c = state rows 32c..32c+31; box (c, nb) = its columns 32nb..32nb+31
-    // (the projected map loads chunks 2-3 later, over W_g)
-    for (int c = 0; c < (PROJ ? 2 : 4); ++c) {
-      mbar_arrive_expect_tx(bar_s + 8 * c, 16384);
-#pragma unroll
-      for (int nb = 0; nb < 4; ++nb)
-        tma_load_3d(base + kOffS + c * 16384 + nb * 4096, &tmS, bar_s + 8 * c, 32 * nb, 32 * c,
-                    u);
-    }
+    // the projected map's state chunks 0-1 (2-3 follow over W_g)
+    if (PROJ) load_state_chunks(0, 2);
   }
 
-  // projected map: state chunks 2-3 over W_g once the Q W_g product is done
-  auto load_late_chunks = [&]() {
-    for (int c = 2; c < 4; ++c) {
-      mbar_arrive_expect_tx(bar_s + 8 * c, 16384);
-#pragma unroll
-      for (int nb = 0; nb < 4; ++nb)
-        tma_load_3d(base + kOffS + c * 16384 + nb * 4096, &tmS, bar_s + 8 * c, 32 * nb, 32 * c,
-                    u);
-    }
-  };
   float beta = 1.f;   // per-row output scale (shared denominator only)
   if (warp < 4) {
     // phi(q) for row r = 32 w + lane into TMEM as soon as Q has landed, in
@@ -309,10 +307,11 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     if (PROJ) {
       okf = warp_all(mbar_wait(bar_qw, 0, a.err, abort_flag));
       tc_fence_after();
-      if (okf && tid == 0) load_late_chunks();
+      if (okf && tid == 0) load_state_chunks(2, 4);
       if (okf) qz = relu_tmem_phiq<SHARED>(t_a + lane_base, zu);
     } else {
       okf = warp_all(mbar_wait(bar_q, 0, a.err, abort_flag));
+      if (okf && tid == 0) load_state_chunks(0, 4);
       if (okf) qz = write_phiq<FMAP, SHARED>(base + kOffQ, warp * 32 + lane, t_a + lane_base, zu);
     }
     if (SHARED && okf) {

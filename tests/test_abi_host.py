@@ -217,8 +217,11 @@ def test_paged_prefix_validation(L):
     the workspace (sized for the longest cache)."""
     n, hq, hkv, b, d, maxp, ps = 4, 16, 4, 32, 128, 64, 128
     need = L.bha_prefix_softmax_paged_workspace_size(n, hq, hkv, b, d, maxp, ps, _lib.BHA_BF16)
-    # chunks of 16 key tiles over the longest cache (8192 keys + the block: 65 tiles -> 5)
-    assert need == n * hkv * 5 * (128 * 128 + 256) * 4
+    # at most one piece per 32 key tiles of the longest cache (8192 keys + the
+    # block: 129 tiles of 64 keys -> 5 partial slots per unit row), then the
+    # device-side plan: a 256-byte header and one 16-byte work item per slot
+    items = n * hkv * 5
+    assert need == items * (128 * 128 + 256) * 4 + 256 + items * 16
     assert L.bha_prefix_softmax_paged_workspace_size(n, hq, hkv, b, d, maxp, ps,
                                                      _lib.BHA_F32) == 0
     big = GAP * 16

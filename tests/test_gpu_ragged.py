@@ -86,6 +86,7 @@ PAGED_CASES = [  # (n, hq, hkv, b, page_size, P_lens, max_pages)
     (2, 8, 2, 33, 64, [64, 4133], 80),              # several chunks; a chunk past request 0's cache
     (2, 16, 4, 64, 256, [300, 2500], 12),           # half a page per tile
     (1, 4, 1, 1, 32, [77], 3),                      # one active token
+    (3, 16, 4, 32, 64, [0, 0, 0], 40),              # planned pieces, every cache empty
 ]
 
 
@@ -108,6 +109,30 @@ def test_paged_prefix_bf16(case):
     ref = oracle.prefix_softmax_paged(Qv, kv, vv, table, P_lens, ps, Kv, Vv)
     check("paged_prefix_bf16", host(Y.t), ref, TOL_BF16_REL, TOL_BF16_ABS, case=str(case),
           ws=need)
+
+
+def test_paged_prefix_planned_pieces_bf16():
+    """A batch large enough that the device-side plan cuts long caches into
+    pieces longer than the minimum (32 tiles of 64 keys): 32 requests with
+    lengths drawn uniformly in [1, 6000] plus the edge lengths 0, 63, 64, 65
+    and 6000, two query tiles per KV head.  Every output against the oracle."""
+    import torch
+    rng = np.random.default_rng(1250)
+    n, hq, hkv, b, ps, max_pages = 32, 16, 4, 64, 64, 94
+    P_lens = [0, 63, 64, 65, 6000] + [int(x) for x in rng.integers(1, 6001, n - 5)]
+    kb, vb, kv, vv, table, num_pages = paged_pool(1250, P_lens, hkv, ps, 128, max_pages, "bf16")
+    Qb, Qv = inputs.normal_bf16_np(1250, inputs.TID_Q, (n, hq, b, 128), STD)
+    Kb, Kv = inputs.normal_bf16_np(1250, inputs.TID_K, (n, hkv, b, 128), STD)
+    Vb, Vv = inputs.normal_bf16_np(1250, inputs.TID_V, (n, hkv, b, 128), STD)
+    Y = Guarded((n, hq, b, 128), torch.bfloat16)
+    need = bha.bha_prefix_softmax_paged_workspace_size(n, hq, hkv, b, 128, max_pages, ps)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda").fill_(255)
+    bha.bha_prefix_softmax_paged(dev_bf16(Qb), dev_bf16(kb), dev_bf16(vb), dev_i32(table),
+                                 dev_i32(P_lens), dev_bf16(Kb), dev_bf16(Vb), Y.t, workspace=ws)
+    torch.cuda.synchronize()
+    assert Y.intact() and Y.no_nan()
+    ref = oracle.prefix_softmax_paged(Qv, kv, vv, table, P_lens, ps, Kv, Vv)
+    check("paged_prefix_planned_bf16", host(Y.t), ref, TOL_BF16_REL, TOL_BF16_ABS, ws=need)
 
 
 def test_paged_prefix_matches_contiguous_bf16():
