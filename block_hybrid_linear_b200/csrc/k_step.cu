@@ -59,6 +59,9 @@ constexpr uint32_t kOffS = kQBytes;
 constexpr uint32_t kOffK = kQBytes + kSBytes;
 constexpr uint32_t kOffW = kOffS + kSBytes / 2;   // projected map: over state chunks 2-3
 constexpr uint32_t kCtrlBytes = 256;
+// Shared denominator: largest log2 scale put into P instead of phi(q) (P <=
+// 2^92, its row sum <= 64 * 2^92: far inside fp32 and bf16 range).
+constexpr float kSharedShiftLog2 = 92.f;
 
 struct StepArgs {
   const float* z;     // [units][128] (shared mode)
@@ -450,15 +453,19 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         const bool oka = warp_all(mbar_wait(bar_a, 0, a.err, abort_flag));
         tc_fence_after();
         const float qz = oka ? tmem_ld1_sync(t_qz + lane_base) : 0.f;
-        // y = (sum_j e_j v_j + e^{-m_s} phi(q) S) / (l + e^{-m_s} phi(q).z),
-        // m_s = scale * m; the factor that stays <= 1 is applied to phi(q)
-        // (m_s >= 0) or to P (m_s < 0), so nothing overflows.
-        if (m >= 0.f) {
-          ascale = exp2f(-m * a.scale_log2);
+        // y = (sum_j e^{s_j - c} v_j + e^{-c} phi(q) S) / (sum_j e^{s_j - c} +
+        // e^{-c} phi(q).z) for any c; e_j = e^{s_j - m_s} above, m_s = scale * m.
+        // c = 0 (P = e_j e^{m_s}, phi(q) as it is) while 2^kSharedShiftLog2
+        // bounds P; past that c = m_s and e^{-m_s} goes into phi(q) in TMEM.
+        // The common case thus leaves phi(Q) untouched: no TMEM pass on the
+        // way to the phi(Q) S products.
+        const float m2 = m * a.scale_log2;
+        if (m2 > kSharedShiftLog2) {
+          ascale = exp2f(-m2);
           pscale = 1.f;
           beta = 1.f / (l + ascale * qz);
         } else {
-          pscale = exp2f(m * a.scale_log2);
+          pscale = exp2f(m2);
           beta = 1.f / (pscale * l + qz);
         }
       } else {

@@ -97,6 +97,26 @@ def test_step_bf16_scale_and_zero_state():
     check_bf16("step_bf16_scale", host(Y), ref)
 
 
+@pytest.mark.parametrize("scale", [1.0, 4.0])
+def test_step_bf16_shared_large_scores(scale):
+    """Shared denominator with unit-variance inputs: row maxima of the scaled
+    scores reach about 30 (scale 1: the factor goes into P) and above 64
+    (scale 4: some rows put e^{-max} into phi(q) instead)."""
+    import torch
+    n, hq, hkv, b = 2, 16, 4, 32
+    Q, Qv = bf16_case((8, 0), (n, hq, b, 128), 1.0)
+    K, Kv = bf16_case((8, 1), (n, hkv, b, 128), 1.0)
+    V, Vv = bf16_case((8, 2), (n, hkv, b, 128), 1.0)
+    Sv, zv = inputs.synthetic_state_np(8, n, hkv, 128, 4096, STD)
+    Y = Guarded((n, hq, b, 128), torch.bfloat16)
+    bha.bha_hybrid_step(Q, K, V, dev_f32(Sv), Y.t, z=dev_f32(zv), scale=scale,
+                        flags=bha.BHA_FLAG_SHARED_DENOM)
+    torch.cuda.synchronize()
+    assert Y.intact() and Y.no_nan()
+    ref = oracle.hybrid_step(Qv, Kv, Vv, Sv, zv, scale=scale, shared=True)
+    check_bf16("step_bf16_shared_large", host(Y.t), ref, scale=scale)
+
+
 @pytest.mark.parametrize("d", [16, 64, 128])
 @pytest.mark.parametrize("shared", [False, True], ids=["default", "shared"])
 def test_step_f32(d, shared):
