@@ -88,13 +88,20 @@ struct StepLayout {
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
 
+// z[k] of the 128-vector spread over a warp (lane l holds z[4l .. 4l+3]);
+// k is a compile-time index, every lane calls it.
+__device__ __forceinline__ float z_at(float4 zl, int k) {
+  const float c = (k & 3) == 0 ? zl.x : (k & 3) == 1 ? zl.y : (k & 3) == 2 ? zl.z : zl.w;
+  return __shfl_sync(0xffffffffu, c, k >> 2);
+}
+
 // phi(q_r) as fp32 into TMEM (this thread's lane, columns [0, 128) from
 // `tcol`), read from row r of the SW128 Q tile; one wait for all four
 // 32-column stores.  Elementwise maps only (phi of a bf16 pair is a bf16
 // pair; the tensor core reads the values as tf32).  QZ: also returns
-// phi(q_r) . z (the shared denominator's term), z from global memory.
+// phi(q_r) . z (the shared denominator's term); lane l holds z[4l .. 4l+3].
 template <int FMAP, bool QZ>
-__device__ __forceinline__ float write_phiq(uint32_t qtile, int r, uint32_t tcol, const float* zu) {
+__device__ __forceinline__ float write_phiq(uint32_t qtile, int r, uint32_t tcol, float4 zl) {
   float qz = 0.f;
 #pragma unroll
   for (int cg = 0; cg < 4; ++cg) {
@@ -111,12 +118,8 @@ __device__ __forceinline__ float write_phiq(uint32_t qtile, int r, uint32_t tcol
         f[8 * q + 2 * e + 1] = __uint_as_float(p2 & 0xFFFF0000u);
       }
       if (QZ) {
-        // columns cg * 32 + 8 q .. + 7
-        const float4 z0 = __ldg(reinterpret_cast<const float4*>(zu + cg * 32 + 8 * q));
-        const float4 z1 = __ldg(reinterpret_cast<const float4*>(zu + cg * 32 + 8 * q + 4));
-        const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e) qz = fmaf(f[8 * q + e], zz[e], qz);
+        for (int e = 0; e < 8; ++e) qz = fmaf(f[8 * q + e], z_at(zl, cg * 32 + 8 * q + e), qz);
       }
     }
     tmem_st32(tcol + cg * 32, f);
@@ -127,9 +130,9 @@ __device__ __forceinline__ float write_phiq(uint32_t qtile, int r, uint32_t tcol
 
 // Projected map: the Q W_g product sits in TMEM (this thread's lane, 128
 // columns from `tcol`); replace it by max(., 0).  QZ: also returns
-// phi(q_r) . z.
+// phi(q_r) . z (z spread over the lanes as for write_phiq).
 template <bool QZ>
-__device__ __forceinline__ float relu_tmem_phiq(uint32_t tcol, const float* zu) {
+__device__ __forceinline__ float relu_tmem_phiq(uint32_t tcol, float4 zl) {
   float qz = 0.f;
 #pragma unroll
   for (int cg = 0; cg < 4; ++cg) {
@@ -139,13 +142,7 @@ __device__ __forceinline__ float relu_tmem_phiq(uint32_t tcol, const float* zu) 
     for (int q = 0; q < 32; ++q) f[q] = fmaxf(f[q], 0.f);
     if (QZ) {
 #pragma unroll
-      for (int q = 0; q < 32; q += 4) {
-        const float4 zz = __ldg(reinterpret_cast<const float4*>(zu + cg * 32 + q));
-        qz = fmaf(f[q], zz.x, qz);
-        qz = fmaf(f[q + 1], zz.y, qz);
-        qz = fmaf(f[q + 2], zz.z, qz);
-        qz = fmaf(f[q + 3], zz.w, qz);
-      }
+      for (int q = 0; q < 32; ++q) qz = fmaf(f[q], z_at(zl, cg * 32 + q), qz);
     }
     tmem_st32(tcol + cg * 32, f);
   }
@@ -259,10 +256,10 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   const uint32_t t_a = tmem + 128;     // [128, 256): phi(Q) as tf32 (the MMA's A)
   // Scores sit in the accumulator's first columns (P V overwrites them once
   // read), so phi(Q) is built in parallel.  With the shared denominator,
-  // warps 0-3 also hand each row's phi(q) . z to the row owners through the
-  // accumulator's last column, which P V overwrites only after it is read.
+  // warps 0-3 hand each row's phi(q) . z to the row owners through that
+  // row's own bytes of the consumed Q tile (row r of Q is read by thread r
+  // alone, and by the MMAs that bar_sc / bar_qw complete).
   const uint32_t t_sc = t_d;
-  const uint32_t t_qz = t_d + kD - 1;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   pdl_wait();   // inputs may come from the previous kernel of the stream
 
@@ -304,23 +301,25 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   if (warp < 4) {
     // phi(q) for row r = 32 w + lane into TMEM as soon as Q has landed, in
     // parallel with the score MMA and the softmax (and phi(q) . z)
-    const float* zu = SHARED ? a.z + static_cast<size_t>(u) * kD : nullptr;
+    // z (shared denominator), four values a lane, requested before Q lands
+    float4 zl = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (SHARED) zl = __ldg(reinterpret_cast<const float4*>(a.z + static_cast<size_t>(u) * kD) + lane);
     float qz = 0.f;
     bool okf;
     if (PROJ) {
       okf = warp_all(mbar_wait(bar_qw, 0, a.err, abort_flag));
       tc_fence_after();
       if (okf && tid == 0) load_state_chunks(2, 4);
-      if (okf) qz = relu_tmem_phiq<SHARED>(t_a + lane_base, zu);
+      if (okf) qz = relu_tmem_phiq<SHARED>(t_a + lane_base, zl);
     } else {
       okf = warp_all(mbar_wait(bar_q, 0, a.err, abort_flag));
-      if (okf && tid == 0) load_state_chunks(0, 4);
-      if (okf) qz = write_phiq<FMAP, SHARED>(base + kOffQ, warp * 32 + lane, t_a + lane_base, zu);
+      // state chunk w from warp w: the issue cost is spread over the warps
+      // that build phi(Q), which the phi(Q) S products wait for
+      if (okf && lane == 0) load_state_chunks(warp, warp + 1);
+      if (okf) qz = write_phiq<FMAP, SHARED>(base + kOffQ, warp * 32 + lane, t_a + lane_base, zl);
     }
-    if (SHARED && okf) {
-      tmem_st1(t_qz + lane_base, qz);
-      tmem_wait_st();
-    }
+    if (SHARED && okf && (PROJ || warp_all(mbar_wait(bar_sc, 0, a.err, abort_flag))))
+      st_shared_f32(base + kOffQ + tid * 128, qz);
     tc_fence_before();
     mbar_arrive(bar_a);
     if (COMMIT && PROJ) {
@@ -426,6 +425,8 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     const bool ok = warp_all(mbar_wait(bar_sc, 0, a.err, abort_flag));
     tc_fence_after();
     float ascale = 1.f;
+    // shared denominator: the row max in log2 units, the row sum, P's factor
+    float m2 = 0.f, lsum = 1.f, pscale = 1.f;
     if (ok) {
       float sc[BPAD];
 #pragma unroll
@@ -447,27 +448,16 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         sc[j] = exp2f((sc[j] - m) * a.scale_log2);
         l += sc[j];
       }
-      float pscale;
       if (SHARED) {
-        // phi(q) . z from warps 0-3 (with phi(Q), unscaled, in TMEM)
-        const bool oka = warp_all(mbar_wait(bar_a, 0, a.err, abort_flag));
-        tc_fence_after();
-        const float qz = oka ? tmem_ld1_sync(t_qz + lane_base) : 0.f;
         // y = (sum_j e^{s_j - c} v_j + e^{-c} phi(q) S) / (sum_j e^{s_j - c} +
         // e^{-c} phi(q).z) for any c; e_j = e^{s_j - m_s} above, m_s = scale * m.
         // c = 0 (P = e_j e^{m_s}, phi(q) as it is) while 2^kSharedShiftLog2
-        // bounds P; past that c = m_s and e^{-m_s} goes into phi(q) in TMEM.
-        // The common case thus leaves phi(Q) untouched: no TMEM pass on the
-        // way to the phi(Q) S products.
-        const float m2 = m * a.scale_log2;
-        if (m2 > kSharedShiftLog2) {
-          ascale = exp2f(-m2);
-          pscale = 1.f;
-          beta = 1.f / (l + ascale * qz);
-        } else {
-          pscale = exp2f(m2);
-          beta = 1.f / (pscale * l + qz);
-        }
+        // bounds P; past that c = m_s and e^{-m_s} goes into phi(q) in TMEM
+        // below.  P depends on the scores alone, so P V never waits for
+        // phi(Q); only the output's 1 / denominator needs phi(q) . z.
+        m2 = m * a.scale_log2;
+        pscale = m2 > kSharedShiftLog2 ? 1.f : exp2f(m2);
+        lsum = l;
       } else {
         pscale = 1.f / l;   // default: P is normalised, the terms add as they are
       }
@@ -490,18 +480,12 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     tc_fence_before();
     mbar_arrive(bar_p);
 
-    if (SHARED) {
-      // the row's factor e^{-m_s} into its phi(q) (rows with m_s < 0 put
-      // theirs into P instead)
-      if (ok && __any_sync(0xffffffffu, ascale != 1.f)) scale_tmem_row(t_a + lane_base, ascale);
-      tc_fence_before();
-      mbar_arrive(bar_a2);
-    }
-
+    // MMA issuer (a row owner too): P V as soon as P and V are in, before
+    // its own row's shared-denominator work below
+    bool ok2 = true;
     if (tid == 128) {
-      // MMA issuer for P V and the per-chunk phi(Q) S products
-      bool ok2 = mbar_wait(bar_p, 0, a.err, abort_flag) && mbar_wait(bar_v, 0, a.err, abort_flag) &&
-                 (!(COMMIT && PROJ) || mbar_wait(bar_kwr, 0, a.err, abort_flag));
+      ok2 = mbar_wait(bar_p, 0, a.err, abort_flag) && mbar_wait(bar_v, 0, a.err, abort_flag) &&
+            (!(COMMIT && PROJ) || mbar_wait(bar_kwr, 0, a.err, abort_flag));
       if (ok2) {
         tc_fence_after();
         constexpr uint32_t idesc = make_idesc_bf16(128, 128, 0, 1);
@@ -512,8 +496,31 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
               make_sdesc(base + Lay::kOffV + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
           mma_bf16_ss(t_d, da, db, idesc, ks > 0 ? 1u : 0u);
         }
-        ok2 = mbar_wait(SHARED ? bar_a2 : bar_a, 0, a.err, abort_flag);
       }
+    }
+
+    if (SHARED) {
+      // phi(q) . z from warps 0-3; the output's 1 / denominator, and for rows
+      // past the shift bound the factor e^{-m_s} into their phi(q)
+      const bool oka = warp_all(ok && mbar_wait(bar_a, 0, a.err, abort_flag));
+      tc_fence_after();
+      if (oka) {
+        const float qz = ld_shared_f32(base + kOffQ + r * 128);
+        if (m2 > kSharedShiftLog2) {
+          ascale = exp2f(-m2);
+          beta = 1.f / (lsum + ascale * qz);
+        } else {
+          beta = 1.f / (pscale * lsum + qz);
+        }
+        if (__any_sync(0xffffffffu, ascale != 1.f)) scale_tmem_row(t_a + lane_base, ascale);
+      }
+      tc_fence_before();
+      mbar_arrive(bar_a2);
+    }
+
+    if (tid == 128) {
+      // then the per-chunk phi(Q) S products
+      if (ok2) ok2 = mbar_wait(SHARED ? bar_a2 : bar_a, 0, a.err, abort_flag);
       for (int c = 0; c < 4 && ok2; ++c) {
         ok2 = mbar_wait(bar_s + 8 * c, 0, a.err, abort_flag);
         if (!ok2) break;
