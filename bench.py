@@ -53,7 +53,8 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--no-compare", action="store_true", help="skip the exact-path comparison")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--only", choices=["step", "step_commit", "commit", "prefill", "prefix"],
+    ap.add_argument("--only", choices=["step", "step_commit", "commit", "prefill", "prefix",
+                                       "paged"],
                     help="launch just this kernel warmup + steps times (small case for ncu)")
     ap.add_argument("--prefix", type=int, default=8192,
                     help="prompt / cache length used by --only prefill|prefix")
@@ -622,6 +623,15 @@ def run_only(args):
         need = bha.bha_prefix_softmax_workspace_size(N_, HQ, HKV, B_, D_, P)
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         fn = lambda: bha.bha_prefix_softmax(Q, Kp, Vp, P, K, V, Y, workspace=ws)
+    elif args.only == "paged":
+        # the ragged workload's paged exact path (batch 64, lengths in [1, 16384])
+        _, max_pages, Kpool, Vpool, tab, plen, Q, K, V = _ragged_paged_batch(N_, dev)
+        Y = torch.empty_like(Q)
+        need = bha.bha_prefix_softmax_paged_workspace_size(N_, HQ, HKV, B_, D_, max_pages,
+                                                           RAGGED_PAGE)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        fn = lambda: bha.bha_prefix_softmax_paged(Q, Kpool, Vpool, tab, plen, K, V, Y,
+                                                  workspace=ws)
     elif args.only == "commit":
         fn = lambda: bha.bha_state_commit(K, V, S, z)
     elif args.only == "step_commit":
@@ -794,22 +804,19 @@ def run_feature_maps(args):
         "rotating_sets": R, "peak_gbs": peak, "maps": out}), flush=True)
 
 
-def run_ragged(args):
-    """Batch 64, 16q/4kv, d=128, B=32 with per-request prefix lengths drawn
-    uniformly from [1, 16384] (mean about 8192, seeded): the exact path over a
-    paged KV cache (pages of 128 tokens) against the same path padded to the
-    longest cache, the hybrid step, the ragged prefill of the same prompts, and
-    the 20-layer stack (6 hybrid + 14 exact layers) memory per request and
-    largest batch before out-of-memory with paged and with padded caches."""
+RAGGED_PAGE, RAGGED_LMAX = 128, 16384
+
+
+def _ragged_paged_batch(n, dev):
+    """The ragged workload's batch: prefix lengths drawn uniformly from
+    [1, 16384] (seeded), each request's cache in its own pages of 128 tokens
+    of one pool in a seeded random order, and the active block's Q, K, V."""
     import numpy as np
     import torch
-    import block_hybrid_linear_b200 as bha
-    from block_hybrid_linear_b200 import build, inputs
-    build.build()
-    dev = torch.device("cuda", 0)
-    n, ps, Lmax, layers, hyb = N_, 128, 16384, 20, 6
+    from block_hybrid_linear_b200 import inputs
+    ps = RAGGED_PAGE
     std = 1.0 / math.sqrt(D_)
-    lengths = np.random.default_rng(6000).integers(1, Lmax + 1, size=8192)
+    lengths = np.random.default_rng(6000).integers(1, RAGGED_LMAX + 1, size=8192)
     P_lens = lengths[:n]
     pages = (P_lens + ps - 1) // ps
     num_pages, max_pages = int(pages.sum()), int(pages.max())
@@ -826,6 +833,27 @@ def run_ragged(args):
     Q = inputs.normal_bf16_torch(6000, inputs.TID_Q, (n, HQ, B_, D_), std, dev)
     K = inputs.normal_bf16_torch(6000, inputs.TID_K, (n, HKV, B_, D_), std, dev)
     V = inputs.normal_bf16_torch(6000, inputs.TID_V, (n, HKV, B_, D_), std, dev)
+    return P_lens, max_pages, Kpool, Vpool, tab, plen, Q, K, V
+
+
+def run_ragged(args):
+    """Batch 64, 16q/4kv, d=128, B=32 with per-request prefix lengths drawn
+    uniformly from [1, 16384] (mean about 8192, seeded): the exact path over a
+    paged KV cache (pages of 128 tokens) against the same path padded to the
+    longest cache, the hybrid step, the ragged prefill of the same prompts, and
+    the 20-layer stack (6 hybrid + 14 exact layers) memory per request and
+    largest batch before out-of-memory with paged and with padded caches."""
+    import numpy as np
+    import torch
+    import block_hybrid_linear_b200 as bha
+    from block_hybrid_linear_b200 import build, inputs
+    build.build()
+    dev = torch.device("cuda", 0)
+    n, ps, Lmax, layers, hyb = N_, RAGGED_PAGE, RAGGED_LMAX, 20, 6
+    std = 1.0 / math.sqrt(D_)
+    P_lens, max_pages, Kpool, Vpool, tab, plen, Q, K, V = _ragged_paged_batch(n, dev)
+    # the stack's memory per request over the first 8192 draws of the same lengths
+    lengths = np.random.default_rng(6000).integers(1, Lmax + 1, size=8192)
     Y = torch.empty_like(Q)
     S = torch.randn(n, HKV, D_, D_, device=dev)
     stream = torch.cuda.Stream(device=dev)
