@@ -735,6 +735,7 @@ def run_single_step(args):
                         "frac_of_peak": bytes_step / (step_us / 1e6) / 1e9 / peak,
                         "algorithmic_bytes": bytes_step},
         "prefix_softmax": {"launch_us": exact_us, "tokens_per_s": n * B_ / (exact_us / 1e6)},
+        "same_bytes_copy": same_bytes_copy(bytes_step, R, stream, dev, peak),
         "note": "4.7 MB per step: bound by launch latency, not by HBM"}), flush=True)
 
 

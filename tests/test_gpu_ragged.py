@@ -87,6 +87,8 @@ PAGED_CASES = [  # (n, hq, hkv, b, page_size, P_lens, max_pages)
     (2, 16, 4, 64, 256, [300, 2500], 12),           # half a page per tile
     (1, 4, 1, 1, 32, [77], 3),                      # one active token
     (3, 16, 4, 32, 64, [0, 0, 0], 40),              # planned pieces, every cache empty
+    (12, 16, 4, 32, 64, [9000] + [1, 2, 3, 5, 8, 13, 21, 34, 55, 89, 0], 150),  # one long
+                                                    # request among tiny ones: 5 pieces + 11 single
 ]
 
 
