@@ -23,12 +23,13 @@
 // P_lens[i] tokens, token t at row t % page_size of page block_table[i][t /
 // page_size] of a pool [pages][hkv][page_size][128].  A 64-key tile is one
 // TMA box per page (page_size < 64: 64 / page_size boxes, pages past the
-// request's cache not loaded; page_size >= 64: part of one page).  The plan
-// covers the longest possible cache in chunks of 32 tiles (2048 keys) so
-// that short and long requests balance over the SMs; a chunk past a
-// request's cache does nothing, and the merge reads only the chunks its
-// request has.  Rows past the cache in its last tile hold stale pool data:
-// their scores are masked and their V rows zeroed before P V.
+// request's cache not loaded; page_size >= 64: part of one page).  A
+// one-CTA planning kernel reads the lengths on the device and cuts each
+// request into pieces of equal length plus a remainder, longest first (see
+// k_prefix_paged_plan); each CTA takes one piece, a request of one piece
+// writes Y itself, and the merge combines the pieces of the others.  Rows
+// past the cache in its last tile hold stale pool data: their scores are
+// masked and their V rows zeroed before P V.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <math.h>

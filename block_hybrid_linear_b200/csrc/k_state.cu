@@ -22,7 +22,7 @@
 // one chunk) and a second kernel adds the chunks in a fixed order.
 //
 // Feature maps (the method details' kernel-function approximation): elu + 1
-// is applied in place like ReLU (computed in fp32, rounded to bf16).  The
+// is applied in place like ReLU (packed bf16 arithmetic, elu1_bf16x2).  The
 // projected map phi(k) = ReLU(k W_g) takes one more MMA per K tile, the
 // transposed projection (K W_g)^T = W_g^T K^T (M = 128 features, N =
 // tokens, K = 128 inputs; A = W_g MN-major as it sits in memory, B = the K
