@@ -82,12 +82,37 @@ def measured_peaks():
     return 6650.0, "fallback"
 
 
+def code_only(text):
+    """C/C++ source without its comments, whitespace runs collapsed: what the
+    compiler sees, so that editing a comment does not retire a capture."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def source_sha256(src_file):
-    """sha256 over a kernel's source file and the device helpers it includes."""
+    """sha256 over the code (comments aside) of a kernel's source file and of
+    the device helpers it includes."""
     h = hashlib.sha256()
     for name in (src_file, "bha_ptx.cuh"):
-        with open(os.path.join(ROOT, "block_hybrid_linear_b200", "csrc", name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "block_hybrid_linear_b200", "csrc", name)) as f:
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()
 
 

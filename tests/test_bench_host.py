@@ -68,3 +68,14 @@ def test_reference_arm_prints_one_line():
     assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["metric"] == bench.METRIC
+
+
+def test_source_hash_ignores_comments_only():
+    """The ncu traffic record stays valid across comment edits and is retired
+    by any change to the code itself."""
+    import bench
+    src = 'int f(int a) { // add one\n  return a + 1; /* done */ }\nconst char* s = "// kept";\n'
+    assert bench.code_only(src) == bench.code_only(src.replace("add one", "increment"))
+    assert bench.code_only(src) != bench.code_only(src.replace("a + 1", "a + 2"))
+    assert "// kept" in bench.code_only(src)
+    assert "add one" not in bench.code_only(src) and "done" not in bench.code_only(src)
