@@ -175,7 +175,12 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t tcol, float s) {
 // tile to a TMA reduce-add into S.  P then lives in the consumed Q tile so that K survives for the commit MMA,
 // and phi(K)^T V accumulates in the TMEM columns phi(Q) used.  Default mode
 // and a single 128-row tile per unit only.
-template <int BPAD, bool SHARED, bool COMMIT, int FMAP>
+// HALF (small grids): a pair of adjacent CTAs shares a unit, each computing
+// 64 of the 128 output columns: it loads the whole Q and K (the pair's second
+// reads hit L2) but only its half of V and of every state chunk, and runs
+// P V and phi(Q) S at N = 64.  The scores and the softmax are computed by
+// both.  This doubles the CTAs of a grid that would leave most SMs idle.
+template <int BPAD, bool SHARED, bool COMMIT, int FMAP, bool HALF>
 __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     k_step_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
@@ -183,6 +188,9 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
                 const StepArgs a) {
   static_assert(!(SHARED && COMMIT), "the fused commit runs in the default mode only");
   constexpr bool PROJ = FMAP == kFmapReluProj;
+  static_assert(!(HALF && (COMMIT || PROJ)), "column halves: plain step, elementwise maps");
+  constexpr int kN = HALF ? 64 : 128;                   // output columns of this CTA
+  constexpr uint32_t kChunkS = HALF ? 8192 : 16384;     // bytes of one state chunk here
   using Lay = StepLayout<BPAD>;
   // P (the softmax weights, bf16, K-major) goes over the consumed K tile, or
   // over the consumed Q tile when K is still needed by the commit
@@ -190,7 +198,9 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int u = blockIdx.x / a.mtiles, mt = blockIdx.x % a.mtiles;
+  const int half = HALF ? static_cast<int>(blockIdx.x & 1u) : 0;   // column half
+  const int item = HALF ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int u = item / a.mtiles, mt = item % a.mtiles;
   const int g = u % a.hkv;
 
   const uint32_t raw = smem_u32(smem_raw);
@@ -234,10 +244,11 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       tma_prefetch_l2_3d(&tmQ, 64, row0, u);
       tma_prefetch_l2_3d(&tmK, 0, 0, u);
       tma_prefetch_l2_3d(&tmK, 64, 0, u);
-      tma_prefetch_l2_3d(&tmV, 0, 0, u);
-      tma_prefetch_l2_3d(&tmV, 64, 0, u);
+      for (int vb = 0; vb < 2; ++vb)
+        if (!HALF || vb == half) tma_prefetch_l2_3d(&tmV, 64 * vb, 0, u);
       for (int c = 0; c < 4; ++c)
-        for (int nb = 0; nb < 4; ++nb) tma_prefetch_l2_3d(&tmS, 32 * nb, 32 * c, u);
+        for (int nb = 0; nb < 4; ++nb)
+          if (!HALF || (nb >> 1) == half) tma_prefetch_l2_3d(&tmS, 32 * nb, 32 * c, u);
       if (PROJ) {
         tma_prefetch_l2_3d(&tmW, 0, 0, g);
         tma_prefetch_l2_3d(&tmW, 64, 0, g);
@@ -264,13 +275,16 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   pdl_wait();   // inputs may come from the previous kernel of the stream
 
   // chunk c = state rows 32c..32c+31; box (c, nb) = its columns 32nb..32nb+31
+  // (HALF: only the half's two boxes of every chunk, packed)
   auto load_state_chunks = [&](int c0, int c1) {
     for (int c = c0; c < c1; ++c) {
-      mbar_arrive_expect_tx(bar_s + 8 * c, 16384);
+      mbar_arrive_expect_tx(bar_s + 8 * c, kChunkS);
 #pragma unroll
-      for (int nb = 0; nb < 4; ++nb)
-        tma_load_3d(base + kOffS + c * 16384 + nb * 4096, &tmS, bar_s + 8 * c, 32 * nb, 32 * c,
+      for (int nn = 0; nn < kN / 32; ++nn) {
+        const int nb = HALF ? 2 * half + nn : nn;
+        tma_load_3d(base + kOffS + c * kChunkS + nn * 4096, &tmS, bar_s + 8 * c, 32 * nb, 32 * c,
                     u);
+      }
     }
   };
 
@@ -285,9 +299,14 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     mbar_arrive_expect_tx(bar_k, Lay::kKV);
     tma_load_3d(base + kOffK, &tmK, bar_k, 0, 0, u);
     tma_load_3d(base + kOffK + BPAD * 128, &tmK, bar_k, 64, 0, u);
-    mbar_arrive_expect_tx(bar_v, Lay::kKV);
-    tma_load_3d(base + Lay::kOffV, &tmV, bar_v, 0, 0, u);
-    tma_load_3d(base + Lay::kOffV + BPAD * 128, &tmV, bar_v, 64, 0, u);
+    if (HALF) {
+      mbar_arrive_expect_tx(bar_v, Lay::kKV / 2);
+      tma_load_3d(base + Lay::kOffV, &tmV, bar_v, 64 * half, 0, u);
+    } else {
+      mbar_arrive_expect_tx(bar_v, Lay::kKV);
+      tma_load_3d(base + Lay::kOffV, &tmV, bar_v, 0, 0, u);
+      tma_load_3d(base + Lay::kOffV + BPAD * 128, &tmV, bar_v, 64, 0, u);
+    }
     if (PROJ) {
       mbar_arrive_expect_tx(bar_w, 2 * 16384);
       tma_load_3d(base + kOffW, &tmW, bar_w, 0, 0, g);
@@ -488,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
             (!(COMMIT && PROJ) || mbar_wait(bar_kwr, 0, a.err, abort_flag));
       if (ok2) {
         tc_fence_after();
-        constexpr uint32_t idesc = make_idesc_bf16(128, 128, 0, 1);
+        constexpr uint32_t idesc = make_idesc_bf16(128, kN, 0, 1);
 #pragma unroll
         for (int ks = 0; ks < BPAD / 16; ++ks) {
           const uint64_t da = make_sdesc(base + kOffP + ks * 32, 16, 8 * Lay::kRowB, Lay::kPLayout);
@@ -525,12 +544,12 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         ok2 = mbar_wait(bar_s + 8 * c, 0, a.err, abort_flag);
         if (!ok2) break;
         tc_fence_after();
-        constexpr uint32_t idesc = make_idesc_tf32(128, 128, 0, 1);
+        constexpr uint32_t idesc = make_idesc_tf32(128, kN, 0, 1);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
           // state rows 32c + 8kk .. +7 of every 32-column box: two 4-row
           // atoms of the 32-byte-chunk swizzle (MN-major tf32 layout)
-          const uint64_t db = make_sdesc(base + kOffS + c * 16384 + kk * 1024, 4096, 512,
+          const uint64_t db = make_sdesc(base + kOffS + c * kChunkS + kk * 1024, 4096, 512,
                                          kLayoutSW128_32B);
           mma_tf32_ts(t_d, t_a + 32 * c + 8 * kk, db, idesc, 1u);
         }
@@ -574,6 +593,31 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     named_barrier_sync(1, kThreads);
     beta = rs[r];
   }
+  if (HALF) {
+    // warp w: rows 32(w%4).., columns 32(w/4).. of the CTA's 64; one SW128
+    // box in the (consumed) Q region, one TMA store
+    if (okd) {
+      const uint32_t row = base + kOffQ + r * 128;
+      float acc[32];
+      tmem_ld32_sync(t_d + lane_base + hb * 32, acc);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int j = hb * 4 + q;
+        const float* e = acc + 8 * q;
+        st_shared_v4(row + ((j ^ (r & 7)) << 4), pack_bf16x2(e[0] * beta, e[1] * beta),
+                     pack_bf16x2(e[2] * beta, e[3] * beta),
+                     pack_bf16x2(e[4] * beta, e[5] * beta),
+                     pack_bf16x2(e[6] * beta, e[7] * beta));
+      }
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    named_barrier_sync(2, kThreads);
+    if (tid == 0 && !*abort_flag) {
+      tma_store_3d(&tmY, base + kOffQ, 64 * half, mt * kMT, u);
+      bulk_commit_group();
+    }
+  } else {
   if (okd) {
     // bf16 tile of this 64-column half -> the (consumed) Q region, SW128
     const uint32_t row = base + kOffQ + hb * 16384 + r * 128;
@@ -598,6 +642,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   if ((tid & 127) == 0 && !*abort_flag) {
     tma_store_3d(&tmY, base + kOffQ + hb * 16384, 64 * hb, mt * kMT, u);
     bulk_commit_group();
+  }
   }
   if (COMMIT) {
     // phi(K)^T V over the consumed state tile (32-byte-chunk swizzle: chunk
@@ -642,20 +687,25 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   if ((tid & 127) == 0) bulk_wait_group_read0();   // shared memory stays until read
 }
 
-template <int BPAD, bool SHARED, bool COMMIT, int FMAP>
+template <int BPAD, bool SHARED, bool COMMIT, int FMAP, bool HALF = false>
 int launch_cfg(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int grid) {
   using Lay = StepLayout<BPAD>;
-  auto kern = k_step_bf16<BPAD, SHARED, COMMIT, FMAP>;
+  auto kern = k_step_bf16<BPAD, SHARED, COMMIT, FMAP, HALF>;
   static std::atomic<uint64_t> prepared{0};
   if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
-  return launch_pdl(kern, grid, kThreads, Lay::kSmem, c.stream, tm[0], tm[1], tm[2], tm[3], tm[4],
-                    tm[5], a);
+  return launch_pdl(kern, (HALF ? 2 : 1) * grid, kThreads, Lay::kSmem, c.stream, tm[0], tm[1],
+                    tm[2], tm[3], tm[4], tm[5], a);
 }
 
+// Column halves when the grid would fill at most one CTA per SM (and the
+// variant allows them: no fused commit, an elementwise map).
 template <int BPAD, int FMAP>
 int launch_fmap(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int grid, int shared,
                 int commit) {
   if (commit) return launch_cfg<BPAD, false, true, FMAP>(c, tm, a, grid);
+  if (FMAP != kFmapReluProj && grid <= c.sm_count)
+    return shared ? launch_cfg<BPAD, true, false, FMAP, FMAP != kFmapReluProj>(c, tm, a, grid)
+                  : launch_cfg<BPAD, false, false, FMAP, FMAP != kFmapReluProj>(c, tm, a, grid);
   return shared ? launch_cfg<BPAD, true, false, FMAP>(c, tm, a, grid)
                 : launch_cfg<BPAD, false, false, FMAP>(c, tm, a, grid);
 }

@@ -88,6 +88,7 @@ STEP_CASES = [  # (n, hq, hkv, b)
     (1, 4, 1, 1),      # one active token
     (2, 8, 1, 33),     # BPAD 64, three M tiles with a ragged tail
     (1, 16, 4, 64),    # two M tiles
+    (38, 16, 4, 32),   # 152 unit rows: whole units (the cases above run as column halves)
 ]
 
 

@@ -59,6 +59,12 @@ STEP_CASES = [  # (n, hq, hkv, b)
     (2, 8, 1, 33),     # BPAD 64, G*b = 264 rows: three M tiles, ragged tail
     (1, 16, 4, 64),    # b = 64, G*b = 256 rows: two M tiles
     (2, 2, 1, 16),
+    # The cases above are grids of at most one CTA per SM, which run as column
+    # halves (two CTAs per unit); these exceed the SM count and run whole units.
+    (37, 16, 4, 32),   # 148 unit rows: the largest grid still split (296 CTAs)
+    (38, 16, 4, 32),   # 152 unit rows: whole units, BPAD 32
+    (40, 8, 4, 10),    # whole units, BPAD 16
+    (75, 4, 1, 33),    # 75 units x two M tiles = 150 unit rows: whole units, BPAD 64
 ]
 
 
