@@ -98,19 +98,17 @@ def synthetic_state_np(seed, n, hkv, d, T, sigma):
     return S, np.abs(z).astype(np.float32)
 
 
-# Workloads: the worked example and the four attention-layer configurations
-# of a 16B dLLM (16 query / 4 KV heads, head dim 128, active block 32).
-CONFIGS = {
-    1: dict(name="worked-example", n=1, hq=1, hkv=1, d=16, L=10, B=4,
-            dtype="f32", std=1.0, seed=1000),
-    2: dict(name="single-step", n=8, hq=16, hkv=4, d=128, b=32, P=4096,
-            dtype="bf16", std=1.0 / math.sqrt(128), seed=2000),
-    3: dict(name="generation-loop", n=32, hq=16, hkv=4, d=128, b=32,
-            prompt=1024, blocks=32, steps=8, dtype="bf16",
-            std=1.0 / math.sqrt(128), seed=3000),
-    4: dict(name="long-prefix", n=64, hq=16, hkv=4, d=128, b=32, P=32768,
-            dtype="bf16", std=1.0 / math.sqrt(128), seed=4000),
-    5: dict(name="stack-sweep", layers=20, hybrid_layers=6, hq=16, hkv=4,
-            d=128, b=32, P=8192, dtype="bf16", std=1.0 / math.sqrt(128),
-            seed=5000),
+# Workloads by name: the worked example and the four attention-layer
+# workloads of a 16B dLLM (16 query / 4 KV heads, head dim 128, active block 32).
+WORKLOADS = {
+    "worked-example": dict(n=1, hq=1, hkv=1, d=16, L=10, B=4, dtype="f32", std=1.0,
+                           seed=1000),
+    "single-step": dict(n=8, hq=16, hkv=4, d=128, b=32, P=4096, dtype="bf16",
+                        std=1.0 / math.sqrt(128), seed=2000),
+    "generation-loop": dict(n=32, hq=16, hkv=4, d=128, b=32, prompt=1024, blocks=32, steps=8,
+                            dtype="bf16", std=1.0 / math.sqrt(128), seed=3000),
+    "long-prefix": dict(n=64, hq=16, hkv=4, d=128, b=32, P=32768, dtype="bf16",
+                        std=1.0 / math.sqrt(128), seed=4000),
+    "stack-sweep": dict(layers=20, hybrid_layers=6, hq=16, hkv=4, d=128, b=32, P=8192,
+                        dtype="bf16", std=1.0 / math.sqrt(128), seed=5000),
 }

@@ -58,7 +58,7 @@ def test_worked_example_decoding_loop_fp32():
     """Worked example: L=10 in blocks 4,4,2 (partition from the library), fp32
     N(0,1), phi=ReLU; block 1 softmax only, block 2 uses S_1, block 3 S_1+S_2."""
     import torch
-    cfg = inputs.CONFIGS[1]
+    cfg = inputs.WORKLOADS["worked-example"]
     L, B, d = cfg["L"], cfg["B"], cfg["d"]
     bounds = bha.bha_block_partition(L, B)
     assert bounds == oracle.block_partition(L, B) == [0, 4, 8, 10]
@@ -86,7 +86,7 @@ def test_worked_example_decoding_loop_fp32():
 def test_single_step_config_all_units():
     """Batch 8, 16q/4kv, B=32, prefix 4096 folded into S by the prefill."""
     import torch
-    cfg = inputs.CONFIGS[2]
+    cfg = inputs.WORKLOADS["single-step"]
     n, hq, hkv, b, P, seed = cfg["n"], cfg["hq"], cfg["hkv"], cfg["b"], cfg["P"], cfg["seed"]
     Kp, Kpv = bf16_case((seed, inputs.TID_KP), (n, hkv, P, 128), STD)
     Vp, Vpv = bf16_case((seed, inputs.TID_VP), (n, hkv, P, 128), STD)
@@ -116,7 +116,7 @@ def test_generation_loop_first_blocks():
     """Batch 32, prompt 1024 -> S, then 3 blocks x 2 denoising steps with a
     commit per block, chained on the GPU and in the oracle independently."""
     import torch
-    cfg = inputs.CONFIGS[3]
+    cfg = inputs.WORKLOADS["generation-loop"]
     n, hq, hkv, b, T, seed = cfg["n"], cfg["hq"], cfg["hkv"], cfg["b"], cfg["prompt"], cfg["seed"]
     nblk, nstep = 3, 2
     Kp, Kpv = bf16_case((seed, inputs.TID_KP), (n, hkv, T, 128), STD)
@@ -153,7 +153,7 @@ def test_long_prefix_step_and_commit_all_units():
     """Batch 64, 16q/4kv, B=32, a 32k-token prefix state (drawn with a 32k
     prefill's statistics): the step and the commit on all 256 units."""
     import torch
-    cfg = inputs.CONFIGS[4]
+    cfg = inputs.WORKLOADS["long-prefix"]
     n, hq, hkv, b, P, seed = cfg["n"], cfg["hq"], cfg["hkv"], cfg["b"], cfg["P"], cfg["seed"]
     Q, Qv = bf16_case((seed, inputs.TID_Q), (n, hq, b, 128), STD)
     K, Kv = bf16_case((seed, inputs.TID_K), (n, hkv, b, 128), STD)
@@ -176,7 +176,7 @@ def test_long_prefix_prefill_and_exact_path_sampled():
     prefill (8 chunks per unit) and the exact prefix softmax over the same
     32k cache, checked on units {first, middle, last} against the oracle."""
     import torch
-    cfg = inputs.CONFIGS[4]
+    cfg = inputs.WORKLOADS["long-prefix"]
     n, hq, hkv, b, P, seed = cfg["n"], cfg["hq"], cfg["hkv"], cfg["b"], cfg["P"], cfg["seed"]
     Kp = inputs.normal_bf16_torch(seed, inputs.TID_KP, (n, hkv, P, 128), STD, "cuda")
     Vp = inputs.normal_bf16_torch(seed, inputs.TID_VP, (n, hkv, P, 128), STD, "cuda")

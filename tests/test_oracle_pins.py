@@ -301,7 +301,7 @@ def test_worked_example_structure():
     """L=10, B=4, d=16, phi=ReLU, fp32 N(0,1) inputs from seed: block 1 is
     softmax only; block 2 adds phi(Q_2) S_1; block 3 uses S_1 + S_2."""
     g = json.load(open(os.path.join(GOLDEN, "worked_example.json")))
-    cfg = inputs.CONFIGS[1]
+    cfg = inputs.WORKLOADS["worked-example"]
     d, L = cfg["d"], g["L"]
     bounds = oracle.block_partition(L, g["B"])
     seq_q = inputs.normal_f32_np(cfg["seed"], inputs.TID_Q, (1, 1, L, d)).astype(np.float64)
