@@ -58,6 +58,8 @@ def parse():
                     help="launch just this kernel warmup + steps times (small case for ncu)")
     ap.add_argument("--prefix", type=int, default=8192,
                     help="prompt / cache length used by --only prefill|prefix")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="batch used by --only step|step_commit|commit (default 64)")
     ap.add_argument("--workload", default="long-prefix",
                     choices=["long-prefix", "single-step", "generation-loop", "stack",
                              "feature-maps", "ragged"],
@@ -640,28 +642,29 @@ def run_only(args):
     dev = torch.device("cuda", 0)
     std = 1.0 / math.sqrt(D_)
     P = args.prefix
-    Q = inputs.normal_bf16_torch(1, inputs.TID_Q, (N_, HQ, B_, D_), std, dev)
-    K = inputs.normal_bf16_torch(1, inputs.TID_K, (N_, HKV, B_, D_), std, dev)
-    V = inputs.normal_bf16_torch(1, inputs.TID_V, (N_, HKV, B_, D_), std, dev)
+    nb = args.batch if args.batch and args.only in ("step", "step_commit", "commit") else N_
+    Q = inputs.normal_bf16_torch(1, inputs.TID_Q, (nb, HQ, B_, D_), std, dev)
+    K = inputs.normal_bf16_torch(1, inputs.TID_K, (nb, HKV, B_, D_), std, dev)
+    V = inputs.normal_bf16_torch(1, inputs.TID_V, (nb, HKV, B_, D_), std, dev)
     Y = torch.empty_like(Q)
-    S = torch.randn(N_, HKV, D_, D_, device=dev)
-    z = torch.rand(N_, HKV, D_, device=dev)
+    S = torch.randn(nb, HKV, D_, D_, device=dev)
+    z = torch.rand(nb, HKV, D_, device=dev)
     if args.only in ("prefill", "prefix"):
-        Kp = inputs.normal_bf16_torch(1, inputs.TID_KP, (N_, HKV, P, D_), std, dev)
-        Vp = inputs.normal_bf16_torch(1, inputs.TID_VP, (N_, HKV, P, D_), std, dev)
+        Kp = inputs.normal_bf16_torch(1, inputs.TID_KP, (nb, HKV, P, D_), std, dev)
+        Vp = inputs.normal_bf16_torch(1, inputs.TID_VP, (nb, HKV, P, D_), std, dev)
     if args.only == "prefill":
-        need = bha.bha_state_prefill_workspace_size(N_, HKV, P, D_)
+        need = bha.bha_state_prefill_workspace_size(nb, HKV, P, D_)
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         fn = lambda: bha.bha_state_prefill(Kp, Vp, S, z, workspace=ws)
     elif args.only == "prefix":
-        need = bha.bha_prefix_softmax_workspace_size(N_, HQ, HKV, B_, D_, P)
+        need = bha.bha_prefix_softmax_workspace_size(nb, HQ, HKV, B_, D_, P)
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         fn = lambda: bha.bha_prefix_softmax(Q, Kp, Vp, P, K, V, Y, workspace=ws)
     elif args.only == "paged":
         # the ragged workload's paged exact path (batch 64, lengths in [1, 16384])
-        _, max_pages, Kpool, Vpool, tab, plen, Q, K, V = _ragged_paged_batch(N_, dev)
+        _, max_pages, Kpool, Vpool, tab, plen, Q, K, V = _ragged_paged_batch(nb, dev)
         Y = torch.empty_like(Q)
-        need = bha.bha_prefix_softmax_paged_workspace_size(N_, HQ, HKV, B_, D_, max_pages,
+        need = bha.bha_prefix_softmax_paged_workspace_size(nb, HQ, HKV, B_, D_, max_pages,
                                                            RAGGED_PAGE)
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         fn = lambda: bha.bha_prefix_softmax_paged(Q, Kpool, Vpool, tab, plen, K, V, Y,
