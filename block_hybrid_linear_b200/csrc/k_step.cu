@@ -180,6 +180,8 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t tcol, float s) {
 // reads hit L2) but only its half of V and of every state chunk, and runs
 // P V and phi(Q) S at N = 64.  The scores and the softmax are computed by
 // both.  This doubles the CTAs of a grid that would leave most SMs idle.
+// With the fused commit each CTA adds its half of phi(K)^T V to S, and the
+// first of the pair adds the block's sum of phi(k) to z.
 template <int BPAD, bool SHARED, bool COMMIT, int FMAP, bool HALF>
 __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     k_step_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -188,7 +190,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
                 const StepArgs a) {
   static_assert(!(SHARED && COMMIT), "the fused commit runs in the default mode only");
   constexpr bool PROJ = FMAP == kFmapReluProj;
-  static_assert(!(HALF && (COMMIT || PROJ)), "column halves: plain step, elementwise maps");
+  static_assert(!(HALF && PROJ), "column halves: elementwise maps only");
   constexpr int kN = HALF ? 64 : 128;                   // output columns of this CTA
   constexpr uint32_t kChunkS = HALF ? 8192 : 16384;     // bytes of one state chunk here
   using Lay = StepLayout<BPAD>;
@@ -385,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       fence_proxy_async_smem();
       named_barrier_sync(4, 128);   // the whole phi(K) tile is written
       mbar_arrive(bar_phik);
-      if (okk && a.zc != nullptr) {
+      if (okk && a.zc != nullptr && half == 0) {
         const int rr = tid;
         const uint32_t col = base + kOffK + (rr >> 6) * (BPAD * 128) + (rr & 7) * 2;
         float zs = 0.f;
@@ -563,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
           tc_fence_after();
           // A = phi(K)^T: MN-major phi(K) in place, or K-major rows of the
           // projected map's features
-          constexpr uint32_t idesc = make_idesc_bf16(128, 128, PROJ ? 0 : 1, 1);
+          constexpr uint32_t idesc = make_idesc_bf16(128, kN, PROJ ? 0 : 1, 1);
 #pragma unroll
           for (int ks = 0; ks < BPAD / 16; ++ks) {
             const uint64_t da =
@@ -652,12 +654,13 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     tc_fence_after();
     if (okc) {
       const int rr = r & 31;
-      const uint32_t rowb = base + kOffS + (r >> 5) * 16384 + rr * 128;
+      const uint32_t rowb = base + kOffS + (r >> 5) * kChunkS + rr * 128;
+      // warp w: columns (kN / 2) (w / 4).. of the CTA's dS, 32 at a time
 #pragma unroll
-      for (int cc = 0; cc < 2; ++cc) {
+      for (int cc = 0; cc < kN / 64; ++cc) {
         float dsv[32];
-        tmem_ld32_sync(t_a + lane_base + hb * 64 + cc * 32, dsv);
-        const uint32_t box = rowb + (2 * hb + cc) * 4096;
+        tmem_ld32_sync(t_a + lane_base + hb * (kN / 2) + cc * 32, dsv);
+        const uint32_t box = rowb + (hb * (kN / 64) + cc) * 4096;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const uint32_t addr = box + ((j ^ (rr & 3)) << 5);
@@ -673,8 +676,9 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     __syncthreads();
     if (tid == 0 && okc && !*abort_flag) {
       for (int c = 0; c < 4; ++c)
-        for (int nb = 0; nb < 4; ++nb)
-          tma_reduce_add_3d(&tmS, base + kOffS + c * 16384 + nb * 4096, 32 * nb, 32 * c, u);
+        for (int nn = 0; nn < kN / 32; ++nn)
+          tma_reduce_add_3d(&tmS, base + kOffS + c * kChunkS + nn * 4096,
+                            32 * (HALF ? 2 * half + nn : nn), 32 * c, u);
       bulk_commit_group();
     }
   }
@@ -698,12 +702,15 @@ int launch_cfg(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int 
 }
 
 // Column halves when the grid would fill at most one CTA per SM (and the
-// variant allows them: no fused commit, an elementwise map).
+// map is elementwise).
 template <int BPAD, int FMAP>
 int launch_fmap(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int grid, int shared,
                 int commit) {
-  if (commit) return launch_cfg<BPAD, false, true, FMAP>(c, tm, a, grid);
-  if (FMAP != kFmapReluProj && grid <= c.sm_count)
+  const bool halves = FMAP != kFmapReluProj && grid <= c.sm_count;
+  if (commit)
+    return halves ? launch_cfg<BPAD, false, true, FMAP, FMAP != kFmapReluProj>(c, tm, a, grid)
+                  : launch_cfg<BPAD, false, true, FMAP>(c, tm, a, grid);
+  if (halves)
     return shared ? launch_cfg<BPAD, true, false, FMAP, FMAP != kFmapReluProj>(c, tm, a, grid)
                   : launch_cfg<BPAD, false, false, FMAP, FMAP != kFmapReluProj>(c, tm, a, grid);
   return shared ? launch_cfg<BPAD, true, false, FMAP>(c, tm, a, grid)

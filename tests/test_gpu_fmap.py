@@ -248,7 +248,8 @@ def test_prefill_fmap_f32(fmap):
 
 @pytest.mark.parametrize("mode", ["default", "shared"])
 @pytest.mark.parametrize("fmap", list(FMAPS), ids=list(FMAPS))
-@pytest.mark.parametrize("case", [(2, 16, 4, 32), (2, 8, 2, 17), (2, 8, 1, 33)],
+@pytest.mark.parametrize("case", [(2, 16, 4, 32), (2, 8, 2, 17), (2, 8, 1, 33),
+                                  (38, 16, 4, 32)],   # the last on whole units
                          ids=lambda c: "n%d_hq%d_hkv%d_b%d" % c)
 def test_step_commit_fmap_bf16(case, fmap, mode):
     """In the default mode with G*b <= 128 both maps run the fused kernel

@@ -320,6 +320,8 @@ FUSED_CASES = [  # (n, hq, hkv, b): the first five run as one kernel in the defa
     (2, 16, 4, 32), (3, 4, 4, 32), (2, 8, 2, 17), (2, 8, 2, 10), (1, 4, 1, 1),
     (2, 8, 1, 33),   # G*b = 264 rows: step + commit kernels
     (1, 16, 4, 64),  # 256 rows
+    (38, 16, 4, 32), # 152 unit rows: the fused kernel on whole units (the five above
+                     # run as column halves)
 ]
 
 
