@@ -8,7 +8,8 @@
 // projection W_g (the method details' kernel-function approximation).
 //
 // One CTA per (request n, KV head g, 128-row tile of the G*b query rows that
-// share g).  TMA brings Q, K, V first; the fp32 state S (four 32-row chunks)
+// share g); on grids of at most one CTA per SM, two CTAs per tile, each
+// computing half of the output columns (HALF, below).  TMA brings Q, K, V first; the fp32 state S (four 32-row chunks)
 // is requested once this CTA's Q has landed, so that across the grid the
 // softmax operands are not queued behind the state (measured: 2 % faster in
 // the default mode, 4 % with the shared denominator):
