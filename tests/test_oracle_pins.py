@@ -599,6 +599,18 @@ def test_paged_prefix_page_order_invariance():
     assert np.array_equal(Y, Y2)
 
 
+def test_paged_prefix_page_size_invariance():
+    """The same caches laid out in pages of 1, 4 and 16 tokens (each in its own
+    random page order) give bit-identical outputs: the result depends on the
+    tokens a request sees, not on how its pages cut them."""
+    P_lens = [0, 9, 31, 16]
+    outs = []
+    for ps in (1, 4, 16):
+        Q, K, V, _, _, Kpool, Vpool, table = _paged_case(14, P_lens, ps)
+        outs.append(oracle.prefix_softmax_paged(Q, Kpool, Vpool, table, P_lens, ps, K, V))
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
+
+
 def test_paged_prefix_pins_catch_planted_mistakes():
     """A gather reading the wrong row of a page, or every request through
     request 0's table, fails the per-request SDPA pin."""
