@@ -39,6 +39,7 @@ DENOISE = 8
 UNIT_BYTES_STEP = (HQ // HKV) * B_ * D_ * 2 * 2 + 2 * B_ * D_ * 2 + D_ * D_ * 4  # Q+Y, K+V, S
 UNIT_BYTES_COMMIT = 2 * B_ * D_ * 2 + 2 * D_ * D_ * 4                           # K+V, S r+w
 UNIT_BYTES_FUSED = UNIT_BYTES_STEP + D_ * D_ * 4                                # + S write
+UNIT_BYTES_SHARED = UNIT_BYTES_STEP + D_ * 4                                     # + z read
 WORKLOAD = ("long-prefix: batch 64, 16q/4kv heads, d=128, active block B=32, prefix 32768 "
             "in fp32 state; step = one block: 8 hybrid denoising steps, the last fused with "
             "the block commit")
@@ -53,6 +54,8 @@ def parse():
     ap.add_argument("--no-cpu", action="store_true", help="skip the CPU-oracle baseline")
     ap.add_argument("--no-compare", action="store_true", help="skip the exact-path comparison")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the secondary workloads in the benchmark line")
     ap.add_argument("--only", choices=["step", "step_commit", "commit", "prefill", "prefix",
                                        "paged"],
                     help="launch just this kernel warmup + steps times (small case for ncu)")
@@ -191,6 +194,23 @@ def max_over_ranks(value, dist, device):
     return float(t.item())
 
 
+def graph_schedule(steps, cycles_per_graph):
+    """Replays that run exactly `steps` block cycles: (replays of the graph of
+    `cycles_per_graph` cycles, single-cycle graphs after them)."""
+    steps = max(0, int(steps))
+    return steps // cycles_per_graph, steps % cycles_per_graph
+
+
+E2E_MIN_CYCLES, E2E_MIN_WARMUP = 50, 10
+
+
+def e2e_counts(steps, warmup):
+    """Timed and warm-up block cycles of the end-to-end leg: --steps and
+    --warmup, floored at 50 and 10 (30 timed cycles after 3 warm-up cycles
+    under-measured the copies: 5.4e6 tokens/s where 50 after 3 gave 8.5e6)."""
+    return max(E2E_MIN_CYCLES, int(steps)), max(E2E_MIN_WARMUP, int(warmup))
+
+
 def job_throughput(tokens_per_rank, world, time_ms):
     """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
     return tokens_per_rank * world / (time_ms / 1e3)
@@ -273,31 +293,57 @@ def run_reference(args, rank, world):
 
 
 def cpu_baseline_native():
-    """Oracle timed on this host's cores on a bounded sample (~10-30 s)."""
+    """The oracle on this host's cores, on bounded samples (about 20 s in all):
+    the block cycle on all cores (the reported value) and on one thread, and,
+    per batch row (one request: 4 KV heads, 16 query heads), the 32768-token
+    prefill and the exact path over a 32768-token cache on all cores."""
     import oracle
     from block_hybrid_linear_b200 import inputs
     cores = len(os.sched_getaffinity(0))
-    oracle.set_threads(cores)
     std = 1.0 / math.sqrt(D_)
     nreq = 16
     Qb, Qv = inputs.normal_bf16_np(4000, inputs.TID_Q, (nreq, HQ, B_, D_), std)
     Kb, Kv = inputs.normal_bf16_np(4000, inputs.TID_K, (nreq, HKV, B_, D_), std)
     Vb, Vv = inputs.normal_bf16_np(4000, inputs.TID_V, (nreq, HKV, B_, D_), std)
     Sv, zv = inputs.synthetic_state_np(4000, nreq, HKV, D_, P_, std)
+
+    def cycles_for(nr, seconds, max_cycles):
+        t0 = time.perf_counter()
+        cycles = 0
+        while True:
+            for _ in range(DENOISE):
+                oracle.hybrid_step(Qv[:nr], Kv[:nr], Vv[:nr], Sv[:nr], zv[:nr])
+            oracle.state_commit(Sv[:nr], zv[:nr], Kv[:nr], Vv[:nr])
+            cycles += 1
+            if time.perf_counter() - t0 > seconds or cycles >= max_cycles:
+                break
+        return cycles, time.perf_counter() - t0
+
+    oracle.set_threads(cores)
+    cycles, dt = cycles_for(nreq, 8.0, 50)
+    out = {"value": nreq * B_ * DENOISE * cycles / dt, "unit": "tokens/s", "cores": cores,
+           "kind": "oracle",
+           "sample": "%d of 64 requests x %d block cycles (8 steps + commit), fp64 oracle, "
+                     "%.1f s on %d threads" % (nreq, cycles, dt, cores)}
+    oracle.set_threads(1)
+    c1, dt1 = cycles_for(1, 4.0, 50)
+    out["single_thread"] = {"value": B_ * DENOISE * c1 / dt1, "unit": "tokens/s", "cores": 1,
+                            "sample": "1 of 64 requests x %d block cycles, %.1f s" % (c1, dt1)}
+    # per row: one request of the long-prefix workload
+    oracle.set_threads(cores)
+    _, Kp = inputs.normal_bf16_np(4001, inputs.TID_KP, (1, HKV, P_, D_), std)
+    _, Vp = inputs.normal_bf16_np(4001, inputs.TID_VP, (1, HKV, P_, D_), std)
     t0 = time.perf_counter()
-    cycles = 0
-    while True:
-        for _ in range(DENOISE):
-            oracle.hybrid_step(Qv, Kv, Vv, Sv, zv)
-        oracle.state_commit(Sv, zv, Kv, Vv)
-        cycles += 1
-        if time.perf_counter() - t0 > 10.0 or cycles >= 50:
-            break
-    dt = time.perf_counter() - t0
-    return {"value": nreq * B_ * DENOISE * cycles / dt, "unit": "tokens/s", "cores": cores,
-            "kind": "oracle",
-            "sample": "%d of 64 requests x %d block cycles (8 steps + commit), fp64 oracle, "
-                      "%.1f s" % (nreq, cycles, dt)}
+    oracle.state_prefill(Kp, Vp)
+    out["per_row_prefill_32k_s"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    oracle.prefix_softmax(Qv[:1], Kp, Vp, P_, Kv[:1], Vv[:1])
+    out["per_row_exact_32k_s"] = time.perf_counter() - t0
+    out["per_row_note"] = ("per-row: one request (4 KV heads, 16 query heads x 32 active "
+                           "tokens) with a 32768-token prompt / cache, fp64 oracle on %d "
+                           "threads; per_row_exact_32k_s is one denoising step of the exact "
+                           "path" % cores)
+    return out
 
 
 # ---------------------------------------------------------------- native
@@ -397,18 +443,29 @@ def run_native(args, rank, world, local):
         bha.bha_hybrid_step_commit(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"],
                                    stream=stream)
 
-    # graph of R cycles: every set is touched in each role, rotation period R
+    # graph of R cycles: every set is touched in each role, rotation period R;
+    # and one graph per single cycle c < R for step counts that are not a
+    # multiple of R (exactly --steps block cycles are timed)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for c in range(2):
             cycle(c)
+        st = sets[0]   # (each kernel variant runs once before any capture)
+        bha.bha_hybrid_step(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"],
+                            flags=bha.BHA_FLAG_SHARED_DENOM, stream=stream)
     stream.synchronize()
     g_cycles = R
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for c in range(g_cycles):
             cycle(c)
-    # kernel-only graphs for the per-launch durations of the two kernels
+    singles = []
+    for c in range(g_cycles):
+        g1 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g1, stream=stream):
+            cycle(c)
+        singles.append(g1)
+    # kernel-only graphs for the per-launch durations of the kernels
     g_step = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step, stream=stream):
         for k in range(4 * R):
@@ -421,14 +478,24 @@ def run_native(args, rank, world, local):
             st = sets[k % R]
             bha.bha_hybrid_step_commit(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"],
                                        stream=stream)
+    g_shared = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_shared, stream=stream):
+        for k in range(4 * R):
+            st = sets[k % R]
+            bha.bha_hybrid_step(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"],
+                                flags=bha.BHA_FLAG_SHARED_DENOM, stream=stream)
     torch.cuda.synchronize()
 
-    reps = max(1, math.ceil(args.steps / g_cycles))
-    steps = reps * g_cycles
-    warm = max(1, math.ceil(args.warmup / g_cycles))
+    steps, warmup = max(1, args.steps), max(0, args.warmup)
     torch.cuda.set_stream(stream)   # graph replays launch on the current stream
-    for _ in range(warm):
-        graph.replay()
+
+    def run_cycles(k):
+        full, rem = graph_schedule(k, g_cycles)
+        for _ in range(full):
+            graph.replay()
+        for c in range(rem):
+            singles[c].replay()
+    run_cycles(warmup)
     torch.cuda.synchronize()
     assert bha.bha_device_error(True) == 0
 
@@ -436,29 +503,36 @@ def run_native(args, rank, world, local):
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ks0, ks1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     kc0, kc1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    kd0, kd1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
     ev0.record(stream)
-    for _ in range(reps):
-        graph.replay()
+    run_cycles(steps)
     ev1.record(stream)
     # per-kernel durations, measured in the same run on the launching stream
+    # (at least 60 launches of each)
+    kreps = max(1, math.ceil(steps / (4 * g_cycles)))
     ks0.record(stream)
-    for _ in range(max(1, reps // 4)):
+    for _ in range(kreps):
         g_step.replay()
     ks1.record(stream)
     kc0.record(stream)
-    for _ in range(max(1, reps // 4)):
+    for _ in range(kreps):
         g_commit.replay()
     kc1.record(stream)
+    kd0.record(stream)
+    for _ in range(kreps):
+        g_shared.replay()
+    kd1.record(stream)
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     t_ms = ev0.elapsed_time(ev1)
-    step_launch_ms = ks0.elapsed_time(ks1) / (max(1, reps // 4) * 4 * R)
-    commit_launch_ms = kc0.elapsed_time(kc1) / (max(1, reps // 4) * 2 * R)
+    step_launch_ms = ks0.elapsed_time(ks1) / (kreps * 4 * R)
+    commit_launch_ms = kc0.elapsed_time(kc1) / (kreps * 2 * R)
+    shared_launch_ms = kd0.elapsed_time(kd1) / (kreps * 4 * R)
     assert bha.bha_device_error(True) == 0
     t_ms = max_over_ranks(t_ms, pg, dev)
     value = job_throughput(steps * N_ * B_ * DENOISE, world, t_ms)
@@ -467,9 +541,10 @@ def run_native(args, rank, world, local):
     step_bytes = N_ * HKV * UNIT_BYTES_STEP
     achieved = step_bytes / (step_launch_ms / 1e3) / 1e9
     fused_bytes = N_ * HKV * UNIT_BYTES_FUSED
+    shared_bytes = N_ * HKV * UNIT_BYTES_SHARED
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
-        "steps": steps, "warmup": warm * g_cycles, "ms_per_step": t_ms / steps,
+        "steps": steps, "warmup": warmup, "ms_per_step": t_ms / steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": DATA,
         "config": {"workload": WORKLOAD, "batch": N_, "heads_q": HQ, "heads_kv": HKV,
@@ -482,7 +557,13 @@ def run_native(args, rank, world, local):
                      "peak_kind": peak_kind,
                      "traffic": traffic_record("k_step_bf16", "k_step.cu"),
                      "algorithmic_bytes_per_launch": step_bytes,
-                     "launch_us": step_launch_ms * 1e3},
+                     "launch_us": step_launch_ms * 1e3,
+                     "shared_denom": {
+                         "kernel": "k_step_bf16 (shared denominator)",
+                         "launch_us": shared_launch_ms * 1e3,
+                         "algorithmic_bytes_per_launch": shared_bytes,
+                         "achieved": shared_bytes / (shared_launch_ms / 1e3) / 1e9,
+                         "frac": shared_bytes / (shared_launch_ms / 1e3) / 1e9 / peak}},
         "hbm_roofline_frac": achieved / peak,
         "step_commit": {"kernel": "k_step_bf16 (fused commit)",
                         "launch_us": commit_launch_ms * 1e3,
@@ -493,6 +574,8 @@ def run_native(args, rank, world, local):
         "prefill": {"ms": prefill_ms, "tokens": N_ * P_,
                     "achieved_gbs": prefill_bytes / (prefill_ms / 1e3) / 1e9},
         "gpu_launches": steps * DENOISE,
+        "timed_block_cycles": {"full_graphs_of_%d" % g_cycles: graph_schedule(steps, g_cycles)[0],
+                               "single_cycle_graphs": graph_schedule(steps, g_cycles)[1]},
         "clocks": clk,
     }
 
@@ -505,7 +588,7 @@ def run_native(args, rank, world, local):
 
     # ---- exact prefix softmax on identical shapes (the comparison path)
     if not args.no_compare:
-        del graph, g_step, g_commit
+        del graph, g_step, g_commit, g_shared, singles
         cap = P_ + B_
         Kc = torch.empty(N_, HKV, cap, D_, dtype=torch.bfloat16, device=dev)
         Vc = torch.empty_like(Kc)
@@ -581,9 +664,7 @@ def run_native(args, rank, world, local):
         for b in range(2):
             for e in (ev_comp[b], ev_out[b]):
                 e.record(stream)
-        # a fixed count, whatever --steps is: 30 cycles after 3 warm-up cycles
-        # measured 5.4e6 tokens/s where 50 after 3 measured 8.5e6
-        n_e2e, warm_e2e = 50, 10
+        n_e2e, warm_e2e = e2e_counts(args.steps, args.warmup)
 
         def e2e_cycle():
             for s in range(DENOISE):
@@ -620,16 +701,34 @@ def run_native(args, rank, world, local):
         d2h = DENOISE * hY.numel() * 2
         line["e2e"] = {"value": job_throughput(n_e2e * N_ * B_ * DENOISE, world, e2e_ms),
                        "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                       "d2h_bytes_per_step": d2h}
+                       "d2h_bytes_per_step": d2h, "steps": n_e2e, "warmup": warm_e2e,
+                       "note": "block cycles: --steps and --warmup, at least %d and %d"
+                               % (E2E_MIN_CYCLES, E2E_MIN_WARMUP)}
         line["gpu_launches_e2e"] = n_e2e * DENOISE
 
-    if rank == 0 and not args.no_cpu:
-        line["cpu_baseline"] = cpu_baseline_native()
+    # every rank has finished its collective steps; rank 0 alone goes on
     if pg is not None:
         pg.barrier()
         pg.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    if rank != 0:
+        return
+    # ---- secondary workloads on this GPU, from a clean device: the single
+    # step (batch 8), the generation loop against the exact path, and the
+    # 20-layer stack's largest batch before out-of-memory
+    if not args.no_secondary:
+        # drop every device buffer of the benchmark line
+        sets = S0 = z0 = ws = st = dbuf = Kp = Vp = Kc = Vc = Yx = wsp = None
+        graph = singles = g_step = g_commit = g_shared = None
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        line["secondary"] = {
+            "single_step_batch8": measure_single_step(dev),
+            "generation_loop": measure_generation_loop(dev),
+            "stack_memory": stack_oom(dev),
+        }
+    if not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline_native()
+    print(json.dumps(line), flush=True)
 
 
 def run_only(args):
@@ -714,14 +813,13 @@ def _time_graph(g, stream, reps):
     return e0.elapsed_time(e1) / reps
 
 
-def run_single_step(args):
+def measure_single_step(dev):
     """Batch 8, 16q/4kv, B=32, prefix 4096 in the state: one denoising step
-    (launch-latency bound at this size), beside the exact path."""
+    (launch-latency bound at this size), beside the exact path and a plain
+    copy of the same bytes."""
     import torch
     import block_hybrid_linear_b200 as bha
-    from block_hybrid_linear_b200 import build, inputs
-    build.build()
-    dev = torch.device("cuda", 0)
+    from block_hybrid_linear_b200 import inputs
     n, P = 8, 4096
     std = 1.0 / math.sqrt(D_)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -737,15 +835,23 @@ def run_single_step(args):
     sets = [dict(Q=inputs.normal_bf16_torch(r, inputs.TID_Q, (n, HQ, B_, D_), std, dev),
                  K=inputs.normal_bf16_torch(r, inputs.TID_K, (n, HKV, B_, D_), std, dev),
                  V=inputs.normal_bf16_torch(r, inputs.TID_V, (n, HKV, B_, D_), std, dev),
-                 S=S0.clone(), Y=torch.empty(n, HQ, B_, D_, dtype=torch.bfloat16, device=dev))
+                 S=S0.clone(), z=z0.clone(),
+                 Y=torch.empty(n, HQ, B_, D_, dtype=torch.bfloat16, device=dev))
             for r in range(R)]
     stream = torch.cuda.Stream(device=dev)
 
-    def steps():
+    def steps(flags=0, commit=False):
+        call = bha.bha_hybrid_step_commit if commit else bha.bha_hybrid_step
         for st in sets:
-            bha.bha_hybrid_step(st["Q"], st["K"], st["V"], st["S"], st["Y"], stream=stream)
+            call(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"], flags=flags,
+                 stream=stream)
     g = _graph(steps, stream)
     step_us = _time_graph(g, stream, 50) * 1e3 / R
+    g = _graph(lambda: steps(flags=bha.BHA_FLAG_SHARED_DENOM), stream)
+    shared_us = _time_graph(g, stream, 50) * 1e3 / R
+    g = _graph(lambda: steps(commit=True), stream)
+    commit_us = _time_graph(g, stream, 50) * 1e3 / R
+    del g
     needp = bha.bha_prefix_softmax_workspace_size(n, HQ, HKV, B_, D_, P)
     wsp = torch.empty(max(needp, 16), dtype=torch.uint8, device=dev)
     st = sets[0]
@@ -755,18 +861,31 @@ def run_single_step(args):
                                stream=stream)
     gx = _graph(exact, stream)
     exact_us = _time_graph(gx, stream, 50) * 1e3
+    del gx
     bytes_step = n * HKV * UNIT_BYTES_STEP
     peak, _ = measured_peaks()
-    print(json.dumps({
+    torch.cuda.synchronize()
+    assert bha.bha_device_error(True) == 0
+    return {
         "workload": "single-step: batch 8, 16q/4kv, d=128, B=32, prefix 4096 in the state",
-        "metric": METRIC, "unit": "tokens/s",
         "hybrid_step": {"launch_us": step_us, "tokens_per_s": n * B_ / (step_us / 1e6),
                         "achieved_gbs": bytes_step / (step_us / 1e6) / 1e9,
                         "frac_of_peak": bytes_step / (step_us / 1e6) / 1e9 / peak,
                         "algorithmic_bytes": bytes_step},
+        "hybrid_step_shared_denom_us": shared_us,
+        "hybrid_step_commit_us": commit_us,
         "prefix_softmax": {"launch_us": exact_us, "tokens_per_s": n * B_ / (exact_us / 1e6)},
         "same_bytes_copy": same_bytes_copy(bytes_step, R, stream, dev, peak),
-        "note": "4.7 MB per step: bound by launch latency, not by HBM"}), flush=True)
+        "note": "4.7 MB per step: bound by per-CTA latency, not by HBM"}
+
+
+def run_single_step(args):
+    import torch
+    from block_hybrid_linear_b200 import build
+    build.build()
+    out = measure_single_step(torch.device("cuda", 0))
+    out["metric"], out["unit"] = METRIC, "tokens/s"
+    print(json.dumps(out), flush=True)
 
 
 def run_feature_maps(args):
@@ -978,15 +1097,14 @@ def run_ragged(args):
           flush=True)
 
 
-def run_generation_loop(args):
-    """Batch 32, prompt 1024 -> state, 32 blocks x 8 denoising steps (one
-    commit per block), against exact attention over the growing KV cache
-    (appending each finished block).  Whole loops replayed as CUDA graphs."""
+def measure_generation_loop(dev):
+    """Batch 32, prompt 1024 -> state, 32 blocks x 8 denoising steps (the
+    last step of each block fused with its commit), against exact attention
+    over the growing KV cache (appending each finished block).  Whole loops
+    replayed as CUDA graphs."""
     import torch
     import block_hybrid_linear_b200 as bha
-    from block_hybrid_linear_b200 import build, inputs
-    build.build()
-    dev = torch.device("cuda", 0)
+    from block_hybrid_linear_b200 import inputs
     n, T, nblk, nst = 32, 1024, 32, DENOISE
     std = 1.0 / math.sqrt(D_)
     cap = T + nblk * B_
@@ -1029,15 +1147,26 @@ def run_generation_loop(args):
     gx = _graph(exact_loop, stream)
     h_ms = _time_graph(gh, stream, 5)
     x_ms = _time_graph(gx, stream, 5)
+    del gh, gx
+    torch.cuda.synchronize()
+    assert bha.bha_device_error(True) == 0
     tokens = n * B_ * nblk * nst
-    print(json.dumps({
+    return {
         "workload": "generation-loop: batch 32, 16q/4kv, d=128, prompt 1024 prefilled, "
                     "32 blocks x 8 denoising steps, B=32",
-        "metric": METRIC, "unit": "tokens/s",
         "hybrid": {"loop_ms": h_ms, "tokens_per_s": tokens / (h_ms / 1e3),
                    "launches": 2 + nblk * nst},
         "exact_prefix_softmax": {"loop_ms": x_ms, "tokens_per_s": tokens / (x_ms / 1e3)},
-        "speedup": x_ms / h_ms}), flush=True)
+        "speedup": x_ms / h_ms}
+
+
+def run_generation_loop(args):
+    import torch
+    from block_hybrid_linear_b200 import build
+    build.build()
+    out = measure_generation_loop(torch.device("cuda", 0))
+    out["metric"], out["unit"] = METRIC, "tokens/s"
+    print(json.dumps(out), flush=True)
 
 
 def run_stack(args):
@@ -1052,10 +1181,6 @@ def run_stack(args):
     dev = torch.device("cuda", 0)
     P, layers, hyb = 8192, 20, 6
     std = 1.0 / math.sqrt(D_)
-    kv_req = HKV * P * D_ * 2 * 2             # one exact layer, per request
-    st_req = HKV * (D_ * D_ + D_) * 4         # one hybrid layer, per request
-    hybrid_req = hyb * st_req + (layers - hyb) * kv_req
-    exact_req = layers * kv_req
     stream = torch.cuda.Stream(device=dev)
     rows = []
     batches = [1, 2, 4, 8, 16, 32, 64, 128, 256]
@@ -1099,6 +1224,27 @@ def run_stack(args):
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
 
+    out = {"workload": "stack: 20 attention layers (6 hybrid + 14 exact), 16q/4kv, d=128, "
+                       "B=32, prefix 8192; one denoising step through the stack",
+           "metric": METRIC, "unit": "tokens/s", "sweep": rows}
+    out.update(stack_oom(dev))
+    print(json.dumps(out), flush=True)
+
+
+def stack_oom(dev):
+    """The 20-layer stack (6 hybrid + 14 exact layers) at prefix 8192 with
+    contiguous caches: device bytes per request and the largest batch whose
+    per-request state fits in the free device memory (doubling, then
+    bisection, by allocation with out-of-memory caught)."""
+    import torch
+    P, layers, hyb = 8192, 20, 6
+    kv_req = HKV * P * D_ * 2 * 2             # one exact layer, per request
+    st_req = HKV * (D_ * D_ + D_) * 4         # one hybrid layer, per request
+    hybrid_req = hyb * st_req + (layers - hyb) * kv_req
+    exact_req = layers * kv_req
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+
     def fits(per_req, n):
         try:
             buf = torch.empty(int(per_req) * n, dtype=torch.uint8, device=dev)
@@ -1118,16 +1264,13 @@ def run_stack(args):
             lo, hi = (mid, hi) if fits(per_req, mid) else (lo, mid)
         return lo
     free, total = torch.cuda.mem_get_info(dev)
-    print(json.dumps({
-        "workload": "stack: 20 attention layers (6 hybrid + 14 exact), 16q/4kv, d=128, B=32, "
-                    "prefix 8192; one denoising step through the stack",
-        "metric": METRIC, "unit": "tokens/s", "sweep": rows,
-        "bytes_per_request": {"hybrid_layer_state": st_req, "exact_layer_kv": kv_req,
-                              "hybrid_stack": hybrid_req, "all_exact_stack": exact_req},
-        "max_batch_before_oom": {"hybrid_stack": max_batch(hybrid_req),
-                                 "all_exact_stack": max_batch(exact_req),
-                                 "device_free_bytes": free, "device_total_bytes": total}}),
-          flush=True)
+    return {"layout": "contiguous KV caches of 8192 tokens per exact layer, an fp32 S and z "
+                      "per hybrid layer",
+            "bytes_per_request": {"hybrid_layer_state": st_req, "exact_layer_kv": kv_req,
+                                  "hybrid_stack": hybrid_req, "all_exact_stack": exact_req},
+            "max_batch_before_oom": {"hybrid_stack": max_batch(hybrid_req),
+                                     "all_exact_stack": max_batch(exact_req),
+                                     "device_free_bytes": free, "device_total_bytes": total}}
 
 
 def main():

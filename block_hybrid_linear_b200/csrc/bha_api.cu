@@ -25,6 +25,7 @@ constexpr int kMaxDevices = 64;
 
 struct DeviceInfo {
   std::atomic<bool> ready{false};
+  std::atomic<unsigned long long> ctx_id{0};   // context the entry was read in
   int* dev_err = nullptr;
   int sm_count = 0;
   int cc_major = 0;
@@ -36,23 +37,43 @@ std::mutex g_dev_mutex;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+PfnCtxGetCurrent g_ctx_current = nullptr;
+PfnCtxGetId g_ctx_id = nullptr;
+std::once_flag g_ctx_once;
+
+// Per-device entries (the error word's address, the SM count) belong to the
+// context they were read in: after cudaDeviceReset the runtime creates a new
+// primary context, where the library's device symbols may sit elsewhere.  The
+// entry is re-read whenever the current context's ID differs from the one it
+// was read in (without the driver's context-ID call, once per device).
 int device_info(DeviceInfo** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BHA_ERR_CUDA;
   DeviceInfo& d = g_devices[dev];
-  if (!d.ready.load(std::memory_order_acquire)) {
+  const unsigned long long id = current_context_id();
+  if (!d.ready.load(std::memory_order_acquire) || (id != 0 && d.ctx_id.load() != id)) {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
-    if (!d.ready.load(std::memory_order_relaxed)) {
+    if (!d.ready.load(std::memory_order_relaxed) || (id != 0 && d.ctx_id.load() != id)) {
+      d.ready.store(false, std::memory_order_relaxed);
       void* p = nullptr;
-      if (cudaGetSymbolAddress(&p, g_dev_error) != cudaSuccess) return BHA_ERR_CUDA;
+      // (also creates the runtime's context on this device if there is none yet)
+      if (cudaGetSymbolAddress(&p, g_dev_error) != cudaSuccess) {
+        cudaGetLastError();   // leave no error behind for a later call to find
+        return BHA_ERR_CUDA;
+      }
       if (cudaDeviceGetAttribute(&d.sm_count, cudaDevAttrMultiProcessorCount, dev) !=
               cudaSuccess ||
           cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) !=
               cudaSuccess ||
           cudaDeviceGetAttribute(&d.cc_minor, cudaDevAttrComputeCapabilityMinor, dev) !=
-              cudaSuccess)
+              cudaSuccess) {
+        cudaGetLastError();
         return BHA_ERR_CUDA;
+      }
       d.dev_err = static_cast<int*>(p);
+      d.ctx_id.store(current_context_id());
       d.ready.store(true, std::memory_order_release);
     }
   }
@@ -69,6 +90,8 @@ int make_ctx(bha_stream_t stream, bha_dtype dtype, Ctx* c) {
   c->stream = reinterpret_cast<cudaStream_t>(stream);
   c->dev_err = d->dev_err;
   c->sm_count = d->sm_count;
+  c->dev = static_cast<int>(d - g_devices);
+  c->ctx_id = d->ctx_id.load();
   return BHA_OK;
 }
 
@@ -139,6 +162,28 @@ __global__ void k_selftest_timeout(int* err, unsigned limit_us) {
 }
 
 }  // namespace
+
+unsigned long long current_context_id() {
+  std::call_once(g_ctx_once, [] {
+    void* f0 = nullptr;
+    void* f1 = nullptr;
+    cudaDriverEntryPointQueryResult q0, q1;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f0, cudaEnableDefault, &q0) == cudaSuccess &&
+        q0 == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &f1, cudaEnableDefault, &q1) == cudaSuccess &&
+        q1 == cudaDriverEntryPointSuccess) {
+      g_ctx_current = reinterpret_cast<PfnCtxGetCurrent>(f0);
+      g_ctx_id = reinterpret_cast<PfnCtxGetId>(f1);
+    }
+    cudaGetLastError();
+  });
+  if (g_ctx_current == nullptr || g_ctx_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (g_ctx_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id + 1;   // 0 stays "unknown"
+}
 
 bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const void* gaddr,
                  const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,

@@ -15,6 +15,19 @@ struct Ctx {
   cudaStream_t stream;
   int* dev_err;    // device error word of the current device
   int sm_count;    // SMs of the current device
+  int dev;         // the current device
+  unsigned long long ctx_id;   // its current context (0: not known)
+};
+
+// ID of the calling thread's current CUDA context plus one (distinct for
+// every context a process creates, so a context re-created after
+// cudaDeviceReset gets a new one); 0 when none is current or the driver
+// lacks the call.
+unsigned long long current_context_id();
+
+// For each device, the context in which a kernel's attributes were last set.
+struct Prepared {
+  std::atomic<unsigned long long> ctx[64] = {};
 };
 
 // Tensor-map encoder fetched from the driver at run time (no libcuda link).
@@ -24,18 +37,17 @@ bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int rank, const vo
                  CUtensorMapSwizzle swizzle);
 
 // Sets a kernel's dynamic shared-memory limit and the maximum shared-memory
-// carveout once per device (bit `dev` of `done`), outside any hot path.
+// carveout once per device and context (`done`), outside any hot path.
 template <typename Kernel>
-bool prepare_kernel(Kernel kern, int smem_bytes, std::atomic<uint64_t>& done) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  const uint64_t bit = 1ull << dev;
-  if (done.load(std::memory_order_acquire) & bit) return true;
+bool prepare_kernel(const Ctx& c, Kernel kern, int smem_bytes, Prepared& done) {
+  if (c.dev < 0 || c.dev >= 64) return false;
+  const unsigned long long stamp = c.ctx_id == 0 ? 1ull : c.ctx_id;
+  if (done.ctx[c.dev].load(std::memory_order_acquire) == stamp) return true;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
       cudaSuccess)
     return false;
   cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-  done.fetch_or(bit, std::memory_order_release);
+  done.ctx[c.dev].store(stamp, std::memory_order_release);
   return true;
 }
 

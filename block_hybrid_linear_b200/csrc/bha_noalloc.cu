@@ -10,16 +10,21 @@
 // workspace from a fixed-size array that lives in this library's device
 // memory instead, so the call itself allocates nothing.
 //
-// Cost: every GPU that loads this part of the library keeps kScratchBytes
-// (32 MiB) of device memory until the process exits.  All calls on a device
-// share that one array: two calls whose kernels overlap on the GPU (for
-// example on two streams without ordering between them) race on it.  The
-// chunk partials are fully rewritten by each call, so nothing in the array
-// needs clearing between calls.
+// Cost: kScratchBytes (32 MiB) of device memory on every GPU where this
+// library's device code is loaded, until the process exits.  Under lazy
+// module loading (the CUDA default, CUDA_MODULE_LOADING=LAZY) that happens at
+// the first call of this entry point on a device; under eager loading
+// (CUDA_MODULE_LOADING=EAGER) every context that loads the library holds the
+// array from its creation, whether or not this entry point is ever called.
+// All calls on a device share that one array: two calls whose kernels overlap
+// on the GPU (for example on two streams without ordering between them) race
+// on it.  The chunk partials are fully rewritten by each call, so nothing in
+// the array needs clearing between calls.
 //
-// The device address of the array is looked up once per device, on the
-// first call made with that device current; make that first call before any
-// stream capture begins.
+// The device address of the array is looked up on the first call made in
+// each CUDA context (the first call on a device, and again after
+// cudaDeviceReset has replaced the device's context); make that first call
+// before any stream capture begins.
 #include <cuda_runtime.h>
 
 #include <atomic>
@@ -27,6 +32,7 @@
 #include <mutex>
 
 #include "../../include/bha.h"
+#include "bha_internal.h"
 
 namespace {
 
@@ -36,23 +42,34 @@ constexpr int kMaxDevices = 64;
 // Chunk partials of the prefill (see bha_state_prefill_workspace_size).
 static __device__ __align__(256) unsigned char g_prefill_scratch[kScratchBytes];
 
-std::atomic<void*> g_scratch_ptr[kMaxDevices];
+// Per device: the array's address and the context it was looked up in.
+struct ScratchEntry {
+  std::atomic<void*> ptr{nullptr};
+  std::atomic<unsigned long long> ctx_id{0};
+};
+ScratchEntry g_scratch[kMaxDevices];
 std::mutex g_scratch_mutex;
 
-// Device address of the scratch array on the current device (set-up once per
-// device).  In host code the array's name only stands in for the symbol; its
-// device address must come from the runtime.
+// Device address of the scratch array in the current context (looked up once
+// per context).  In host code the array's name only stands in for the
+// symbol; its device address must come from the runtime.
 int scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return BHA_ERR_CUDA;
-  void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
+  ScratchEntry& e = g_scratch[dev];
+  const unsigned long long id = bha::current_context_id();
+  void* p = e.ptr.load(std::memory_order_acquire);
+  if (p == nullptr || (id != 0 && e.ctx_id.load() != id)) {
     std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    p = g_scratch_ptr[dev].load(std::memory_order_relaxed);
-    if (p == nullptr) {
-      if (cudaGetSymbolAddress(&p, g_prefill_scratch) != cudaSuccess || p == nullptr)
+    p = e.ptr.load(std::memory_order_relaxed);
+    if (p == nullptr || (id != 0 && e.ctx_id.load() != id)) {
+      p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_prefill_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();   // leave no error behind for a later call to find
         return BHA_ERR_CUDA;
-      g_scratch_ptr[dev].store(p, std::memory_order_release);
+      }
+      e.ctx_id.store(bha::current_context_id());
+      e.ptr.store(p, std::memory_order_release);
     }
   }
   *out = p;

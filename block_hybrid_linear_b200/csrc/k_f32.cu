@@ -243,8 +243,8 @@ int launch_step_f32(const Ctx& c, const float* Q, const float* K, const float* V
                     const float* S, const float* z, float* Y, int n, int hq, int hkv, int b,
                     int d, float scale, int shared, int fmap, const float* W) {
   const size_t smem = (size_t)(2 * b * d + 2 * d + b) * sizeof(float);
-  static std::atomic<uint64_t> prepared{0};
-  if (!prepare_kernel(k_step_f32, (2 * 64 * 128 + 2 * 128 + 64) * 4, prepared)) return -5;
+  static Prepared prepared;
+  if (!prepare_kernel(c, k_step_f32, (2 * 64 * 128 + 2 * 128 + 64) * 4, prepared)) return -5;
   k_step_f32<<<n * hq, kThreads, smem, c.stream>>>(Q, K, V, S, z, Y, hq, hkv, b, d, scale,
                                                    shared, fmap, W);
   return finish_launch();

@@ -721,13 +721,13 @@ int launch_prefix_impl(const Ctx& c, const void* Q, const void* Kc, const void* 
     if (launch_pdl(k_prefix_paged_plan, 1u, kPlanThreads, 0u, c.stream, pa)) return -5;
   }
   if (pg != nullptr) {
-    static std::atomic<uint64_t> prepared{0};
-    if (!prepare_kernel(k_prefix_bf16<true>, (int)kSmem, prepared)) return -5;
+    static Prepared prepared;
+    if (!prepare_kernel(c, k_prefix_bf16<true>, (int)kSmem, prepared)) return -5;
     rc = launch_pdl(k_prefix_bf16<true>, (unsigned)plan_grid, kThreads, kSmem, c.stream, tq, tkc, tvc,
                     tka, tva, ty, to, a);
   } else {
-    static std::atomic<uint64_t> prepared{0};
-    if (!prepare_kernel(k_prefix_bf16<false>, (int)kSmem, prepared)) return -5;
+    static Prepared prepared;
+    if (!prepare_kernel(c, k_prefix_bf16<false>, (int)kSmem, prepared)) return -5;
     rc = launch_pdl(k_prefix_bf16<false>, (unsigned)items, kThreads, kSmem, c.stream, tq, tkc,
                     tvc, tka, tva, ty, to, a);
   }

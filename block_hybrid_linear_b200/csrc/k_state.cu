@@ -878,14 +878,14 @@ int launch_commit_cfg(const Ctx& c, const CUtensorMap& tk, const CUtensorMap& tv
   if constexpr (FMAP == kFmapReluProj) {
     using Lay = CommitProjLayout<BPAD>;
     auto kern = k_commit_proj_bf16<BPAD>;
-    static std::atomic<uint64_t> prepared{0};
-    if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
+    static Prepared prepared;
+    if (!prepare_kernel(c, kern, (int)Lay::kSmem, prepared)) return -5;
     return launch_pdl(kern, units, kThreads, Lay::kSmem, c.stream, tk, tv, ts, tw, a);
   } else {
     using Lay = CommitLayout<BPAD>;
     auto kern = k_commit_bf16<BPAD, FMAP>;
-    static std::atomic<uint64_t> prepared{0};
-    if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
+    static Prepared prepared;
+    if (!prepare_kernel(c, kern, (int)Lay::kSmem, prepared)) return -5;
     return launch_pdl(kern, units, kThreads, Lay::kSmem, c.stream, tk, tv, ts, a);
   }
 }
@@ -958,19 +958,19 @@ int launch_prefill_bf16(const Ctx& c, const void* K, const void* V, int units, i
   PrefillArgs a{outZ, c.dev_err, T, splits, tp, hkv, T_lens};
   int rc;
   if (fmap == kFmapReluProj) {
-    static std::atomic<uint64_t> prepared_p{0};
-    if (!prepare_kernel(k_prefill_proj_bf16, (int)kPrefSmem, prepared_p)) return -5;
+    static Prepared prepared_p;
+    if (!prepare_kernel(c, k_prefill_proj_bf16, (int)kPrefSmem, prepared_p)) return -5;
     const PrefillProjArgs pa{a, static_cast<const uint16_t*>(W)};
     rc = launch_pdl(k_prefill_proj_bf16, units * splits, kThreads, kPrefSmem, c.stream, tk, tv,
                     to, pa);
   } else if (fmap == kFmapElu1) {
-    static std::atomic<uint64_t> prepared_e{0};
-    if (!prepare_kernel(k_prefill_bf16<kFmapElu1>, (int)kPrefSmem, prepared_e)) return -5;
+    static Prepared prepared_e;
+    if (!prepare_kernel(c, k_prefill_bf16<kFmapElu1>, (int)kPrefSmem, prepared_e)) return -5;
     rc = launch_pdl(k_prefill_bf16<kFmapElu1>, units * splits, kThreads, kPrefSmem, c.stream, tk,
                     tv, to, a);
   } else {
-    static std::atomic<uint64_t> prepared_r{0};
-    if (!prepare_kernel(k_prefill_bf16<kFmapRelu>, (int)kPrefSmem, prepared_r)) return -5;
+    static Prepared prepared_r;
+    if (!prepare_kernel(c, k_prefill_bf16<kFmapRelu>, (int)kPrefSmem, prepared_r)) return -5;
     rc = launch_pdl(k_prefill_bf16<kFmapRelu>, units * splits, kThreads, kPrefSmem, c.stream, tk,
                     tv, to, a);
   }

@@ -696,8 +696,8 @@ template <int BPAD, bool SHARED, bool COMMIT, int FMAP, bool HALF = false>
 int launch_cfg(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int grid) {
   using Lay = StepLayout<BPAD>;
   auto kern = k_step_bf16<BPAD, SHARED, COMMIT, FMAP, HALF>;
-  static std::atomic<uint64_t> prepared{0};
-  if (!prepare_kernel(kern, (int)Lay::kSmem, prepared)) return -5;
+  static Prepared prepared;
+  if (!prepare_kernel(c, kern, (int)Lay::kSmem, prepared)) return -5;
   return launch_pdl(kern, (HALF ? 2 : 1) * grid, kThreads, Lay::kSmem, c.stream, tm[0], tm[1],
                     tm[2], tm[3], tm[4], tm[5], a);
 }

@@ -25,17 +25,25 @@
  * S and z are always fp32, and every path accumulates in fp32.
  *
  * Ownership: the caller allocates and owns every buffer, the workspace and
- * the stream.  The library allocates no memory.  It holds one 4-byte device
- * word per GPU that records a kernel-side error (read with
- * bha_device_error), and a per-device host cache of that word's address;
- * bha_state_prefill_noalloc also keeps a fixed 32 MiB device array per GPU.
+ * the stream.  No call allocates memory.  The library's device code holds
+ * one 4-byte word per GPU that records a kernel-side error (read with
+ * bha_device_error) and the fixed 32 MiB array of bha_state_prefill_noalloc
+ * (below); both exist wherever the CUDA runtime has loaded the library's
+ * device code into a context.  Under lazy module loading (the default) that
+ * is the first call on a device; under eager loading
+ * (CUDA_MODULE_LOADING=EAGER) every context holds both from its creation,
+ * the 32 MiB included, whether or not bha_state_prefill_noalloc is called.
+ * The host side caches each device's symbol addresses per CUDA context and
+ * looks them up again after cudaDeviceReset has replaced the context.
  *
  * Behaviour: every compute call validates its arguments before any launch,
  * returns a negative bha_status on failure (nothing launched), otherwise
  * enqueues its kernels on `stream` and returns BHA_OK without waiting.  A
  * launch failure reported by the runtime returns BHA_ERR_CUDA.  Kernels wait
  * on their own asynchronous copies with a bounded spin; if a wait runs out
- * they record BHA_ERR_TIMEOUT in the device error word and return.
+ * they record BHA_ERR_TIMEOUT in the device error word and return.  The
+ * outputs of that call, and the state S, z of a call that updates them in
+ * place, are then undefined.
  * Pointers must be 16-byte aligned (BHA_ERR_MISALIGNED).  Outputs must not
  * overlap inputs (BHA_ERR_INVALID_ARG).  n = 0 is a valid empty call.
  *
@@ -109,9 +117,11 @@ int bha_state_prefill(const void *K, const void *V, int n, int hkv, int T,
  * on every GPU that uses it, until the process exits.  Returns
  * BHA_ERR_WORKSPACE, launching nothing, when bha_state_prefill_workspace_size
  * exceeds 32 MiB.  The array's device address is looked up on the first
- * call made on each device (make that call before any stream capture).  All
+ * call made in each CUDA context: the first call on a device, and the first
+ * after cudaDeviceReset (make that call before any stream capture).  All
  * calls on a device share the array: calls whose kernels overlap on the GPU
- * race on it.  It holds nothing that must start at zero.
+ * race on it.  It holds nothing that must start at zero.  Where the array is
+ * reserved depends on module loading: see Ownership above.
  */
 int bha_state_prefill_noalloc(const void *K, const void *V, int n, int hkv,
                               int T, int d, bha_dtype dtype, float *S,
@@ -148,7 +158,11 @@ int bha_hybrid_step(const void *Qa, const void *Ka, const void *Va,
  * S_{1,2} = S_1 + phi(K_2)^T V_2).  In the default mode with G * b <= 128
  * this is one kernel that reads the state once; otherwise it launches the
  * step and the commit kernels back to back.  Y must not overlap any input,
- * S or z; S and z must not overlap the inputs.
+ * S or z; S and z must not overlap the inputs.  If a kernel of this call
+ * records BHA_ERR_TIMEOUT (bha_device_error), the contents of S and z are
+ * undefined afterwards: the update is not atomic per (request, KV head) --
+ * on small grids two CTAs each add half of the columns -- so rebuild the
+ * state (for example by a prefill) before using it again.
  */
 int bha_hybrid_step_commit(const void *Qa, const void *Ka, const void *Va,
                            float *S, float *z, void *Y, int n, int hq,

@@ -237,19 +237,25 @@ def block_partition(L: int, B: int):
 
 
 def generate(Q_steps, K_steps, V_steps, K_prompt=None, V_prompt=None,
-             scale=0.0, shared=False, fmap=FMAP_RELU, W=None):
+             scale=0.0, shared=False, fmap=FMAP_RELU, W=None, S0=None, z0=None):
     """Blockwise decoding loop of the worked example, on given inputs.
 
     Q_steps[blk][step] etc. hold the active block's tensors at each
     denoising step ([n, hq, b_blk, d] / [n, hkv, b_blk, d]).  The prompt
-    (optional) is folded into S first; every block's outputs use the state
-    of all earlier blocks, and after its last step the block is committed
-    with the K/V of that step.  Returns outputs[blk][step] and the final S, z.
+    (optional) is folded into S first -- or the state the prompt left
+    (S0, z0, e.g. from state_prefill run piecewise) is given instead; every
+    block's outputs use the state of all earlier blocks, and after its last
+    step the block is committed with the K/V of that step.  Returns
+    outputs[blk][step] and the final S, z.
     """
     first_k = K_steps[0][0]
     n, hkv, _, dd = first_k.shape
     if K_prompt is not None:
+        assert S0 is None and z0 is None
         S, z = state_prefill(K_prompt, V_prompt, fmap=fmap, W=W)
+    elif S0 is not None:
+        S = _f64(S0)
+        z = _f64(z0) if z0 is not None else np.zeros((n, hkv, dd))
     else:
         S = np.zeros((n, hkv, dd, dd))
         z = np.zeros((n, hkv, dd))

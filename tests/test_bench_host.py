@@ -79,3 +79,14 @@ def test_source_hash_ignores_comments_only():
     assert bench.code_only(src) != bench.code_only(src.replace("a + 1", "a + 2"))
     assert "// kept" in bench.code_only(src)
     assert "add one" not in bench.code_only(src) and "done" not in bench.code_only(src)
+
+
+def test_graph_schedule_runs_exactly_the_requested_cycles():
+    for steps in (0, 1, 5, 14, 15, 16, 20, 29, 30, 31, 20000):
+        full, rem = bench.graph_schedule(steps, 15)
+        assert full * 15 + rem == steps and 0 <= rem < 15
+
+
+def test_e2e_counts_follow_steps_with_a_floor():
+    assert bench.e2e_counts(20, 5) == (bench.E2E_MIN_CYCLES, bench.E2E_MIN_WARMUP)
+    assert bench.e2e_counts(200, 40) == (200, 40)

@@ -149,6 +149,100 @@ def test_generation_loop_first_blocks():
     check_rel("config3_final_z", host(z), ref_z, TOL_STATE_REL)
 
 
+def _timed_loop_case(seed, nblk, nstep, T):
+    """Inputs of the benchmark's block cycle at its shape (batch 64, 16q/4kv,
+    d = 128, B = 32): a T-token prompt and Q, K, V for every (block, step),
+    seeded per row; the oracle's prefix state of the prompt, built piecewise
+    (16 requests at a time) to bound host memory."""
+    cfg = inputs.WORKLOADS["long-prefix"]
+    n, hq, hkv, b = cfg["n"], cfg["hq"], cfg["hkv"], cfg["b"]
+    Kp, Kpv = bf16_case((seed, inputs.TID_KP), (n, hkv, T, 128), STD)
+    Vp, Vpv = bf16_case((seed, inputs.TID_VP), (n, hkv, T, 128), STD)
+    S0 = np.empty((n, hkv, 128, 128))
+    z0 = np.empty((n, hkv, 128))
+    for r0 in range(0, n, 16):
+        S0[r0:r0 + 16], z0[r0:r0 + 16] = oracle.state_prefill(Kpv[r0:r0 + 16], Vpv[r0:r0 + 16])
+    del Kpv, Vpv
+    steps = {}
+    for name, tid, h in (("Q", inputs.TID_Q, hq), ("K", inputs.TID_K, hkv),
+                         ("V", inputs.TID_V, hkv)):
+        steps[name] = [[bf16_case((seed, inputs.step_tid(tid, blk, s)), (n, h, b, 128), STD)
+                        for s in range(nstep)] for blk in range(nblk)]
+    return (n, hq, hkv, b), Kp, Vp, S0, z0, steps
+
+
+def _run_timed_loop(shared, seed):
+    """The benchmark's decoding loop on the GPU: a prefill-built state, then
+    4 blocks x 8 denoising steps -- 7 x bha_hybrid_step and the last step
+    through bha_hybrid_step_commit -- captured in one CUDA graph on one stream
+    and replayed once, with no host synchronisation inside the loop (every
+    step writes its own output buffer).  Every step's output and the final
+    state are compared with the oracle's decoding loop from the oracle's own
+    prefill of the same prompt."""
+    import torch
+    nblk, nstep, T = 4, 8, 4096
+    (n, hq, hkv, b), Kp, Vp, S0v, z0v, st = _timed_loop_case(seed, nblk, nstep, T)
+    flags = bha.BHA_FLAG_SHARED_DENOM if shared else 0
+    ref_out, ref_S, ref_z = oracle.generate(
+        [[x[1] for x in r] for r in st["Q"]], [[x[1] for x in r] for r in st["K"]],
+        [[x[1] for x in r] for r in st["V"]], shared=shared, S0=S0v, z0=z0v)
+    S = torch.empty(n, hkv, 128, 128, device="cuda")
+    z = torch.empty(n, hkv, 128, device="cuda")
+    need = bha.bha_state_prefill_workspace_size(n, hkv, T, 128)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device="cuda")
+    Ys = [[torch.empty(n, hq, b, 128, dtype=torch.bfloat16, device="cuda")
+           for _ in range(nstep)] for _ in range(nblk)]
+    stream = torch.cuda.Stream()
+
+    def loop(S_, z_):
+        for blk in range(nblk):
+            for s in range(nstep):
+                call = bha.bha_hybrid_step_commit if s == nstep - 1 else bha.bha_hybrid_step
+                call(st["Q"][blk][s][0], st["K"][blk][s][0], st["V"][blk][s][0], S_,
+                     Ys[blk][s], z=z_, flags=flags, stream=stream)
+
+    # warm-up (kernel attributes are set on first use) on a throw-away state
+    with torch.cuda.stream(stream):
+        loop(torch.zeros_like(S), torch.zeros_like(z))
+    stream.synchronize()
+    bha.bha_state_prefill(Kp, Vp, S, z, workspace=ws, stream=stream)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        loop(S, z)
+    for Yrow in Ys:
+        for Y in Yrow:
+            Y.fill_(float("nan"))
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    assert bha.bha_device_error(True) == 0
+    tag = "timed_loop_shared" if shared else "timed_loop"
+    for blk in range(nblk):
+        for s in range(nstep):
+            check_bf16(tag, host(Ys[blk][s]), ref_out[blk][s], blk=blk, step=s)
+    check_rel(tag + "_final_S", host(S), ref_S, TOL_STATE_REL)
+    check_rel(tag + "_final_z", host(z), ref_z, TOL_STATE_REL)
+    del g
+
+
+def test_generation_loop_fused_timed_shape():
+    """The exact launch sequence the benchmark times (batch 64, 16q/4kv, B=32;
+    each block's last step fused with its commit, one CUDA graph, no host sync):
+    every output of 4 blocks x 8 steps and the final S, z against the oracle.
+    Block 2 reads the state block 1's fused commit left (worked example: block
+    2 uses S_1, block 3 uses S_1 + S_2)."""
+    _run_timed_loop(False, 4100)
+
+
+def test_generation_loop_shared_denominator_timed_shape():
+    """The same loop with the shared denominator (the last step of each block
+    runs as a step kernel then a commit kernel, the fused kernel being
+    default-mode only)."""
+    _run_timed_loop(True, 4200)
+
+
 def test_long_prefix_step_and_commit_all_units():
     """Batch 64, 16q/4kv, B=32, a 32k-token prefix state (drawn with a 32k
     prefill's statistics): the step and the commit on all 256 units."""
