@@ -56,6 +56,11 @@ def _load():
         lib.oracle_prefix_softmax.argtypes = [dp, dp, dp, L, L, dp, dp, dp, L,
                                               L, L, L, L, ctypes.c_double]
         lib.oracle_prefix_softmax.restype = None
+        lib.oracle_losa_select.argtypes = [dp, dp, L, L, L, L, L, lp, dp]
+        lib.oracle_losa_select.restype = None
+        lib.oracle_losa_apply.argtypes = [dp, dp, dp, L, L, dp, dp, lp, dp, dp, dp,
+                                          L, L, L, L, L, ctypes.c_double]
+        lib.oracle_losa_apply.restype = None
         lib.oracle_block_partition.argtypes = [L, L, lp]
         lib.oracle_block_partition.restype = L
         _lib = lib
@@ -224,6 +229,89 @@ def state_prefill_ragged(K, V, T_lens, with_z=True, fmap=FMAP_RELU, W=None):
         if with_z:
             z[i] = zi[0]
     return S, z
+
+
+def losa_select(Q, Qprev, k):
+    """Locality scores and active tokens (LoSA page, 3. 方法论: 局部性剪枝).
+
+    Q, Qprev [n, hq, b, d]: the block's queries at this and at the previous
+    denoising step.  score[ni, i] is the MSE of token i's query change over
+    all query heads and dimensions; the k tokens with the largest score (ties
+    to the lower index) are active.  Returns (active [n, min(k, b)] int64,
+    increasing token order; score [n, b] float64).
+    """
+    Q, Qprev = _f64(Q), _f64(Qprev)
+    n, hq, b, d = Q.shape
+    assert Qprev.shape == Q.shape
+    k = max(0, min(int(k), b))
+    active = np.zeros((n, max(k, 1)), dtype=np.int64)
+    score = np.zeros((n, b))
+    _load().oracle_losa_select(_ptr(Q), _ptr(Qprev), n, hq, b, d, k,
+                               active.ctypes.data_as(ctypes.POINTER(ctypes.c_long)),
+                               _ptr(score))
+    return active[:, :k], score
+
+
+def losa_apply(Q, Kc, Vc, P, K, V, is_active, O_pre, L_pre, scale=0.0):
+    """Cache reuse and merge for a given active set (LoSA page, 缓存复用 and
+    技术细节): active tokens get a dense prefix pass with this step's queries
+    (their entries of the cache are replaced), stable tokens keep their cached
+    prefix output and log-normaliser, and every token's block attention is
+    merged with its prefix part by the online-softmax identity.
+
+    is_active [n, b] (nonzero = active); O_pre [n, hq, b, d], L_pre [n, hq, b]
+    (natural-log normalisers; may be None when every token is active).
+    Returns (Y, O_pre, L_pre) as new float64 arrays.
+    """
+    Q, Kc, Vc, K, V = _f64(Q), _f64(Kc), _f64(Vc), _f64(K), _f64(V)
+    n, hq, b, d = Q.shape
+    hkv, cap = Kc.shape[1], Kc.shape[2]
+    assert 0 <= P <= cap and Kc.shape == (n, hkv, cap, d) and hq % hkv == 0
+    act = np.ascontiguousarray(np.asarray(is_active).reshape(n, b) != 0, dtype=np.int64)
+    if O_pre is None:
+        assert act.all(), "a cache is needed unless every token is active"
+        O = np.zeros((n, hq, b, d))
+        Lp = np.full((n, hq, b), -np.inf)
+    else:
+        O = _f64(O_pre).copy()
+        Lp = _f64(L_pre).copy()
+    Y = np.zeros((n, hq, b, d))
+    _load().oracle_losa_apply(_ptr(Q), _ptr(Kc), _ptr(Vc), int(P), cap, _ptr(K), _ptr(V),
+                              act.ctypes.data_as(ctypes.POINTER(ctypes.c_long)), _ptr(O),
+                              _ptr(Lp), _ptr(Y), n, hq, hkv, b, d, float(scale))
+    return Y, O, Lp
+
+
+def losa_step(Q, Qprev, Kc, Vc, P, K, V, O_pre=None, L_pre=None, k=0, scale=0.0):
+    """One denoising step of the exact path with reuse for stable tokens.
+
+    Qprev None: the block's first step, dense (every token active, the LoSA
+    page's 初始化策略).  Otherwise the k tokens whose queries changed most
+    since Qprev are active.  Returns (Y, O_pre, L_pre, active [n, k'])."""
+    n, hq, b, d = np.shape(Q)
+    if Qprev is None:
+        active = np.tile(np.arange(b, dtype=np.int64), (n, 1))
+    else:
+        active, _ = losa_select(Q, Qprev, k)
+    is_active = np.zeros((n, b), dtype=np.int64)
+    for ni in range(n):
+        is_active[ni, active[ni]] = 1
+    Y, O, Lp = losa_apply(Q, Kc, Vc, P, K, V, is_active, O_pre, L_pre, scale)
+    return Y, O, Lp, active
+
+
+def losa_block(Q_steps, K_steps, V_steps, Kc, Vc, P, k, scale=0.0):
+    """The denoising steps of one block with reuse: the first step dense, each
+    later step with the k most-changed tokens active.  Returns the outputs,
+    the active sets of every step and the final cache (O_pre, L_pre)."""
+    O = Lp = None
+    outs, acts = [], []
+    for t in range(len(Q_steps)):
+        Y, O, Lp, act = losa_step(Q_steps[t], None if t == 0 else Q_steps[t - 1], Kc, Vc, P,
+                                  K_steps[t], V_steps[t], O, Lp, k, scale)
+        outs.append(Y)
+        acts.append(act)
+    return outs, acts, O, Lp
 
 
 def block_partition(L: int, B: int):

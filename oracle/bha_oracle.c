@@ -304,6 +304,149 @@ void oracle_prefix_softmax(const double *Q, const double *Kc, const double *Vc,
 }
 
 /*
+ * Reuse of prefix attention for stable tokens, the method of the LoSA page
+ * (gist.science explainer of arXiv 2604.12056, section "3. 方法论 LoSA":
+ * 局部性剪枝 locality pruning, 缓存复用 cache reuse, 初始化策略 initialisation;
+ * and "技术细节" technical details), applied to the exact comparison path with
+ * a dense prefix pass over the active tokens (the page's sparse selector,
+ * QUEST, is not part of this path).  One denoising step of a block:
+ *
+ *   1. locality score of block token i of request ni (the MSE of its query
+ *      between this denoising step and the previous one, over the token's
+ *      whole query: every query head, every dimension):
+ *        score_i = (1 / (hq d)) sum_h sum_c (Q[ni][h][i][c] - Qprev[ni][h][i][c])^2
+ *   2. the active set A of request ni: the k tokens with the largest score
+ *      (ties to the lower token index); the others are stable tokens;
+ *   3. for an active token, every query head's prefix attention over the
+ *      cache, as a normalised output and its log-normaliser,
+ *        o_p = sum_{j<P} e^{s_j} v_j / sum_{j<P} e^{s_j},
+ *        lse_p = log sum_{j<P} e^{s_j},       s_j = scale q . k_j,
+ *      replaces the token's entries of the cache (O_pre, L_pre); a stable
+ *      token keeps the entries of the previous step (the previous step's q);
+ *   4. the block's own attention of every token, o_b and lse_b likewise over
+ *      the b block tokens with the current q, merged with the cached prefix
+ *      part by the online-softmax identity
+ *        y = (e^{lse_p - M} o_p + e^{lse_b - M} o_b) / (e^{lse_p - M} + e^{lse_b - M}),
+ *        M = max(lse_p, lse_b)      (P = 0: lse_p = -inf, y = o_b).
+ * The first denoising step of a block has no cache: every token is active
+ * (the page's dense initialisation).  The cache holds b x (d + 1) values per
+ * query head, as the page counts.
+ */
+
+/* Locality scores and the active set: active[ni * k + a], a < k, lists
+ * request ni's active tokens in increasing token order. */
+void oracle_losa_select(const double *Q, const double *Qprev, long n, long hq,
+                        long b, long d, long k, long *active, double *score)
+{
+    long ni;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (ni = 0; ni < n; ++ni) {
+        double *sc = score + ni * b;
+        for (long i = 0; i < b; ++i) {
+            double acc = 0.0;
+            for (long h = 0; h < hq; ++h) {
+                const double *q = Q + ((ni * hq + h) * b + i) * d;
+                const double *p = Qprev + ((ni * hq + h) * b + i) * d;
+                for (long c = 0; c < d; ++c)
+                    acc += (q[c] - p[c]) * (q[c] - p[c]);
+            }
+            sc[i] = acc / (double)(hq * d);
+        }
+        long a = 0;
+        for (long i = 0; i < b && a < k; ++i) {
+            /* rank of token i: tokens with a larger score, or an equal score
+             * and a lower index, come first */
+            long rank = 0;
+            for (long j = 0; j < b; ++j)
+                if (sc[j] > sc[i] || (sc[j] == sc[i] && j < i)) ++rank;
+            if (rank < k) active[ni * k + a++] = i;
+        }
+    }
+}
+
+/* Steps 3 and 4 for a given active set (is_active[ni * b + i] != 0): updates
+ * O_pre [n][hq][b][d] and L_pre [n][hq][b] for the active tokens, writes Y. */
+void oracle_losa_apply(const double *Q, const double *Kc, const double *Vc,
+                       long P, long cap, const double *K, const double *V,
+                       const long *is_active, double *O_pre, double *L_pre,
+                       double *Y, long n, long hq, long hkv, long b, long d,
+                       double scale)
+{
+    if (scale <= 0.0) scale = 1.0 / sqrt((double)d);
+    const long G = hq / hkv;
+    long nh;
+#pragma omp parallel for num_threads(g_threads) schedule(static)
+    for (nh = 0; nh < n * hq; ++nh) {
+        const long ni = nh / hq, h = nh % hq, g = h / G;
+        const double *Kcg = Kc + (ni * hkv + g) * cap * d;
+        const double *Vcg = Vc + (ni * hkv + g) * cap * d;
+        const double *Kg = K + (ni * hkv + g) * b * d;
+        const double *Vg = V + (ni * hkv + g) * b * d;
+        const long L = P > b ? P : b;
+        double *s = (double *)malloc(sizeof(double) * (size_t)(L > 0 ? L : 1));
+        double *ob = (double *)malloc(sizeof(double) * (size_t)d);
+        for (long i = 0; i < b; ++i) {
+            const long row = (ni * hq + h) * b + i;
+            const double *q = Q + row * d;
+            double *op = O_pre + row * d;
+            if (is_active[ni * b + i]) {
+                /* dense prefix pass with this step's q */
+                double m = -INFINITY;
+                for (long j = 0; j < P; ++j) {
+                    double dot = 0.0;
+                    for (long c = 0; c < d; ++c)
+                        dot += q[c] * Kcg[j * d + c];
+                    s[j] = scale * dot;
+                    if (s[j] > m) m = s[j];
+                }
+                double l = 0.0;
+                for (long j = 0; j < P; ++j) {
+                    s[j] = exp(s[j] - m);
+                    l += s[j];
+                }
+                for (long c = 0; c < d; ++c) {
+                    double acc = 0.0;
+                    for (long j = 0; j < P; ++j)
+                        acc += (s[j] / l) * Vcg[j * d + c];
+                    op[c] = P > 0 ? acc : 0.0;
+                }
+                L_pre[row] = P > 0 ? m + log(l) : -INFINITY;
+            }
+            /* the block's attention with this step's q */
+            double mb = -INFINITY;
+            for (long j = 0; j < b; ++j) {
+                double dot = 0.0;
+                for (long c = 0; c < d; ++c)
+                    dot += q[c] * Kg[j * d + c];
+                s[j] = scale * dot;
+                if (s[j] > mb) mb = s[j];
+            }
+            double lb = 0.0;
+            for (long j = 0; j < b; ++j) {
+                s[j] = exp(s[j] - mb);
+                lb += s[j];
+            }
+            for (long c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (long j = 0; j < b; ++j)
+                    acc += (s[j] / lb) * Vg[j * d + c];
+                ob[c] = acc;
+            }
+            const double lse_b = mb + log(lb);
+            const double lse_p = L_pre[row];
+            const double M = lse_p > lse_b ? lse_p : lse_b;
+            const double wp = lse_p == -INFINITY ? 0.0 : exp(lse_p - M);
+            const double wb = exp(lse_b - M);
+            double *y = Y + row * d;
+            for (long c = 0; c < d; ++c)
+                y[c] = (wp * op[c] + wb * ob[c]) / (wp + wb);
+        }
+        free(ob);
+        free(s);
+    }
+}
+
+/*
  * Block partition of a length-L sequence into blocks of B tokens; the last
  * block may be short (worked example: L=10, B=4 gives tokens 1-4, 5-8, 9-10).
  * Writes the boundaries 0 = bounds[0] < bounds[1] < ... < bounds[k] = L and
