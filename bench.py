@@ -56,8 +56,8 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the secondary workloads in the benchmark line")
-    ap.add_argument("--only", choices=["step", "step_commit", "commit", "prefill", "prefix",
-                                       "paged"],
+    ap.add_argument("--only", choices=["step", "step_shared", "step_commit", "commit", "prefill",
+                                       "prefix", "paged"],
                     help="launch just this kernel warmup + steps times (small case for ncu)")
     ap.add_argument("--prefix", type=int, default=8192,
                     help="prompt / cache length used by --only prefill|prefix")
@@ -65,7 +65,7 @@ def parse():
                     help="batch used by --only step|step_commit|commit (default 64)")
     ap.add_argument("--workload", default="long-prefix",
                     choices=["long-prefix", "single-step", "generation-loop", "stack",
-                             "feature-maps", "ragged"],
+                             "feature-maps", "ragged", "reuse"],
                     help="long-prefix is the benchmark line; the others are the secondary "
                          "workloads (one JSON line each)")
     return ap.parse_args()
@@ -194,11 +194,21 @@ def max_over_ranks(value, dist, device):
     return float(t.item())
 
 
-def graph_schedule(steps, cycles_per_graph):
-    """Replays that run exactly `steps` block cycles: (replays of the graph of
-    `cycles_per_graph` cycles, single-cycle graphs after them)."""
+def graph_plan(steps, cycles_per_graph):
+    """CUDA-graph replays that run exactly `steps` block cycles: a list of
+    (cycles in the graph, replays).  Up to 4 rotation periods run as one
+    graph of exactly `steps` cycles; beyond that, replays of the graph of one
+    period and one graph of the remainder (every graph boundary costs a
+    launch gap, so there are at most two graphs)."""
     steps = max(0, int(steps))
-    return steps // cycles_per_graph, steps % cycles_per_graph
+    if steps == 0:
+        return []
+    if steps <= 4 * cycles_per_graph:
+        return [(steps, 1)]
+    plan = [(cycles_per_graph, steps // cycles_per_graph)]
+    if steps % cycles_per_graph:
+        plan.append((steps % cycles_per_graph, 1))
+    return plan
 
 
 E2E_MIN_CYCLES, E2E_MIN_WARMUP = 50, 10
@@ -443,9 +453,8 @@ def run_native(args, rank, world, local):
         bha.bha_hybrid_step_commit(st["Q"], st["K"], st["V"], st["S"], st["Y"], z=st["z"],
                                    stream=stream)
 
-    # graph of R cycles: every set is touched in each role, rotation period R;
-    # and one graph per single cycle c < R for step counts that are not a
-    # multiple of R (exactly --steps block cycles are timed)
+    # graphs of whole block cycles (every set is touched in each role, rotation
+    # period R), so that exactly --steps cycles are timed (graph_plan)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for c in range(2):
@@ -455,16 +464,15 @@ def run_native(args, rank, world, local):
                             flags=bha.BHA_FLAG_SHARED_DENOM, stream=stream)
     stream.synchronize()
     g_cycles = R
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph, stream=stream):
-        for c in range(g_cycles):
-            cycle(c)
-    singles = []
-    for c in range(g_cycles):
-        g1 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g1, stream=stream):
-            cycle(c)
-        singles.append(g1)
+    steps, warmup = max(1, args.steps), max(0, args.warmup)
+    graphs = {}
+    for ncyc, _ in graph_plan(steps, g_cycles) + graph_plan(warmup, g_cycles):
+        if ncyc not in graphs:
+            g1 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g1, stream=stream):
+                for c in range(ncyc):
+                    cycle(c)
+            graphs[ncyc] = g1
     # kernel-only graphs for the per-launch durations of the kernels
     g_step = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_step, stream=stream):
@@ -486,21 +494,39 @@ def run_native(args, rank, world, local):
                                 flags=bha.BHA_FLAG_SHARED_DENOM, stream=stream)
     torch.cuda.synchronize()
 
-    steps, warmup = max(1, args.steps), max(0, args.warmup)
     torch.cuda.set_stream(stream)   # graph replays launch on the current stream
 
     def run_cycles(k):
-        full, rem = graph_schedule(k, g_cycles)
-        for _ in range(full):
-            graph.replay()
-        for c in range(rem):
-            singles[c].replay()
+        for ncyc, reps in graph_plan(k, g_cycles):
+            for _ in range(reps):
+                graphs[ncyc].replay()
+    # The timing events: when the K cycles are one graph, they are recorded by
+    # the graph itself (event-record nodes before the first and after the
+    # last kernel), so that the host's graph submission, which precedes the
+    # first kernel on an idle stream, is not counted as device time of the K
+    # steps (measured: 2.9 us per cycle at K = 20).
+    ev0 = torch.cuda.Event(enable_timing=True, external=True)
+    ev1 = torch.cuda.Event(enable_timing=True, external=True)
+    timed_graph = None
+    if len(graph_plan(steps, g_cycles)) == 1:
+        timed_graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(timed_graph, stream=stream):
+            ev0.record(stream)
+            for c in range(steps):
+                cycle(c)
+            ev1.record(stream)
+    # every graph is launched once before the warm-up: the first launch of an
+    # instantiated graph uploads it to the device (measured: a timed region
+    # holding a graph's first launch ran 0.082 ms per cycle against 0.066)
+    for g_ in list(graphs.values()) + [g_step, g_commit, g_shared] + (
+            [timed_graph] if timed_graph is not None else []):
+        g_.replay()
+    torch.cuda.synchronize()
     run_cycles(warmup)
     torch.cuda.synchronize()
     assert bha.bha_device_error(True) == 0
 
     clocks = ClockSampler(local)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     ks0, ks1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     kc0, kc1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     kd0, kd1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -508,9 +534,12 @@ def run_native(args, rank, world, local):
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
-    ev0.record(stream)
-    run_cycles(steps)
-    ev1.record(stream)
+    if timed_graph is not None:
+        timed_graph.replay()
+    else:
+        ev0.record(stream)
+        run_cycles(steps)
+        ev1.record(stream)
     # per-kernel durations, measured in the same run on the launching stream
     # (at least 60 launches of each)
     kreps = max(1, math.ceil(steps / (4 * g_cycles)))
@@ -574,8 +603,12 @@ def run_native(args, rank, world, local):
         "prefill": {"ms": prefill_ms, "tokens": N_ * P_,
                     "achieved_gbs": prefill_bytes / (prefill_ms / 1e3) / 1e9},
         "gpu_launches": steps * DENOISE,
-        "timed_block_cycles": {"full_graphs_of_%d" % g_cycles: graph_schedule(steps, g_cycles)[0],
-                               "single_cycle_graphs": graph_schedule(steps, g_cycles)[1]},
+        "timed_graphs": {"plan": [{"cycles": c, "replays": r}
+                                  for c, r in graph_plan(steps, g_cycles)],
+                         "events": "inside the graph" if timed_graph is not None
+                                   else "on the stream around the replays",
+                         "note": "CUDA graphs of whole block cycles, each launched once "
+                                 "(uploaded) before the warm-up"},
         "clocks": clk,
     }
 
@@ -588,7 +621,7 @@ def run_native(args, rank, world, local):
 
     # ---- exact prefix softmax on identical shapes (the comparison path)
     if not args.no_compare:
-        del graph, g_step, g_commit, g_shared, singles
+        del graphs, g_step, g_commit, g_shared, timed_graph
         cap = P_ + B_
         Kc = torch.empty(N_, HKV, cap, D_, dtype=torch.bfloat16, device=dev)
         Vc = torch.empty_like(Kc)
@@ -718,7 +751,7 @@ def run_native(args, rank, world, local):
     if not args.no_secondary:
         # drop every device buffer of the benchmark line
         sets = S0 = z0 = ws = st = dbuf = Kp = Vp = Kc = Vc = Yx = wsp = None
-        graph = singles = g_step = g_commit = g_shared = None
+        graphs = g_step = g_commit = g_shared = timed_graph = None
         torch.cuda.synchronize()
         torch.cuda.empty_cache()
         line["secondary"] = {
@@ -741,7 +774,8 @@ def run_only(args):
     dev = torch.device("cuda", 0)
     std = 1.0 / math.sqrt(D_)
     P = args.prefix
-    nb = args.batch if args.batch and args.only in ("step", "step_commit", "commit") else N_
+    nb = (args.batch if args.batch and args.only in ("step", "step_shared", "step_commit", "commit")
+          else N_)
     Q = inputs.normal_bf16_torch(1, inputs.TID_Q, (nb, HQ, B_, D_), std, dev)
     K = inputs.normal_bf16_torch(1, inputs.TID_K, (nb, HKV, B_, D_), std, dev)
     V = inputs.normal_bf16_torch(1, inputs.TID_V, (nb, HKV, B_, D_), std, dev)
@@ -770,6 +804,8 @@ def run_only(args):
                                                   workspace=ws)
     elif args.only == "commit":
         fn = lambda: bha.bha_state_commit(K, V, S, z)
+    elif args.only == "step_shared":
+        fn = lambda: bha.bha_hybrid_step(Q, K, V, S, Y, z=z, flags=bha.BHA_FLAG_SHARED_DENOM)
     elif args.only == "step_commit":
         fn = lambda: bha.bha_hybrid_step_commit(Q, K, V, S, Y, z=z)
     else:
@@ -1160,6 +1196,94 @@ def measure_generation_loop(dev):
         "speedup": x_ms / h_ms}
 
 
+def measure_reuse(dev, ks=(8, 4, 16)):
+    """The exact path with reuse for stable tokens at the long-prefix shape
+    (batch 64, 16q/4kv, d=128, B=32, a 32768-token cache): one block of 8
+    denoising steps -- the first dense, the other 7 selecting the k tokens
+    whose queries changed most -- against 8 steps of the exact path, as CUDA
+    graphs.  Queries drift from step to step with a per-token weight (a few
+    tokens change much, most little); timing does not depend on the values."""
+    import torch
+    import block_hybrid_linear_b200 as bha
+    from block_hybrid_linear_b200 import inputs
+    n, P = N_, P_
+    std = 1.0 / math.sqrt(D_)
+    Kc = inputs.normal_bf16_torch(4400, inputs.TID_KC, (n, HKV, P, D_), std, dev)
+    Vc = inputs.normal_bf16_torch(4400, inputs.TID_VC, (n, HKV, P, D_), std, dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(4401)
+    q = torch.randn(n, HQ, B_, D_, generator=g, device=dev) * std
+    Qs = [q.to(torch.bfloat16)]
+    for _ in range(1, DENOISE):
+        w = torch.empty(n, 1, B_, 1, device=dev).exponential_(generator=g) ** 2
+        q = q + 0.3 * w * torch.randn(q.shape, generator=g, device=dev) * std
+        Qs.append(q.to(torch.bfloat16))
+    Ks = [inputs.normal_bf16_torch(4402 + t, inputs.TID_K, (n, HKV, B_, D_), std, dev)
+          for t in range(DENOISE)]
+    Vs = [inputs.normal_bf16_torch(4402 + t, inputs.TID_V, (n, HKV, B_, D_), std, dev)
+          for t in range(DENOISE)]
+    Y = torch.empty(n, HQ, B_, D_, dtype=torch.bfloat16, device=dev)
+    O = torch.empty(n, HQ, B_, D_, device=dev)
+    L = torch.empty(n, HQ, B_, device=dev)
+    need = max(bha.bha_prefix_softmax_reuse_workspace_size(n, HQ, HKV, B_, D_, P, k)
+               for k in ks)
+    ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    needx = bha.bha_prefix_softmax_workspace_size(n, HQ, HKV, B_, D_, P)
+    wsx = torch.empty(max(needx, 16), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    peak, _ = measured_peaks()
+    kv_bytes = n * HKV * P * D_ * 2 * 2
+
+    def exact_block():
+        for t in range(DENOISE):
+            bha.bha_prefix_softmax(Qs[t], Kc, Vc, P, Ks[t], Vs[t], Y, workspace=wsx,
+                                   stream=stream)
+    gx = _graph(exact_block, stream)
+    x_ms = _time_graph(gx, stream, 5)
+    del gx
+    out = {"workload": "reuse: batch 64, 16q/4kv, d=128, B=32, cache 32768; one block of 8 "
+                       "denoising steps (the first dense)",
+           "kv_cache_bytes_per_step": kv_bytes,
+           "exact_block_ms": x_ms, "exact_step_ms": x_ms / DENOISE}
+    for k in ks:
+        def reuse_block():
+            for t in range(DENOISE):
+                bha.bha_prefix_softmax_reuse(Qs[t], None if t == 0 else Qs[t - 1], Kc, Vc, P,
+                                             Ks[t], Vs[t], Y, O, L, k, workspace=ws,
+                                             stream=stream)
+
+        def reuse_steps():   # the selecting steps alone
+            for t in range(1, DENOISE):
+                bha.bha_prefix_softmax_reuse(Qs[t], Qs[t - 1], Kc, Vc, P, Ks[t], Vs[t], Y, O,
+                                             L, k, workspace=ws, stream=stream)
+        gr = _graph(reuse_block, stream)
+        r_ms = _time_graph(gr, stream, 5)
+        del gr
+        gs = _graph(reuse_steps, stream)
+        s_ms = _time_graph(gs, stream, 5) / (DENOISE - 1)
+        del gs
+        out["k%d" % k] = {"block_ms": r_ms, "speedup_vs_exact": x_ms / r_ms,
+                          "selecting_step_ms": s_ms,
+                          "selecting_step_kv_gbs": kv_bytes / (s_ms / 1e3) / 1e9,
+                          "selecting_step_frac_of_peak": kv_bytes / (s_ms / 1e3) / 1e9 / peak,
+                          "tokens_per_s": n * B_ * DENOISE / (r_ms / 1e3)}
+    torch.cuda.synchronize()
+    assert bha.bha_device_error(True) == 0
+    out["note"] = ("a dense prefix pass over the active tokens still reads the whole cache "
+                   "(kv_cache_bytes_per_step) whenever a KV head has one: reuse saves the "
+                   "stable tokens' prefix arithmetic, not cache traffic")
+    return out
+
+
+def run_reuse(args):
+    import torch
+    from block_hybrid_linear_b200 import build
+    build.build()
+    out = measure_reuse(torch.device("cuda", 0))
+    out["metric"], out["unit"] = METRIC, "tokens/s"
+    print(json.dumps(out), flush=True)
+
+
 def run_generation_loop(args):
     import torch
     from block_hybrid_linear_b200 import build
@@ -1283,7 +1407,7 @@ def main():
         if rank == 0:
             {"single-step": run_single_step, "generation-loop": run_generation_loop,
              "stack": run_stack, "feature-maps": run_feature_maps,
-             "ragged": run_ragged}[args.workload](args)
+             "ragged": run_ragged, "reuse": run_reuse}[args.workload](args)
         return
     if args.impl == "reference":
         run_reference(args, rank, world)

@@ -15,7 +15,8 @@ from ._lib import (  # noqa: F401
     bha_block_partition, bha_device_error, bha_hybrid_step, bha_hybrid_step_commit,
     bha_hybrid_step_commit_fm, bha_hybrid_step_fm, bha_state_commit_fm, bha_state_prefill_fm,
     bha_prefix_softmax, bha_prefix_softmax_paged, bha_prefix_softmax_paged_workspace_size,
-    bha_prefix_softmax_workspace_size, bha_state_prefill_ragged, bha_selftest_timeout, bha_state_commit,
+    bha_prefix_softmax_workspace_size, bha_prefix_softmax_reuse,
+    bha_prefix_softmax_reuse_workspace_size, bha_state_prefill_ragged, bha_selftest_timeout, bha_state_commit,
     bha_state_prefill,
     bha_state_prefill_noalloc, bha_state_prefill_workspace_size, bha_version, lib,
     status_string,

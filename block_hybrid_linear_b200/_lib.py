@@ -36,6 +36,7 @@ EXPORTED = [
     "bha_hybrid_step_fm", "bha_hybrid_step_commit_fm", "bha_prefix_softmax_paged_workspace_size",
     "bha_prefix_softmax_paged", "bha_state_prefill_ragged",
     "bha_prefix_softmax_workspace_size", "bha_prefix_softmax",
+    "bha_prefix_softmax_reuse_workspace_size", "bha_prefix_softmax_reuse",
     "bha_block_partition", "bha_device_error", "bha_selftest_timeout",
 ]
 
@@ -100,6 +101,11 @@ def lib():
         L.bha_prefix_softmax.argtypes = [vp, vp, vp, i, i, vp, vp, vp, i, i, i, i,
                                          i, fl, i, vp, sz, vp]
         L.bha_prefix_softmax.restype = i
+        L.bha_prefix_softmax_reuse_workspace_size.argtypes = [i, i, i, i, i, i, i, i]
+        L.bha_prefix_softmax_reuse_workspace_size.restype = sz
+        L.bha_prefix_softmax_reuse.argtypes = [vp, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp, i,
+                                               i, i, i, i, i, fl, i, vp, sz, vp]
+        L.bha_prefix_softmax_reuse.restype = i
         L.bha_block_partition.argtypes = [i, i, ctypes.POINTER(ctypes.c_int), i]
         L.bha_block_partition.restype = i
         L.bha_device_error.argtypes = [i]
@@ -266,6 +272,28 @@ def bha_prefix_softmax(Q, Kc, Vc, P, K, V, Y, scale=0.0, workspace=None, stream=
                                     _ptr(V), _ptr(Y), n, hq, hkv, b, d, float(scale),
                                     _dtype(Q), _ptr(workspace), ws_bytes, _stream(stream)),
            "bha_prefix_softmax")
+
+
+def bha_prefix_softmax_reuse_workspace_size(n, hq, hkv, b, d, P, k, dtype=BHA_BF16):
+    return lib().bha_prefix_softmax_reuse_workspace_size(n, hq, hkv, b, d, P, k, dtype)
+
+
+def bha_prefix_softmax_reuse(Q, Qprev, Kc, Vc, P, K, V, Y, O_pre, L_pre, k, active=None,
+                             scale=0.0, workspace=None, stream=None):
+    """One denoising step of the exact path with reuse for stable tokens.
+
+    Qprev: the previous step's queries, or None for the block's first step
+    (every token active).  O_pre [n, hq, b, d] / L_pre [n, hq, b] fp32: the
+    reuse cache (read for stable tokens, written for active ones).  active:
+    optional [n, k] int32 output of the selected tokens."""
+    n, hq, b, d = Q.shape
+    hkv, cap = Kc.shape[1], Kc.shape[2]
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().bha_prefix_softmax_reuse(_ptr(Q), _ptr(Qprev), _ptr(Kc), _ptr(Vc), int(P), cap,
+                                          _ptr(K), _ptr(V), _ptr(Y), _ptr(O_pre), _ptr(L_pre),
+                                          _ptr(active), int(k), n, hq, hkv, b, d, float(scale),
+                                          _dtype(Q), _ptr(workspace), ws_bytes,
+                                          _stream(stream)), "bha_prefix_softmax_reuse")
 
 
 def bha_prefix_softmax_paged_workspace_size(n, hq, hkv, b, d, max_pages, page_size,

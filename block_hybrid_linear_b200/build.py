@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 LIB = os.path.join(HERE, "libbha.so")
-SOURCES = ["bha_api.cu", "k_f32.cu", "k_step.cu", "k_state.cu", "k_prefix.cu",
+SOURCES = ["bha_api.cu", "k_f32.cu", "k_step.cu", "k_state.cu", "k_prefix.cu", "k_reuse.cu",
            "bha_noalloc.cu"]
 HEADERS = ["bha_internal.h", "bha_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

@@ -547,6 +547,71 @@ int bha_prefix_softmax(const void* Qa, const void* Kc, const void* Vc, int P, in
                                           workspace, workspace_bytes));
 }
 
+size_t bha_prefix_softmax_reuse_workspace_size(int n, int hq, int hkv, int b, int d, int P,
+                                               int k, bha_dtype dtype) {
+  if (dtype != BHA_BF16 || n <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0 || b < 1 || b > 64 ||
+      d != 128 || P < 0 || k < 0)
+    return 0;
+  const size_t first = reuse_bf16_workspace(n, hq, hkv, b, P, k, 0);
+  const size_t later = reuse_bf16_workspace(n, hq, hkv, b, P, k, 1);
+  return first > later ? first : later;
+}
+
+int bha_prefix_softmax_reuse(const void* Qa, const void* Qprev, const void* Kc, const void* Vc,
+                             int P, int cap, const void* Ka, const void* Va, void* Y,
+                             float* O_pre, float* L_pre, int* active, int k, int n, int hq,
+                             int hkv, int b, int d, float scale, bha_dtype dtype, void* workspace,
+                             size_t workspace_bytes, bha_stream_t stream) {
+  int st = check_dims(dtype, d, b);
+  if (st != BHA_OK) return st;
+  if (dtype != BHA_BF16) return BHA_ERR_UNSUPPORTED;
+  if (n < 0 || hq < 1 || hkv < 1 || hq % hkv != 0 || P < 0 || cap < P || k < 0)
+    return BHA_ERR_INVALID_ARG;
+  if (static_cast<long long>(hq) * b > 8192) return BHA_ERR_UNSUPPORTED;   // selection scratch
+  if (n == 0) return BHA_OK;
+  if (Qa == nullptr || Ka == nullptr || Va == nullptr || Y == nullptr || O_pre == nullptr ||
+      L_pre == nullptr || (P > 0 && (Kc == nullptr || Vc == nullptr)))
+    return BHA_ERR_INVALID_ARG;
+  if (misaligned(Qa) || misaligned(Qprev) || misaligned(Kc) || misaligned(Vc) ||
+      misaligned(Ka) || misaligned(Va) || misaligned(Y) || misaligned(O_pre) ||
+      misaligned(L_pre) || misaligned4(active) || misaligned(workspace))
+    return BHA_ERR_MISALIGNED;
+  const size_t es = esize(dtype);
+  const size_t q_bytes = static_cast<size_t>(n) * hq * b * d * es;
+  const size_t kv_bytes = static_cast<size_t>(n) * hkv * b * d * es;
+  const size_t c_bytes = static_cast<size_t>(n) * hkv * cap * d * es;
+  const size_t o_bytes = static_cast<size_t>(n) * hq * b * d * 4;
+  const size_t l_bytes = static_cast<size_t>(n) * hq * b * 4;
+  const bool selects = Qprev != nullptr && k > 0 && k < b;
+  const size_t a_bytes = selects && active != nullptr ? static_cast<size_t>(n) * k * 4 : 0;
+  const void* ins[6] = {Qa, Qprev, Ka, Va, Kc, Vc};
+  const size_t in_bytes[6] = {q_bytes, Qprev ? q_bytes : 0, kv_bytes, kv_bytes,
+                              P > 0 ? c_bytes : 0, P > 0 ? c_bytes : 0};
+  const void* outs[4] = {Y, O_pre, L_pre, a_bytes ? active : nullptr};
+  const size_t out_bytes[4] = {q_bytes, o_bytes, l_bytes, a_bytes};
+  for (int o = 0; o < 4; ++o) {
+    for (int i = 0; i < 6; ++i)
+      if (overlap(outs[o], out_bytes[o], ins[i], in_bytes[i])) return BHA_ERR_INVALID_ARG;
+    for (int o2 = o + 1; o2 < 4; ++o2)
+      if (overlap(outs[o], out_bytes[o], outs[o2], out_bytes[o2])) return BHA_ERR_INVALID_ARG;
+  }
+  const size_t need = bha_prefix_softmax_reuse_workspace_size(n, hq, hkv, b, d, P, k, dtype);
+  if (need > 0 && (workspace == nullptr || workspace_bytes < need)) return BHA_ERR_WORKSPACE;
+  if (need > 0) {
+    for (int i = 0; i < 6; ++i)
+      if (overlap(workspace, need, ins[i], in_bytes[i])) return BHA_ERR_INVALID_ARG;
+    for (int o = 0; o < 4; ++o)
+      if (overlap(workspace, need, outs[o], out_bytes[o])) return BHA_ERR_INVALID_ARG;
+  }
+  Ctx c;
+  st = make_ctx(stream, dtype, &c);
+  if (st != BHA_OK) return st;
+  return launch_status(launch_prefix_reuse_bf16(c, Qa, Qprev, Kc, Vc, P, cap, Ka, Va, Y, O_pre,
+                                                L_pre, active, k, n, hq, hkv, b,
+                                                resolve_scale(scale, d), workspace,
+                                                workspace_bytes));
+}
+
 size_t bha_prefix_softmax_paged_workspace_size(int n, int hq, int hkv, int b, int d,
                                                int max_pages, int page_size, bha_dtype dtype) {
   if (dtype != BHA_BF16 || n <= 0 || hq <= 0 || hkv <= 0 || hq % hkv != 0 || b < 1 || b > 64 ||

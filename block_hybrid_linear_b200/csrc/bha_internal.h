@@ -123,4 +123,23 @@ int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* 
                        int cap, const void* K, const void* V, void* Y, int n, int hq, int hkv,
                        int b, float scale, void* ws, size_t ws_bytes);
 
+// ---- reuse of prefix attention for stable tokens (bf16, d = 128) ----
+// Chunking of the reuse path's prefix pass (cache tiles only).
+void prefix_only_plan(int units, int rows, int P, int* splits, int* tiles_per);
+// The exact path's kernel over the cache alone for `rows` packed query rows
+// per unit (Q [units][rows][128]): every chunk's numerators, row max (log2
+// units) and row sum to wsO [items][128][128] / wsML [items][256]; P > 0.
+int launch_prefix_partials_bf16(const Ctx& c, const void* Q, int rows, const void* Kc,
+                                const void* Vc, int P, int cap, int units, int hkv, float scale,
+                                float* wsO, float* wsML);
+// Block attention of every query row merged with its cached prefix part.
+int launch_reuse_block_bf16(const Ctx& c, const void* Q, const void* K, const void* V,
+                            const float* O_pre, const float* L_pre, void* Y, int n, int hq,
+                            int hkv, int b, float scale);
+size_t reuse_bf16_workspace(int n, int hq, int hkv, int b, int P, int k, int have_prev);
+int launch_prefix_reuse_bf16(const Ctx& c, const void* Q, const void* Qprev, const void* Kc,
+                             const void* Vc, int P, int cap, const void* K, const void* V,
+                             void* Y, float* O_pre, float* L_pre, int* active, int k, int n,
+                             int hq, int hkv, int b, float scale, void* ws, size_t ws_bytes);
+
 }  // namespace bha

@@ -82,6 +82,7 @@ struct PrefixArgs {
   int splits;
   int tiles_per;
   float sl2;         // scale * log2(e)
+  int prefix_only;   // reuse path: cache tiles only (no block tile), partials always
 };
 
 __device__ __forceinline__ bool warp_all(bool v) { return __all_sync(0xffffffffu, v); }
@@ -158,7 +159,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int nreq = u / a.hkv, g = u % a.hkv;
   const int P = PAGED ? min(max(__ldg(a.P_lens + nreq), 0), a.Pmax) : a.P;
   const int ncache_tiles = PAGED ? (P + kTK - 1) / kTK : a.ncache_tiles;
-  const int nt = planned ? max(0, min(nt_plan, ncache_tiles + 1 - tile0)) : 0;
+  const int key_tiles = ncache_tiles + (a.prefix_only ? 0 : 1);
+  const int nt = planned ? max(0, min(nt_plan, key_tiles - tile0)) : 0;
   // false for a chunk past a paged request's cache, or past the plan's pieces
   const bool live = nt > 0;
   // pieces of this unit row: one writes Y directly, more write partials
@@ -167,6 +169,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     const int L = __ldcg(a.hdr);
     npieces = min(a.splits, (ncache_tiles + 1 + L - 1) / L);
   }
+  // the reuse path's prefix pass hands every chunk to its merge as a partial
+  const bool direct = npieces == 1 && !a.prefix_only;
   const int slot = umt * a.splits + sp;   // partial numerator slot
 
   if (tid == 0 && live) {
@@ -267,7 +271,37 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int r = (warp & 3) * 32 + lane;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   bool ok = true;
-  if (warp >= 4 && live) {
+  // a warp whose 32 query rows are all past the tile's valid rows (a ragged
+  // last query tile, the reuse path's packed active rows) computes no
+  // softmax: it keeps the barrier protocol and (paged) its share of clearing
+  // the V rows past the cache, which every output row's P V reads
+  const bool rows_live = mt * 128 + (warp & 3) * 32 < a.rows;
+  if (warp >= 4 && live && !rows_live) {
+    for (int i = 0; i < nt; ++i) {
+      const int st = i & 1;
+      const int gi = tile0 + i;
+      if (i > 0) {
+        ok = warp_all(ok && mbar_wait(bar_pv, (i - 1) & 1, a.err, abort_flag));
+        if (!ok) break;
+      }
+      if (PAGED && gi < ncache_tiles && P - gi * kTK < kTK) {
+        ok = warp_all(ok && mbar_wait(bar_vf + 8 * st, (i >> 1) & 1, a.err, abort_flag));
+        if (!ok) break;
+        if (r >= P - gi * kTK && r < kTK) {
+          const uint32_t vrow = base + kOffV + st * kTileBytes + r * 128;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            st_shared_v4(vrow + q * 16, 0u, 0u, 0u, 0u);
+            st_shared_v4(vrow + kBox + q * 16, 0u, 0u, 0u, 0u);
+          }
+        }
+        fence_proxy_async_smem();
+      }
+      tc_fence_before();
+      mbar_arrive(bar_pf);
+    }
+    if (ok && nt > 0) ok = warp_all(mbar_wait(bar_pv, (nt - 1) & 1, a.err, abort_flag));
+  } else if (warp >= 4 && live) {
     for (int i = 0; i < nt; ++i) {
       const int st = i & 1;
       const int gi = tile0 + i;
@@ -352,7 +386,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     if (ok && nt > 0) ok = warp_all(mbar_wait(bar_pv, (nt - 1) & 1, a.err, abort_flag));
     tc_fence_after();
     if (ok) {
-      if (npieces == 1) {
+      if (direct) {
         const float inv = 1.f / l;
 #pragma unroll 1
         for (int cc = 0; cc < 4; ++cc) {
@@ -389,7 +423,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   tc_fence_before();
   __syncthreads();
   if (tid == 0 && live && !*abort_flag) {
-    if (npieces == 1) {
+    if (direct) {
       tma_store_3d(&tmY, base + kOffQ, 0, mt * 128, u);
       tma_store_3d(&tmY, base + kOffQ + 16384, 64, mt * 128, u);
     } else {
@@ -571,9 +605,10 @@ void prefix_plan_paged(int P, int* splits, int* tiles_per) {
 // that is not chunk partials (64 KB numerator + row statistics, written and
 // read back, per chunk).  Depends only on the shapes, so the workspace query
 // and the launch agree.
-void prefix_plan(int units, int mtiles, int P, int* splits, int* tiles_per) {
+void prefix_plan(int units, int mtiles, int P, int* splits, int* tiles_per,
+                 int block_tiles = 1) {
   constexpr double kSlots = 296.0;
-  const int ntot = (P + kTK - 1) / kTK + 1;
+  const int ntot = (P + kTK - 1) / kTK + block_tiles;
   const int items = units * mtiles;
   const int cap = (ntot + kMinTilesPerChunk - 1) / kMinTilesPerChunk;
   const double unit_bytes = static_cast<double>(ntot) * kTK * kD * 2 * 2;   // K and V
@@ -714,6 +749,7 @@ int launch_prefix_impl(const Ctx& c, const void* Q, const void* Kc, const void* 
   a.splits = splits;
   a.tiles_per = tp;
   a.sl2 = scale * 1.4426950408889634f;
+  a.prefix_only = 0;
   int rc;
   if (planned) {
     const PlanArgs pa{pg->P_lens, n, hkv * mtiles, P, splits, 2 * c.sm_count,
@@ -753,6 +789,53 @@ int launch_prefix_impl(const Ctx& c, const void* Q, const void* Kc, const void* 
 }
 
 }  // namespace
+
+// The reuse path's prefix pass: `rows` packed query rows per unit, the cache
+// only (no block tile), every chunk a partial (wsO, wsML), P > 0.
+void prefix_only_plan(int units, int rows, int P, int* splits, int* tiles_per) {
+  prefix_plan(units, (rows + 127) / 128, P, splits, tiles_per, 0);
+}
+
+int launch_prefix_partials_bf16(const Ctx& c, const void* Q, int rows, const void* Kc,
+                                const void* Vc, int P, int cap, int units, int hkv, float scale,
+                                float* wsO, float* wsML) {
+  const int mtiles = (rows + 127) / 128;
+  int splits, tp;
+  prefix_only_plan(units, rows, P, &splits, &tp);
+  const size_t items = static_cast<size_t>(units) * mtiles * splits;
+  CUtensorMap tq, tkc, tvc, to;
+  bool ok = bf16_rows_tmap(&tq, Q, rows, rows, units, 128) &&
+            bf16_rows_tmap(&tkc, Kc, P, cap, units, kTK) &&
+            bf16_rows_tmap(&tvc, Vc, P, cap, units, kTK);
+  const uint64_t dims[3] = {(uint64_t)kD, (uint64_t)kD, items};
+  const uint64_t strides[2] = {kD * 4ull, (uint64_t)kD * kD * 4ull};
+  const uint32_t box[3] = {32, 128, 1};
+  ok = ok && encode_tmap(&to, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, wsO, dims, strides, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return -5;
+  PrefixArgs a = {};
+  a.err = c.dev_err;
+  a.hkv = hkv;
+  a.Pmax = P;
+  a.wsO = wsO;
+  a.wsML = wsML;
+  a.rows = rows;
+  a.mtiles = mtiles;
+  a.P = P;
+  a.b = 0;
+  a.ncache_tiles = (P + kTK - 1) / kTK;
+  a.splits = splits;
+  a.tiles_per = tp;
+  a.sl2 = scale * 1.4426950408889634f;
+  a.prefix_only = 1;
+  static Prepared prepared;
+  if (!prepare_kernel(c, k_prefix_bf16<false>, (int)kSmem, prepared)) return -5;
+  // the block maps are never read (no block tile) and Y is never written
+  return launch_pdl(k_prefix_bf16<false>, (unsigned)items, kThreads, kSmem, c.stream, tq, tkc,
+                    tvc, tkc, tvc, tq, to, a)
+             ? -5
+             : 0;
+}
 
 int launch_prefix_bf16(const Ctx& c, const void* Q, const void* Kc, const void* Vc, int P,
                        int cap, const void* K, const void* V, void* Y, int n, int hq, int hkv,

@@ -66,6 +66,7 @@ constexpr float kSharedShiftLog2 = 92.f;
 
 struct StepArgs {
   const float* z;     // [units][128] (shared mode)
+  const float* lpre;  // reuse: [units][rows] cached prefix log-normalisers (natural log)
   float* zc;          // [units][128] updated by the fused commit, or null
   int* err;           // device error word
   int hkv;            // KV heads (unit u uses W[u % hkv])
@@ -103,7 +104,7 @@ __device__ __forceinline__ float z_at(float4 zl, int k) {
 // phi(q_r) . z (the shared denominator's term); lane l holds z[4l .. 4l+3].
 template <int FMAP, bool QZ>
 __device__ __forceinline__ float write_phiq(uint32_t qtile, int r, uint32_t tcol, float4 zl) {
-  float qz = 0.f;
+  float qz[4] = {0.f, 0.f, 0.f, 0.f};   // four independent partial sums
 #pragma unroll
   for (int cg = 0; cg < 4; ++cg) {
     float f[32];
@@ -118,15 +119,15 @@ __device__ __forceinline__ float write_phiq(uint32_t qtile, int r, uint32_t tcol
         f[8 * q + 2 * e] = __uint_as_float(p2 << 16);
         f[8 * q + 2 * e + 1] = __uint_as_float(p2 & 0xFFFF0000u);
       }
-      if (QZ) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) qz = fmaf(f[8 * q + e], z_at(zl, cg * 32 + 8 * q + e), qz);
-      }
     }
     tmem_st32(tcol + cg * 32, f);
+    if (QZ) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) qz[e & 3] = fmaf(f[e], z_at(zl, cg * 32 + e), qz[e & 3]);
+    }
   }
   tmem_wait_st();
-  return qz;
+  return (qz[0] + qz[1]) + (qz[2] + qz[3]);
 }
 
 // Projected map: the Q W_g product sits in TMEM (this thread's lane, 128
@@ -134,21 +135,22 @@ __device__ __forceinline__ float write_phiq(uint32_t qtile, int r, uint32_t tcol
 // phi(q_r) . z (z spread over the lanes as for write_phiq).
 template <bool QZ>
 __device__ __forceinline__ float relu_tmem_phiq(uint32_t tcol, float4 zl) {
-  float qz = 0.f;
+  // the same four partial sums, in the same order, as write_phiq
+  float qz[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
   for (int cg = 0; cg < 4; ++cg) {
     float f[32];
     tmem_ld32_sync(tcol + cg * 32, f);
 #pragma unroll
     for (int q = 0; q < 32; ++q) f[q] = fmaxf(f[q], 0.f);
+    tmem_st32(tcol + cg * 32, f);
     if (QZ) {
 #pragma unroll
-      for (int q = 0; q < 32; ++q) qz = fmaf(f[q], z_at(zl, cg * 32 + q), qz);
+      for (int q = 0; q < 32; ++q) qz[q & 3] = fmaf(f[q], z_at(zl, cg * 32 + q), qz[q & 3]);
     }
-    tmem_st32(tcol + cg * 32, f);
   }
   tmem_wait_st();
-  return qz;
+  return (qz[0] + qz[1]) + (qz[2] + qz[3]);
 }
 
 // Shared denominator: this thread's row of phi(Q) in TMEM times s.
@@ -183,13 +185,22 @@ __device__ __forceinline__ void scale_tmem_row(uint32_t tcol, float s) {
 // both.  This doubles the CTAs of a grid that would leave most SMs idle.
 // With the fused commit each CTA adds its half of phi(K)^T V to S, and the
 // first of the pair adds the block's sum of phi(k) to z.
-template <int BPAD, bool SHARED, bool COMMIT, int FMAP, bool HALF>
+// REUSE (the exact path with reuse for stable tokens, LoSA page, cache
+// reuse and technical details): the "state" tile is this 128-row tile's
+// cached prefix outputs O_pre (fp32, one row per query row, normalised) and
+// no phi(Q) S product runs; the row owners also compute the block's
+// log-normaliser and, with the row's cached prefix log-normaliser, the
+// online-softmax weights a, b (a + b = 1), and the epilogue writes
+// y = a (P V) + b O_pre.
+template <int BPAD, bool SHARED, bool COMMIT, int FMAP, bool HALF, bool REUSE = false>
 __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     k_step_bf16(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmS,
                 const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmW,
                 const StepArgs a) {
   static_assert(!(SHARED && COMMIT), "the fused commit runs in the default mode only");
+  static_assert(!(REUSE && (SHARED || COMMIT || FMAP != kFmapRelu)),
+                "the reuse block pass has no state, commit or feature map");
   constexpr bool PROJ = FMAP == kFmapReluProj;
   static_assert(!(HALF && PROJ), "column halves: elementwise maps only");
   constexpr int kN = HALF ? 64 : 128;                   // output columns of this CTA
@@ -205,6 +216,9 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   const int item = HALF ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int u = item / a.mtiles, mt = item % a.mtiles;
   const int g = u % a.hkv;
+  // first row of this tile in the state-shaped operand: the d x d state, or
+  // (reuse) this tile's rows of the cached prefix outputs
+  const int srow0 = REUSE ? mt * kMT : 0;
 
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -213,9 +227,13 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   const uint32_t bar_q = ctrl, bar_k = ctrl + 8, bar_v = ctrl + 16, bar_s = ctrl + 24,
                  bar_sc = ctrl + 56, bar_p = ctrl + 64, bar_a = ctrl + 72, bar_done = ctrl + 80,
                  bar_phik = ctrl + 96, bar_ds = ctrl + 104, bar_w = ctrl + 112,
-                 bar_qw = ctrl + 120, bar_kwr = ctrl + 128, bar_a2 = ctrl + 136;
+                 bar_qw = ctrl + 120, bar_kwr = ctrl + 128, bar_a2 = ctrl + 136,
+                 bar_qz = ctrl + 144;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 88);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 92);
+  // shared denominator: set by a row owner whose row scales its phi(q) (row
+  // max past the shift bound), before it arrives on bar_p
+  volatile int* rescale_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 152);
 
   if (warp == 0) {
     if (lane == 0) {
@@ -226,7 +244,11 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       mbar_init(bar_sc, 1);
       mbar_init(bar_p, 128);
       mbar_init(bar_a, 128);
-      if (SHARED) mbar_init(bar_a2, 128);
+      if (SHARED) {
+        mbar_init(bar_a2, 128);
+        mbar_init(bar_qz, 128);
+        *rescale_flag = 0;
+      }
       mbar_init(bar_done, 1);
       if (COMMIT) {
         mbar_init(bar_phik, 128);
@@ -251,11 +273,13 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         if (!HALF || vb == half) tma_prefetch_l2_3d(&tmV, 64 * vb, 0, u);
       for (int c = 0; c < 4; ++c)
         for (int nb = 0; nb < 4; ++nb)
-          if (!HALF || (nb >> 1) == half) tma_prefetch_l2_3d(&tmS, 32 * nb, 32 * c, u);
+          if (!HALF || (nb >> 1) == half) tma_prefetch_l2_3d(&tmS, 32 * nb, srow0 + 32 * c, u);
       if (PROJ) {
         tma_prefetch_l2_3d(&tmW, 0, 0, g);
         tma_prefetch_l2_3d(&tmW, 64, 0, g);
       }
+      if (SHARED)
+        for (int l = 0; l < 4; ++l) prefetch_l2(a.z + static_cast<size_t>(u) * kD + 32 * l);
     }
     __syncwarp();
     tmem_alloc(smem_u32(tmem_slot), 256);
@@ -285,8 +309,8 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
 #pragma unroll
       for (int nn = 0; nn < kN / 32; ++nn) {
         const int nb = HALF ? 2 * half + nn : nn;
-        tma_load_3d(base + kOffS + c * kChunkS + nn * 4096, &tmS, bar_s + 8 * c, 32 * nb, 32 * c,
-                    u);
+        tma_load_3d(base + kOffS + c * kChunkS + nn * 4096, &tmS, bar_s + 8 * c, 32 * nb,
+                    srow0 + 32 * c, u);
       }
     }
   };
@@ -320,7 +344,13 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   }
 
   float beta = 1.f;   // per-row output scale (shared denominator only)
-  if (warp < 4) {
+  // reuse: the row's weights of P V and of its cached prefix output
+  float ralpha = 1.f, rbeta = 0.f;
+  if (REUSE && warp < 4) {
+    // only the cached prefix rows to request, once Q has landed
+    const bool okq = warp_all(mbar_wait(bar_q, 0, a.err, abort_flag));
+    if (okq && lane == 0) load_state_chunks(warp, warp + 1);
+  } else if (warp < 4) {
     // phi(q) for row r = 32 w + lane into TMEM as soon as Q has landed, in
     // parallel with the score MMA and the softmax (and phi(q) . z)
     // z (shared denominator), four values a lane, requested before Q lands
@@ -340,10 +370,15 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       if (okf && lane == 0) load_state_chunks(warp, warp + 1);
       if (okf) qz = write_phiq<FMAP, SHARED>(base + kOffQ, warp * 32 + lane, t_a + lane_base, zl);
     }
-    if (SHARED && okf && (PROJ || warp_all(mbar_wait(bar_sc, 0, a.err, abort_flag))))
-      st_shared_f32(base + kOffQ + tid * 128, qz);
     tc_fence_before();
-    mbar_arrive(bar_a);
+    mbar_arrive(bar_a);   // phi(Q) is in TMEM
+    if (SHARED) {
+      // phi(q) . z to the row owners, over row tid of the Q tile once the
+      // score MMA (or, projected, Q W_g) has read it
+      if (okf && (PROJ || warp_all(mbar_wait(bar_sc, 0, a.err, abort_flag))))
+        st_shared_f32(base + kOffQ + tid * 128, qz);
+      mbar_arrive(bar_qz);
+    }
     if (COMMIT && PROJ) {
       // thread = feature r: row r of (K W_g)^T (landed with Q W_g) out of
       // TMEM, which P V may then overwrite; ReLU, bf16, z, and row r of
@@ -405,6 +440,11 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   if (warp >= 4) {
     // ---- row owners: thread = query row r of the tile = TMEM lane r
     const int r = (warp - 4) * 32 + lane;
+    // reuse: the row's cached prefix log-normaliser (rows past the unit's:
+    // none), read before the scores land
+    float lp2 = -INFINITY;
+    if (REUSE && mt * kMT + r < a.rows)
+      lp2 = __ldg(a.lpre + static_cast<size_t>(u) * a.rows + mt * kMT + r) * 1.4426950408889634f;
     if (tid == 128) {
       if (mbar_wait(bar_q, 0, a.err, abort_flag) && mbar_wait(bar_k, 0, a.err, abort_flag)) {
         tc_fence_after();
@@ -480,8 +520,19 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         m2 = m * a.scale_log2;
         pscale = m2 > kSharedShiftLog2 ? 1.f : exp2f(m2);
         lsum = l;
+        if (m2 > kSharedShiftLog2) *rescale_flag = 1;   // before this row's bar_p arrive
       } else {
         pscale = 1.f / l;   // default: P is normalised, the terms add as they are
+      }
+      if (REUSE) {
+        // online-softmax merge of the block part (log2-normaliser lb2) with
+        // the cached prefix part (lp2): y = wb/(wp+wb) o_b + wp/(wp+wb) o_p
+        const float lb2 = m * a.scale_log2 + __log2f(l);
+        const float M2 = fmaxf(lp2, lb2);
+        const float wp = exp2f(lp2 - M2), wb = exp2f(lb2 - M2);
+        const float inv = 1.f / (wp + wb);
+        ralpha = wb * inv;
+        rbeta = wp * inv;
       }
       // P row r (K-major, swizzle width = row bytes); over the Q tile only
       // once phi(Q) has been read out of it
@@ -521,28 +572,13 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       }
     }
 
-    if (SHARED) {
-      // phi(q) . z from warps 0-3; the output's 1 / denominator, and for rows
-      // past the shift bound the factor e^{-m_s} into their phi(q)
-      const bool oka = warp_all(ok && mbar_wait(bar_a, 0, a.err, abort_flag));
-      tc_fence_after();
-      if (oka) {
-        const float qz = ld_shared_f32(base + kOffQ + r * 128);
-        if (m2 > kSharedShiftLog2) {
-          ascale = exp2f(-m2);
-          beta = 1.f / (lsum + ascale * qz);
-        } else {
-          beta = 1.f / (pscale * lsum + qz);
-        }
-        if (__any_sync(0xffffffffu, ascale != 1.f)) scale_tmem_row(t_a + lane_base, ascale);
-      }
-      tc_fence_before();
-      mbar_arrive(bar_a2);
-    }
-
-    if (tid == 128) {
-      // then the per-chunk phi(Q) S products
-      if (ok2) ok2 = mbar_wait(SHARED ? bar_a2 : bar_a, 0, a.err, abort_flag);
+    // the phi(Q) S products: issued right after P V unless (shared
+    // denominator) a row of the tile has to scale its phi(q) first, in which
+    // case they follow the row owners' shared-denominator work (bar_a2)
+    bool rescale = false;
+    if (SHARED && tid == 128 && ok2) rescale = *rescale_flag != 0;
+    auto issue_products = [&]() {
+      if (ok2) ok2 = mbar_wait(SHARED && rescale ? bar_a2 : bar_a, 0, a.err, abort_flag);
       for (int c = 0; c < 4 && ok2; ++c) {
         ok2 = mbar_wait(bar_s + 8 * c, 0, a.err, abort_flag);
         if (!ok2) break;
@@ -558,6 +594,35 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         }
       }
       if (ok2) mma_commit(bar_done);
+    };
+    if (!REUSE && tid == 128 && !rescale) issue_products();
+
+    if (SHARED) {
+      // phi(q) . z from warps 0-3; the output's 1 / denominator, and for rows
+      // past the shift bound the factor e^{-m_s} into their phi(q)
+      const bool oka = warp_all(ok && mbar_wait(bar_qz, 0, a.err, abort_flag));
+      tc_fence_after();
+      if (oka) {
+        const float qz = ld_shared_f32(base + kOffQ + r * 128);
+        if (m2 > kSharedShiftLog2) {
+          ascale = exp2f(-m2);
+          beta = 1.f / (lsum + ascale * qz);
+        } else {
+          beta = 1.f / (pscale * lsum + qz);
+        }
+        if (__any_sync(0xffffffffu, ascale != 1.f)) scale_tmem_row(t_a + lane_base, ascale);
+        // the row's 1 / denominator for warps 0-3 (the other column half),
+        // beside phi(q) . z in the row's bytes of the consumed Q tile
+        if (!HALF) st_shared_f32(base + kOffQ + r * 128 + 4, beta);
+      }
+      tc_fence_before();
+      mbar_arrive(bar_a2);
+    }
+
+    if (REUSE && tid == 128) {
+      if (ok2) mma_commit(bar_done);   // P V is the whole product
+    } else if (tid == 128) {
+      if (rescale) issue_products();
       if (COMMIT && ok2) {
         // phi(K)^T V over the block's tokens into the columns phi(Q) used,
         // once the products that read them are complete
@@ -588,21 +653,56 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   const int hb = warp >> 2;
   const bool okd = warp_all(mbar_wait(bar_done, 0, a.err, abort_flag));
   tc_fence_after();
-  if (SHARED) {
-    // row scales from the row owners to the other column half, through the
-    // (consumed) V tile
+  if (SHARED && !HALF) {
+    // warps 0-3 take their rows' 1 / denominator from the row owners (bar_a2:
+    // the row owners are done with the Q tile's half these warps overwrite);
+    // each column half then finishes on its own
+    if (warp < 4) {
+      const bool okb = warp_all(mbar_wait(bar_a2, 0, a.err, abort_flag));
+      beta = okb ? ld_shared_f32(base + kOffQ + r * 128 + 4) : 1.f;
+    }
+  } else if (SHARED) {
+    // column halves: both halves share each row's swizzled staging bytes, so
+    // the row scales go through the (consumed) V tile and a CTA barrier
     float* rs = reinterpret_cast<float*>(smem_raw + (base - raw) + Lay::kOffV);
     if (warp >= 4) rs[r] = beta;
     named_barrier_sync(1, kThreads);
     beta = rs[r];
   }
+  bool oko = true;
+  if (REUSE) {
+    // the merge weights likewise, and this warp's rows of O_pre in place
+    float* rs = reinterpret_cast<float*>(smem_raw + (base - raw) + Lay::kOffV);
+    if (warp >= 4) {
+      rs[r] = ralpha;
+      rs[kMT + r] = rbeta;
+    }
+    named_barrier_sync(1, kThreads);
+    ralpha = rs[r];
+    rbeta = rs[kMT + r];
+    oko = warp_all(mbar_wait(bar_s + 8 * (warp & 3), 0, a.err, abort_flag));
+  }
+  // reuse: y = a D + b O_pre for the 32 columns of D in `acc` whose first
+  // column is the start of 32 x 32 box `box` of the O_pre tile (row r)
+  auto blend = [&](float (&acc)[32], uint32_t box) {
+    const uint32_t ob = box + (r & 31) * 128;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float4 lo = ld_shared_f4(ob + ((j ^ (r & 3)) << 5));
+      const float4 hi = ld_shared_f4(ob + ((j ^ (r & 3)) << 5) + 16);
+      const float o[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) acc[8 * j + q] = fmaf(ralpha, acc[8 * j + q], rbeta * o[q]);
+    }
+  };
   if (HALF) {
     // warp w: rows 32(w%4).., columns 32(w/4).. of the CTA's 64; one SW128
     // box in the (consumed) Q region, one TMA store
-    if (okd) {
+    if (okd && oko) {
       const uint32_t row = base + kOffQ + r * 128;
       float acc[32];
       tmem_ld32_sync(t_d + lane_base + hb * 32, acc);
+      if (REUSE) blend(acc, base + kOffS + (r >> 5) * kChunkS + hb * 4096);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int j = hb * 4 + q;
@@ -621,13 +721,14 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       bulk_commit_group();
     }
   } else {
-  if (okd) {
+  if (okd && oko) {
     // bf16 tile of this 64-column half -> the (consumed) Q region, SW128
     const uint32_t row = base + kOffQ + hb * 16384 + r * 128;
 #pragma unroll
     for (int cc = 0; cc < 2; ++cc) {
       float acc[32];
       tmem_ld32_sync(t_d + lane_base + hb * 64 + cc * 32, acc);
+      if (REUSE) blend(acc, base + kOffS + (r >> 5) * kChunkS + (hb * 2 + cc) * 4096);
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int j = cc * 4 + q;
@@ -692,10 +793,10 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   if ((tid & 127) == 0) bulk_wait_group_read0();   // shared memory stays until read
 }
 
-template <int BPAD, bool SHARED, bool COMMIT, int FMAP, bool HALF = false>
+template <int BPAD, bool SHARED, bool COMMIT, int FMAP, bool HALF = false, bool REUSE = false>
 int launch_cfg(const Ctx& c, const CUtensorMap (&tm)[6], const StepArgs& a, int grid) {
   using Lay = StepLayout<BPAD>;
-  auto kern = k_step_bf16<BPAD, SHARED, COMMIT, FMAP, HALF>;
+  auto kern = k_step_bf16<BPAD, SHARED, COMMIT, FMAP, HALF, REUSE>;
   static Prepared prepared;
   if (!prepare_kernel(c, kern, (int)Lay::kSmem, prepared)) return -5;
   return launch_pdl(kern, (HALF ? 2 : 1) * grid, kThreads, Lay::kSmem, c.stream, tm[0], tm[1],
@@ -774,6 +875,7 @@ int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, 
 
   StepArgs a;
   a.z = z;
+  a.lpre = nullptr;
   a.zc = commit ? commit_z : nullptr;
   a.err = c.dev_err;
   a.hkv = hkv;
@@ -787,6 +889,65 @@ int launch_step_bf16(const Ctx& c, const void* Q, const void* K, const void* V, 
     case 16: return launch_bpad<16>(c, tm, a, grid, shared, commit, fmap);
     case 32: return launch_bpad<32>(c, tm, a, grid, shared, commit, fmap);
     default: return launch_bpad<64>(c, tm, a, grid, shared, commit, fmap);
+  }
+}
+
+// The reuse path's block pass: every query row's attention over the active
+// block, merged with its cached prefix part (O_pre [units][rows][128] fp32,
+// L_pre [units][rows] natural-log normalisers; rows = G * b).
+int launch_reuse_block_bf16(const Ctx& c, const void* Q, const void* K, const void* V,
+                            const float* O_pre, const float* L_pre, void* Y, int n, int hq,
+                            int hkv, int b, float scale) {
+  const int G = hq / hkv;
+  const int rows = G * b;
+  const int units = n * hkv;
+  const int bpad = b <= 16 ? 16 : (b <= 32 ? 32 : 64);
+  const int mtiles = (rows + kMT - 1) / kMT;
+  CUtensorMap tm[6];
+  const uint64_t dq[3] = {(uint64_t)kD, (uint64_t)rows, (uint64_t)units};
+  const uint64_t sq[2] = {kD * 2ull, (uint64_t)rows * kD * 2ull};
+  const uint32_t bq[3] = {64, kMT, 1};
+  const uint64_t dk[3] = {(uint64_t)kD, (uint64_t)b, (uint64_t)units};
+  const uint64_t sk[2] = {kD * 2ull, (uint64_t)b * kD * 2ull};
+  const uint32_t bk[3] = {64, (uint32_t)bpad, 1};
+  const uint64_t dob[3] = {(uint64_t)kD, (uint64_t)rows, (uint64_t)units};
+  const uint64_t sob[2] = {kD * 4ull, (uint64_t)rows * kD * 4ull};
+  const uint32_t bob[3] = {32, 32, 1};
+  if (!encode_tmap(&tm[0], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Q, dq, sq, bq,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&tm[4], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, Y, dq, sq, bq,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&tm[1], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, K, dk, sk, bk,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&tm[2], CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, V, dk, sk, bk,
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !encode_tmap(&tm[3], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, O_pre, dob, sob, bob,
+                   CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B))
+    return -5;
+  tm[5] = tm[0];
+  StepArgs a;
+  a.z = nullptr;
+  a.lpre = L_pre;
+  a.zc = nullptr;
+  a.err = c.dev_err;
+  a.hkv = hkv;
+  a.rows = rows;
+  a.b = b;
+  a.mtiles = mtiles;
+  a.scale = scale;
+  a.scale_log2 = scale * 1.4426950408889634f;
+  const int grid = units * mtiles;
+  const bool halves = grid <= c.sm_count;
+  switch (bpad) {
+    case 16:
+      return halves ? launch_cfg<16, false, false, kFmapRelu, true, true>(c, tm, a, grid)
+                    : launch_cfg<16, false, false, kFmapRelu, false, true>(c, tm, a, grid);
+    case 32:
+      return halves ? launch_cfg<32, false, false, kFmapRelu, true, true>(c, tm, a, grid)
+                    : launch_cfg<32, false, false, kFmapRelu, false, true>(c, tm, a, grid);
+    default:
+      return halves ? launch_cfg<64, false, false, kFmapRelu, true, true>(c, tm, a, grid)
+                    : launch_cfg<64, false, false, kFmapRelu, false, true>(c, tm, a, grid);
   }
 }
 

@@ -285,6 +285,56 @@ int bha_state_prefill_ragged(const void *K, const void *V, const int *T_lens,
                              bha_stream_t stream);
 
 /*
+ * Reuse of prefix attention for stable tokens (the LoSA page: gist.science
+ * explainer of arXiv 2604.12056, section "3. 方法论 LoSA" -- 局部性剪枝
+ * locality pruning, 缓存复用 cache reuse, 初始化策略 initialisation -- and
+ * "技术细节" technical details), applied to the exact comparison path with a
+ * dense prefix pass over the active tokens (the page's sparse selector is not
+ * part of this library).  One denoising step of a block:
+ *   1. score_i = mean over every query head h and dimension c of
+ *      (Qa[n][h][i][c] - Qprev[n][h][i][c])^2, the MSE of token i's query
+ *      since the previous denoising step (evaluated in fp64: per head the
+ *      squares summed in column order, then the heads summed in order, so
+ *      the selection is reproducible bit for bit);
+ *   2. the active set of request n: the k tokens with the largest score,
+ *      ties to the lower token index;
+ *   3. for an active token, every query head's softmax attention over the
+ *      cache alone, as its normalised output and natural-log normaliser
+ *      lse_p = log sum_{j<P} exp(scale q . k_j), replaces the token's entries
+ *      of the reuse cache (O_pre, L_pre); a stable token keeps the entries
+ *      the previous step left (computed with an earlier query);
+ *   4. y = (e^{lse_p - M} o_p + e^{lse_b - M} o_b) / (e^{lse_p - M} + e^{lse_b - M}),
+ *      M = max(lse_p, lse_b), with o_b, lse_b the token's softmax attention
+ *      over the b block tokens with its current query (P = 0: y = o_b).
+ * Qprev == NULL (the block's first denoising step, the page's dense
+ * initialisation) or k >= b makes every token active; the result is then
+ * that of bha_prefix_softmax.  k = 0 makes every token stable.
+ *   Qa, Qprev     [n][hq][b][d]     this and the previous step's queries
+ *   O_pre         [n][hq][b][d] fp32, L_pre [n][hq][b] fp32: the reuse
+ *                 cache, b x (d + 1) values per query head, read for stable
+ *                 tokens and written for active ones; it must come from the
+ *                 previous step of the same block (any contents when every
+ *                 token is active)
+ *   active        [n][k] int32 or NULL: the active tokens of each request in
+ *                 increasing order, written on steps that select (Qprev set,
+ *                 0 < k < b), untouched otherwise
+ * Other arguments as for bha_prefix_softmax.  bf16 only (BHA_F32 returns
+ * BHA_ERR_UNSUPPORTED), and hq * b <= 8192 (else BHA_ERR_UNSUPPORTED).  The workspace size covers both kinds of step (first
+ * and later) for the given k.  Y must not overlap any input or the cache;
+ * O_pre, L_pre and active must not overlap the inputs or each other.
+ */
+size_t bha_prefix_softmax_reuse_workspace_size(int n, int hq, int hkv, int b,
+                                               int d, int P, int k,
+                                               bha_dtype dtype);
+int bha_prefix_softmax_reuse(const void *Qa, const void *Qprev,
+                             const void *Kc, const void *Vc, int P, int cap,
+                             const void *Ka, const void *Va, void *Y,
+                             float *O_pre, float *L_pre, int *active, int k,
+                             int n, int hq, int hkv, int b, int d, float scale,
+                             bha_dtype dtype, void *workspace,
+                             size_t workspace_bytes, bha_stream_t stream);
+
+/*
  * Block partition of a length-L sequence into blocks of B tokens, the last
  * one possibly short (worked example: L=10, B=4 -> tokens 1-4, 5-8, 9-10).
  * Host-only.  Writes bounds[0..k] = {0, B, 2B, ..., L} and returns k, the

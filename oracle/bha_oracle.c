@@ -343,12 +343,15 @@ void oracle_losa_select(const double *Q, const double *Qprev, long n, long hq,
     for (ni = 0; ni < n; ++ni) {
         double *sc = score + ni * b;
         for (long i = 0; i < b; ++i) {
+            /* the squared change summed per head, then over the heads */
             double acc = 0.0;
             for (long h = 0; h < hq; ++h) {
                 const double *q = Q + ((ni * hq + h) * b + i) * d;
                 const double *p = Qprev + ((ni * hq + h) * b + i) * d;
+                double sh = 0.0;
                 for (long c = 0; c < d; ++c)
-                    acc += (q[c] - p[c]) * (q[c] - p[c]);
+                    sh += (q[c] - p[c]) * (q[c] - p[c]);
+                acc += sh;
             }
             sc[i] = acc / (double)(hq * d);
         }

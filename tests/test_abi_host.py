@@ -269,3 +269,48 @@ def test_ragged_prefill_validation(L):
     import torch
     if not torch.cuda.is_available():
         assert f() == _lib.BHA_ERR_CUDA
+
+
+def test_reuse_validation_and_workspace(L):
+    """bha_prefix_softmax_reuse: bf16 only, k >= 0, the cache and the active
+    list required to be disjoint from the inputs and each other, and a
+    workspace that covers both the dense first step and a selecting step."""
+    n, hq, hkv, b, d, P, k = 64, 16, 4, 32, 128, 32768, 8
+    need = L.bha_prefix_softmax_reuse_workspace_size(n, hq, hkv, b, d, P, k, _lib.BHA_BF16)
+    assert need > 0 and need % 16 == 0
+    assert L.bha_prefix_softmax_reuse_workspace_size(n, hq, hkv, b, d, P, k, _lib.BHA_F32) == 0
+    assert L.bha_prefix_softmax_reuse_workspace_size(n, hq, hkv, b, d, P, -1,
+                                                     _lib.BHA_BF16) == 0
+    # the dense first step (every token active) needs at least the exact path's partials
+    assert need >= L.bha_prefix_softmax_reuse_workspace_size(n, hq, hkv, b, d, P, 0,
+                                                             _lib.BHA_BF16)
+    big = GAP * 16
+    Qp, O, Lp, act = GAP * 7, GAP * 8, GAP * 9, GAP * 10
+
+    def f(**kw):
+        return L.bha_prefix_softmax_reuse(
+            kw.get("Q", A), kw.get("Qprev", Qp), kw.get("Kc", big), kw.get("Vc", 2 * big),
+            kw.get("P", P), kw.get("cap", P), B, C, kw.get("Y", D), kw.get("O", O),
+            kw.get("Lp", Lp), kw.get("act", act), kw.get("k", k), n, hq, hkv, b, d, 0.0,
+            kw.get("dtype", _lib.BHA_BF16), kw.get("ws", 3 * big), kw.get("ws_bytes", need),
+            None)
+    assert f(dtype=_lib.BHA_F32) == _lib.BHA_ERR_UNSUPPORTED
+    assert f(k=-1) == _lib.BHA_ERR_INVALID_ARG
+    assert f(cap=100) == _lib.BHA_ERR_INVALID_ARG
+    assert f(O=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(Lp=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(Kc=None) == _lib.BHA_ERR_INVALID_ARG
+    assert f(ws=None) == _lib.BHA_ERR_WORKSPACE
+    assert f(ws_bytes=need - 16) == _lib.BHA_ERR_WORKSPACE
+    assert f(Y=A) == _lib.BHA_ERR_INVALID_ARG         # Y aliases Q
+    assert f(Y=O) == _lib.BHA_ERR_INVALID_ARG         # Y aliases the cache
+    assert f(O=Qp) == _lib.BHA_ERR_INVALID_ARG        # the cache aliases Qprev
+    assert f(Lp=O + 64) == _lib.BHA_ERR_INVALID_ARG   # L_pre inside O_pre
+    assert f(act=Lp) == _lib.BHA_ERR_INVALID_ARG      # the list over L_pre
+    assert f(O=O + 8) == _lib.BHA_ERR_MISALIGNED
+    assert f(act=act + 2) == _lib.BHA_ERR_MISALIGNED
+    assert f(ws=big + 64) == _lib.BHA_ERR_INVALID_ARG  # workspace inside the cache
+    # without a device the valid call gets as far as the runtime
+    assert f() == _lib.BHA_ERR_CUDA
+    assert f(Qprev=None, act=None) == _lib.BHA_ERR_CUDA
+    assert f(Kc=None, Vc=None, P=0, cap=0) == _lib.BHA_ERR_CUDA

@@ -81,10 +81,13 @@ def test_source_hash_ignores_comments_only():
     assert "add one" not in bench.code_only(src) and "done" not in bench.code_only(src)
 
 
-def test_graph_schedule_runs_exactly_the_requested_cycles():
-    for steps in (0, 1, 5, 14, 15, 16, 20, 29, 30, 31, 20000):
-        full, rem = bench.graph_schedule(steps, 15)
-        assert full * 15 + rem == steps and 0 <= rem < 15
+def test_graph_plan_runs_exactly_the_requested_cycles():
+    for steps in (0, 1, 5, 14, 15, 16, 20, 29, 30, 31, 59, 60, 61, 75, 20000):
+        plan = bench.graph_plan(steps, 15)
+        assert sum(c * r for c, r in plan) == steps
+        assert len(plan) <= 2 and all(c >= 1 and r >= 1 for c, r in plan)
+    assert bench.graph_plan(20, 15) == [(20, 1)]
+    assert bench.graph_plan(61, 15) == [(15, 4), (1, 1)]
 
 
 def test_e2e_counts_follow_steps_with_a_floor():
