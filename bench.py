@@ -57,7 +57,7 @@ def parse():
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the secondary workloads in the benchmark line")
     ap.add_argument("--only", choices=["step", "step_shared", "step_commit", "commit", "prefill",
-                                       "prefix", "paged"],
+                                       "prefix", "paged", "reuse"],
                     help="launch just this kernel warmup + steps times (small case for ncu)")
     ap.add_argument("--prefix", type=int, default=8192,
                     help="prompt / cache length used by --only prefill|prefix")
@@ -592,7 +592,8 @@ def run_native(args, rank, world, local):
                          "launch_us": shared_launch_ms * 1e3,
                          "algorithmic_bytes_per_launch": shared_bytes,
                          "achieved": shared_bytes / (shared_launch_ms / 1e3) / 1e9,
-                         "frac": shared_bytes / (shared_launch_ms / 1e3) / 1e9 / peak}},
+                         "frac": shared_bytes / (shared_launch_ms / 1e3) / 1e9 / peak,
+                         "traffic": traffic_record("k_step_bf16_shared", "k_step.cu")}},
         "hbm_roofline_frac": achieved / peak,
         "step_commit": {"kernel": "k_step_bf16 (fused commit)",
                         "launch_us": commit_launch_ms * 1e3,
@@ -782,7 +783,7 @@ def run_only(args):
     Y = torch.empty_like(Q)
     S = torch.randn(nb, HKV, D_, D_, device=dev)
     z = torch.rand(nb, HKV, D_, device=dev)
-    if args.only in ("prefill", "prefix"):
+    if args.only in ("prefill", "prefix", "reuse"):
         Kp = inputs.normal_bf16_torch(1, inputs.TID_KP, (nb, HKV, P, D_), std, dev)
         Vp = inputs.normal_bf16_torch(1, inputs.TID_VP, (nb, HKV, P, D_), std, dev)
     if args.only == "prefill":
@@ -793,6 +794,18 @@ def run_only(args):
         need = bha.bha_prefix_softmax_workspace_size(nb, HQ, HKV, B_, D_, P)
         ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
         fn = lambda: bha.bha_prefix_softmax(Q, Kp, Vp, P, K, V, Y, workspace=ws)
+    elif args.only == "reuse":
+        # a selecting step (k = 8 of 32 tokens) of the exact path with reuse; the
+        # cache comes from one dense step first
+        k = 8
+        Q1 = inputs.normal_bf16_torch(2, inputs.TID_Q, (nb, HQ, B_, D_), std, dev)
+        O = torch.empty(nb, HQ, B_, D_, device=dev)
+        L = torch.empty(nb, HQ, B_, device=dev)
+        need = bha.bha_prefix_softmax_reuse_workspace_size(nb, HQ, HKV, B_, D_, P, k)
+        ws = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+        bha.bha_prefix_softmax_reuse(Q, None, Kp, Vp, P, K, V, Y, O, L, k, workspace=ws)
+        fn = lambda: bha.bha_prefix_softmax_reuse(Q1, Q, Kp, Vp, P, K, V, Y, O, L, k,
+                                                  workspace=ws)
     elif args.only == "paged":
         # the ragged workload's paged exact path (batch 64, lengths in [1, 16384])
         _, max_pages, Kpool, Vpool, tab, plen, Q, K, V = _ragged_paged_batch(nb, dev)
