@@ -564,7 +564,6 @@ int bha_prefix_softmax_reuse(const void* Qa, const void* Qprev, const void* Kc, 
                              size_t workspace_bytes, bha_stream_t stream) {
   int st = check_dims(dtype, d, b);
   if (st != BHA_OK) return st;
-  if (dtype != BHA_BF16) return BHA_ERR_UNSUPPORTED;
   if (n < 0 || hq < 1 || hkv < 1 || hq % hkv != 0 || P < 0 || cap < P || k < 0)
     return BHA_ERR_INVALID_ARG;
   if (static_cast<long long>(hq) * b > 8192) return BHA_ERR_UNSUPPORTED;   // selection scratch
@@ -606,6 +605,12 @@ int bha_prefix_softmax_reuse(const void* Qa, const void* Qprev, const void* Kc, 
   Ctx c;
   st = make_ctx(stream, dtype, &c);
   if (st != BHA_OK) return st;
+  if (dtype == BHA_F32)
+    return launch_status(launch_prefix_reuse_f32(
+        c, static_cast<const float*>(Qa), static_cast<const float*>(Qprev),
+        static_cast<const float*>(Kc), static_cast<const float*>(Vc), P, cap,
+        static_cast<const float*>(Ka), static_cast<const float*>(Va), static_cast<float*>(Y),
+        O_pre, L_pre, active, k, n, hq, hkv, b, d, resolve_scale(scale, d)));
   return launch_status(launch_prefix_reuse_bf16(c, Qa, Qprev, Kc, Vc, P, cap, Ka, Va, Y, O_pre,
                                                 L_pre, active, k, n, hq, hkv, b,
                                                 resolve_scale(scale, d), workspace,

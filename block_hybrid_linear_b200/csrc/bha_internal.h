@@ -116,6 +116,10 @@ struct PagedCache {
 int launch_prefix_paged_bf16(const Ctx& c, const void* Q, const void* Kpool, const void* Vpool,
                              const PagedCache& pg, const void* K, const void* V, void* Y, int n,
                              int hq, int hkv, int b, float scale, void* ws, size_t ws_bytes);
+int launch_prefix_reuse_f32(const Ctx& c, const float* Q, const float* Qprev, const float* Kc,
+                            const float* Vc, int P, int cap, const float* K, const float* V,
+                            float* Y, float* O_pre, float* L_pre, int* active, int k, int n,
+                            int hq, int hkv, int b, int d, float scale);
 int launch_prefix_paged_f32(const Ctx& c, const float* Q, const float* Kpool, const float* Vpool,
                             const PagedCache& pg, const float* K, const float* V, float* Y, int n,
                             int hq, int hkv, int b, int d, float scale);

@@ -233,6 +233,144 @@ __global__ void __launch_bounds__(kThreads) k_prefix_f32(
   for (int c = threadIdx.x; c < d; c += kThreads) Y[row + c] = acc[c] / l_run;
 }
 
+// The exact path with reuse for stable tokens (the LoSA page's cache reuse),
+// fp32 reference mode: one CTA per (request, head, token row).  Each CTA
+// evaluates its request's selection itself (the same fp64 nested sum and
+// ranking as the bf16 path's selection kernel), then -- if its token is active
+// (or every token is) -- its row's softmax over the cache alone (normalised
+// output and natural-log normaliser into O_pre / L_pre), else reads them from
+// there; then its attention over the b block tokens and the online-softmax
+// merge of the two.  `active` ([n][k], or null) gets the active tokens in
+// increasing order (written by the head-0 CTAs).
+__global__ void __launch_bounds__(kThreads) k_reuse_f32(
+    const float* __restrict__ Q, const float* __restrict__ Qprev, const float* __restrict__ Kc,
+    const float* __restrict__ Vc, int P, int cap, const float* __restrict__ K,
+    const float* __restrict__ V, float* __restrict__ Y, float* __restrict__ O_pre,
+    float* __restrict__ L_pre, int* __restrict__ active, int k, int hq, int hkv, int b, int d,
+    float scale) {
+  extern __shared__ double dsm[];
+  double* part = dsm;                                   // [hq * b] (selecting steps)
+  float* sq = reinterpret_cast<float*>(dsm + (Qprev ? hq * b : 0));   // [d]
+  float* se = sq + d;                                   // [kThreads]
+  float* acc = se + kThreads;                           // [d]
+  __shared__ float red[kThreads / 32];
+  __shared__ double sc[64];
+  __shared__ int is_act;
+
+  const int id = blockIdx.x;
+  const int i = id % b, nh = id / b;
+  const int ni = nh / hq, h = nh % hq, g = h / (hq / hkv);
+  const size_t row = (((size_t)ni * hq + h) * b + i) * d;
+  if (threadIdx.x == 0) is_act = 1;
+  if (Qprev != nullptr && k < b) {
+    // per (head, token) row: groups of 8 columns, then the groups, in order
+    for (int t = threadIdx.x; t < hq * b; t += kThreads) {
+      const size_t rr = ((size_t)ni * hq * b + t) * d;
+      double sh = 0.0;
+      for (int c0 = 0; c0 < d; c0 += 8) {
+        double sg = 0.0;
+        for (int c = c0; c < c0 + 8 && c < d; ++c) {
+          const double df = __dsub_rn((double)Q[rr + c], (double)Qprev[rr + c]);
+          sg = __dadd_rn(sg, __dmul_rn(df, df));
+        }
+        sh = __dadd_rn(sh, sg);
+      }
+      part[t] = sh;
+    }
+    __syncthreads();
+    if (threadIdx.x < b) {
+      double a = 0.0;
+      for (int hh = 0; hh < hq; ++hh) a = __dadd_rn(a, part[hh * b + threadIdx.x]);
+      const double s = __ddiv_rn(a, (double)hq * d);
+      sc[threadIdx.x] = s != s ? -INFINITY : s;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int rank = 0, pos = 0;
+      for (int j = 0; j < b; ++j) rank += (sc[j] > sc[i] || (sc[j] == sc[i] && j < i)) ? 1 : 0;
+      is_act = rank < k;
+      if (is_act && h == 0 && active != nullptr) {
+        for (int t = 0; t < i; ++t) {
+          int rt = 0;
+          for (int j = 0; j < b; ++j) rt += (sc[j] > sc[t] || (sc[j] == sc[t] && j < t)) ? 1 : 0;
+          pos += rt < k;
+        }
+        if (pos < k) active[(size_t)ni * k + pos] = i;
+      }
+    }
+  } else if (Qprev != nullptr && k == 0 && threadIdx.x == 0) {
+    is_act = 0;
+  }
+  for (int c = threadIdx.x; c < d; c += kThreads) sq[c] = Q[row + c];
+  __syncthreads();
+  const bool act = is_act != 0;
+  const size_t lrow = ((size_t)ni * hq + h) * b + i;
+  float lse_p;
+  if (act) {
+    const float* Kcg = Kc + ((size_t)ni * hkv + g) * cap * d;
+    const float* Vcg = Vc + ((size_t)ni * hkv + g) * cap * d;
+    for (int c = threadIdx.x; c < d; c += kThreads) acc[c] = 0.f;
+    float m_run = -INFINITY, l_run = 0.f;
+    for (int j0 = 0; j0 < P; j0 += kThreads) {
+      const int j = j0 + threadIdx.x;
+      float s = -INFINITY;
+      if (j < P) {
+        float a = 0.f;
+        for (int c = 0; c < d; ++c) a = fmaf(sq[c], Kcg[(size_t)j * d + c], a);
+        s = a * scale;
+      }
+      const float m_new = fmaxf(m_run, block_reduce_max(s, red));
+      const float e = j < P ? expf(s - m_new) : 0.f;
+      const float corr = expf(m_run - m_new);
+      se[threadIdx.x] = e;
+      l_run = l_run * corr + block_reduce_sum(e, red);
+      m_run = m_new;
+      __syncthreads();
+      const int cnt = min(kThreads, P - j0);
+      for (int c = threadIdx.x; c < d; c += kThreads) {
+        float a = acc[c] * corr;
+        for (int t = 0; t < cnt; ++t) a = fmaf(se[t], Vcg[(size_t)(j0 + t) * d + c], a);
+        acc[c] = a;
+      }
+      __syncthreads();
+    }
+    for (int c = threadIdx.x; c < d; c += kThreads) {
+      acc[c] = P > 0 ? acc[c] / l_run : 0.f;
+      O_pre[row + c] = acc[c];
+    }
+    lse_p = P > 0 ? m_run + logf(l_run) : -INFINITY;
+    if (threadIdx.x == 0) L_pre[lrow] = lse_p;
+  } else {
+    for (int c = threadIdx.x; c < d; c += kThreads) acc[c] = O_pre[row + c];
+    lse_p = L_pre[lrow];
+  }
+  __syncthreads();
+  // the block's attention with this step's query
+  const float* Kg = K + ((size_t)ni * hkv + g) * b * d;
+  const float* Vg = V + ((size_t)ni * hkv + g) * b * d;
+  float s = -INFINITY;
+  if (threadIdx.x < b) {
+    float a = 0.f;
+    for (int c = 0; c < d; ++c) a = fmaf(sq[c], Kg[(size_t)threadIdx.x * d + c], a);
+    s = a * scale;
+  }
+  const float mb = block_reduce_max(s, red);
+  const float e = threadIdx.x < b ? expf(s - mb) : 0.f;
+  const float lb = block_reduce_sum(e, red);
+  se[threadIdx.x] = e;
+  __syncthreads();
+  const float lse_b = mb + logf(lb);
+  const float M = fmaxf(lse_p, lse_b);
+  const float wp = lse_p == -INFINITY ? 0.f : expf(lse_p - M);
+  const float wb = expf(lse_b - M);
+  for (int c = threadIdx.x; c < d; c += kThreads) {
+    float ob = 0.f;
+    for (int j = 0; j < b; ++j) ob = fmaf(se[j], Vg[(size_t)j * d + c], ob);
+    ob /= lb;
+    Y[row + c] = (wp * acc[c] + wb * ob) / (wp + wb);
+  }
+}
+
 int finish_launch() {
   return cudaGetLastError() == cudaSuccess ? 0 : -5;
 }
@@ -271,6 +409,19 @@ int launch_prefix_f32(const Ctx& c, const float* Q, const float* Kc, const float
   const size_t smem = (size_t)(2 * d + kThreads) * sizeof(float);
   k_prefix_f32<<<n * hq * b, kThreads, smem, c.stream>>>(Q, Kc, Vc, P, cap, K, V, Y, hq, hkv,
                                                          b, d, scale, PagedF32{});
+  return finish_launch();
+}
+
+int launch_prefix_reuse_f32(const Ctx& c, const float* Q, const float* Qprev, const float* Kc,
+                            const float* Vc, int P, int cap, const float* K, const float* V,
+                            float* Y, float* O_pre, float* L_pre, int* active, int k, int n,
+                            int hq, int hkv, int b, int d, float scale) {
+  const size_t smem = (Qprev ? (size_t)hq * b * sizeof(double) : 0) +
+                      (size_t)(2 * d + kThreads) * sizeof(float);
+  static Prepared prepared;
+  if (!prepare_kernel(c, k_reuse_f32, 8192 * 8 + (2 * 128 + kThreads) * 4, prepared)) return -5;
+  k_reuse_f32<<<n * hq * b, kThreads, smem, c.stream>>>(Q, Qprev, Kc, Vc, P, cap, K, V, Y, O_pre,
+                                                        L_pre, active, k, hq, hkv, b, d, scale);
   return finish_launch();
 }
 

@@ -14,9 +14,9 @@
 // Launch sequence of one step (each kernel with programmatic dependent
 // launch, so every one waits for its predecessor before touching memory):
 //   k_reuse_select       one CTA per request: the locality scores (the MSE of
-//                        each token's query change over all heads, fp64, summed
-//                        in index order so that the selection is reproducible
-//                        bit for bit), the top-k active set (ties to the lower
+//                        each token's query change over all heads, fp64, a
+//                        nested sum in a fixed order so that the selection is
+//                        reproducible bit for bit), the top-k active set (ties to the lower
 //                        index), the active tokens' query rows packed per KV
 //                        head into the workspace [units][G k][128];
 //   k_prefix_bf16        (prefix-only mode) the exact path's flash kernel over
@@ -57,28 +57,21 @@ struct SelectArgs {
   int hq, hkv, b, k;
 };
 
-// 16-byte read-only global load, issued in program order (the score loop
-// requests a half row of both query sets before it uses any of it)
-__device__ __forceinline__ uint4 ldg_v4_ordered(const uint4* p) {
-  uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p)
-               : "memory");
-  return v;
-}
-
 __device__ __forceinline__ double bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ double bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // One CTA per request (kSelThreads threads, dynamic shared memory of hq * b
-// doubles).  The score of token i is evaluated as the plain nested sum --
-// per head h the squared query change summed column by column in fp64, then
-// those hq partial sums added head by head, then divided by hq * 128 -- with
-// every product and sum rounded on its own (no fused multiply-add): the same
-// operations in the same order as a straightforward loop, so equal inputs give
-// bit-identical scores wherever they are computed.  Thread t takes the
-// (head, token) rows t, t + kSelThreads, ... (token fastest).
+// doubles).  The score of token i is evaluated as a plain nested sum in fp64,
+// each level in index order and every product and sum rounded on its own (no
+// fused multiply-add): per head h and group of 8 columns, the squared query
+// change summed column by column; per head the 16 group sums; over the heads
+// the hq head sums; then divided by hq * 128.  Equal inputs give bit-identical
+// scores wherever this is computed.  A half warp takes one (head, token) row:
+// lane j of it loads columns 8j .. 8j+7 of Q and Qprev (a coalesced 256-byte
+// row per half warp) and sums its group; the half warp's lane 0 then adds the
+// 16 group sums in order.
+constexpr int kRowsPerPass = kSelThreads / 16;   // rows in flight per pass
+constexpr int kPassUnroll = 4;                   // passes whose loads issue together
 __global__ void __launch_bounds__(kSelThreads) k_reuse_select(const SelectArgs a) {
   extern __shared__ double part[];   // [hq][b] per-head sums
   __shared__ double sc[kMaxB];
@@ -88,36 +81,42 @@ __global__ void __launch_bounds__(kSelThreads) k_reuse_select(const SelectArgs a
   pdl_wait();
   const int ni = blockIdx.x, tid = threadIdx.x;
   const int b = a.b, hq = a.hq;
-  for (int t = tid; t < hq * b; t += kSelThreads) {
-    const int h = t / b, i = t % b;
-    const size_t row = (static_cast<size_t>(ni) * hq + h) * b + i;
-    const uint4* q = reinterpret_cast<const uint4*>(a.Q + row * kD);
-    const uint4* p = reinterpret_cast<const uint4*>(a.Qprev + row * kD);
-    double sh = 0.0;
+  const int rows = hq * b;
+  const int hw = tid >> 4, j = tid & 15;   // half warp = row slot, lane = column group
+  const uint4* Q4 = reinterpret_cast<const uint4*>(a.Q) + static_cast<size_t>(ni) * rows * 16;
+  const uint4* P4 = reinterpret_cast<const uint4*>(a.Qprev) + static_cast<size_t>(ni) * rows * 16;
+  for (int r0 = 0; r0 < rows; r0 += kRowsPerPass * kPassUnroll) {
+    uint4 qv[kPassUnroll], pv[kPassUnroll];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint4 qv[8], pv[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        qv[j] = ldg_v4_ordered(q + 8 * half + j);
-        pv[j] = ldg_v4_ordered(p + 8 * half + j);
+    for (int p = 0; p < kPassUnroll; ++p) {
+      const int t = r0 + p * kRowsPerPass + hw;   // row t = h * b + i
+      if (t < rows) {
+        qv[p] = __ldg(Q4 + static_cast<size_t>(t) * 16 + j);
+        pv[p] = __ldg(P4 + static_cast<size_t>(t) * 16 + j);
       }
+    }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t qw[4] = {qv[j].x, qv[j].y, qv[j].z, qv[j].w};
-        const uint32_t pw[4] = {pv[j].x, pv[j].y, pv[j].z, pv[j].w};
+    for (int p = 0; p < kPassUnroll; ++p) {
+      const int t = r0 + p * kRowsPerPass + hw;
+      double g = 0.0;   // this lane's group of 8 columns
+      if (t < rows) {
+        const uint32_t qw[4] = {qv[p].x, qv[p].y, qv[p].z, qv[p].w};
+        const uint32_t pw[4] = {pv[p].x, pv[p].y, pv[p].z, pv[p].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const double d0 = __dsub_rn(bf16_lo(qw[e]), bf16_lo(pw[e]));
-          sh = __dadd_rn(sh, __dmul_rn(d0, d0));
+          g = __dadd_rn(g, __dmul_rn(d0, d0));
           const double d1 = __dsub_rn(bf16_hi(qw[e]), bf16_hi(pw[e]));
-          sh = __dadd_rn(sh, __dmul_rn(d1, d1));
+          g = __dadd_rn(g, __dmul_rn(d1, d1));
         }
       }
+      // the row's 16 group sums, in order, by the half warp's lane 0
+      double row = 0.0;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) row = __dadd_rn(row, __shfl_sync(0xffffffffu, g, (tid & 16) + q));
+      if (j == 0 && t < rows) part[t] = row;
     }
-    part[t] = sh;
   }
-  if (tid < kMaxB) lst[tid] = 0;
   __syncthreads();
   if (tid < b) {
     double acc = 0.0;
@@ -127,12 +126,13 @@ __global__ void __launch_bounds__(kSelThreads) k_reuse_select(const SelectArgs a
     // stays total and exactly k tokens are selected)
     sc[tid] = s != s ? -INFINITY : s;
   }
+  if (tid < kMaxB) lst[tid] = 0;
   __syncthreads();
   if (tid < b) {
     // rank: tokens with a larger score, or an equal one and a lower index
     const double s = sc[tid];
     int rank = 0;
-    for (int j = 0; j < b; ++j) rank += (sc[j] > s || (sc[j] == s && j < tid)) ? 1 : 0;
+    for (int jj = 0; jj < b; ++jj) rank += (sc[jj] > s || (sc[jj] == s && jj < tid)) ? 1 : 0;
     act[tid] = rank < a.k ? 1 : 0;
   }
   __syncthreads();

@@ -318,8 +318,9 @@ int bha_state_prefill_ragged(const void *K, const void *V, const int *T_lens,
  *   active        [n][k] int32 or NULL: the active tokens of each request in
  *                 increasing order, written on steps that select (Qprev set,
  *                 0 < k < b), untouched otherwise
- * Other arguments as for bha_prefix_softmax.  bf16 only (BHA_F32 returns
- * BHA_ERR_UNSUPPORTED), and hq * b <= 8192 (else BHA_ERR_UNSUPPORTED).  The workspace size covers both kinds of step (first
+ * Other arguments as for bha_prefix_softmax, and hq * b <= 8192 (else
+ * BHA_ERR_UNSUPPORTED).  BHA_F32 is the CUDA-core reference mode (one CTA
+ * per query row; no workspace).  The workspace size covers both kinds of step (first
  * and later) for the given k.  Y must not overlap any input or the cache;
  * O_pre, L_pre and active must not overlap the inputs or each other.
  */

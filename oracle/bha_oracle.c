@@ -343,14 +343,19 @@ void oracle_losa_select(const double *Q, const double *Qprev, long n, long hq,
     for (ni = 0; ni < n; ++ni) {
         double *sc = score + ni * b;
         for (long i = 0; i < b; ++i) {
-            /* the squared change summed per head, then over the heads */
+            /* the squared change summed over groups of 8 columns, the groups
+             * of a head, then the heads: each level in index order */
             double acc = 0.0;
             for (long h = 0; h < hq; ++h) {
                 const double *q = Q + ((ni * hq + h) * b + i) * d;
                 const double *p = Qprev + ((ni * hq + h) * b + i) * d;
                 double sh = 0.0;
-                for (long c = 0; c < d; ++c)
-                    sh += (q[c] - p[c]) * (q[c] - p[c]);
+                for (long c0 = 0; c0 < d; c0 += 8) {
+                    double sg = 0.0;
+                    for (long c = c0; c < c0 + 8 && c < d; ++c)
+                        sg += (q[c] - p[c]) * (q[c] - p[c]);
+                    sh += sg;
+                }
                 acc += sh;
             }
             sc[i] = acc / (double)(hq * d);

@@ -294,7 +294,11 @@ def test_reuse_validation_and_workspace(L):
             kw.get("Lp", Lp), kw.get("act", act), kw.get("k", k), n, hq, hkv, b, d, 0.0,
             kw.get("dtype", _lib.BHA_BF16), kw.get("ws", 3 * big), kw.get("ws_bytes", need),
             None)
-    assert f(dtype=_lib.BHA_F32) == _lib.BHA_ERR_UNSUPPORTED
+    # fp32 reference mode: validated like bf16, no workspace, reaches the runtime
+    assert f(dtype=_lib.BHA_F32, ws=None, ws_bytes=0) == _lib.BHA_ERR_CUDA
+    assert L.bha_prefix_softmax_reuse(A, Qp, big, 2 * big, P, P, B, C, D, O, Lp, act, k, n, 512,
+                                      4, b, d, 0.0, _lib.BHA_BF16, 3 * big, need,
+                                      None) == _lib.BHA_ERR_UNSUPPORTED   # hq * b > 8192
     assert f(k=-1) == _lib.BHA_ERR_INVALID_ARG
     assert f(cap=100) == _lib.BHA_ERR_INVALID_ARG
     assert f(O=None) == _lib.BHA_ERR_INVALID_ARG

@@ -228,3 +228,54 @@ def test_reuse_selection_ties_go_to_the_lower_index():
     torch.cuda.synchronize()
     assert np.array_equal(act.cpu().numpy(), ract)
     assert list(ract[0]) == [5, 9, 20]
+
+
+F32_CASES = [  # (n, hq, hkv, b, d, P, k)
+    (1, 1, 1, 4, 16, 6, 2),      # the worked example's head size
+    (2, 4, 2, 13, 64, 37, 5),    # GQA, ragged block
+    (1, 8, 2, 32, 128, 300, 8),  # the model's head dim, several key chunks
+    (2, 4, 1, 5, 16, 0, 2),      # no cache
+]
+
+
+@pytest.mark.parametrize("n,hq,hkv,b,d,P,k", F32_CASES)
+def test_reuse_f32_block_loop(n, hq, hkv, b, d, P, k):
+    """fp32 reference mode: three denoising steps against the oracle at 1e-4
+    relative L2 (outputs and cache), the active lists bit-exact."""
+    import torch
+    from gpu_util import TOL_F32_REL
+    seed = 1500 + d + b + k
+    rng = np.random.default_rng(seed)
+    Kc = inputs.normal_f32_np(seed, inputs.TID_KC, (n, hkv, P + 3, d), 1.0)
+    Vc = inputs.normal_f32_np(seed, inputs.TID_VC, (n, hkv, P + 3, d), 1.0)
+    q = inputs.normal_f32_np(seed, inputs.TID_Q, (n, hq, b, d), 1.0)
+    Qs = [q]
+    for t in range(1, 3):
+        w = rng.exponential(1.0, size=(n, 1, b, 1)).astype(np.float32) ** 2
+        Qs.append((Qs[-1] + 0.3 * w * inputs.normal_f32_np(seed + t, 0, (n, hq, b, d), 1.0))
+                  .astype(np.float32))
+    Ks = [inputs.normal_f32_np(seed + 10 + t, inputs.TID_K, (n, hkv, b, d), 1.0) for t in range(3)]
+    Vs = [inputs.normal_f32_np(seed + 10 + t, inputs.TID_V, (n, hkv, b, d), 1.0) for t in range(3)]
+    O = torch.full((n, hq, b, d), float("nan"), device="cuda")
+    L = torch.full((n, hq, b), float("nan"), device="cuda")
+    Y = torch.empty(n, hq, b, d, device="cuda")
+    act = torch.full((n, max(k, 1)), -1, dtype=torch.int32, device="cuda")
+    rO = rL = None
+    dKc, dVc = dev_f32(Kc), dev_f32(Vc)
+    for t in range(3):
+        bha.bha_prefix_softmax_reuse(dev_f32(Qs[t]), None if t == 0 else dev_f32(Qs[t - 1]), dKc,
+                                     dVc, P, dev_f32(Ks[t]), dev_f32(Vs[t]), Y, O, L, k,
+                                     active=act)
+        torch.cuda.synchronize()
+        rY, rO, rL, ract = oracle.losa_step(Qs[t], None if t == 0 else Qs[t - 1], Kc, Vc, P,
+                                            Ks[t], Vs[t], rO, rL, k)
+        e = rel_l2(host(Y), rY)
+        log_parity("reuse_f32_y", rel_l2=e, step=t, d=d, b=b, k=k)
+        assert e <= TOL_F32_REL, (t, e)
+        assert rel_l2(host(O), rO) <= TOL_F32_REL or not np.any(rO)
+        fin = np.isfinite(rL)
+        assert np.array_equal(np.isfinite(host(L)), fin)
+        if fin.any():
+            assert float(np.max(np.abs(host(L)[fin] - rL[fin]))) <= 1e-4
+        if t > 0 and 0 < k < b:
+            assert np.array_equal(act.cpu().numpy()[:, :k], ract)
