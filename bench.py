@@ -747,8 +747,9 @@ def run_native(args, rank, world, local):
     if rank != 0:
         return
     # ---- secondary workloads on this GPU, from a clean device: the single
-    # step (batch 8), the generation loop against the exact path, and the
-    # 20-layer stack's largest batch before out-of-memory
+    # step (batch 8), the generation loop against the exact path, the exact
+    # path with reuse for stable tokens, and the 20-layer stack's largest
+    # batch before out-of-memory
     if not args.no_secondary:
         # drop every device buffer of the benchmark line
         sets = S0 = z0 = ws = st = dbuf = Kp = Vp = Kc = Vc = Yx = wsp = None
@@ -758,6 +759,7 @@ def run_native(args, rank, world, local):
         line["secondary"] = {
             "single_step_batch8": measure_single_step(dev),
             "generation_loop": measure_generation_loop(dev),
+            "reuse": measure_reuse(dev),
             "stack_memory": stack_oom(dev),
         }
     if not args.no_cpu:

@@ -318,3 +318,23 @@ def test_reuse_validation_and_workspace(L):
     assert f() == _lib.BHA_ERR_CUDA
     assert f(Qprev=None, act=None) == _lib.BHA_ERR_CUDA
     assert f(Kc=None, Vc=None, P=0, cap=0) == _lib.BHA_ERR_CUDA
+
+
+def test_product_path_and_oracle_share_nothing():
+    """The CUDA package never imports or loads the oracle, and the oracle never
+    imports the package (the seeded input generators live in the package's
+    `inputs` module, which holds no arithmetic of the method and is imported by
+    tests and the benchmark, not by the oracle)."""
+    pkg = os.path.join(ROOT, "block_hybrid_linear_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                text = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
+                assert "liboracle" not in text and "bha_oracle" not in text, f
+    odir = os.path.join(ROOT, "oracle")
+    for f in os.listdir(odir):
+        if f.endswith((".py", ".c", ".h")):
+            text = open(os.path.join(odir, f)).read()
+            assert not re.search(r"^\s*(import|from)\s+block_hybrid_linear_b200\b", text, re.M), f
+            assert "libbha" not in text and "#include \"bha" not in text, f
