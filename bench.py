@@ -527,9 +527,6 @@ def run_native(args, rank, world, local):
     assert bha.bha_device_error(True) == 0
 
     clocks = ClockSampler(local)
-    ks0, ks1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    kc0, kc1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    kd0, kd1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize()
     clocks.start()
@@ -540,28 +537,40 @@ def run_native(args, rank, world, local):
         ev0.record(stream)
         run_cycles(steps)
         ev1.record(stream)
-    # per-kernel durations, measured in the same run on the launching stream
-    # (at least 60 launches of each)
-    kreps = max(1, math.ceil(steps / (4 * g_cycles)))
-    ks0.record(stream)
-    for _ in range(kreps):
-        g_step.replay()
-    ks1.record(stream)
-    kc0.record(stream)
-    for _ in range(kreps):
-        g_commit.replay()
-    kc1.record(stream)
-    kd0.record(stream)
-    for _ in range(kreps):
-        g_shared.replay()
-    kd1.record(stream)
+    # per-kernel durations, measured in the same run on the launching stream:
+    # every replay of a kernel-only graph (60 or 30 back-to-back launches) timed
+    # on its own, at least 5 replays; the mean over replays is the roofline's
+    # launch time, the spread over replays is reported beside it
+    kreps = max(5, math.ceil(steps / (4 * g_cycles)))
+
+    def time_replays(g):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(kreps)]
+        for a_, b_ in evs:
+            a_.record(stream)
+            g.replay()
+            b_.record(stream)
+        return evs
+    ev_step, ev_commit, ev_shared = (time_replays(g_step), time_replays(g_commit),
+                                     time_replays(g_shared))
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
     t_ms = ev0.elapsed_time(ev1)
-    step_launch_ms = ks0.elapsed_time(ks1) / (kreps * 4 * R)
-    commit_launch_ms = kc0.elapsed_time(kc1) / (kreps * 2 * R)
-    shared_launch_ms = kd0.elapsed_time(kd1) / (kreps * 4 * R)
+
+    def per_launch(evs, launches):
+        return [a_.elapsed_time(b_) / launches for a_, b_ in evs]
+    step_ms_all = per_launch(ev_step, 4 * R)
+    commit_ms_all = per_launch(ev_commit, 2 * R)
+    shared_ms_all = per_launch(ev_shared, 4 * R)
+    step_launch_ms = sum(step_ms_all) / len(step_ms_all)
+    commit_launch_ms = sum(commit_ms_all) / len(commit_ms_all)
+    shared_launch_ms = sum(shared_ms_all) / len(shared_ms_all)
+
+    def spread_us(v):
+        q = sorted(x * 1e3 for x in v)
+        pick = lambda f: q[min(len(q) - 1, int(round(f * (len(q) - 1))))]
+        return {"p10": pick(0.1), "p50": pick(0.5), "p90": pick(0.9), "replays": len(q)}
     assert bha.bha_device_error(True) == 0
     t_ms = max_over_ranks(t_ms, pg, dev)
     value = job_throughput(steps * N_ * B_ * DENOISE, world, t_ms)
@@ -587,9 +596,11 @@ def run_native(args, rank, world, local):
                      "traffic": traffic_record("k_step_bf16", "k_step.cu"),
                      "algorithmic_bytes_per_launch": step_bytes,
                      "launch_us": step_launch_ms * 1e3,
+                     "launch_us_spread": spread_us(step_ms_all),
                      "shared_denom": {
                          "kernel": "k_step_bf16 (shared denominator)",
                          "launch_us": shared_launch_ms * 1e3,
+                         "launch_us_spread": spread_us(shared_ms_all),
                          "algorithmic_bytes_per_launch": shared_bytes,
                          "achieved": shared_bytes / (shared_launch_ms / 1e3) / 1e9,
                          "frac": shared_bytes / (shared_launch_ms / 1e3) / 1e9 / peak,
@@ -597,6 +608,7 @@ def run_native(args, rank, world, local):
         "hbm_roofline_frac": achieved / peak,
         "step_commit": {"kernel": "k_step_bf16 (fused commit)",
                         "launch_us": commit_launch_ms * 1e3,
+                        "launch_us_spread": spread_us(commit_ms_all),
                         "achieved_gbs": fused_bytes / (commit_launch_ms / 1e3) / 1e9,
                         "frac_of_peak": fused_bytes / (commit_launch_ms / 1e3) / 1e9 / peak,
                         "algorithmic_bytes_per_launch": fused_bytes,

@@ -111,6 +111,11 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 104);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 108);
 
+  // softmax warps with query rows in this tile (a ragged last tile, the reuse
+  // path's packed active rows); with a contiguous cache the others take no
+  // part in P's barrier at all
+  const int mt0 = (item / a.splits) % a.mtiles;
+  const int live_warps = PAGED ? 4 : min(4, max(1, (a.rows - mt0 * 128 + 31) / 32));
   if (warp == 0) {
     if (lane == 0) {
       mbar_init(bar_q, 1);
@@ -121,7 +126,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         mbar_init(bar_ve + 8 * s, 1);
         mbar_init(bar_sf + 8 * s, 1);
       }
-      mbar_init(bar_pf, 128);
+      mbar_init(bar_pf, 32 * live_warps);
       mbar_init(bar_pv, 1);
       *abort_flag = 0;
       fence_mbar_init();
@@ -273,10 +278,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   bool ok = true;
   // a warp whose 32 query rows are all past the tile's valid rows (a ragged
   // last query tile, the reuse path's packed active rows) computes no
-  // softmax: it keeps the barrier protocol and (paged) its share of clearing
+  // softmax; paged, it keeps the barrier protocol and its share of clearing
   // the V rows past the cache, which every output row's P V reads
   const bool rows_live = mt * 128 + (warp & 3) * 32 < a.rows;
-  if (warp >= 4 && live && !rows_live) {
+  if (warp >= 4 && live && !rows_live && PAGED) {
     for (int i = 0; i < nt; ++i) {
       const int st = i & 1;
       const int gi = tile0 + i;
@@ -301,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       mbar_arrive(bar_pf);
     }
     if (ok && nt > 0) ok = warp_all(mbar_wait(bar_pv, (nt - 1) & 1, a.err, abort_flag));
-  } else if (warp >= 4 && live) {
+  } else if (warp >= 4 && live && rows_live) {
     for (int i = 0; i < nt; ++i) {
       const int st = i & 1;
       const int gi = tile0 + i;
