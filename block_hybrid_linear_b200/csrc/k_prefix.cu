@@ -62,6 +62,32 @@ constexpr float kRescaleLog2 = 8.f;             // rescale O when max grows > 2^
 constexpr int kMinTilesPerChunk = 16;           // 1024 keys
 constexpr int kPagedTilesPerChunk = 32;         // 2048 keys
 
+// Two fp32 lanes at once (sm_100's packed fp32 pipe): d = a * b + c and
+// d = a + b, each lane rounded to nearest.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
+        "l"(*reinterpret_cast<uint64_t*>(&c)));
+  return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
+}
+// 2^x by the special-function unit (PTX ex2.approx, relative error below
+// 2^-22; results below 2^-126 flush to 0): the softmax weights of a tile,
+// x <= 0, relative to a row maximum of weight 1.
+__device__ __forceinline__ float ex2_sfu(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 struct PrefixArgs {
   int* err;
   const int* table;  // paged: [n][max_pages] page numbers
@@ -178,53 +204,59 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool direct = npieces == 1 && !a.prefix_only;
   const int slot = umt * a.splits + sp;   // partial numerator slot
 
+  // loads one K or V tile of the cache (through the page table) or of the block
+  auto load_tile = [&](const CUtensorMap* mc, const CUtensorMap* ma, uint32_t dst, uint32_t bar,
+                       int gi) {
+    if (gi >= ncache_tiles) {
+      mbar_arrive_expect_tx(bar, kTileBytes);
+      tma_load_3d(dst, ma, bar, 0, 0, u);
+      tma_load_3d(dst + kBox, ma, bar, 64, 0, u);
+    } else if (!PAGED) {
+      mbar_arrive_expect_tx(bar, kTileBytes);
+      tma_load_3d(dst, mc, bar, 0, gi * kTK, u);
+      tma_load_3d(dst + kBox, mc, bar, 64, gi * kTK, u);
+    } else {
+      const int t0 = gi * kTK;
+      const int* trow = a.table + static_cast<size_t>(nreq) * a.max_pages;
+      if (a.ps_log2 >= 6) {
+        // part of one page
+        const int pg = __ldg(trow + (t0 >> a.ps_log2));
+        const int row = t0 & ((1 << a.ps_log2) - 1);
+        mbar_arrive_expect_tx(bar, kTileBytes);
+        tma_load_3d(dst, mc, bar, 0, row, pg * a.hkv + g);
+        tma_load_3d(dst + kBox, mc, bar, 64, row, pg * a.hkv + g);
+      } else {
+        // 64 / page_size pages; only those holding cached tokens
+        const int ps = 1 << a.ps_log2;
+        const int npg = min(kTK >> a.ps_log2, (P - t0 + ps - 1) >> a.ps_log2);
+        mbar_arrive_expect_tx(bar, static_cast<uint32_t>(npg) * ps * 256);
+        for (int j = 0; j < npg; ++j) {
+          const int pg = __ldg(trow + (t0 >> a.ps_log2) + j);
+          tma_load_3d(dst + j * ps * 128, mc, bar, 0, 0, pg * a.hkv + g);
+          tma_load_3d(dst + kBox + j * ps * 128, mc, bar, 64, 0, pg * a.hkv + g);
+        }
+      }
+    }
+  };
   if (tid == 0 && live) {
-    // ---------------- TMA producer
+    // ---------------- TMA producer of Q and the K ring: a K stage is free
+    // once the score MMA has read it, well before P V frees the V stage of
+    // the same tile, so the two rings are refilled by separate threads
     const int row0 = mt * 128;
     mbar_arrive_expect_tx(bar_q, kQBytes);
     tma_load_3d(base + kOffQ, &tmQ, bar_q, 0, row0, u);
     tma_load_3d(base + kOffQ + 16384, &tmQ, bar_q, 64, row0, u);
-    // loads one K or V tile of the cache (through the page table) or of the block
-    auto load_tile = [&](const CUtensorMap* mc, const CUtensorMap* ma, uint32_t dst, uint32_t bar,
-                         int gi) {
-      if (gi >= ncache_tiles) {
-        mbar_arrive_expect_tx(bar, kTileBytes);
-        tma_load_3d(dst, ma, bar, 0, 0, u);
-        tma_load_3d(dst + kBox, ma, bar, 64, 0, u);
-      } else if (!PAGED) {
-        mbar_arrive_expect_tx(bar, kTileBytes);
-        tma_load_3d(dst, mc, bar, 0, gi * kTK, u);
-        tma_load_3d(dst + kBox, mc, bar, 64, gi * kTK, u);
-      } else {
-        const int t0 = gi * kTK;
-        const int* trow = a.table + static_cast<size_t>(nreq) * a.max_pages;
-        if (a.ps_log2 >= 6) {
-          // part of one page
-          const int pg = __ldg(trow + (t0 >> a.ps_log2));
-          const int row = t0 & ((1 << a.ps_log2) - 1);
-          mbar_arrive_expect_tx(bar, kTileBytes);
-          tma_load_3d(dst, mc, bar, 0, row, pg * a.hkv + g);
-          tma_load_3d(dst + kBox, mc, bar, 64, row, pg * a.hkv + g);
-        } else {
-          // 64 / page_size pages; only those holding cached tokens
-          const int ps = 1 << a.ps_log2;
-          const int npg = min(kTK >> a.ps_log2, (P - t0 + ps - 1) >> a.ps_log2);
-          mbar_arrive_expect_tx(bar, static_cast<uint32_t>(npg) * ps * 256);
-          for (int j = 0; j < npg; ++j) {
-            const int pg = __ldg(trow + (t0 >> a.ps_log2) + j);
-            tma_load_3d(dst + j * ps * 128, mc, bar, 0, 0, pg * a.hkv + g);
-            tma_load_3d(dst + kBox + j * ps * 128, mc, bar, 64, 0, pg * a.hkv + g);
-          }
-        }
-      }
-    };
     for (int i = 0; i < nt; ++i) {
       const int st = i & 1;
-      const int gi = tile0 + i;
       if (i >= 2 && !mbar_wait(bar_ke + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
-      load_tile(&tmKc, &tmKa, base + kOffK + st * kTileBytes, bar_kf + 8 * st, gi);
+      load_tile(&tmKc, &tmKa, base + kOffK + st * kTileBytes, bar_kf + 8 * st, tile0 + i);
+    }
+  } else if (tid == 64 && live) {
+    // ---------------- TMA producer of the V ring
+    for (int i = 0; i < nt; ++i) {
+      const int st = i & 1;
       if (i >= 2 && !mbar_wait(bar_ve + 8 * st, ((i >> 1) - 1) & 1, a.err, abort_flag)) break;
-      load_tile(&tmVc, &tmVa, base + kOffV + st * kTileBytes, bar_vf + 8 * st, gi);
+      load_tile(&tmVc, &tmVa, base + kOffV + st * kTileBytes, bar_vf + 8 * st, tile0 + i);
     }
   } else if (tid == 32 && live) {
     // ---------------- MMA issuer
@@ -322,12 +354,19 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int q = 0; q < 32; ++q) s[c + q] = t[q];
       }
-      float tmax = -INFINITY;
+      // keys past the cache (the last cache tile) or the block (its tile)
+      if (valid < kTK) {
 #pragma unroll
-      for (int j = 0; j < kTK; ++j) {
-        if (j >= valid) s[j] = -INFINITY;
-        tmax = fmaxf(tmax, s[j]);
+        for (int j = 0; j < kTK; ++j)
+          if (j >= valid) s[j] = -INFINITY;
       }
+      float m4[4] = {s[0], s[1], s[2], s[3]};
+#pragma unroll
+      for (int j = 4; j < kTK; j += 4) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], s[j + q]);
+      }
+      const float tmax = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
       float corr = 1.f;
       bool resc = false;
       if (mx == -INFINITY) {
@@ -337,13 +376,22 @@ __global__ void __launch_bounds__(kThreads, 2)
         mx = tmax;
         resc = true;
       }
-      float ls = 0.f;
+      // p = 2^{(s - mx) scale log2 e}, as s * (scale log2 e) - mx (scale log2 e)
+      const float2 sl = make_float2(a.sl2, a.sl2);
+      const float2 nb = make_float2(-mx * a.sl2, -mx * a.sl2);
+      float2 ls4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int j = 0; j < kTK; ++j) {
-        s[j] = exp2f((s[j] - mx) * a.sl2);
-        ls += s[j];
+      for (int j = 0; j < kTK; j += 2) {
+        float2 x = fma2(make_float2(s[j], s[j + 1]), sl, nb);
+        x.x = ex2_sfu(x.x);
+        x.y = ex2_sfu(x.y);
+        s[j] = x.x;
+        s[j + 1] = x.y;
+        ls4[(j >> 1) & 3] = add2(ls4[(j >> 1) & 3], x);
       }
-      l = l * corr + ls;
+      const float2 ls2 = add2(add2(ls4[0], ls4[1]), add2(ls4[2], ls4[3]));
+      l = l * corr + (ls2.x + ls2.y);
       // P and O are free once P V of the previous tile has completed
       if (i > 0) {
         ok = warp_all(mbar_wait(bar_pv, (i - 1) & 1, a.err, abort_flag));
