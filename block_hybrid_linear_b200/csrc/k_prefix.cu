@@ -527,16 +527,28 @@ __global__ void __launch_bounds__(256) k_prefix_merge(const float* __restrict__ 
   for (int s = 0; s < splits; ++s) M = fmaxf(M, wsML[(item0 + s) * 256 + r]);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float* ml = wsML + (item0 + s) * 256;
-    const float w = exp2f(ml[r] - M);
-    if (w == 0.f) continue;   // no weight (a row underflow): skip the read
-    den = fmaf(w, ml[128 + r], den);
-    const float4 o = reinterpret_cast<const float4*>(wsO + (item0 + s) * kD * kD + r * kD)[c4];
-    acc.x = fmaf(w, o.x, acc.x);
-    acc.y = fmaf(w, o.y, acc.y);
-    acc.z = fmaf(w, o.z, acc.z);
-    acc.w = fmaf(w, o.w, acc.w);
+  // eight chunks' loads in flight at a time; a chunk of no weight (a row
+  // underflow) contributes nothing, whatever its partial holds
+  for (int s0 = 0; s0 < splits; s0 += 8) {
+    float w[8], l[8];
+    float4 o[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int s = s0 + j < splits ? s0 + j : s0;
+      const float* ml = wsML + (item0 + s) * 256;
+      w[j] = s0 + j < splits ? exp2f(ml[r] - M) : 0.f;
+      l[j] = ml[128 + r];
+      o[j] = reinterpret_cast<const float4*>(wsO + (item0 + s) * kD * kD + r * kD)[c4];
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (w[j] == 0.f) continue;
+      den = fmaf(w[j], l[j], den);
+      acc.x = fmaf(w[j], o[j].x, acc.x);
+      acc.y = fmaf(w[j], o[j].y, acc.y);
+      acc.z = fmaf(w[j], o[j].z, acc.z);
+      acc.w = fmaf(w[j], o[j].w, acc.w);
+    }
   }
   const float inv = 1.f / den;
   __nv_bfloat162* out = reinterpret_cast<__nv_bfloat162*>(
