@@ -527,28 +527,35 @@ __global__ void __launch_bounds__(256) k_prefix_merge(const float* __restrict__ 
   for (int s = 0; s < splits; ++s) M = fmaxf(M, wsML[(item0 + s) * 256 + r]);
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   float den = 0.f;
-  // eight chunks' loads in flight at a time; a chunk of no weight (a row
-  // underflow) contributes nothing, whatever its partial holds
-  for (int s0 = 0; s0 < splits; s0 += 8) {
-    float w[8], l[8];
-    float4 o[8];
+  // four chunks' loads in flight at a time, then one by one; a chunk of no
+  // weight (a row underflow) contributes nothing, whatever its partial holds
+  auto add = [&](float w, float l, float4 o) {
+    if (w == 0.f) return;
+    den = fmaf(w, l, den);
+    acc.x = fmaf(w, o.x, acc.x);
+    acc.y = fmaf(w, o.y, acc.y);
+    acc.z = fmaf(w, o.z, acc.z);
+    acc.w = fmaf(w, o.w, acc.w);
+  };
+  int s = 0;
+  for (; s + 4 <= splits; s += 4) {
+    float w[4], l[4];
+    float4 o[4];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int s = s0 + j < splits ? s0 + j : s0;
-      const float* ml = wsML + (item0 + s) * 256;
-      w[j] = s0 + j < splits ? exp2f(ml[r] - M) : 0.f;
+    for (int j = 0; j < 4; ++j) {
+      const float* ml = wsML + (item0 + s + j) * 256;
+      w[j] = exp2f(ml[r] - M);
       l[j] = ml[128 + r];
-      o[j] = reinterpret_cast<const float4*>(wsO + (item0 + s) * kD * kD + r * kD)[c4];
+      o[j] = reinterpret_cast<const float4*>(wsO + (item0 + s + j) * kD * kD + r * kD)[c4];
     }
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (w[j] == 0.f) continue;
-      den = fmaf(w[j], l[j], den);
-      acc.x = fmaf(w[j], o[j].x, acc.x);
-      acc.y = fmaf(w[j], o[j].y, acc.y);
-      acc.z = fmaf(w[j], o[j].z, acc.z);
-      acc.w = fmaf(w[j], o[j].w, acc.w);
-    }
+    for (int j = 0; j < 4; ++j) add(w[j], l[j], o[j]);
+  }
+  for (; s < splits; ++s) {
+    const float* ml = wsML + (item0 + s) * 256;
+    const float w = exp2f(ml[r] - M);
+    if (w == 0.f) continue;
+    add(w, ml[128 + r], reinterpret_cast<const float4*>(wsO + (item0 + s) * kD * kD + r * kD)[c4]);
   }
   const float inv = 1.f / den;
   __nv_bfloat162* out = reinterpret_cast<__nv_bfloat162*>(
