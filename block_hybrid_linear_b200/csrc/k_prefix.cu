@@ -62,32 +62,6 @@ constexpr float kRescaleLog2 = 8.f;             // rescale O when max grows > 2^
 constexpr int kMinTilesPerChunk = 16;           // 1024 keys
 constexpr int kPagedTilesPerChunk = 32;         // 2048 keys
 
-// Two fp32 lanes at once (sm_100's packed fp32 pipe): d = a * b + c and
-// d = a + b, each lane rounded to nearest.
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-  uint64_t d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
-        "l"(*reinterpret_cast<uint64_t*>(&c)));
-  return *reinterpret_cast<float2*>(&d);
-}
-__device__ __forceinline__ float2 add2(float2 a, float2 b) {
-  uint64_t d;
-  asm("add.rn.f32x2 %0, %1, %2;"
-      : "=l"(d)
-      : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
-  return *reinterpret_cast<float2*>(&d);
-}
-// 2^x by the special-function unit (PTX ex2.approx, relative error below
-// 2^-22; results below 2^-126 flush to 0): the softmax weights of a tile,
-// x <= 0, relative to a row maximum of weight 1.
-__device__ __forceinline__ float ex2_sfu(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
 struct PrefixArgs {
   int* err;
   const int* table;  // paged: [n][max_pages] page numbers

@@ -498,18 +498,35 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
 #pragma unroll
         for (int q = 0; q < 16; ++q) sc[j + q] = t[q];
       }
-      float m = -INFINITY;
+      // keys past the block (padding of the MMA's N)
+      if (a.b < BPAD) {
 #pragma unroll
-      for (int j = 0; j < BPAD; ++j) {
-        if (j >= a.b) sc[j] = -INFINITY;
-        m = fmaxf(m, sc[j]);
+        for (int j = 0; j < BPAD; ++j)
+          if (j >= a.b) sc[j] = -INFINITY;
       }
-      float l = 0.f;
+      float m4[4] = {sc[0], sc[1], sc[2], sc[3]};
 #pragma unroll
-      for (int j = 0; j < BPAD; ++j) {
-        sc[j] = exp2f((sc[j] - m) * a.scale_log2);
-        l += sc[j];
+      for (int j = 4; j < BPAD; j += 4) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) m4[q] = fmaxf(m4[q], sc[j + q]);
       }
+      const float m = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+      // e_j = 2^{s_j scale log2 e - m scale log2 e}, on the packed fp32 pipe
+      const float2 sl = make_float2(a.scale_log2, a.scale_log2);
+      const float2 nb = make_float2(-m * a.scale_log2, -m * a.scale_log2);
+      float2 l4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                      make_float2(0.f, 0.f)};
+#pragma unroll
+      for (int j = 0; j < BPAD; j += 2) {
+        float2 x = fma2(make_float2(sc[j], sc[j + 1]), sl, nb);
+        x.x = ex2_sfu(x.x);
+        x.y = ex2_sfu(x.y);
+        sc[j] = x.x;
+        sc[j + 1] = x.y;
+        l4[(j >> 1) & 3] = add2(l4[(j >> 1) & 3], x);
+      }
+      const float2 l2 = add2(add2(l4[0], l4[1]), add2(l4[2], l4[3]));
+      const float l = l2.x + l2.y;
       if (SHARED) {
         // y = (sum_j e^{s_j - c} v_j + e^{-c} phi(q) S) / (sum_j e^{s_j - c} +
         // e^{-c} phi(q).z) for any c; e_j = e^{s_j - m_s} above, m_s = scale * m.
@@ -540,13 +557,14 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       const uint32_t prow = base + kOffP + (r >> 3) * (8 * Lay::kRowB) + (r & 7) * Lay::kRowB;
       const uint32_t swz = Lay::kRowB == 128 ? (r & 7) : Lay::kRowB == 64 ? ((r & 7) >> 1)
                                                                           : ((r & 7) >> 2);
+      const float2 ps = make_float2(pscale, pscale);
 #pragma unroll
       for (int jj = 0; jj < BPAD / 8; ++jj) {
         const float* e = sc + 8 * jj;
-        st_shared_v4(prow + ((jj ^ swz) << 4), pack_bf16x2(e[0] * pscale, e[1] * pscale),
-                     pack_bf16x2(e[2] * pscale, e[3] * pscale),
-                     pack_bf16x2(e[4] * pscale, e[5] * pscale),
-                     pack_bf16x2(e[6] * pscale, e[7] * pscale));
+        const float2 p0 = mul2(make_float2(e[0], e[1]), ps), p1 = mul2(make_float2(e[2], e[3]), ps),
+                     p2 = mul2(make_float2(e[4], e[5]), ps), p3 = mul2(make_float2(e[6], e[7]), ps);
+        st_shared_v4(prow + ((jj ^ swz) << 4), pack_bf16x2(p0.x, p0.y), pack_bf16x2(p1.x, p1.y),
+                     pack_bf16x2(p2.x, p2.y), pack_bf16x2(p3.x, p3.y));
       }
     }
     fence_proxy_async_smem();
