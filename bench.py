@@ -221,6 +221,34 @@ def e2e_counts(steps, warmup):
     return max(E2E_MIN_CYCLES, int(steps)), max(E2E_MIN_WARMUP, int(warmup))
 
 
+def parse_cpulist(text):
+    """CPU numbers of a sysfs cpulist ("0-3,8,10-11" -> {0, 1, 2, 3, 8, 10, 11})."""
+    cpus = set()
+    for part in text.strip().split(","):
+        if not part:
+            continue
+        lo, _, hi = part.partition("-")
+        cpus.update(range(int(lo), int(hi or lo) + 1))
+    return cpus
+
+
+def gpu_host_locality(dev):
+    """(NUMA node, CPUs of that node this process may use) of the GPU's PCI
+    device, from sysfs; (None, set()) when the platform does not say."""
+    import torch
+    p = torch.cuda.get_device_properties(dev)
+    path = "/sys/bus/pci/devices/%04x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id,
+                                                       p.pci_device_id)
+    try:
+        with open(os.path.join(path, "numa_node")) as f:
+            node = int(f.read())
+        with open(os.path.join(path, "local_cpulist")) as f:
+            cpus = parse_cpulist(f.read())
+    except (OSError, ValueError):
+        return None, set()
+    return node, cpus & os.sched_getaffinity(0)
+
+
 def job_throughput(tokens_per_rank, world, time_ms):
     """Whole-job tokens/s: every rank's tokens over the slowest rank's time."""
     return tokens_per_rank * world / (time_ms / 1e3)
@@ -691,11 +719,22 @@ def run_native(args, rank, world, local):
     if not args.no_e2e:
         st = sets[0]
         nq, nk = st["Q"].numel(), st["K"].numel()
-        hQKV = torch.cat([st[k].reshape(-1).cpu() for k in ("Q", "K", "V")]).pin_memory()
+        # the pinned buffers on the GPU's own NUMA node: allocated and first
+        # written by this thread while it runs on that node's CPUs (copies
+        # from a far node's memory cross the socket link on every step)
+        numa_node, local_cpus = gpu_host_locality(dev)
+        old_cpus = os.sched_getaffinity(0)
+        if local_cpus:
+            os.sched_setaffinity(0, local_cpus)
+        try:
+            hQKV = torch.cat([st[k].reshape(-1).cpu() for k in ("Q", "K", "V")]).pin_memory()
+            hY = torch.empty(st["Y"].shape, dtype=torch.bfloat16).pin_memory()
+            hY.zero_()
+        finally:
+            os.sched_setaffinity(0, old_cpus)
         hQ = hQKV[:nq].view(st["Q"].shape)
         hK = hQKV[nq:nq + nk].view(st["K"].shape)
         hV = hQKV[nq + nk:].view(st["V"].shape)
-        hY = torch.empty(st["Y"].shape, dtype=torch.bfloat16).pin_memory()
         dbuf = []
         for _ in range(2):
             flat = torch.empty_like(hQKV, device=dev)
@@ -745,9 +784,23 @@ def run_native(args, rank, world, local):
         e2e_ms = max_over_ranks(e2e_ms, pg, dev)
         h2d = DENOISE * (hQ.numel() + hK.numel() + hV.numel()) * 2
         d2h = DENOISE * hY.numel() * 2
+        # the link alone: one copy each way of the same buffers, after the loop
+        link = {}
+        for name, dst, src, nbytes in (("h2d_gbs", dbuf[0]["QKV"], hQKV, hQKV.numel() * 2),
+                                       ("d2h_gbs", hY, dbuf[0]["Y"], hY.numel() * 2)):
+            e0l, e1l = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0l.record(stream)
+            with torch.cuda.stream(stream):
+                for _ in range(5):
+                    dst.copy_(src, non_blocking=True)
+            e1l.record(stream)
+            torch.cuda.synchronize()
+            link[name] = 5 * nbytes / (e0l.elapsed_time(e1l) / 1e3) / 1e9
         line["e2e"] = {"value": job_throughput(n_e2e * N_ * B_ * DENOISE, world, e2e_ms),
                        "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                        "d2h_bytes_per_step": d2h, "steps": n_e2e, "warmup": warm_e2e,
+                       "host_numa_node": numa_node, "host_buffers_local": bool(local_cpus),
+                       "link_alone": link,
                        "note": "block cycles: --steps and --warmup, at least %d and %d"
                                % (E2E_MIN_CYCLES, E2E_MIN_WARMUP)}
         line["gpu_launches_e2e"] = n_e2e * DENOISE

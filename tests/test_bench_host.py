@@ -93,3 +93,10 @@ def test_graph_plan_runs_exactly_the_requested_cycles():
 def test_e2e_counts_follow_steps_with_a_floor():
     assert bench.e2e_counts(20, 5) == (bench.E2E_MIN_CYCLES, bench.E2E_MIN_WARMUP)
     assert bench.e2e_counts(200, 40) == (200, 40)
+
+
+def test_parse_cpulist():
+    """The sysfs cpulist format of a PCI device's local CPUs."""
+    assert bench.parse_cpulist("0-3,8,10-11\n") == {0, 1, 2, 3, 8, 10, 11}
+    assert bench.parse_cpulist("5") == {5}
+    assert bench.parse_cpulist("\n") == set()
