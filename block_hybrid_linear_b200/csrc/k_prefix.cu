@@ -10,11 +10,14 @@
 //     tiles first, the active block last; 113 KB of shared memory and 256
 //     TMEM columns, so two CTAs share an SM and one's prologue, pipeline
 //     fill and epilogue overlap the other's stream;
-//   * a TMA thread streams K and V tiles through 2-stage rings, an MMA
-//     thread issues S = Q K^T into one of two TMEM buffers and O += P V into
-//     a TMEM accumulator, and four softmax warps (thread = query row = TMEM
-//     lane) run the online softmax in registers, rescaling O only when a row
-//     max grows by more than 2^8 (the stale max is exact for the final ratio);
+//   * two TMA threads stream K and V tiles through 2-stage rings (a K stage
+//     is refilled once the score MMA has read it, without waiting for the V
+//     stage of the same tile), an MMA thread issues S = Q K^T into one of two
+//     TMEM buffers and O += P V into a TMEM accumulator, and four softmax
+//     warps (thread = query row = TMEM lane) run the online softmax in
+//     registers -- exponentials on the packed fp32 pipe and the SFU, the key
+//     mask only in a partial tile -- rescaling O only when a row max grows by
+//     more than 2^8 (the stale max is exact for the final ratio);
 //   * chunks are combined by log-sum-exp in a second kernel, the way the
 //     LoSA page describes merging prefix and block attention with online
 //     softmax.  With one chunk the CTA normalises and stores Y itself.
