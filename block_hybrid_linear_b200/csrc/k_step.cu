@@ -204,6 +204,11 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   constexpr bool PROJ = FMAP == kFmapReluProj;
   static_assert(!(HALF && PROJ), "column halves: elementwise maps only");
   constexpr int kN = HALF ? 64 : 128;                   // output columns of this CTA
+  // Column halves in the default mode (small grids, latency bound): the
+  // state is requested with Q, the scores sit in the accumulator's unused
+  // upper half, and tid 0 (once phi(Q) is in) issues the phi(Q) S products
+  // as the state lands, then P V, while the row owners run the softmax.
+  constexpr bool EARLY = HALF && !SHARED && !COMMIT && !REUSE;
   constexpr uint32_t kChunkS = HALF ? 8192 : 16384;     // bytes of one state chunk here
   using Lay = StepLayout<BPAD>;
   // P (the softmax weights, bf16, K-major) goes over the consumed K tile, or
@@ -297,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   // warps 0-3 hand each row's phi(q) . z to the row owners through that
   // row's own bytes of the consumed Q tile (row r of Q is read by thread r
   // alone, and by the MMAs that bar_sc / bar_qw complete).
-  const uint32_t t_sc = t_d;
+  const uint32_t t_sc = EARLY ? t_d + 64 : t_d;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   pdl_wait();   // inputs may come from the previous kernel of the stream
 
@@ -341,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     }
     // the projected map's state chunks 0-1 (2-3 follow over W_g)
     if (PROJ) load_state_chunks(0, 2);
+    if (EARLY) load_state_chunks(0, 4);
   }
 
   float beta = 1.f;   // per-row output scale (shared denominator only)
@@ -367,11 +373,42 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       okf = warp_all(mbar_wait(bar_q, 0, a.err, abort_flag));
       // state chunk w from warp w: the issue cost is spread over the warps
       // that build phi(Q), which the phi(Q) S products wait for
-      if (okf && lane == 0) load_state_chunks(warp, warp + 1);
+      if (!EARLY && okf && lane == 0) load_state_chunks(warp, warp + 1);
       if (okf) qz = write_phiq<FMAP, SHARED>(base + kOffQ, warp * 32 + lane, t_a + lane_base, zl);
     }
     tc_fence_before();
     mbar_arrive(bar_a);   // phi(Q) is in TMEM
+    if (EARLY && tid == 0) {
+      // the four state chunks' products as they land (the state was
+      // requested with Q, so it usually lands before P is ready), then P V:
+      // a fixed order, so that the result does not depend on timing
+      bool ok3 = mbar_wait(bar_a, 0, a.err, abort_flag);
+      for (int c = 0; c < 4 && ok3; ++c) {
+        ok3 = mbar_wait(bar_s + 8 * c, 0, a.err, abort_flag);
+        if (!ok3) break;
+        tc_fence_after();
+        constexpr uint32_t idesc = make_idesc_tf32(128, kN, 0, 1);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+          const uint64_t db = make_sdesc(base + kOffS + c * kChunkS + kk * 1024, 4096, 512,
+                                         kLayoutSW128_32B);
+          mma_tf32_ts(t_d, t_a + 32 * c + 8 * kk, db, idesc, (c | kk) ? 1u : 0u);
+        }
+      }
+      ok3 = ok3 && mbar_wait(bar_p, 0, a.err, abort_flag) && mbar_wait(bar_v, 0, a.err, abort_flag);
+      if (ok3) {
+        tc_fence_after();
+        constexpr uint32_t idesc = make_idesc_bf16(128, kN, 0, 1);
+#pragma unroll
+        for (int ks = 0; ks < BPAD / 16; ++ks) {
+          const uint64_t da = make_sdesc(base + kOffP + ks * 32, 16, 8 * Lay::kRowB, Lay::kPLayout);
+          const uint64_t db =
+              make_sdesc(base + Lay::kOffV + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
+          mma_bf16_ss(t_d, da, db, idesc, 1u);
+        }
+        mma_commit(bar_done);
+      }
+    }
     if (SHARED) {
       // phi(q) . z to the row owners, over row tid of the Q tile once the
       // score MMA (or, projected, Q W_g) has read it
@@ -574,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     // MMA issuer (a row owner too): P V as soon as P and V are in, before
     // its own row's shared-denominator work below
     bool ok2 = true;
-    if (tid == 128) {
+    if (!EARLY && tid == 128) {
       ok2 = mbar_wait(bar_p, 0, a.err, abort_flag) && mbar_wait(bar_v, 0, a.err, abort_flag) &&
             (!(COMMIT && PROJ) || mbar_wait(bar_kwr, 0, a.err, abort_flag));
       if (ok2) {
@@ -613,7 +650,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       }
       if (ok2) mma_commit(bar_done);
     };
-    if (!REUSE && tid == 128 && !rescale) issue_products();
+    if (!REUSE && !EARLY && tid == 128 && !rescale) issue_products();
 
     if (SHARED) {
       // phi(q) . z from warps 0-3; the output's 1 / denominator, and for rows
