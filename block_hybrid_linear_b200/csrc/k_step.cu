@@ -208,7 +208,11 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
   // state is requested with Q, the scores sit in the accumulator's unused
   // upper half, and tid 0 (once phi(Q) is in) issues the phi(Q) S products
   // as the state lands, then P V, while the row owners run the softmax.
-  constexpr bool EARLY = HALF && !SHARED && !COMMIT && !REUSE;
+  // With the shared denominator the products go first only when no row of
+  // the tile moves e^{-m} into its phi(q) (the row owners say so on bar_m
+  // once their row maxima are known); otherwise P V goes first and the
+  // products follow the rows' rescaling, as in the whole-unit order.
+  constexpr bool EARLY = HALF && !COMMIT && !REUSE;
   constexpr uint32_t kChunkS = HALF ? 8192 : 16384;     // bytes of one state chunk here
   using Lay = StepLayout<BPAD>;
   // P (the softmax weights, bf16, K-major) goes over the consumed K tile, or
@@ -233,7 +237,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
                  bar_sc = ctrl + 56, bar_p = ctrl + 64, bar_a = ctrl + 72, bar_done = ctrl + 80,
                  bar_phik = ctrl + 96, bar_ds = ctrl + 104, bar_w = ctrl + 112,
                  bar_qw = ctrl + 120, bar_kwr = ctrl + 128, bar_a2 = ctrl + 136,
-                 bar_qz = ctrl + 144;
+                 bar_qz = ctrl + 144, bar_m = ctrl + 160;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(ctrl_ptr + 88);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(ctrl_ptr + 92);
   // shared denominator: set by a row owner whose row scales its phi(q) (row
@@ -252,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       if (SHARED) {
         mbar_init(bar_a2, 128);
         mbar_init(bar_qz, 128);
+        if (EARLY) mbar_init(bar_m, 128);
         *rescale_flag = 0;
       }
       mbar_init(bar_done, 1);
@@ -378,25 +383,33 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     }
     tc_fence_before();
     mbar_arrive(bar_a);   // phi(Q) is in TMEM
-    if (EARLY && tid == 0) {
+    auto issue_early = [&]() {
       // the four state chunks' products as they land (the state was
       // requested with Q, so it usually lands before P is ready), then P V:
       // a fixed order, so that the result does not depend on timing
       bool ok3 = mbar_wait(bar_a, 0, a.err, abort_flag);
-      for (int c = 0; c < 4 && ok3; ++c) {
-        ok3 = mbar_wait(bar_s + 8 * c, 0, a.err, abort_flag);
-        if (!ok3) break;
-        tc_fence_after();
-        constexpr uint32_t idesc = make_idesc_tf32(128, kN, 0, 1);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          const uint64_t db = make_sdesc(base + kOffS + c * kChunkS + kk * 1024, 4096, 512,
-                                         kLayoutSW128_32B);
-          mma_tf32_ts(t_d, t_a + 32 * c + 8 * kk, db, idesc, (c | kk) ? 1u : 0u);
-        }
+      bool late = false;   // shared denominator: some row rescales its phi(q)
+      if (SHARED && ok3) {
+        ok3 = mbar_wait(bar_m, 0, a.err, abort_flag);
+        late = ok3 && *rescale_flag != 0;
       }
-      ok3 = ok3 && mbar_wait(bar_p, 0, a.err, abort_flag) && mbar_wait(bar_v, 0, a.err, abort_flag);
-      if (ok3) {
+      auto products = [&](bool acc) {
+        for (int c = 0; c < 4 && ok3; ++c) {
+          ok3 = mbar_wait(bar_s + 8 * c, 0, a.err, abort_flag);
+          if (!ok3) break;
+          tc_fence_after();
+          constexpr uint32_t idesc = make_idesc_tf32(128, kN, 0, 1);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t db = make_sdesc(base + kOffS + c * kChunkS + kk * 1024, 4096, 512,
+                                           kLayoutSW128_32B);
+            mma_tf32_ts(t_d, t_a + 32 * c + 8 * kk, db, idesc, (acc || c || kk) ? 1u : 0u);
+          }
+        }
+      };
+      auto pv = [&](bool acc) {
+        ok3 = ok3 && mbar_wait(bar_p, 0, a.err, abort_flag) && mbar_wait(bar_v, 0, a.err, abort_flag);
+        if (!ok3) return;
         tc_fence_after();
         constexpr uint32_t idesc = make_idesc_bf16(128, kN, 0, 1);
 #pragma unroll
@@ -404,17 +417,28 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
           const uint64_t da = make_sdesc(base + kOffP + ks * 32, 16, 8 * Lay::kRowB, Lay::kPLayout);
           const uint64_t db =
               make_sdesc(base + Lay::kOffV + ks * 2048, BPAD * 128, 1024, kLayoutSW128);
-          mma_bf16_ss(t_d, da, db, idesc, 1u);
+          mma_bf16_ss(t_d, da, db, idesc, (acc || ks) ? 1u : 0u);
         }
-        mma_commit(bar_done);
+      };
+      if (!late) {
+        products(false);
+        pv(true);
+      } else {
+        // the rescaled phi(q) rows are in TMEM once bar_a2 completes
+        pv(false);
+        ok3 = ok3 && mbar_wait(bar_a2, 0, a.err, abort_flag);
+        products(true);
       }
-    }
+      if (ok3) mma_commit(bar_done);
+    };
+    if (EARLY && !SHARED && tid == 0) issue_early();
     if (SHARED) {
       // phi(q) . z to the row owners, over row tid of the Q tile once the
       // score MMA (or, projected, Q W_g) has read it
       if (okf && (PROJ || warp_all(mbar_wait(bar_sc, 0, a.err, abort_flag))))
         st_shared_f32(base + kOffQ + tid * 128, qz);
       mbar_arrive(bar_qz);
+      if (EARLY && tid == 0) issue_early();
     }
     if (COMMIT && PROJ) {
       // thread = feature r: row r of (K W_g)^T (landed with Q W_g) out of
@@ -575,6 +599,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
         pscale = m2 > kSharedShiftLog2 ? 1.f : exp2f(m2);
         lsum = l;
         if (m2 > kSharedShiftLog2) *rescale_flag = 1;   // before this row's bar_p arrive
+        if (EARLY) mbar_arrive(bar_m);
       } else {
         pscale = 1.f / l;   // default: P is normalised, the terms add as they are
       }
@@ -604,6 +629,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
                      pack_bf16x2(p2.x, p2.y), pack_bf16x2(p3.x, p3.y));
       }
     }
+    if (SHARED && EARLY && !ok) mbar_arrive(bar_m);
     fence_proxy_async_smem();
     tc_fence_before();
     mbar_arrive(bar_p);
@@ -631,7 +657,7 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
     // denominator) a row of the tile has to scale its phi(q) first, in which
     // case they follow the row owners' shared-denominator work (bar_a2)
     bool rescale = false;
-    if (SHARED && tid == 128 && ok2) rescale = *rescale_flag != 0;
+    if (SHARED && !EARLY && tid == 128 && ok2) rescale = *rescale_flag != 0;
     auto issue_products = [&]() {
       if (ok2) ok2 = mbar_wait(SHARED && rescale ? bar_a2 : bar_a, 0, a.err, abort_flag);
       for (int c = 0; c < 4 && ok2; ++c) {
