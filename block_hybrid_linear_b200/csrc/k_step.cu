@@ -9,18 +9,21 @@
 //
 // One CTA per (request n, KV head g, 128-row tile of the G*b query rows that
 // share g); on grids of at most one CTA per SM, two CTAs per tile, each
-// computing half of the output columns (HALF, below).  TMA brings Q, K, V first; the fp32 state S (four 32-row chunks)
-// is requested once this CTA's Q has landed, so that across the grid the
-// softmax operands are not queued behind the state (measured: 2 % faster in
-// the default mode, 4 % with the shared denominator):
+// computing half of the output columns (HALF, below).  TMA brings Q, K, V
+// first; the fp32 state S (four 32-row chunks) is requested once this CTA's
+// Q has landed, so that across the grid the softmax operands are not queued
+// behind the state (measured: 2 % faster in the default mode, 4 % with the
+// shared denominator); column halves outside the fused commit request it
+// with Q (EARLY, below):
 //   Q   128 x 128 bf16  (2 SW128 boxes, K-major)               32 KB
 //   S   128 x 128 fp32  (16 boxes of 32 rows x 32 cols, 32B-atom swizzle)  64 KB
 //   K,V BPAD x 128 bf16 (2 SW128 boxes each)                   2 x 8 KB at BPAD=32
-// Work (TMEM columns: D = [0,128), scores then phi(Q) = [128,256)):
+// Work (TMEM columns: D = [0,128), the scores in its first BPAD columns until
+// P V overwrites them; phi(Q) = [128,256)):
 //   MMA (bf16)  scores = Q K^T                    M=128 N=BPAD K=128
-//   warps 4-7 (thread = query row = TMEM lane): row softmax in registers,
-//        P -> smem over the consumed K tile; then phi(q) as fp32 into TMEM
-//        over the consumed scores
+//   warps 0-3 (thread = query row = TMEM lane): phi(q) as fp32 into TMEM
+//   warps 4-7 (likewise): row softmax in registers, P -> smem over the
+//        consumed K tile
 //   MMA (bf16)  D  = P V                          M=128 N=128 K=BPAD
 //   MMA (tf32)  D += phi(Q)[TMEM] S[smem]  per state chunk, as it lands
 //   all 8 warps: D -> bf16 -> swizzled tile -> TMA store, per 64-column half
