@@ -103,6 +103,30 @@ def test_step_bf16_scale_and_zero_state():
     check_bf16("step_bf16_scale", host(Y), ref)
 
 
+@pytest.mark.parametrize("n", [2, 64], ids=["halves", "whole_units"])
+def test_step_bf16_is_deterministic(n):
+    """The MMA order is fixed in every path (column halves issue the state
+    products and P V in a set order, not in the order their operands land),
+    so repeated calls on the same inputs give the same bits; scale 4 makes
+    some rows of the shared-denominator tile take the rescaled order."""
+    import torch
+    hq, hkv, b = 16, 4, 32
+    Q, _ = bf16_case((9, 0), (n, hq, b, 128), 1.0)
+    K, _ = bf16_case((9, 1), (n, hkv, b, 128), 1.0)
+    V, _ = bf16_case((9, 2), (n, hkv, b, 128), 1.0)
+    Sv, zv = inputs.synthetic_state_np(9, n, hkv, 128, 4096, STD)
+    S, z = dev_f32(Sv), dev_f32(zv)
+    for flags, scale in ((0, 0.0), (bha.BHA_FLAG_SHARED_DENOM, 0.0),
+                         (bha.BHA_FLAG_SHARED_DENOM, 4.0)):
+        outs = []
+        for _ in range(3):
+            Y = torch.empty(n, hq, b, 128, dtype=torch.bfloat16, device="cuda")
+            bha.bha_hybrid_step(Q, K, V, S, Y, z=z, scale=scale, flags=flags)
+            outs.append(Y)
+        torch.cuda.synchronize()
+        assert all(torch.equal(outs[0], o) for o in outs[1:]), (n, flags, scale)
+
+
 @pytest.mark.parametrize("scale", [1.0, 4.0])
 def test_step_bf16_shared_large_scores(scale):
     """Shared denominator with unit-variance inputs: row maxima of the scaled
