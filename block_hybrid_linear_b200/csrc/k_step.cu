@@ -133,6 +133,22 @@ __device__ __forceinline__ float write_phiq(uint32_t qtile, int r, uint32_t tcol
   return (qz[0] + qz[1]) + (qz[2] + qz[3]);
 }
 
+// phi(q_r) . z from phi(q_r) as written to TMEM (this thread's lane, 128
+// columns from `tcol`): the same values and the same four partial sums, in
+// the same order, as write_phiq<FMAP, true>, read back after phi(Q) has been
+// handed to the tensor core so that the products need not wait for them.
+__device__ __forceinline__ float qz_from_tmem(uint32_t tcol, float4 zl) {
+  float qz[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int cg = 0; cg < 4; ++cg) {
+    float f[32];
+    tmem_ld32_sync(tcol + cg * 32, f);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) qz[e & 3] = fmaf(f[e], z_at(zl, cg * 32 + e), qz[e & 3]);
+  }
+  return (qz[0] + qz[1]) + (qz[2] + qz[3]);
+}
+
 // Projected map: the Q W_g product sits in TMEM (this thread's lane, 128
 // columns from `tcol`); replace it by max(., 0).  QZ: also returns
 // phi(q_r) . z (z spread over the lanes as for write_phiq).
@@ -382,10 +398,14 @@ __global__ void __launch_bounds__(kThreads, BPAD <= 32 ? 2 : 1)
       // state chunk w from warp w: the issue cost is spread over the warps
       // that build phi(Q), which the phi(Q) S products wait for
       if (!EARLY && okf && lane == 0) load_state_chunks(warp, warp + 1);
-      if (okf) qz = write_phiq<FMAP, SHARED>(base + kOffQ, warp * 32 + lane, t_a + lane_base, zl);
+      // shared denominator: phi(q) . z along the way with column halves
+      // (their products wait for it, see issue_early), read back from TMEM
+      // once phi(Q) is handed over otherwise (the products need not wait)
+      if (okf) qz = write_phiq<FMAP, SHARED && HALF>(base + kOffQ, warp * 32 + lane, t_a + lane_base, zl);
     }
     tc_fence_before();
     mbar_arrive(bar_a);   // phi(Q) is in TMEM
+    if (SHARED && !HALF && !PROJ && okf) qz = qz_from_tmem(t_a + lane_base, zl);
     auto issue_early = [&]() {
       // the four state chunks' products as they land (the state was
       // requested with Q, so it usually lands before P is ready), then P V:
