@@ -232,13 +232,9 @@ def parse_cpulist(text):
     return cpus
 
 
-def gpu_host_locality(dev):
-    """(NUMA node, CPUs of that node this process may use) of the GPU's PCI
-    device, from sysfs; (None, set()) when the platform does not say."""
-    import torch
-    p = torch.cuda.get_device_properties(dev)
-    path = "/sys/bus/pci/devices/%04x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id,
-                                                       p.pci_device_id)
+def pci_locality(path, allowed):
+    """(NUMA node, CPUs of that node among `allowed`) of the PCI device whose
+    sysfs folder is `path`; (None, set()) when the platform does not say."""
     try:
         with open(os.path.join(path, "numa_node")) as f:
             node = int(f.read())
@@ -246,7 +242,16 @@ def gpu_host_locality(dev):
             cpus = parse_cpulist(f.read())
     except (OSError, ValueError):
         return None, set()
-    return node, cpus & os.sched_getaffinity(0)
+    return node, cpus & set(allowed)
+
+
+def gpu_host_locality(dev):
+    """pci_locality of the GPU's PCI device, for the CPUs this process may use."""
+    import torch
+    p = torch.cuda.get_device_properties(dev)
+    path = "/sys/bus/pci/devices/%04x:%02x:%02x.0" % (p.pci_domain_id, p.pci_bus_id,
+                                                       p.pci_device_id)
+    return pci_locality(path, os.sched_getaffinity(0))
 
 
 def job_throughput(tokens_per_rank, world, time_ms):

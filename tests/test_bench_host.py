@@ -100,3 +100,14 @@ def test_parse_cpulist():
     assert bench.parse_cpulist("0-3,8,10-11\n") == {0, 1, 2, 3, 8, 10, 11}
     assert bench.parse_cpulist("5") == {5}
     assert bench.parse_cpulist("\n") == set()
+
+
+def test_pci_locality_reads_sysfs_and_intersects(tmp_path):
+    """The e2e leg's host-buffer placement: the GPU's NUMA node and its CPUs
+    among those this process may use; nothing when sysfs does not say."""
+    (tmp_path / "numa_node").write_text("1\n")
+    (tmp_path / "local_cpulist").write_text("8-15,24\n")
+    assert bench.pci_locality(str(tmp_path), {0, 8, 9, 24, 30}) == (1, {8, 9, 24})
+    assert bench.pci_locality(str(tmp_path / "missing"), {0, 1}) == (None, set())
+    (tmp_path / "numa_node").write_text("-1\n")
+    assert bench.pci_locality(str(tmp_path), range(32))[0] == -1
